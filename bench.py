@@ -1,0 +1,370 @@
+"""Benchmark of the rotate-then-quantize hot path on B200 (one JSON line).
+
+Workload: the attention-projection layer shape of the image DiTs in the
+OrbitQuant write-up (hotelren.com/news/3376620, §3): d_in = d_out = 3072,
+4608 tokens (a 64 x 64 latent patch grid + 512 text tokens), W4A4, RPBH h = 64.
+Synthetic seeded data: Student-t(3) activations with 1% of channels x30,
+N(0, 0.02^2) weights, both BF16.
+
+One step = one pass of the whole path over one batch:
+  rotate_quantize_act (x' = Pi x, norm, Lloyd-Max codes)  [HBM-bound]
+  quantize_weights    (the same fused kernel on W's rows)  [HBM-bound]
+  qlinear             (codes -> fp16 tiles -> tcgen05 MMA)  [tensor-bound]
+Each kernel is bracketed by CUDA events on the launching stream.  Inputs
+rotate over enough buffer sets that every step reads from HBM, not L2.
+
+`value` is rotate_quantize_act throughput in GB/s of algorithmic bytes
+(2d bytes in + d*b/8 + 4 bytes out per token); the qlinear TFLOP/s, the
+roofline of the dominant kernel and the CPU oracle's own throughput ride
+along.  --impl reference times the fp64 CPU oracle on the same workload.
+"""
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
+METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
+WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
+
+
+def act_bytes_per_token(d=D, bits=BITS_A):
+    return 2 * d + d * bits // 8 + 4
+
+
+def weight_bytes_per_row(d=D, bits=BITS_W):
+    return 2 * d + d * bits // 8 + 2
+
+
+def to_bf16_tensor(x, dev):
+    """BF16-valued fp32 numpy array -> torch.bfloat16 tensor on `dev`."""
+    import torch
+    return torch.from_numpy(synth.bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx),
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 3:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+                mask = int(parts[2], 16)
+            except ValueError:
+                continue
+            for bit, name in _REASONS.items():
+                if mask & bit and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world):
+    import torch
+    import rotation_bit_ptq_b200 as rbq
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    data = synth.attn_proj(seed=SEED + rank)
+    X_host = data["X"]
+    W_host = data["W"]
+    r = rbq.RPBH(D, SEED)
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_set = X_host.nbytes // 2 + W_host.nbytes // 2
+    nsets = max(2, int(np.ceil(3 * l2 / per_set)))
+    Xs = [to_bf16_tensor(X_host, dev) for _ in range(nsets)]
+    Ws = [to_bf16_tensor(W_host, dev) for _ in range(nsets)]
+    a_codes = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev) for _ in range(nsets)]
+    norms = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(nsets)]
+    w_codes = [torch.empty((D, D * BITS_W // 8), dtype=torch.uint8, device=dev) for _ in range(nsets)]
+    rnorm = [torch.empty((D,), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    Y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+
+    def step(i, ev=None):
+        k = i % nsets
+        if ev:
+            ev[0].record(stream)
+        rbq.rotate_quantize_act(r, Xs[k], BITS_A, a_codes[k], norms[k], stream=stream)
+        if ev:
+            ev[1].record(stream)
+        rbq.quantize_weights(r, Ws[k], BITS_W, "lloydmax", w_codes[k], rnorm[k], stream=stream)
+        if ev:
+            ev[2].record(stream)
+        rbq.qlinear(a_codes[k], norms[k], BITS_A, w_codes[k], rnorm[k], BITS_W, D, Y, stream=stream)
+        if ev:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    k1 = [e[0].elapsed_time(e[1]) for e in evs]
+    k1w = [e[1].elapsed_time(e[2]) for e in evs]
+    k2 = [e[2].elapsed_time(e[3]) for e in evs]
+    times = torch.tensor([total_ms, sum(k1), sum(k1w), sum(k2)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, k1_ms, k1w_ms, k2_ms = times.tolist()
+
+    act_bytes = act_bytes_per_token() * T
+    flops = 2.0 * T * D * D
+    gbs = act_bytes * args.steps * world / (k1_ms * 1e-3) / 1e9
+    k1_avg_s = k1_ms / args.steps * 1e-3
+    k2_avg_s = k2_ms / args.steps * 1e-3
+    tflops = flops * args.steps * world / (k2_ms * 1e-3) / 1e12
+    wgbs = weight_bytes_per_row() * D * args.steps * world / (k1w_ms * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 or world > 1:
+        e2e = run_e2e(r, X_host, dev, stream, args)
+
+    res = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; BF16 Student-t(3) activations with 1% outlier channels x30, N(0,0.02^2) weights)",
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": T, "d_in": D, "d_out": D, "bits_a": BITS_A,
+                   "bits_w": BITS_W, "parallelism": f"replicas x{world} (tokens sharded, no collective)",
+                   "l2": f"{nsets} rotating input sets ({nsets * per_set / 2**20:.0f} MiB > L2 {l2 / 2**20:.0f} MiB)"},
+        "rotate_quantize": {"GB/s": round(gbs, 2), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                            "avg_us": round(k1_avg_s * 1e6, 3)},
+        "quantize_weights": {"GB/s": round(wgbs, 2), "frac_hbm": round(wgbs / pk["hbm_gbs"], 4),
+                             "avg_us": round(k1w_ms / args.steps * 1e3, 3)},
+        "qlinear": {"TFLOP/s": round(tflops, 2), "frac_bf16": round(tflops / pk["bf16_tflops"], 4),
+                    "avg_us": round(k2_avg_s * 1e6, 3)},
+        "roofline": {"kernel": "qlinear", "bound": "tensor", "achieved": round(flops / k2_avg_s / 1e12, 2),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": None,
+                     "peak_source": pk["source"] + " bf16 burst"},
+        "roofline_rotate_quantize": {"kernel": "rotate_quantize_act", "bound": "hbm",
+                                     "achieved": round(act_bytes / k1_avg_s / 1e9, 2), "peak": pk["hbm_gbs"],
+                                     "unit": "GB/s", "frac": round(act_bytes / k1_avg_s / 1e9 / pk["hbm_gbs"], 4),
+                                     "traffic": None, "peak_source": pk["source"]},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    return res
+
+
+def run_e2e(r, X_host, dev, stream, args):
+    """rotate_quantize_act through the public API from pinned host memory:
+    H2D of X, the kernel, D2H of codes and norms, every step."""
+    import torch
+    import rotation_bit_ptq_b200 as rbq
+    xh = torch.from_numpy(synth.bf16_bits(X_host).view(np.int16)).view(torch.bfloat16).pin_memory()
+    xd = torch.empty_like(xh, device=dev)
+    ch = torch.empty((T, D * BITS_A // 8), dtype=torch.uint8).pin_memory()
+    nh = torch.empty((T,), dtype=torch.float32).pin_memory()
+    cd = torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev)
+    nd = torch.empty((T,), dtype=torch.float32, device=dev)
+
+    def one():
+        xd.copy_(xh, non_blocking=True)
+        rbq.rotate_quantize_act(r, xd, BITS_A, cd, nd, stream=stream)
+        ch.copy_(cd, non_blocking=True)
+        nh.copy_(nd, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    return {"value": round(act_bytes_per_token() * T * args.steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(ch.numel() + nh.numel() * 4)}
+
+
+# ---------------------------------------------------------------------------
+# oracle (CPU) timings
+# ---------------------------------------------------------------------------
+
+def oracle_rotq_gbs(tokens, min_seconds, rank_seed=0):
+    """The fp64 oracle's rotate-then-quantize on `tokens` tokens of the workload,
+    repeated until `min_seconds` passed.  Returns (GB/s, seconds, reps)."""
+    import oracle
+    data = synth.attn_proj(seed=rank_seed)
+    X = data["X"][:tokens].astype(np.float64)
+    perm, signs = oracle.rpbh_draw(D, SEED)
+    Pi = oracle.rpbh_matrix(perm, signs)
+    _, bounds = oracle.lloydmax_table(D, BITS_A)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        out = oracle.quantize_act(X, Pi, bounds)
+        oracle.pack_codes(out["codes"], BITS_A)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return act_bytes_per_token() * tokens * reps / el / 1e9, el, reps
+
+
+def cpu_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args):
+    """The oracle, as it stands, timed per step on a bounded token sample."""
+    tokens = 512
+    for _ in range(args.warmup):
+        oracle_rotq_gbs(tokens, 0.0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_rotq_gbs(tokens, 0.0)
+    el = time.perf_counter() - t0
+    gbs = act_bytes_per_token() * tokens * args.steps / el / 1e9
+    cores = cpu_cores()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": {"workload": WORKLOAD, "tokens_per_step": tokens},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{tokens} of {T} tokens per step, dense fp64 Pi (numpy)"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            gbs, el, reps = oracle_rotq_gbs(T, 10.0)
+            res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                                   "sample": f"all {T} tokens x {reps} reps ({el:.1f} s), dense fp64 Pi (numpy)"}
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,206 @@
+/*
+ * rbq.h -- C ABI of the B200 rotate-then-quantize library (librbq.so).
+ *
+ * The library implements the data-parallel hot path of rotation-based
+ * post-training quantisation for diffusion-transformer linear layers:
+ *
+ *   OrbitQuant (write-up at hotelren.com/news/3376620):
+ *     §2.3  the random-permuted block-Hadamard rotation (RPBH)
+ *           Pi_d = blkdiag(H_64 D_1, ..., H_64 D_{d/64}) · P_pi;
+ *     §1, §4.2  one Lloyd-Max codebook per input width d for N(0, 1/d);
+ *     §2.1  offline weights: W' = W Pi^T, row norms r' (BF16), direction codes;
+ *     §2.2  online activations: x' = Pi x, norm s, direction codes; the rotation
+ *           cancels inside the linear, y = r' s sum_k C_w[q] C_a[p].
+ *   INT8-convrot ("INT8旋转量化是什么", cloud.baidu.com/article/9430339) §4 and
+ *   the rotated-model explainer (cloud.baidu.com/article/9432521) §4:
+ *     rotate, then symmetric INT8 with a per-output-channel scale; inference
+ *     either dequantises or runs an INT8 operator (here: W8A16).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor arguments are DEVICE pointers to memory the caller allocated
+ *   (for example with PyTorch); the library never frees them.  Row-major,
+ *   no padding between rows.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *   stream).  Kernel calls are asynchronous on that stream; there is no hidden
+ *   device-wide synchronisation.
+ * - The return value is RBQ_OK (0) or a negative RBQ_E* code.  Arguments are
+ *   validated before anything is launched, so a call that returns
+ *   RBQ_EINVAL / RBQ_EALIGN has written nothing.  RBQ_ECUDA reports a failed
+ *   launch or allocation inside the library; rbq_error_string() names it.
+ * - The first compute call that uses an RPBH handle or a (d, bits) codebook on
+ *   a device uploads small tables to that device synchronously (a few KB).
+ *   Make that first call before capturing a stream into a CUDA graph.
+ * - Dense inputs are BF16 (RBQ_BF16) or fp32 (RBQ_F32), d a multiple of 64.
+ * - Packed codes: code j of a row occupies bits [j*b, j*b+b) of the row's
+ *   little-endian bitstream (LSB first); the row pitch is d*b/8 bytes.
+ *   (The pages do not fix a bit layout; this is the library's.)
+ */
+#ifndef RBQ_H
+#define RBQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ------------------------------------------------------ */
+#define RBQ_OK          0
+#define RBQ_EINVAL     (-1)  /* bad size, bit width, mode, dtype or NULL pointer */
+#define RBQ_EALIGN     (-2)  /* pointer not aligned as documented               */
+#define RBQ_ECUDA      (-3)  /* CUDA launch / allocation / copy failed          */
+#define RBQ_ENOMEM     (-4)  /* host allocation failed                          */
+#define RBQ_ECONVERGE  (-5)  /* Lloyd-Max solver did not converge               */
+#define RBQ_EDEVICE    (-6)  /* kernel reported an internal error (see below)   */
+
+/* ---- element types and modes --------------------------------------------- */
+#define RBQ_F32    0
+#define RBQ_BF16   1
+
+#define RBQ_LLOYDMAX   0   /* OrbitQuant direction codes + BF16 row norms     */
+#define RBQ_INT8_SYM   1   /* symmetric per-output-channel INT8 + fp32 scales */
+
+#define RBQ_ROTATE_ONLY 16 /* `bits` value of rotate_quantize_act: x' only  */
+
+/* ---- RPBH transform (OrbitQuant §2.3) ------------------------------------ */
+
+/* Opaque handle: the permutation pi and signs D of one Pi_d, on the host and
+ * (after first use) on each device that used it. */
+typedef struct rbq_rpbh rbq_rpbh;
+
+/*
+ * rpbh_make -- draw Pi_d = blkdiag(H_h D_1 ... H_h D_{d/h}) · P_pi from `seed`.
+ *   d     input width, a positive multiple of h, at most 32768
+ *   h     Hadamard block size; must be 64
+ *   seed  any 64-bit value
+ *   out   receives the new handle (free with rpbh_free)
+ * The draw is fixed by this library (the pages ask only that it be
+ * reproducible across platforms, OrbitQuant §6.3): SplitMix64 started at
+ * `seed`; Fisher-Yates for i = d-1..1 with j = floor(u*(i+1)/2^64); then d
+ * sign draws, D_k = -1 when the top bit is set.  (P_pi x)_k = x_{pi(k)}.
+ * H_h is the Sylvester-order Walsh-Hadamard matrix scaled by 1/sqrt(h).
+ * Host only: works without a GPU.  Errors: RBQ_EINVAL, RBQ_ENOMEM.
+ */
+int rpbh_make(int d, int h, uint64_t seed, rbq_rpbh** out);
+
+/* rpbh_free -- release a handle and its device copies (NULL is a no-op).
+ * The caller must ensure no launched kernel still uses it. */
+void rpbh_free(rbq_rpbh* r);
+
+/* rpbh_export -- copy pi (int32[d]) and D (int8[d], +-1) to HOST buffers.
+ * Either pointer may be NULL.  Errors: RBQ_EINVAL. */
+int rpbh_export(const rbq_rpbh* r, int32_t* perm_host, int8_t* signs_host);
+
+/* rpbh_dim -- d of a handle, or RBQ_EINVAL for NULL. */
+int rpbh_dim(const rbq_rpbh* r);
+
+/* ---- Lloyd-Max codebook (OrbitQuant §1, §4.2) ---------------------------- */
+
+/*
+ * lloydmax_table -- MSE-optimal 2^bits-level quantiser of N(0, 1/d).
+ *   d       input width (> 0); the table is the N(0,1) table times 1/sqrt(d)
+ *   bits    1..8
+ *   levels  HOST double[2^bits], increasing, antisymmetric (may be NULL)
+ *   bounds  HOST double[2^bits - 1], the midpoints of adjacent levels; the
+ *           middle one is exactly 0 (may be NULL)
+ * Solved in fp64 by Newton's method on the centroid/midpoint conditions.
+ * Host only.  Errors: RBQ_EINVAL, RBQ_ECONVERGE.
+ */
+int lloydmax_table(int d, int bits, double* levels, double* bounds);
+
+/* ---- rotate-then-quantise kernels ---------------------------------------- */
+
+/*
+ * rotate_quantize_act -- online activation quantiser (OrbitQuant §2.2),
+ * one fused kernel per call.  For every token row x of X[T, d]:
+ *   x' = Pi_d x;  s = ||x'||_2 (fp32);  v = x' / (s + 1e-12);
+ *   code_k = #{ j : t_j <= v_k }  over the Lloyd-Max boundaries of (d, bits)
+ *            (nearest level, ties to the upper level);
+ *   codes row = packed codes (LSB-first bitstream, d*bits/8 bytes).
+ *   r       RPBH handle of width d
+ *   X       device, T x d, dtype RBQ_BF16 or RBQ_F32, 16-byte aligned
+ *   T       number of tokens (0 is a valid no-op)
+ *   bits    1..8, or RBQ_ROTATE_ONLY: then `codes_out` receives x' itself as
+ *           BF16 [T, d] (round to nearest even) -- the activation operand of
+ *           qlinear_int8 -- and `norms_out` may be NULL
+ *   codes_out  device, T x (d*bits/8) bytes, 16-byte aligned
+ *   norms_out  device float[T], s per token, 4-byte aligned
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int rotate_quantize_act(const rbq_rpbh* r, const void* X, int dtype, int T,
+                        int bits, void* codes_out, float* norms_out,
+                        void* stream);
+
+/*
+ * quantize_weights -- offline weight quantiser, the same fused kernel run on
+ * the d_out rows of W[d_out, d] (each row w_i becomes w'_i = Pi_d w_i, i.e.
+ * W' = W Pi^T, OrbitQuant §2.1).
+ *   mode RBQ_LLOYDMAX: bits 1..8; `codes_or_q` = packed direction codes
+ *        (d_out x d*bits/8 bytes); `rownorm_or_scale` = uint16 BF16 r'_i =
+ *        bf16(||w'_i||) (round to nearest even).  Directions are w'/(r + 1e-12)
+ *        with the fp32 norm r.
+ *   mode RBQ_INT8_SYM: bits must be 8; `codes_or_q` = int8 q [d_out, d];
+ *        `rownorm_or_scale` = float scale_i = max_k |w'_ik| / 127;
+ *        q = clamp(round_half_even(w' / scale), -127, 127); a zero row gives
+ *        scale 0 and q 0 (INT8-convrot §4; the zero point is 0).
+ *   W  device, d_out x d, dtype RBQ_BF16 or RBQ_F32, 16-byte aligned.
+ *   Output pointers 16-byte (codes/q) and 4-byte (norms/scales) aligned.
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int d_out,
+                     int mode, int bits, void* codes_or_q,
+                     void* rownorm_or_scale, void* stream);
+
+/* ---- quantised linear layers --------------------------------------------- */
+
+/*
+ * qlinear -- OrbitQuant §2.2 (the rotation cancels):
+ *   Y[m, n] = bf16( s[m] * r'[n] * sum_k C_w[q[n,k]] * C_a[p[m,k]] ),
+ * with C_a / C_w the Lloyd-Max levels of (K, bits_a) / (K, bits_w), operands
+ * expanded on the fly into tensor-core tiles, fp32 accumulation.
+ *   a_codes  device, M x (K*bits_a/8) bytes, from rotate_quantize_act
+ *   s        device float[M], norms from rotate_quantize_act
+ *   w_codes  device, N x (K*bits_w/8) bytes, from quantize_weights
+ *   rnorm    device uint16 BF16[N], row norms from quantize_weights
+ *   M, N, K  tokens, output width, input width (K a multiple of 64)
+ *   Y        device uint16 BF16 [M, N], row-major
+ * Alignment: code arrays 16-byte, Y 16-byte, s/rnorm 4-byte.
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int qlinear(const uint8_t* a_codes, const float* s, int bits_a,
+            const uint8_t* w_codes, const uint16_t* rnorm, int bits_w,
+            int M, int N, int K, uint16_t* Y, void* stream);
+
+/*
+ * qlinear_int8 -- W8A16 linear of the INT8 path (INT8-convrot §4):
+ *   Y[m, n] = bf16( scale[n] * sum_k q[n,k] * Xrot[m,k] ),
+ * Xrot = bf16(Pi x) from rotate_quantize_act(bits = RBQ_ROTATE_ONLY), q and
+ * scale from quantize_weights(RBQ_INT8_SYM).  fp32 accumulation.
+ *   Xrot   device uint16 BF16 [M, K];  Wq device int8 [N, K];
+ *   scale  device float[N];  Y device uint16 BF16 [M, N]
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float* scale,
+                 int M, int N, int K, uint16_t* Y, void* stream);
+
+/* ---- diagnostics ----------------------------------------------------------- */
+
+/* Text for a return code (static storage). */
+const char* rbq_error_string(int code);
+
+/*
+ * rbq_device_error -- synchronise `stream`, then read and clear the device
+ * error word of the current device.  Kernels that wait on shared-memory
+ * barriers give every wait an iteration limit; when a limit runs out the
+ * kernel records a non-zero word, abandons the tile and exits instead of
+ * hanging.  Returns 0 when clean, RBQ_EDEVICE after such an event, RBQ_ECUDA
+ * if the synchronisation itself failed.
+ */
+int rbq_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RBQ_H */

@@ -45,7 +45,7 @@ qlinear.*              pure-Python triple loop; equal-code closed form
 """
 
 from .rng import splitmix64, rpbh_draw
-from .rpbh import hadamard, rpbh_matrix, rpbh_apply
+from .rpbh import hadamard, rpbh_matrix, rpbh_rows, rpbh_apply
 from .lloydmax import lloydmax_unit, lloydmax_table, lloydmax_distortion_unit
 from .bf16 import round_to_bf16
 from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
@@ -54,7 +54,7 @@ from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
 from .qlinear import qlinear, qlinear_int8
 
 __all__ = [
-    "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_apply",
+    "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_rows", "rpbh_apply",
     "lloydmax_unit", "lloydmax_table", "lloydmax_distortion_unit",
     "round_to_bf16", "assign_codes", "pack_codes", "unpack_codes",
     "quantize_act", "quantize_weights_lloydmax", "quantize_weights_int8",

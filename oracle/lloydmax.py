@@ -16,10 +16,11 @@ sigma has its optimal quantiser scaled by sigma).
 
 Numerics (our reading of "compute in fp64"): a cell probability on the
 positive side is taken as Q(a) - Q(b) with Q the upper tail, so that the far
-tails keep their relative precision; the iteration stops when no level moves
-by more than ``tol``.  The fixed-point map contracts slowly for many levels
-(rate ~0.9999 at 8 bits), so its answer sits within ~1e-9 of the exact
-optimum at 6-8 bits and within ~1e-14 at <= 4 bits.  The levels are made
+tails keep their relative precision; the iteration runs until the levels stop
+moving (below 1e-15, or no new smallest move for 2000 steps: the fp64
+rounding floor).  The map contracts slowly for many levels (rate ~0.9999 at 8
+bits), which amplifies rounding, so the answer sits within ~1e-11 of the
+exact optimum at 8 bits and ~1e-14 at <= 4 bits.  The levels are made
 exactly antisymmetric at the end, which puts the middle boundary at 0.
 """
 
@@ -53,17 +54,20 @@ def _x_pdf(x):
 
 
 @functools.lru_cache(maxsize=None)
-def lloydmax_unit(bits, tol=1e-13, max_iter=2_000_000):
+def lloydmax_unit(bits, tol=1e-15, stall=2000, max_iter=3_000_000):
     """Lloyd-Max quantiser of N(0,1) with 2**bits levels.
 
     Returns (levels[2**bits], bounds[2**bits - 1], iterations), increasing,
     levels antisymmetric.  Iteration: levels start uniform on (-4, 4); then
-    repeat  t = midpoints(c);  c = centroids(t)  until max |dc| < tol.
+    repeat  t = midpoints(c);  c = centroids(t)  until no level moves by more
+    than ``tol``, or until the largest move has not set a new minimum for
+    ``stall`` iterations (the map has reached its fp64 rounding floor).
     """
     if not 1 <= bits <= 8:
         raise ValueError("bits must be in 1..8")
     L = 2 ** bits
     c = (np.arange(L) - (L - 1) / 2.0) * (8.0 / L)
+    best, since_best = np.inf, 0
     for it in range(1, max_iter + 1):
         t = 0.5 * (c[:-1] + c[1:])
         lo = np.concatenate(([-np.inf], t))
@@ -73,6 +77,12 @@ def lloydmax_unit(bits, tol=1e-13, max_iter=2_000_000):
         c = c_new
         if step < tol:
             break
+        if step < best:
+            best, since_best = step, 0
+        else:
+            since_best += 1
+            if since_best >= stall and best < 1e-12:
+                break
     else:
         raise RuntimeError(f"Lloyd-Max iteration did not converge at {bits} bits")
     c = 0.5 * (c - c[::-1])

@@ -55,20 +55,47 @@ def permutation_matrix(perm):
     return P
 
 
-def rpbh_matrix(perm, signs, h=64):
-    """Dense Pi_d = B · P_pi.
+def rpbh_rows(perm, signs, r0, r1, h=64):
+    """Rows r0 .. r1-1 of the dense Pi_d = B · P_pi (r0, r1 multiples of h).
 
     Row k of P_pi selects input coordinate perm[k], so the product B · P_pi
-    is B with column m moved to column perm[m].  That column move is what is
-    computed here (a d^3 matmul at d = 12288 would take hours); the test-suite
-    checks it against the literal product B @ P at small d.
+    is B with column m moved to column perm[m]; within output block b that
+    places the 64 x 64 piece H_h D_b at the columns perm[64b .. 64b+63].  (A
+    d^3 matmul at d = 12288 would take hours; the test-suite checks this
+    column move against the literal product B @ P at small d.)
     """
-    B = block_part(signs, h)
-    Pi = np.empty_like(B)
-    Pi[:, np.asarray(perm)] = B
-    return Pi
+    perm = np.asarray(perm)
+    signs = np.asarray(signs, dtype=np.float64)
+    d = perm.shape[0]
+    if d % h or r0 % h or r1 % h or not 0 <= r0 <= r1 <= d:
+        raise ValueError("rows must be whole blocks of h")
+    H = hadamard(h)
+    out = np.zeros((r1 - r0, d))
+    for b in range(r0 // h, r1 // h):
+        sl = slice(b * h, (b + 1) * h)
+        out[b * h - r0: (b + 1) * h - r0, perm[sl]] = H @ np.diag(signs[sl])
+    return out
 
 
-def rpbh_apply(Pi, X):
-    """x' = Pi x for each row x of X (OrbitQuant §2.2 step 1)."""
-    return np.asarray(X, dtype=np.float64) @ Pi.T
+def rpbh_matrix(perm, signs, h=64):
+    """The dense d x d Pi_d = B · P_pi."""
+    return rpbh_rows(perm, signs, 0, len(perm), h)
+
+
+def rpbh_apply(Pi, X, chunk=2048):
+    """x' = Pi x for each row x of X (OrbitQuant §2.2 step 1).
+
+    ``Pi`` is the dense matrix, or a (perm, signs) pair for widths whose dense
+    matrix is too large to hold: then Pi is built and applied ``chunk`` rows
+    at a time -- the same dense product, in pieces.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    if isinstance(Pi, tuple):
+        perm, signs = Pi
+        d = len(perm)
+        out = np.empty((X.shape[0], d))
+        for r0 in range(0, d, chunk):
+            r1 = min(d, r0 + chunk)
+            out[:, r0:r1] = X @ rpbh_rows(perm, signs, r0, r1).T
+        return out
+    return X @ Pi.T

@@ -1,0 +1,255 @@
+"""Python binding of librbq.so, the B200 rotate-then-quantize library.
+
+Argument marshalling only: every step of the path runs inside the library's
+CUDA kernels (see include/rbq.h for the C ABI).  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library is
+missing every call raises.
+
+Sources: the OrbitQuant write-up (hotelren.com/news/3376620) §2.1-§2.3 and
+§4.2, and INT8-convrot (cloud.baidu.com/article/9430339) §4.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librbq.so")
+
+RBQ_F32, RBQ_BF16 = 0, 1
+RBQ_LLOYDMAX, RBQ_INT8_SYM = 0, 1
+RBQ_ROTATE_ONLY = 16
+RBQ_OK, RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA, RBQ_ENOMEM, RBQ_ECONVERGE, RBQ_EDEVICE = 0, -1, -2, -3, -4, -5, -6
+
+# name -> (restype, argtypes); mirrors include/rbq.h
+_P, _I, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
+SIGNATURES = {
+    "rpbh_make": (_I, [_I, _I, _U64, ctypes.POINTER(_P)]),
+    "rpbh_free": (None, [_P]),
+    "rpbh_export": (_I, [_P, _P, _P]),
+    "rpbh_dim": (_I, [_P]),
+    "lloydmax_table": (_I, [_I, _I, _P, _P]),
+    "rotate_quantize_act": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
+    "quantize_weights": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "qlinear": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "qlinear_int8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "rbq_error_string": (ctypes.c_char_p, [_I]),
+    "rbq_device_error": (_I, [_P]),
+}
+
+_lib = None
+
+
+class RBQError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        msg = lib().rbq_error_string(code).decode() if _lib is not None else str(code)
+        super().__init__(f"{where}: {msg} ({code})")
+
+
+def lib():
+    """Load librbq.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m rotation_bit_ptq_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(rc, where):
+    if rc != RBQ_OK:
+        raise RBQError(rc, where)
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _need_cuda(t, name, dtype=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return RBQ_BF16
+    if t.dtype == torch.float32:
+        return RBQ_F32
+    raise TypeError("dense inputs must be bfloat16 or float32")
+
+
+# ---------------------------------------------------------------------------
+# RPBH handle and codebook (host)
+# ---------------------------------------------------------------------------
+
+class RPBH:
+    """Pi_d = blkdiag(H_64 D_1, ..., H_64 D_{d/64}) · P_pi drawn from `seed`."""
+
+    def __init__(self, d, seed, h=64):
+        out = ctypes.c_void_p()
+        _check(lib().rpbh_make(int(d), int(h), ctypes.c_uint64(seed & (2 ** 64 - 1)), ctypes.byref(out)),
+               "rpbh_make")
+        self._h = out
+        self.d = int(d)
+        self.seed = int(seed)
+
+    @property
+    def handle(self):
+        if self._h is None:
+            raise ValueError("RPBH handle already freed")
+        return self._h
+
+    def export(self):
+        perm = np.empty(self.d, dtype=np.int32)
+        signs = np.empty(self.d, dtype=np.int8)
+        _check(lib().rpbh_export(self.handle, perm.ctypes.data_as(_P), signs.ctypes.data_as(_P)),
+               "rpbh_export")
+        return perm, signs
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and _lib is not None:
+            _lib.rpbh_free(self._h)
+        self._h = None
+
+    def __del__(self):
+        self.close()
+
+
+def lloydmax_table(d, bits):
+    """(levels[2^bits], bounds[2^bits - 1]) of the N(0, 1/d) Lloyd-Max quantiser."""
+    L = 2 ** int(bits)
+    levels = np.empty(L, dtype=np.float64)
+    bounds = np.empty(L - 1, dtype=np.float64)
+    _check(lib().lloydmax_table(int(d), int(bits), levels.ctypes.data_as(_P), bounds.ctypes.data_as(_P)),
+           "lloydmax_table")
+    return levels, bounds
+
+
+# ---------------------------------------------------------------------------
+# kernels
+# ---------------------------------------------------------------------------
+
+def rotate_quantize_act(rpbh, X, bits, codes=None, norms=None, stream=None):
+    """Packed codes uint8[T, d*bits/8] and norms float32[T] of the rows of X."""
+    import torch
+    _need_cuda(X, "X")
+    T, d = X.shape
+    if d != rpbh.d:
+        raise ValueError("X width does not match the RPBH handle")
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=X.device)
+    if norms is None:
+        norms = torch.empty((T,), dtype=torch.float32, device=X.device)
+    _need_cuda(codes, "codes", torch.uint8)
+    _need_cuda(norms, "norms", torch.float32)
+    _check(lib().rotate_quantize_act(rpbh.handle, _ptr(X), _dtype_code(X), T, int(bits), _ptr(codes),
+                                     _ptr(norms), _stream(stream)), "rotate_quantize_act")
+    return codes, norms
+
+
+def rotate_act(rpbh, X, out=None, norms=None, stream=None):
+    """x' = Pi x in BF16 (the activation operand of qlinear_int8)."""
+    import torch
+    _need_cuda(X, "X")
+    T, d = X.shape
+    if d != rpbh.d:
+        raise ValueError("X width does not match the RPBH handle")
+    if out is None:
+        out = torch.empty((T, d), dtype=torch.bfloat16, device=X.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    if norms is not None:
+        _need_cuda(norms, "norms", torch.float32)
+    _check(lib().rotate_quantize_act(rpbh.handle, _ptr(X), _dtype_code(X), T, RBQ_ROTATE_ONLY, _ptr(out),
+                                     _ptr(norms), _stream(stream)), "rotate_quantize_act")
+    return out
+
+
+def quantize_weights(rpbh, W, bits, mode="lloydmax", out=None, aux=None, stream=None):
+    """Offline weights.  mode='lloydmax': (codes uint8, r' bfloat16[N]);
+    mode='int8': (q int8[N, d], scale float32[N])."""
+    import torch
+    _need_cuda(W, "W")
+    N, d = W.shape
+    if d != rpbh.d:
+        raise ValueError("W width does not match the RPBH handle")
+    if mode == "lloydmax":
+        code = RBQ_LLOYDMAX
+        if out is None:
+            out = torch.empty((N, d * bits // 8), dtype=torch.uint8, device=W.device)
+        if aux is None:
+            aux = torch.empty((N,), dtype=torch.bfloat16, device=W.device)
+        _need_cuda(out, "codes", torch.uint8)
+        _need_cuda(aux, "rnorm", torch.bfloat16)
+    elif mode == "int8":
+        code, bits = RBQ_INT8_SYM, 8
+        if out is None:
+            out = torch.empty((N, d), dtype=torch.int8, device=W.device)
+        if aux is None:
+            aux = torch.empty((N,), dtype=torch.float32, device=W.device)
+        _need_cuda(out, "q", torch.int8)
+        _need_cuda(aux, "scale", torch.float32)
+    else:
+        raise ValueError("mode must be 'lloydmax' or 'int8'")
+    _check(lib().quantize_weights(rpbh.handle, _ptr(W), _dtype_code(W), N, code, int(bits), _ptr(out),
+                                  _ptr(aux), _stream(stream)), "quantize_weights")
+    return out, aux
+
+
+def qlinear(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, stream=None):
+    """y[m, n] = s_m r'_n sum_k C_w[q_nk] C_a[p_mk] as bfloat16 [M, N]."""
+    import torch
+    for t, n, dt in ((a_codes, "a_codes", torch.uint8), (s, "s", torch.float32),
+                     (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16)):
+        _need_cuda(t, n, dt)
+    M, N = a_codes.shape[0], w_codes.shape[0]
+    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
+        raise ValueError("code row widths do not match K and the bit widths")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _check(lib().qlinear(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M, N,
+                         int(K), _ptr(out), _stream(stream)), "qlinear")
+    return out
+
+
+def qlinear_int8(xrot, q, scale, out=None, stream=None):
+    """y[m, n] = scale_n sum_k q_nk x'_mk as bfloat16 [M, N]."""
+    import torch
+    _need_cuda(xrot, "xrot", torch.bfloat16)
+    _need_cuda(q, "q", torch.int8)
+    _need_cuda(scale, "scale", torch.float32)
+    M, K = xrot.shape
+    N = q.shape[0]
+    if q.shape[1] != K:
+        raise ValueError("q and xrot disagree on K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xrot.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _check(lib().qlinear_int8(_ptr(xrot), _ptr(q), _ptr(scale), M, N, K, _ptr(out), _stream(stream)),
+           "qlinear_int8")
+    return out
+
+
+def device_error(stream=None):
+    """Synchronise and read/clear the library's device error word (0 = clean)."""
+    return lib().rbq_device_error(_stream(stream))

@@ -1,0 +1,62 @@
+// Internal declarations shared by the library's translation units.
+// Nothing here is part of the public ABI (include/rbq.h is).
+#pragma once
+
+#include <cstdint>
+#include <cstddef>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "rbq.h"
+
+namespace rbq {
+
+constexpr int kH = 64;            // Hadamard block size (OrbitQuant §2.3: h = 64)
+constexpr int kMaxD = 32768;      // largest supported input width (one token row in shared memory)
+constexpr int kMaxDevices = 64;
+
+// Device-resident copy of one RPBH draw, laid out for the fused kernels.
+struct RpbhDevice {
+  bool ready = false;
+  int32_t* perm = nullptr;        // pi(k), destination order
+  float* sign = nullptr;          // D_k as +-1.0f, destination order
+};
+
+}  // namespace rbq
+
+struct rbq_rpbh {
+  int d = 0;
+  uint64_t seed = 0;
+  std::vector<int32_t> perm;      // pi
+  std::vector<int8_t> sign;       // D
+  rbq::RpbhDevice dev[rbq::kMaxDevices];
+};
+
+namespace rbq {
+
+// Per (device, d, bits) codebook tables for the kernels.
+struct CodebookDevice {
+  int d = 0, bits = 0;
+  float* bounds = nullptr;        // fp32[2^bits - 1], increasing
+  uint16_t* levels_f16 = nullptr; // fp16[2^bits]: levels times sqrt(d) (unit scale)
+  float inv_d = 0.f;              // 1/d: undoes the two sqrt(d) factors in qlinear
+};
+
+// Returns the device tables of `r` on the current device, uploading on first use.
+int rpbh_device(const rbq_rpbh* r, const RpbhDevice** out);
+// Returns the codebook of (d, bits) on the current device, computing and
+// uploading it on first use.
+int codebook_device(int d, int bits, const CodebookDevice** out);
+
+// Records a CUDA error (for rbq_error_string) and maps it to RBQ_ECUDA.
+int cuda_fail(cudaError_t e);
+
+// Device error word (bounded waits record here); defined in rbq_host.cu.
+int device_error_word_ptr(unsigned int** out);
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+}  // namespace rbq

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* librbq.so loads and exports every function include/rbq.h declares;
+* rpbh_make reproduces the oracle's permutation and signs exactly;
+* lloydmax_table (Newton's method, C++) agrees with the oracle's fixed-point
+  iteration (two independent algorithms for the same optimum);
+* invalid arguments are rejected before any device work, with the
+  documented codes (so these calls are safe on a machine without a GPU).
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import rotation_bit_ptq_b200 as rbq
+from rotation_bit_ptq_b200 import build as rbq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(rbq.LIB_PATH):
+        rbq_build.build()
+    return rbq.lib()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "rbq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"rpbh_make", "lloydmax_table", "quantize_weights", "rotate_quantize_act", "qlinear"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in rbq.SIGNATURES, n
+
+
+@pytest.mark.parametrize("d,seed", [(64, 0), (256, 0), (3072, 0), (3072, 12345), (12288, 7),
+                                    (8960, 2 ** 64 - 1)])
+def test_rpbh_make_matches_oracle(lib, d, seed):
+    r = rbq.RPBH(d, seed)
+    perm, signs = r.export()
+    op, os_ = oracle.rpbh_draw(d, seed)
+    assert np.array_equal(perm.astype(np.int64), op)
+    assert np.array_equal(signs.astype(np.int64), os_)
+    assert lib.rpbh_dim(r.handle) == d
+    r.close()
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_lloydmax_table_matches_oracle(lib, bits):
+    d = 3072
+    lv, bd = rbq.lloydmax_table(d, bits)
+    olv, obd = oracle.lloydmax_table(d, bits)
+    # The oracle's plain iteration contracts slowly at 8 bits (rate ~0.9999),
+    # which amplifies fp64 rounding to ~3e-11 sigma; Newton lands on the optimum.
+    tol = 1e-12 if bits <= 7 else 1e-10
+    sigma = 1 / np.sqrt(d)
+    assert np.max(np.abs(lv - olv)) / sigma < tol
+    assert np.max(np.abs(bd - obd)) / sigma < tol
+    assert np.array_equal(lv, -lv[::-1])
+    assert bd[len(bd) // 2] == 0.0
+    assert np.array_equal(bd, 0.5 * (lv[:-1] + lv[1:]))
+
+
+def test_rpbh_make_rejects_bad_arguments(lib):
+    out = ctypes.c_void_p()
+    for d, h in ((0, 64), (-64, 64), (100, 64), (256, 32), (65536 + 64, 64), (32768 + 64, 64)):
+        assert lib.rpbh_make(d, h, 0, ctypes.byref(out)) == rbq.RBQ_EINVAL
+    assert lib.rpbh_make(64, 64, 0, None) == rbq.RBQ_EINVAL
+    assert lib.rpbh_export(None, None, None) == rbq.RBQ_EINVAL
+    assert lib.rpbh_dim(None) == rbq.RBQ_EINVAL
+    lib.rpbh_free(None)
+
+
+def test_lloydmax_rejects_bad_arguments(lib):
+    for d, b in ((0, 4), (64, 0), (64, 9), (-1, 2)):
+        assert lib.lloydmax_table(d, b, None, None) == rbq.RBQ_EINVAL
+
+
+def test_kernel_entry_points_validate_before_launch(lib):
+    r = rbq.RPBH(256, 0)
+    h = r.handle
+    fake = ctypes.c_void_p(0x10000)       # never dereferenced: rejected first
+    odd = ctypes.c_void_p(0x10001)
+    # empty inputs are a successful no-op
+    assert lib.rotate_quantize_act(h, None, rbq.RBQ_BF16, 0, 4, None, None, None) == rbq.RBQ_OK
+    assert lib.quantize_weights(h, None, rbq.RBQ_BF16, 0, rbq.RBQ_LLOYDMAX, 4, None, None, None) == rbq.RBQ_OK
+    assert lib.qlinear(None, None, 4, None, None, 4, 0, 8, 64, None, None) == rbq.RBQ_OK
+    assert lib.qlinear_int8(None, None, None, 8, 0, 64, None, None) == rbq.RBQ_OK
+    # bad arguments
+    assert lib.rotate_quantize_act(None, fake, rbq.RBQ_BF16, 4, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.rotate_quantize_act(h, fake, 7, 4, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.rotate_quantize_act(h, fake, rbq.RBQ_BF16, 4, 9, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.rotate_quantize_act(h, fake, rbq.RBQ_BF16, -1, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.rotate_quantize_act(h, fake, rbq.RBQ_BF16, 4, 4, fake, None, None) == rbq.RBQ_EINVAL
+    assert lib.rotate_quantize_act(h, odd, rbq.RBQ_BF16, 4, 4, fake, fake, None) == rbq.RBQ_EALIGN
+    assert lib.rotate_quantize_act(h, fake, rbq.RBQ_BF16, 4, 4, odd, fake, None) == rbq.RBQ_EALIGN
+    assert lib.quantize_weights(h, fake, rbq.RBQ_BF16, 4, 5, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_weights(h, fake, rbq.RBQ_BF16, 4, rbq.RBQ_INT8_SYM, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_weights(h, odd, rbq.RBQ_BF16, 4, rbq.RBQ_LLOYDMAX, 4, fake, fake, None) == rbq.RBQ_EALIGN
+    assert lib.qlinear(fake, fake, 4, fake, fake, 4, 8, 8, 100, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear(fake, fake, 0, fake, fake, 4, 8, 8, 64, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear(fake, fake, 4, fake, fake, 4, 8, 12, 64, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear(odd, fake, 4, fake, fake, 4, 8, 8, 64, fake, None) == rbq.RBQ_EALIGN
+    assert lib.qlinear_int8(fake, fake, fake, 8, 8, 96, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8(fake, odd, fake, 8, 8, 64, fake, None) == rbq.RBQ_EALIGN
+    r.close()
+
+
+def test_error_strings(lib):
+    for code in (0, -1, -2, -4, -5, -6, -99):
+        assert isinstance(lib.rbq_error_string(code), bytes)

@@ -1,0 +1,272 @@
+"""CUDA path vs oracle, element by element, through the C ABI (needs a B200).
+
+Small cases run the oracle on every row; the full-size workloads run the
+kernel on the whole batch and compare sampled rows (the oracle multiplies by
+the dense d x d rotation, so it computes sampled tokens one by one).  The
+comparison rules (exact outside a 1e-6 band around each decision point) are
+in tests/parity.py.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import (bf16_to_numpy, check_bf16_rounding, check_codes, check_int8, check_rel,
+                    rel_frobenius, torch_bf16)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import rotation_bit_ptq_b200 as rbq  # noqa: E402
+
+NORM_RTOL = 1e-5          # fp32 norm vs fp64 (spec bar)
+QLINEAR_RTOL = 4e-3       # rel. Frobenius, fp16 operands + BF16 output (bar: 2e-2)
+QLINEAR8_RTOL = 3e-3      # rel. Frobenius, exact operands + BF16 output (bar: 2e-2)
+
+
+def _dense(x, dtype):
+    if dtype == "bf16":
+        return torch_bf16(x)
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+def _rpbh(d, seed):
+    """Library handle plus the oracle's Pi (dense matrix, or (perm, signs) for
+    widths whose dense matrix is applied in row chunks)."""
+    perm, signs = oracle.rpbh_draw(d, seed)
+    Pi = oracle.rpbh_matrix(perm, signs) if d <= 4096 else (perm, signs)
+    return rbq.RPBH(d, seed), Pi
+
+
+def _unpack(t, bits, d):
+    return oracle.unpack_codes(t.cpu().numpy(), bits, d)
+
+
+def _act_parity(X, d, bits, seed=0, dtype="bf16", rows=None, Pi=None, r=None):
+    """Run the kernel on all of X; compare rows `rows` (default all) with the oracle."""
+    if r is None:
+        r, Pi = _rpbh(d, seed)
+    xt = _dense(X, dtype)
+    codes, norms = rbq.rotate_quantize_act(r, xt, bits)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
+    levels, bounds = oracle.lloydmax_table(d, bits)
+    ora = oracle.quantize_act(X[rows].astype(np.float64), Pi, bounds)
+    g_codes = _unpack(codes[torch.as_tensor(rows).cuda()], bits, d)
+    n_mis, n_band = check_codes(g_codes, ora["codes"], ora["v"], bounds, d)
+    check_rel(norms.cpu().numpy()[rows], ora["norms"], NORM_RTOL, "norms")
+    return codes, norms, n_mis, n_band
+
+
+# --------------------------------------------------------------------------
+# rotate_quantize_act
+# --------------------------------------------------------------------------
+
+def test_tiny_w4a4_activations():
+    data = synth.tiny()
+    _act_parity(data["X"], 256, 4, dtype="f32")
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_all_bit_widths_ragged_tokens(bits, dtype):
+    X, _ = synth.student_t_act(257, 512, seed=bits)      # 257: ragged against any grouping
+    _act_parity(X, 512, bits, seed=3, dtype=dtype)
+
+
+@pytest.mark.parametrize("d,T", [(64, 1), (64, 130), (128, 3), (1536, 33), (8960, 5), (32768, 2)])
+def test_widths_from_one_block_to_maximum(d, T):
+    X, _ = synth.student_t_act(T, d, seed=d)
+    _act_parity(X, d, 4, seed=1)
+
+
+def test_zero_and_degenerate_rows():
+    d = 256
+    X = synth.tiny()["X"][:8].copy()
+    X[0] = 0.0                       # zero row: s = 0, every code is 2^(b-1)
+    X[1] = 1.0                       # constant row
+    X[2, :] = 0.0
+    X[2, 17] = -3.0                  # one-hot row
+    X[3] = -0.0
+    codes, norms, _, _ = _act_parity(X, d, 4, dtype="f32")
+    g = _unpack(codes, 4, d)
+    assert np.all(g[0] == 8) and np.all(g[3] == 8)
+    assert norms[0].item() == 0.0
+
+
+def test_attention_projection_full_size_sampled():
+    data = synth.attn_proj()
+    X = data["X"]
+    rows = np.unique(np.concatenate([[0, 1, X.shape[0] - 1], np.random.default_rng(0).choice(X.shape[0], 61)]))
+    _, _, n_mis, n_band = _act_parity(X, 3072, 4, rows=rows)
+    print(f"attn_proj A4: {n_mis} in-band mismatches, {n_band} coordinates in band")
+
+
+@pytest.mark.parametrize("bits", [4, 3])
+def test_mlp_down_input_full_size_sampled(bits):
+    X, _ = synth.gelu_act(4608, 12288, seed=1)
+    rows = np.random.default_rng(1).choice(4608, 24, replace=False)
+    _act_parity(X, 12288, bits, seed=5, rows=rows)
+
+
+@pytest.mark.parametrize("d", [1536, 8960])
+def test_video_w4a6_activations_sampled_frames(d):
+    X = synth.video_act(d, layer=3, frames=[0, 20])        # two frames, different scales
+    rows = np.random.default_rng(d).choice(X.shape[0], 32, replace=False)
+    _act_parity(X, d, 6, seed=1000 + 3, rows=rows)
+
+
+# --------------------------------------------------------------------------
+# rotate-only (BF16 x') and offline weights
+# --------------------------------------------------------------------------
+
+def test_rotate_only_bf16():
+    d = 1024
+    X, _ = synth.student_t_act(200, d, seed=9)
+    r, Pi = _rpbh(d, 4)
+    xr = rbq.rotate_act(r, torch_bf16(X))
+    torch.cuda.synchronize()
+    ora = oracle.rotate_only(X.astype(np.float64), Pi)
+    n = check_bf16_rounding(bf16_to_numpy(xr), ora["xr"], "rotate-only")
+    print(f"rotate-only: {n} in-band BF16 rounding differences")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_weights_lloydmax(bits):
+    d = 3072
+    W = synth.attn_proj()["W"][:200]
+    W = W.copy()
+    W[5] = 0.0
+    r, Pi = _rpbh(d, 0)
+    codes, rn = rbq.quantize_weights(r, torch_bf16(W), bits)
+    torch.cuda.synchronize()
+    _, bounds = oracle.lloydmax_table(d, bits)
+    ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
+    check_codes(_unpack(codes, bits, d), ora["codes"], ora["v"], bounds, d)
+    check_bf16_rounding(bf16_to_numpy(rn), ora["rnorm"], "row norms")
+
+
+def test_weights_tiny_fp32():
+    W = synth.tiny()["W"]
+    r, Pi = _rpbh(256, 0)
+    codes, rn = rbq.quantize_weights(r, _dense(W, "f32"), 4)
+    _, bounds = oracle.lloydmax_table(256, 4)
+    ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
+    check_codes(_unpack(codes, 4, 256), ora["codes"], ora["v"], bounds, 256)
+    check_bf16_rounding(bf16_to_numpy(rn), ora["rnorm"], "row norms")
+
+
+@pytest.mark.parametrize("shape", [(256, 256), (320, 4096), (64, 16384)])
+def test_weights_int8(shape):
+    n, d = shape
+    W = synth.int8_dit_weight(0, "q")[:n, :d] if d == 4096 else \
+        synth.gaussian_weights(synth.rng(11, d), n, d, outlier_frac=0.01).astype(np.float32)
+    W = synth.to_bf16(W)
+    W[1] = 0.0
+    r, Pi = _rpbh(d, 2)
+    q, sc = rbq.quantize_weights(r, torch_bf16(W), 8, mode="int8")
+    torch.cuda.synchronize()
+    ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi)
+    n_mis = check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
+    print(f"int8 {shape}: {n_mis} in-band rounding differences")
+
+
+# --------------------------------------------------------------------------
+# qlinear / qlinear_int8
+# --------------------------------------------------------------------------
+
+def _qlinear_case(X, W, d, bits_a, bits_w, seed=0, rows=None, dtype="bf16"):
+    r, Pi = _rpbh(d, seed)
+    a_codes, s = rbq.rotate_quantize_act(r, _dense(X, dtype), bits_a)
+    w_codes, rn = rbq.quantize_weights(r, _dense(W, dtype), bits_w)
+    y = rbq.qlinear(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
+    la, _ = oracle.lloydmax_table(d, bits_a)
+    lw, _ = oracle.lloydmax_table(d, bits_w)
+    pa = _unpack(a_codes[torch.as_tensor(rows).cuda()], bits_a, d)
+    pw = _unpack(w_codes, bits_w, d)
+    ref = oracle.qlinear(pa, s.cpu().numpy()[rows], la, pw, bf16_to_numpy(rn), lw)
+    got = bf16_to_numpy(y[torch.as_tensor(rows).cuda()])
+    err = rel_frobenius(got, ref)
+    return err, got, ref
+
+
+def test_qlinear_tiny_w4a4():
+    data = synth.tiny()
+    err, got, ref = _qlinear_case(data["X"], data["W"], 256, 4, 4, dtype="f32")
+    assert err < QLINEAR_RTOL, err
+    # and the quantised layer approximates the dense one (OrbitQuant §2.2)
+    dense = data["X"].astype(np.float64) @ data["W"].astype(np.float64).T
+    assert rel_frobenius(got, dense) < 0.2
+
+
+@pytest.mark.parametrize("M,N,K,ba,bw", [(1, 8, 64, 4, 4), (130, 136, 128, 4, 2), (257, 264, 320, 3, 3),
+                                         (64, 512, 256, 6, 4), (200, 128, 192, 8, 8), (77, 72, 64, 2, 6)])
+def test_qlinear_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
+    g = np.random.default_rng(M * N)
+    X = synth.to_bf16(g.standard_t(3, (M, K)).astype(np.float32))
+    W = synth.to_bf16((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    err, _, _ = _qlinear_case(X, W, K, ba, bw, seed=M)
+    assert err < QLINEAR_RTOL, err
+
+
+def test_qlinear_attention_projection_full_size_sampled():
+    data = synth.attn_proj()
+    rows = np.random.default_rng(2).choice(4608, 48, replace=False)
+    err, _, _ = _qlinear_case(data["X"], data["W"], 3072, 4, 4, rows=rows)
+    print(f"qlinear attn_proj W4A4 rel. Frobenius error {err:.2e}")
+    assert err < QLINEAR_RTOL
+
+
+@pytest.mark.parametrize("ba,bw", [(4, 2), (3, 3)])
+def test_qlinear_mlp_full_size_sampled(ba, bw):
+    m = synth.mlp()
+    rows = np.random.default_rng(3).choice(4608, 16, replace=False)
+    err_up, _, _ = _qlinear_case(m["X_up"], m["W_up"], 3072, ba, bw, seed=4, rows=rows)
+    err_dn, _, _ = _qlinear_case(m["X_dn"], m["W_dn"], 12288, ba, bw, seed=5, rows=rows)
+    assert err_up < QLINEAR_RTOL and err_dn < QLINEAR_RTOL, (err_up, err_dn)
+
+
+def _int8_case(X, W, d, seed=0, rows=None):
+    r, Pi = _rpbh(d, seed)
+    xr = rbq.rotate_act(r, torch_bf16(X))
+    q, sc = rbq.quantize_weights(r, torch_bf16(W), 8, mode="int8")
+    y = rbq.qlinear_int8(xr, q, sc)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
+    idx = torch.as_tensor(rows).cuda()
+    ref = oracle.qlinear_int8(bf16_to_numpy(xr[idx]), q.cpu().numpy(), sc.cpu().numpy())
+    got = bf16_to_numpy(y[idx])
+    return rel_frobenius(got, ref), got, Pi
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 256, 256), (130, 136, 192), (1, 8, 64)])
+def test_qlinear_int8_small(M, N, K):
+    g = np.random.default_rng(K)
+    X = synth.to_bf16(g.standard_normal((M, K)).astype(np.float32))
+    W = synth.to_bf16(synth.gaussian_weights(g, N, K, outlier_frac=0.01))
+    err, _, _ = _int8_case(X, W, K, seed=K)
+    assert err < QLINEAR8_RTOL, err
+
+
+@pytest.mark.parametrize("name", ["q", "up", "down"])
+def test_qlinear_int8_dit_block_sampled(name):
+    W = synth.int8_dit_weight(0, name)
+    d = W.shape[1]
+    X = synth.int8_dit_act(d)
+    rows = np.random.default_rng(4).choice(4096, 16, replace=False)
+    err, got, Pi = _int8_case(X, W, d, seed=7, rows=rows)
+    assert err < QLINEAR8_RTOL, err
+    # rotated INT8 beats naive INT8 on these outlier weights (INT8-convrot §2)
+    dense = X[rows].astype(np.float64) @ W.astype(np.float64).T
+    naive = oracle.quantize_weights_int8(W.astype(np.float64))
+    y_naive = oracle.qlinear_int8(X[rows].astype(np.float64), naive["q"], naive["scale"])
+    assert rel_frobenius(got, dense) < rel_frobenius(y_naive, dense)

@@ -86,6 +86,15 @@ def test_rpbh_matrix_equals_literal_product():
     assert np.array_equal(Pi, literal)
 
 
+def test_chunked_application_equals_dense():
+    d = 1024
+    perm, signs = oracle.rpbh_draw(d, seed=6)
+    x = np.random.default_rng(3).standard_normal((4, d))
+    dense = oracle.rpbh_apply(oracle.rpbh_matrix(perm, signs), x)
+    assert np.array_equal(oracle.rpbh_apply((perm, signs), x, chunk=192), dense) or \
+        np.allclose(oracle.rpbh_apply((perm, signs), x, chunk=192), dense, rtol=0, atol=1e-14)
+
+
 def test_rpbh_identity_case_is_textbook_hadamard():
     Pi = oracle.rpbh_matrix(np.arange(64), np.ones(64, dtype=int))
     assert np.array_equal(Pi * 8.0, scipy.linalg.hadamard(64).astype(float))
