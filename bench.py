@@ -330,6 +330,37 @@ def run_reference(args):
     }
 
 
+def run_kernel_only(args):
+    """One kernel on a profiling-sized case (for ncu): a few launches, no
+    timing.  rotate_quantize: 32768 tokens x 3072 (201 MB of BF16 input,
+    larger than L2); qlinear: the attention-projection GEMM 4608x3072x3072."""
+    import torch
+    import rotation_bit_ptq_b200 as rbq
+    dev = torch.device("cuda", 0)
+    r = rbq.RPBH(D, SEED)
+    if args.kernel_only in ("rotate_quantize", "rotate_only"):
+        tokens = args.tokens or 32768
+        X = to_bf16_tensor(synth.student_t_act(tokens, D, seed=SEED)[0], dev)
+        for _ in range(args.launches):
+            if args.kernel_only == "rotate_quantize":
+                rbq.rotate_quantize_act(r, X, BITS_A)
+            else:
+                rbq.rotate_act(r, X)
+    elif args.kernel_only == "quantize_weights":
+        W = to_bf16_tensor(synth.attn_proj(seed=SEED)["W"], dev)
+        for _ in range(args.launches):
+            rbq.quantize_weights(r, W, BITS_W)
+    else:
+        data = synth.attn_proj(seed=SEED)
+        a_codes, s = rbq.rotate_quantize_act(r, to_bf16_tensor(data["X"], dev), BITS_A)
+        w_codes, rn = rbq.quantize_weights(r, to_bf16_tensor(data["W"], dev), BITS_W)
+        for _ in range(args.launches):
+            rbq.qlinear(a_codes, s, BITS_A, w_codes, rn, BITS_W, D)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    print(json.dumps({"kernel_only": args.kernel_only, "launches": args.launches, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -337,7 +368,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", choices=["rotate_quantize", "rotate_only", "quantize_weights", "qlinear"],
+                    help="run one kernel on a profiling-sized case (for ncu) instead of the benchmark")
+    ap.add_argument("--tokens", type=int, default=0)
+    ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
+    if args.kernel_only:
+        run_kernel_only(args)
+        return
     args.warmup = max(3, args.warmup)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -36,6 +36,7 @@ SIGNATURES = {
     "qlinear_int8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
+    "rbq_code_grid": (_I, [_I, _I, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -248,6 +249,18 @@ def qlinear_int8(xrot, q, scale, out=None, stream=None):
     _check(lib().qlinear_int8(_ptr(xrot), _ptr(q), _ptr(scale), M, N, K, _ptr(out), _stream(stream)),
            "qlinear_int8")
     return out
+
+
+def code_grid(d, bits):
+    """The kernels' code-search table: (thr float32[n], base int32[n], cells, scale)."""
+    cells, scale = ctypes.c_int(), ctypes.c_float()
+    _check(lib().rbq_code_grid(int(d), int(bits), None, None, ctypes.byref(cells), ctypes.byref(scale)),
+           "rbq_code_grid")
+    thr = np.empty(cells.value + 1, dtype=np.float32)
+    base = np.empty(cells.value + 1, dtype=np.int32)
+    _check(lib().rbq_code_grid(int(d), int(bits), thr.ctypes.data_as(_P), base.ctypes.data_as(_P), None, None),
+           "rbq_code_grid")
+    return thr, base, cells.value, np.float32(scale.value)
 
 
 def device_error(stream=None):

@@ -191,6 +191,83 @@ uint16_t f32_to_f16_bits(float f) {
 }
 
 // ---------------------------------------------------------------------------
+// Code-search grid.  The kernel finds code #{t_j <= v} with one comparison:
+// n = round(sat(v / (2R) + 1/2) * NC) picks cell n of a uniform grid whose
+// cells are centred at -R + n w (w = 2R/NC, n = 0..NC); each cell holds at most
+// one boundary, so the code is the number of boundaries below the cell plus
+// (v >= that boundary).  Rounding can put v one cell off near a cell edge;
+// that gives the same code as long as no boundary sits near an edge, which is
+// checked here (margin 1% of a cell).  NC even puts the boundary at 0 in the
+// middle of cell NC/2; the end cells (which also take the clamped values
+// beyond +-R) hold no boundary.
+// ---------------------------------------------------------------------------
+inline float int_bits_as_float(int v) {
+  float f;
+  std::memcpy(&f, &v, sizeof(f));
+  return f;
+}
+
+struct Grid {
+  int cells = 0;
+  double R = 0.0;
+  std::vector<float2> lut;
+};
+
+bool try_grid(const std::vector<double>& t, int nc, double R, Grid* g) {
+  const double w = 2.0 * R / nc;
+  std::vector<float2> lut(nc + 1);
+  size_t j = 0;   // first boundary not below the current cell's lower edge
+  for (int n = 0; n <= nc; ++n) {
+    const double lo = -R + (n - 0.5) * w, hi = lo + w;
+    if (n == 0) {               // also takes v <= -R: below every boundary
+      if (!t.empty() && t.front() < hi + 0.01 * w) return false;
+      lut[n] = make_float2(INFINITY, int_bits_as_float(0));
+      continue;
+    }
+    if (n == nc) {              // also takes v >= R: above every boundary
+      if (!t.empty() && t.back() >= lo - 0.01 * w) return false;
+      lut[n] = make_float2(INFINITY, int_bits_as_float(static_cast<int>(t.size())));
+      continue;
+    }
+    while (j < t.size() && t[j] < lo) ++j;
+    size_t k = j;
+    int inside = 0;
+    double thr = INFINITY;
+    while (k < t.size() && t[k] < hi) {
+      if (t[k] - lo < 0.01 * w || hi - t[k] < 0.01 * w) return false;
+      thr = t[k];
+      ++inside;
+      ++k;
+    }
+    if (inside > 1) return false;
+    float tf = static_cast<float>(thr);
+    if (inside == 1 && thr == 0.0) tf = -0.0f;   // so that -0.0 counts as >= 0
+    lut[n] = make_float2(tf, int_bits_as_float(static_cast<int>(j)));
+  }
+  g->cells = nc;
+  g->R = R;
+  g->lut = std::move(lut);
+  return true;
+}
+
+int build_grid(const std::vector<double>& bounds, Grid* g) {
+  double tmax = 0.0, gap = INFINITY;
+  for (size_t j = 0; j < bounds.size(); ++j) {
+    tmax = std::fmax(tmax, std::fabs(bounds[j]));
+    if (j) gap = std::fmin(gap, bounds[j] - bounds[j - 1]);
+  }
+  if (bounds.size() == 1) gap = 1.0;           // 1 bit: the single boundary 0
+  const double R0 = tmax > 0.0 ? tmax * 1.05 : 1.0;
+  int nc = static_cast<int>(std::ceil(2.0 * R0 / (0.9 * gap)));
+  nc += nc & 1;
+  if (nc < 2) nc = 2;
+  for (; nc <= 4096; nc += 2)
+    for (int step = 0; step < 64; ++step)
+      if (try_grid(bounds, nc, R0 * (1.0 + 0.003 * step), g)) return RBQ_OK;
+  return RBQ_ECONVERGE;
+}
+
+// ---------------------------------------------------------------------------
 // Per-device caches.
 // ---------------------------------------------------------------------------
 std::map<std::pair<int, long long>, CodebookDevice*>& cb_cache() {
@@ -266,11 +343,17 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
   for (int j = 0; j < L; ++j) lh[j] = f32_to_f16_bits(static_cast<float>(levels[j] * sd));
   if ((rc = upload(bf.data(), bf.size(), &cb->bounds)) != RBQ_OK) { delete cb; return rc; }
   if ((rc = upload(lh.data(), lh.size(), &cb->levels_f16)) != RBQ_OK) { delete cb; return rc; }
+  Grid grid;
+  if ((rc = build_grid(bounds, &grid)) != RBQ_OK) { delete cb; return rc; }
+  cb->grid_cells = grid.cells;
+  cb->grid_scale = static_cast<float>(1.0 / (2.0 * grid.R));
+  if ((rc = upload(grid.lut.data(), grid.lut.size(), &cb->grid)) != RBQ_OK) { delete cb; return rc; }
   std::lock_guard<std::mutex> lk(g_mu);
   auto ins = cb_cache().emplace(key, cb);
   if (!ins.second) {          // another thread won the race; keep its copy
     cudaFree(cb->bounds);
     cudaFree(cb->levels_f16);
+    cudaFree(cb->grid);
     delete cb;
   }
   *out = ins.first->second;
@@ -381,5 +464,25 @@ extern "C" int rbq_device_error(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e);
     return RBQ_EDEVICE;
   }
+  return RBQ_OK;
+}
+
+extern "C" int rbq_code_grid(int d, int bits, float* thr, int32_t* base, int* cells, float* scale) {
+  if (d <= 0 || bits < 1 || bits > 8) return RBQ_EINVAL;
+  std::vector<double> levels, bounds;
+  int rc = full_table(d, bits, levels, bounds);
+  if (rc != RBQ_OK) return rc;
+  Grid g;
+  if ((rc = build_grid(bounds, &g)) != RBQ_OK) return rc;
+  for (size_t n = 0; n < g.lut.size(); ++n) {
+    if (thr) thr[n] = g.lut[n].x;
+    if (base) {
+      int b;
+      std::memcpy(&b, &g.lut[n].y, sizeof(b));
+      base[n] = b;
+    }
+  }
+  if (cells) *cells = g.cells;
+  if (scale) *scale = static_cast<float>(1.0 / (2.0 * g.R));
   return RBQ_OK;
 }

@@ -41,6 +41,12 @@ struct CodebookDevice {
   float* bounds = nullptr;        // fp32[2^bits - 1], increasing
   uint16_t* levels_f16 = nullptr; // fp16[2^bits]: levels times sqrt(d) (unit scale)
   float inv_d = 0.f;              // 1/d: undoes the two sqrt(d) factors in qlinear
+  // Code-search grid: `grid_cells` + 1 cells centred at -R + n*2R/cells;
+  // entry n = {boundary inside cell n or +inf, number of boundaries below
+  // that cell}.  See build_grid() in rbq_host.cu.
+  float2* grid = nullptr;
+  int grid_cells = 0;
+  float grid_scale = 0.f;         // 1 / (2R)
 };
 
 // Returns the device tables of `r` on the current device, uploading on first use.

@@ -178,6 +178,319 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
   }
 }
 
+// ===========================================================================
+// Fast path: BF16 input, 1024 <= d <= 16384.
+//
+// A CTA owns G tokens at a time (G = 4, 2 or 1 so that G*d/64 threads fit).
+// Thread (b, g), tid = b*G + g, produces output block b of token g.
+//
+//  * Staging: each thread streams 16-byte chunks of its token row from HBM
+//    into registers one group ahead, flips the signs of the source positions
+//    (a source-side XOR mask: (D P x)_k = D_k x_pi(k) = s'_{pi(k)} x_{pi(k)}
+//    with s'_j = D_{pi^-1(j)}), and writes them to shared memory in a
+//    chunk-interleaved layout [chunk][token][8 x bf16].  Two stages.
+//  * Gather: a per-CTA table holds, for every output position k, the byte
+//    offset of source position pi(k) in that layout (swizzled so that the
+//    threads of a warp read it without bank conflicts).
+//  * Butterfly: the 64 values sit in 32 fp32x2 registers (y_2m, y_2m+1);
+//    stride 1 runs inside a pair, strides 2..32 use packed f32x2 add/sub.
+//  * Norm: per-thread sum of squares, a shuffle tree over the token's
+//    threads in the warp, then the per-warp partials -- a fixed order, so
+//    every thread of a token gets the same s.
+//  * Codes: one grid lookup and one compare per element (see build_grid()).
+// ===========================================================================
+namespace fast {
+
+struct Params {
+  const __nv_bfloat16* X;
+  long long T;
+  int d, nblk;
+  const int32_t* perm;
+  const float* sign;
+  const float2* grid;     // Lloyd-Max modes
+  int grid_n;             // entries = cells + 1
+  float grid_cells, grid_scale;
+  void* out;
+  void* aux;
+};
+
+__device__ __forceinline__ unsigned long long pk(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk(unsigned long long r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) { return __ldcs(p); }
+
+template <int G>
+struct Layout {
+  // bytes: stage[2] (G*d*2 each) | off (4d) | mask (2d) | red (4*G*32) | grid
+  static __host__ __device__ size_t stage_bytes(int d) { return static_cast<size_t>(G) * d * 2; }
+  static __host__ __device__ size_t off_at(int d) { return 2 * stage_bytes(d); }
+  static __host__ __device__ size_t mask_at(int d) { return off_at(d) + 4 * static_cast<size_t>(d); }
+  static __host__ __device__ size_t red_at(int d) { return mask_at(d) + 2 * static_cast<size_t>(d); }
+  static __host__ __device__ size_t grid_at(int d) { return red_at(d) + 4 * G * 32; }
+  static __host__ __device__ size_t total(int d, int grid_n) { return grid_at(d) + 8 * static_cast<size_t>(grid_n); }
+};
+
+template <int MODE, int BITS, int G>
+__global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  using L = Layout<G>;
+  const int d = p.d, nblk = p.nblk;
+  const int nthreads = blockDim.x;          // G * nblk rounded up to whole warps
+  const int tid = threadIdx.x;
+  const int g = tid % G, b = tid / G;
+  const bool active = b < nblk;             // padding lanes only join shuffles/barriers
+  const uint32_t sbase = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  const uint32_t stage_addr[2] = {sbase, sbase + static_cast<uint32_t>(L::stage_bytes(d))};
+  const uint32_t off_addr = sbase + static_cast<uint32_t>(L::off_at(d));
+  const uint32_t mask_addr = sbase + static_cast<uint32_t>(L::mask_at(d));
+  float* red = reinterpret_cast<float*>(smem + L::red_at(d));
+  const uint32_t grid_addr = sbase + static_cast<uint32_t>(L::grid_at(d));
+  constexpr bool kLloyd = (MODE == kAct || MODE == kWeightLM);
+
+  // ---- per-CTA tables ------------------------------------------------------
+  uint16_t* mask16 = reinterpret_cast<uint16_t*>(smem + L::mask_at(d));
+  uint32_t* off = reinterpret_cast<uint32_t*>(smem + L::off_at(d));
+  for (int k = tid; k < d; k += nthreads) {
+    const int j = __ldg(p.perm + k);
+    mask16[j] = (__ldg(p.sign + k) < 0.f) ? 0x8000u : 0u;
+    const int kb = k >> 6, ki = k & 63;
+    const int slot = 64 * kb + 4 * ((ki >> 2) ^ (kb & 15)) + (ki & 3);
+    off[slot] = static_cast<uint32_t>((j >> 3) * (G * 16) + (j & 7) * 2);
+  }
+  if (kLloyd) {
+    float2* gs = reinterpret_cast<float2*>(smem + L::grid_at(d));
+    for (int n = tid; n < p.grid_n; n += nthreads) gs[n] = p.grid[n];
+  }
+
+  // ---- staging helpers ------------------------------------------------------
+  const int sg = tid % G;              // staged token
+  const int sc0 = tid / G;             // first staged chunk; chunks sc0 + j*nblk
+  const long long ngroups = (p.T + G - 1) / G;
+  uint4 pre[8];
+  auto load_group = [&](long long gi) {
+    const long long row = gi * G + sg;
+    const bool valid = active && (gi < ngroups) && (row < p.T);
+    const uint4* src = reinterpret_cast<const uint4*>(p.X + (valid ? row : 0) * d);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pre[j] = valid ? ldg_stream(src + sc0 + j * nblk) : make_uint4(0, 0, 0, 0);
+  };
+  auto store_group = [&](int st) {
+    if (!active) return;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = sc0 + j * nblk;
+      const uint4 m = lds128(mask_addr + 16 * c);
+      const uint4 v = make_uint4(pre[j].x ^ m.x, pre[j].y ^ m.y, pre[j].z ^ m.z, pre[j].w ^ m.w);
+      sts128(stage_addr[st] + 16 * (c * G + sg), v);
+    }
+  };
+
+  __syncthreads();   // tables ready
+  long long gi = blockIdx.x;
+  load_group(gi);
+  store_group(0);
+  load_group(gi + gridDim.x);
+  __syncthreads();
+
+  const int warp = tid >> 5, lane = tid & 31;
+  const int nwarps = (nthreads + 31) >> 5;
+  int st = 0;
+  for (; gi < ngroups; gi += gridDim.x, st ^= 1) {
+    // ---- gather (signs already applied) -> 32 fp32x2 pairs (y_2m, y_2m+1) ----
+    unsigned long long P[32];
+    if (active) {
+      const uint32_t base = stage_addr[st] + 16 * g;
+#pragma unroll
+      for (int i4 = 0; i4 < 16; ++i4) {
+        const uint4 o = lds128(off_addr + 4 * (64 * b + 4 * (i4 ^ (b & 15))));
+        P[2 * i4] = pk(__uint_as_float(lds_u16(base + o.x) << 16), __uint_as_float(lds_u16(base + o.y) << 16));
+        P[2 * i4 + 1] = pk(__uint_as_float(lds_u16(base + o.z) << 16), __uint_as_float(lds_u16(base + o.w) << 16));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) P[j] = 0ull;
+    }
+    // ---- 64-point Walsh-Hadamard (unnormalised): stride 1 inside a pair,
+    //      strides 2..32 between pairs with packed f32x2 ----
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float lo, hi;
+      upk(P[j], lo, hi);
+      P[j] = pk(lo + hi, lo - hi);
+    }
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if ((j & s) == 0) {
+          const unsigned long long a = P[j], c = P[j + s];
+          P[j] = add2(a, c);
+          P[j + s] = sub2(a, c);
+        }
+      }
+    }
+    // ---- token reduction: sum of squares (or max |z| for INT8) ----
+    float part;
+    if (MODE == kInt8) {
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float lo, hi;
+        upk(P[j], lo, hi);
+        m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+      }
+      part = m;
+    } else {
+      unsigned long long acc = 0ull;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc = fma2(P[j], P[j], acc);
+      float lo, hi;
+      upk(acc, lo, hi);
+      part = lo + hi;
+    }
+    // lanes of the same token in this warp are lane = g (mod G)
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1) {
+      const float other = __shfl_xor_sync(0xffffffffu, part, o);
+      part = (MODE == kInt8) ? fmaxf(part, other) : part + other;
+    }
+    if (lane < G) red[g * 32 + warp] = part;
+    __syncthreads();
+    float tot = 0.f;
+    for (int w = 0; w < nwarps; ++w)
+      tot = (MODE == kInt8) ? fmaxf(tot, red[g * 32 + w]) : tot + red[g * 32 + w];
+
+    // ---- refill the other stage while this one is consumed ----
+    store_group(st ^ 1);
+    load_group(gi + 2 * static_cast<long long>(gridDim.x));
+
+    const long long t = gi * G + g;
+    if (active && t < p.T) {
+      if constexpr (kLloyd) {
+        // z here is 8x the rotated value (H unnormalised): v = z / (||z|| + 8 eps)
+        const float nrm = sqrtf(tot);
+        const float inv = 1.0f / (nrm + 8e-12f);
+        const float A = inv * p.grid_scale;
+        const uint32_t gbase = grid_addr - 0x4B000000u * 8u;
+        uint32_t w[2 * BITS];
+#pragma unroll
+        for (int i = 0; i < 2 * BITS; ++i) w[i] = 0u;
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+          float lo, hi;
+          upk(P[r >> 1], lo, hi);
+          const float z = (r & 1) ? hi : lo;
+          const float u = fma_sat(z, A, 0.5f);
+          const float qf = fmaf(u, p.grid_cells, 8388608.0f);   // 2^23: round(u*NC) in the low bits
+          const float2 e = lds_f2(gbase + __float_as_uint(qf) * 8u);
+          const float diff = fmaf(z, inv, -e.x);
+          const uint32_t code = static_cast<uint32_t>(__float_as_int(e.y)) + ((__float_as_uint(diff) >> 31) ^ 1u);
+          const int bit = r * BITS, wi = bit >> 5, sh = bit & 31;
+          w[wi] |= code << sh;
+          if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
+        }
+        unsigned char* dst = static_cast<unsigned char*>(p.out) + t * (static_cast<long long>(d) * BITS / 8) +
+                             static_cast<long long>(b) * 8 * BITS;
+        if constexpr ((BITS % 2) == 0) {
+#pragma unroll
+          for (int i = 0; i < BITS / 2; ++i)
+            __stcs(reinterpret_cast<uint4*>(dst) + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < BITS; ++i) __stcs(reinterpret_cast<uint2*>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
+        }
+        if (b == 0) {
+          const float sn = nrm * 0.125f;
+          if (MODE == kAct) static_cast<float*>(p.aux)[t] = sn;
+          else static_cast<__nv_bfloat16*>(p.aux)[t] = __float2bfloat16_rn(sn);
+        }
+      } else if constexpr (MODE == kInt8) {
+        const float scale = (tot * 0.125f) / 127.0f;
+        const float rcp = (scale > 0.f) ? 1.0f / scale : 0.f;
+        uint32_t q4[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q4[i] = 0u;
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+          float lo, hi;
+          upk(P[r >> 1], lo, hi);
+          const float z = ((r & 1) ? hi : lo) * 0.125f;
+          int q = __float2int_rn(z * rcp);
+          q = max(-127, min(127, q));
+          q4[r >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (r & 3));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.out) + t * d + 64 * b);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) __stcs(dst + i, make_uint4(q4[4 * i], q4[4 * i + 1], q4[4 * i + 2], q4[4 * i + 3]));
+        if (b == 0) static_cast<float*>(p.aux)[t] = scale;
+      } else {   // kRotate
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + t * d + 64 * b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint32_t u[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float z0, z1;
+            upk(P[4 * i + j], z0, z1);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(z0 * 0.125f, z1 * 0.125f);
+            u[j] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          __stcs(dst + i, make_uint4(u[0], u[1], u[2], u[3]));
+        }
+        if (b == 0 && p.aux) static_cast<float*>(p.aux)[t] = sqrtf(tot) * 0.125f;
+      }
+    }
+    __syncthreads();   // stage st fully read and stage st^1 fully written
+  }
+}
+
+}  // namespace fast
+
 int sm_count() {
   static int n = 0;
   if (!n) {
@@ -228,6 +541,85 @@ int launch_mode(int dtype, int bits, const RotqParams& p, cudaStream_t st) {
                            : launch_one<MODE, 8, float>(p, st);
 }
 
+// ---- fast path launch --------------------------------------------------------
+bool fast_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d >= 1024 && d <= 16384; }
+
+int fast_tokens_per_cta(int nblk) { return (4 * nblk <= 384) ? 4 : (2 * nblk <= 384) ? 2 : 1; }
+
+template <int MODE, int BITS, int G>
+int launch_fast_g(const fast::Params& p, cudaStream_t st) {
+  const int threads = ((G * p.nblk + 31) / 32) * 32;
+  const size_t smem = fast::Layout<G>::total(p.d, p.grid_n);
+  auto kern = fast::rotq_fast_kernel<MODE, BITS, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (per_sm < 1) per_sm = 1;
+  const long long groups = (p.T + G - 1) / G;
+  const long long cap = static_cast<long long>(per_sm) * sm_count();
+  const int grid = static_cast<int>(groups < cap ? groups : cap);
+  kern<<<grid, threads, smem, st>>>(p);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+}
+
+template <int MODE, int BITS>
+int launch_fast_bits(const fast::Params& p, cudaStream_t st) {
+  switch (fast_tokens_per_cta(p.nblk)) {
+    case 4: return launch_fast_g<MODE, BITS, 4>(p, st);
+    case 2: return launch_fast_g<MODE, BITS, 2>(p, st);
+    default: return launch_fast_g<MODE, BITS, 1>(p, st);
+  }
+}
+
+template <int MODE>
+int launch_fast(int bits, const fast::Params& p, cudaStream_t st) {
+  if (MODE != kAct && MODE != kWeightLM) return launch_fast_bits<MODE, 8>(p, st);
+  switch (bits) {
+    case 1: return launch_fast_bits<MODE, 1>(p, st);
+    case 2: return launch_fast_bits<MODE, 2>(p, st);
+    case 3: return launch_fast_bits<MODE, 3>(p, st);
+    case 4: return launch_fast_bits<MODE, 4>(p, st);
+    case 5: return launch_fast_bits<MODE, 5>(p, st);
+    case 6: return launch_fast_bits<MODE, 6>(p, st);
+    case 7: return launch_fast_bits<MODE, 7>(p, st);
+    case 8: return launch_fast_bits<MODE, 8>(p, st);
+    default: return RBQ_EINVAL;
+  }
+}
+
+int run_fast(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
+             cudaStream_t st) {
+  const RpbhDevice* rd = nullptr;
+  int rc = rpbh_device(r, &rd);
+  if (rc != RBQ_OK) return rc;
+  fast::Params p{};
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.T = rows;
+  p.d = r->d;
+  p.nblk = r->d / kH;
+  p.perm = rd->perm;
+  p.sign = rd->sign;
+  p.out = out;
+  p.aux = aux;
+  if (mode == kAct || mode == kWeightLM) {
+    const CodebookDevice* cb = nullptr;
+    if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
+    p.grid = cb->grid;
+    p.grid_n = cb->grid_cells + 1;
+    p.grid_cells = static_cast<float>(cb->grid_cells);
+    p.grid_scale = cb->grid_scale;
+  }
+  switch (mode) {
+    case kAct: return launch_fast<kAct>(bits, p, st);
+    case kWeightLM: return launch_fast<kWeightLM>(bits, p, st);
+    case kInt8: return launch_fast<kInt8>(8, p, st);
+    default: return launch_fast<kRotate>(8, p, st);
+  }
+}
+
 // Tokens per CTA so that a CTA has at least 128 threads (one per block).
 int tokens_per_cta(int nblk) {
   int G = (128 + nblk - 1) / nblk;
@@ -272,8 +664,10 @@ extern "C" int rotate_quantize_act(const rbq_rpbh* r, const void* X, int dtype, 
   if (!X || !codes_out || (!rot && !norms_out)) return RBQ_EINVAL;
   if (!aligned(X, 16) || !aligned(codes_out, 16) || (norms_out && !aligned(norms_out, 4)))
     return RBQ_EALIGN;
-  RotqParams p;
   const int mode = rot ? kRotate : kAct;
+  if (fast_eligible(dtype, r->d))
+    return run_fast(r, mode, bits, T, X, codes_out, norms_out, static_cast<cudaStream_t>(stream));
+  RotqParams p;
   int rc = prepare(r, mode, bits, T, X, codes_out, norms_out, &p);
   if (rc != RBQ_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -294,8 +688,10 @@ extern "C" int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int
   if (!W || !codes_or_q || !rownorm_or_scale) return RBQ_EINVAL;
   if (!aligned(W, 16) || !aligned(codes_or_q, 16) || !aligned(rownorm_or_scale, 4))
     return RBQ_EALIGN;
-  RotqParams p;
   const int m = (mode == RBQ_LLOYDMAX) ? kWeightLM : kInt8;
+  if (fast_eligible(dtype, r->d))
+    return run_fast(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, static_cast<cudaStream_t>(stream));
+  RotqParams p;
   int rc = prepare(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, &p);
   if (rc != RBQ_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

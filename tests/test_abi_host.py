@@ -120,3 +120,36 @@ def test_kernel_entry_points_validate_before_launch(lib):
 def test_error_strings(lib):
     for code in (0, -1, -2, -4, -5, -6, -99):
         assert isinstance(lib.rbq_error_string(code), bytes)
+
+
+@pytest.mark.parametrize("d", [256, 1024, 3072, 8960, 12288])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_code_grid_lookup_matches_oracle(lib, d, bits):
+    """The kernels' one-compare code search, evaluated here in fp32 with the
+    library's table, equals the oracle's boundary count outside the band."""
+    thr, base, cells, scale = rbq.code_grid(d, bits)
+    assert cells % 2 == 0 and len(thr) == cells + 1
+    _, bounds = oracle.lloydmax_table(d, bits)
+    sigma = 1 / np.sqrt(d)
+    g = np.random.default_rng(d * 16 + bits)
+    v = np.concatenate([(g.standard_normal(300000) * sigma).astype(np.float32),
+                        (g.uniform(-1, 1, 20000)).astype(np.float32),
+                        np.float32([0.0, -0.0, 1.0, -1.0]), bounds.astype(np.float32),
+                        np.nextafter(bounds.astype(np.float32), np.float32(np.inf)),
+                        np.nextafter(bounds.astype(np.float32), np.float32(-np.inf))])
+    u = np.clip(v * scale + np.float32(0.5), np.float32(0), np.float32(1)).astype(np.float32)
+    q = (u * np.float32(cells) + np.float32(2.0 ** 23)).astype(np.float32)
+    n = q.view(np.int32) - 0x4B000000
+    assert n.min() >= 0 and n.max() <= cells
+    code = base[n] + (v >= thr[n])
+    ref = oracle.assign_codes(v.astype(np.float64), bounds)
+    near = np.zeros(v.shape, dtype=bool)
+    for t in bounds:
+        near |= np.abs(v.astype(np.float64) - t) <= 1e-6 * max(abs(t), sigma)
+    bad = (code != ref) & ~near
+    assert not np.any(bad), (int(bad.sum()), v[bad][:5])
+    # the zero coordinate takes the upper side of the middle boundary
+    z = np.float32([0.0, -0.0])
+    nz = (np.clip(z * scale + np.float32(0.5), 0, 1) * np.float32(cells) + np.float32(2.0 ** 23)).astype(np.float32)
+    nn = nz.view(np.int32) - 0x4B000000
+    assert np.all(base[nn] + (z >= thr[nn]) == 2 ** (bits - 1))

@@ -79,6 +79,24 @@ def test_all_bit_widths_ragged_tokens(bits, dtype):
     _act_parity(X, 512, bits, seed=3, dtype=dtype)
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_fast_path_all_bit_widths(bits):
+    # d = 1024 takes the fast kernel (4 tokens per CTA); 257 tokens leave a
+    # ragged last group
+    X, _ = synth.student_t_act(257, 1024, seed=10 + bits)
+    _act_parity(X, 1024, bits, seed=bits)
+
+
+@pytest.mark.parametrize("d,T,bits", [(8960, 37, 3), (12288, 9, 5), (16384, 5, 7), (1024, 1, 4),
+                                      (2048, 4099, 2)])
+def test_fast_path_widths(d, T, bits):
+    # 8960 = 140 blocks: 2 tokens per CTA, 280 threads padded to 288;
+    # 16384: 1 token per CTA; 4099 tokens: many groups per CTA
+    X, _ = synth.student_t_act(T, d, seed=d + T)
+    rows = None if T < 600 else np.random.default_rng(0).choice(T, 64, replace=False)
+    _act_parity(X, d, bits, seed=d, rows=rows)
+
+
 @pytest.mark.parametrize("d,T", [(64, 1), (64, 130), (128, 3), (1536, 33), (8960, 5), (32768, 2)])
 def test_widths_from_one_block_to_maximum(d, T):
     X, _ = synth.student_t_act(T, d, seed=d)
@@ -125,8 +143,8 @@ def test_video_w4a6_activations_sampled_frames(d):
 # rotate-only (BF16 x') and offline weights
 # --------------------------------------------------------------------------
 
-def test_rotate_only_bf16():
-    d = 1024
+@pytest.mark.parametrize("d", [512, 1024, 8960])
+def test_rotate_only_bf16(d):
     X, _ = synth.student_t_act(200, d, seed=9)
     r, Pi = _rpbh(d, 4)
     xr = rbq.rotate_act(r, torch_bf16(X))
