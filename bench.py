@@ -124,6 +124,30 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank plumbing (replicas: each rank quantises its own token shard; no
+# data-path collective, only the barrier and the timing reduction)
+# ---------------------------------------------------------------------------
+
+def rank_seed(rank):
+    """Each rank draws its own token batch (a different shard of the job);
+    the rotation and codebook are shared."""
+    return SEED + rank
+
+
+def reduce_job(times_ms, units, group=None, device=None):
+    """Whole-job view of per-rank measurements: the max over ranks of every
+    timing and the sum over ranks of the units processed."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    u = torch.tensor([float(units)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM, group=group)
+    return t.tolist(), u.item()
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
@@ -136,7 +160,7 @@ def run_ours(args, rank, world):
     stream = torch.cuda.current_stream()
     pk = peaks()
 
-    data = synth.attn_proj(seed=SEED + rank)
+    data = synth.attn_proj(seed=rank_seed(rank))
     X_host = data["X"]
     W_host = data["W"]
     r = rbq.RPBH(D, SEED)
@@ -195,23 +219,22 @@ def run_ours(args, rank, world):
     k1 = [e[0].elapsed_time(e[1]) for e in evs]
     k1w = [e[1].elapsed_time(e[2]) for e in evs]
     k2 = [e[2].elapsed_time(e[3]) for e in evs]
-    times = torch.tensor([total_ms, sum(k1), sum(k1w), sum(k2)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, k1_ms, k1w_ms, k2_ms = times.tolist()
+    (total_ms, k1_ms, k1w_ms, k2_ms), job_tokens = reduce_job([total_ms, sum(k1), sum(k1w), sum(k2)],
+                                                              T * args.steps, device=dev)
 
     act_bytes = act_bytes_per_token() * T
     flops = 2.0 * T * D * D
-    gbs = act_bytes * args.steps * world / (k1_ms * 1e-3) / 1e9
+    gbs = act_bytes_per_token() * job_tokens / (k1_ms * 1e-3) / 1e9
     k1_avg_s = k1_ms / args.steps * 1e-3
     k2_avg_s = k2_ms / args.steps * 1e-3
     tflops = flops * args.steps * world / (k2_ms * 1e-3) / 1e12
     wgbs = weight_bytes_per_row() * D * args.steps * world / (k1w_ms * 1e-3) / 1e9
 
-    # end to end through the public API with host buffers
-    e2e = None
-    if rank == 0 or world > 1:
-        e2e = run_e2e(r, X_host, dev, stream, args)
+    # end to end through the public API with host buffers (every rank, its own shard)
+    e2e_ms, h2d, d2h = run_e2e(r, X_host, dev, stream, args)
+    (e2e_ms,), e2e_tokens = reduce_job([e2e_ms], T * args.steps, device=dev)
+    e2e = {"value": round(act_bytes_per_token() * e2e_tokens / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     res = {
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
@@ -244,7 +267,8 @@ def run_ours(args, rank, world):
 
 def run_e2e(r, X_host, dev, stream, args):
     """rotate_quantize_act through the public API from pinned host memory:
-    H2D of X, the kernel, D2H of codes and norms, every step."""
+    H2D of X, the kernel, D2H of codes and norms, every step.  Returns
+    (ms for args.steps steps, H2D bytes per step, D2H bytes per step)."""
     import torch
     import rotation_bit_ptq_b200 as rbq
     xh = torch.from_numpy(synth.bf16_bits(X_host).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -270,9 +294,7 @@ def run_e2e(r, X_host, dev, stream, args):
         one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    return {"value": round(act_bytes_per_token() * T * args.steps / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(ch.numel() + nh.numel() * 4)}
+    return a.elapsed_time(b), int(xh.numel() * 2), int(ch.numel() + nh.numel() * 4)
 
 
 # ---------------------------------------------------------------------------

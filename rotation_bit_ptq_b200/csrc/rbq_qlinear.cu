@@ -247,7 +247,7 @@ int launch_qgemm(const QParams& p, cudaStream_t st) {
 }  // namespace rbq
 
 namespace rbq {
-bool qlinear_fast_eligible(int M, int N, int K);
+bool qlinear_fast_eligible(int M, int N, int K, int bits_a, int bits_w);
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
                         const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st);
@@ -272,7 +272,7 @@ extern "C" int qlinear(const uint8_t* a_codes, const float* s, int bits_a, const
   if ((rc = codebook_device(K, bits_w, &cw)) != RBQ_OK) return rc;
   unsigned int* err = nullptr;
   if ((rc = device_error_word_ptr(&err)) != RBQ_OK) return rc;
-  if (qlinear_fast_eligible(M, N, K))
+  if (qlinear_fast_eligible(M, N, K, bits_a, bits_w))
     return qlinear_fast_launch(a_codes, s, bits_a, w_codes, rnorm, bits_w, M, N, K, Y, ca, cw, err,
                                static_cast<cudaStream_t>(stream));
   QParams p{};

@@ -6,20 +6,21 @@
 //   y[m,n] = s_m r'_n sum_k C_w[q_nk] C_a[p_mk].
 //
 // Each CTA (one per SM) walks a static list of 128 x 256 output tiles.
-//   warp 0          MMA issuer: one thread waits for a filled stage, issues
-//                   four 128x256x16 kind::f16 MMAs into the tile's TMEM
-//                   accumulator and commits them to the stage's "empty"
-//                   barrier; after the last K slice it commits the
-//                   accumulator to the epilogue.
-//   warps 4..7      epilogue: TMEM lane quadrant w%4, one output row per
-//                   thread; scale by s_m r'_n / K, round to BF16, store.
-//   warps 8..19     operand expansion, one row per thread (128 rows of A,
-//                   256 rows of B): read the row's 64 codes of the K slice,
-//                   turn them into fp16 levels (x sqrt(K)), write the row into
-//                   the stage's 128B-swizzled K-major tile.
-// Four shared-memory stages decouple expansion from the MMAs; two TMEM
-// accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs
-// of tile i+1.
+//   warps 0..3   epilogue: TMEM lane quadrant w, one output row per thread;
+//                scale by s_m r'_n / K, round to BF16, store.
+//   warp 4       MMA issuer: one thread waits for a filled operand stage,
+//                issues four 128x256x16 kind::f16 MMAs into the tile's TMEM
+//                accumulator, commits them to the stage's "empty" barrier,
+//                and after the last K slice commits the accumulator.
+//   warp 5       TMA producer: one thread loads the packed codes of two K
+//                slices (64 codes each) for the tile's 128 A rows and 256 B
+//                rows into a ring of code stages (2D tiled bulk copies).
+//   warps 6..17  operand expansion, one row per thread (128 rows of A, 256 of
+//                B): read the row's codes of a K slice from the code stage,
+//                turn them into fp16 levels (x sqrt(K)), write the row into
+//                the operand stage's 128B-swizzled K-major tile.
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i overlap
+// the MMAs of tile i+1.
 //
 // 4-bit codes are expanded in registers: by symmetry C[15-c] = -C[c], the
 // magnitude index m (0..7) selects the two bytes of |C| with byte permutes
@@ -27,12 +28,22 @@
 // eight positive fp16 levels, and the sign lands on the high byte.  Other
 // widths read a 2^b-entry fp16 table in shared memory.
 //
+// Code stages: an operand of even width b is loaded one K slice per box (rows
+// of 8b bytes; 4- and 8-bit rows use the 32B / 64B TMA swizzle so that the
+// expansion threads, one row each, read them without bank conflicts); an odd
+// width is loaded two slices per box (rows of 16b bytes, an odd number of
+// 16-byte chunks, conflict-free as is).
+//
 // Every mbarrier wait is bounded; a thread whose wait runs out raises a
 // shared abort flag (so the others stop waiting at once), records an error
 // in the library's device error word, and the CTA still frees its TMEM.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <mutex>
 
 #include "rbq_internal.h"
 #include "rbq_sm100.cuh"
@@ -42,20 +53,34 @@ namespace qfast {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
-constexpr int kATile = kBM * kBK * 2;          // 16 KB
-constexpr int kBTile = kBN * kBK * 2;          // 32 KB
-constexpr int kStageBytes = kATile + kBTile;   // 48 KB
-constexpr int kThreads = 640;                  // 20 warps
-constexpr int kExpandFirst = 256;              // first expansion thread
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kATile = kBM * kBK * 2;          // 16 KB fp16
+constexpr int kBTile = kBN * kBK * 2;          // 32 KB fp16
+constexpr int kOpStage = kATile + kBTile;      // 48 KB
+constexpr int kMaxF = 4, kMaxC = 4;
+constexpr int kThreads = 576;                  // 18 warps
+constexpr int kMmaWarp = 4, kTmaWarp = 5;
+constexpr int kExpandFirst = 192;              // warp 6
 constexpr int kExpandThreads = kBM + kBN;      // 384
+constexpr size_t kSmemLimit = 227 * 1024;
+
+// Code-stage geometry of one operand.
+struct CodeGeo {
+  uint32_t rows;         // 128 (A) or 256 (B)
+  uint32_t bits;
+  uint32_t offset;       // byte offset of this operand inside a code stage
+  uint32_t bytes;        // bytes of this operand landing per code stage (2 K slices)
+  uint32_t slice_bytes;  // per-slice sub-buffer stride (even widths), else 0
+  uint32_t swz;          // 0 none, 1 = 32B swizzle (4-bit), 2 = 64B swizzle (8-bit)
+};
 
 struct Params {
-  const uint8_t* A;        // activation codes [M, K*bits_a/8]
-  const uint8_t* B;        // weight codes     [N, K*bits_b/8]
   int M, N, K;
   int bits_a, bits_b;
-  const uint16_t* lut_a;   // fp16 levels x sqrt(K), 2^bits entries
+  int F, C;                          // operand stages, code stages
+  uint32_t cstage_bytes;             // bytes per code stage (1024-aligned)
+  CodeGeo ga, gb;
+  const uint16_t* lut_a;             // fp16 levels x sqrt(K), 2^bits entries
   const uint16_t* lut_b;
   const float* s;
   const uint16_t* rnorm;
@@ -65,8 +90,10 @@ struct Params {
 };
 
 struct __align__(8) Tail {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxF];
+  uint64_t empty[kMaxF];
+  uint64_t cfull[kMaxC];
+  uint64_t cempty[kMaxC];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_slot;
@@ -74,8 +101,6 @@ struct __align__(8) Tail {
   uint16_t lut_a[256];
   uint16_t lut_b[256];
 };
-
-constexpr size_t kSmem = 1024 + kStages * kStageBytes + sizeof(Tail);
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
   const long long t0 = clock64();
@@ -95,8 +120,7 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Byte planes of the eight positive fp16 levels C[8..15]: lo/hi bytes of
-// levels 0-3 in p[0]/p[2], of levels 4-7 in p[1]/p[3].
+// Byte planes of the eight positive fp16 levels C[8..15].
 struct Planes4 {
   uint32_t lo0, lo1, hi0, hi1;
 };
@@ -122,8 +146,7 @@ __device__ __forceinline__ Planes4 make_planes4(const uint16_t* lut) {
 __device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint32_t (&w)[4]) {
   const uint32_t neg = (~x >> 3) & 0x11111111u;           // 1 where c < 8
   const uint32_t m = (x ^ (neg * 7u)) & 0x77777777u;      // c<8: 7-c, else c-8
-  // 0xFF bytes where an element is negative, elements 0-3 and 4-7
-  const uint32_t a7 = neg << 7, a3 = neg << 3;
+  const uint32_t a7 = neg << 7, a3 = neg << 3;            // 0xFF bytes where negative
   const uint32_t s_lo = prmt(a7, a3, 0xD9C8u);
   const uint32_t s_hi = prmt(a7, a3, 0xFBEAu);
   const uint32_t m_hi = m >> 16;
@@ -137,10 +160,13 @@ __device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint3
   w[3] = prmt(lo1, hi1, 0x7362u);
 }
 
+template <int BITS>
+constexpr int slice_words() { return 2 * BITS; }
+
 // One row's 64 codes of a K slice -> 8 swizzled 16-byte chunks of fp16.
 template <int BITS>
-__device__ __forceinline__ void expand_row(const uint32_t (&src)[16], const Planes4& P, const uint16_t* lut,
-                                           uint8_t* tile, int r) {
+__device__ __forceinline__ void expand_row(const uint32_t (&src)[slice_words<BITS>()], const Planes4& P,
+                                           const uint16_t* lut, uint8_t* tile, int r) {
   if constexpr (BITS == 4) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -171,66 +197,91 @@ __device__ __forceinline__ void expand_row(const uint32_t (&src)[16], const Plan
   }
 }
 
+// Row r's codes of K slice h (0/1) of a code stage -> 2*BITS words.
 template <int BITS>
-__device__ __forceinline__ void load_row(const uint8_t* row, int kb, bool valid, uint32_t (&dst)[16]) {
-  // 64 codes of slice kb = 8*BITS bytes, 8-byte aligned
-  const uint2* p = reinterpret_cast<const uint2*>(row + static_cast<size_t>(kb) * 8 * BITS);
+__device__ __forceinline__ void read_slice(const uint8_t* part, const CodeGeo& g, int r, int h,
+                                           uint32_t (&dst)[slice_words<BITS>()]) {
+  if constexpr ((BITS & 1) == 0) {
+    // even width: sub-buffer per slice, rows of 8*BITS bytes, maybe swizzled
+    const uint8_t* row = part + h * g.slice_bytes + r * (8 * BITS);
 #pragma unroll
-  for (int i = 0; i < BITS; ++i) {
-    const uint2 v = valid ? __ldg(p + i) : make_uint2(0, 0);
-    dst[2 * i] = v.x;
-    dst[2 * i + 1] = v.y;
-  }
+    for (int c = 0; c < BITS / 2; ++c) {
+      uint32_t pc = c;
+      if constexpr (BITS == 4) pc ^= (r >> 2) & 1;   // 32B swizzle
+      if constexpr (BITS == 8) pc ^= (r >> 1) & 3;   // 64B swizzle
+      const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * pc);
+      dst[4 * c] = v.x;
+      dst[4 * c + 1] = v.y;
+      dst[4 * c + 2] = v.z;
+      dst[4 * c + 3] = v.w;
+    }
+  } else {
+    // odd width: one box of two slices, rows of 16*BITS bytes
+    const uint2* row = reinterpret_cast<const uint2*>(part + r * (16 * BITS) + h * (8 * BITS));
 #pragma unroll
-  for (int i = 2 * BITS; i < 16; ++i) dst[i] = 0u;
-}
-
-template <int BITS>
-__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* stages, bool is_a, int r, int ntiles_m,
-                            int ntiles, Planes4 P, const uint16_t* lut, const uint8_t* base, long long pitch,
-                            int rows_total) {
-  const int KT = p.K / kBK;
-  uint32_t cnt = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int mt = tile % ntiles_m, nt = tile / ntiles_m;
-    const int row = is_a ? mt * kBM + r : nt * kBN + r;
-    const bool valid = row < rows_total;
-    const uint8_t* src = base + (valid ? row : 0) * pitch;
-    uint32_t cur[16], nxt[16];
-    load_row<BITS>(src, 0, valid, cur);
-    for (int kb = 0; kb < KT; ++kb) {
-      if (kb + 1 < KT) load_row<BITS>(src, kb + 1, valid, nxt);
-      const uint32_t s = cnt % kStages;
-      if (cnt >= kStages && !wait_or_abort(&tl->empty[s], ((cnt / kStages) - 1) & 1, tl)) return;
-      uint8_t* tile_ptr = stages + s * kStageBytes + (is_a ? 0 : kATile);
-      expand_row<BITS>(cur, P, lut, tile_ptr, r);
-      fence_proxy_async_smem();
-      mbar_arrive(&tl->full[s]);
-      ++cnt;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) cur[i] = nxt[i];
+    for (int i = 0; i < BITS; ++i) {
+      const uint2 v = row[i];
+      dst[2 * i] = v.x;
+      dst[2 * i + 1] = v.y;
     }
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
+template <int BITS>
+__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, bool is_a,
+                                            int r, int ntiles, Planes4 P, const uint16_t* lut) {
+  const CodeGeo& g = is_a ? p.ga : p.gb;
+  const int KP = p.K / (2 * kBK);
+  uint32_t cf = 0, cc = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    for (int kp = 0; kp < KP; ++kp) {
+      const uint32_t c = cc % p.C;
+      if (!wait_or_abort(&tl->cfull[c], (cc / p.C) & 1, tl)) return;
+      const uint8_t* part = codes + c * p.cstage_bytes + g.offset;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t cur[slice_words<BITS>()];
+        read_slice<BITS>(part, g, r, h, cur);
+        const uint32_t s = cf % p.F;
+        if (cf >= static_cast<uint32_t>(p.F) && !wait_or_abort(&tl->empty[s], ((cf / p.F) - 1) & 1, tl)) return;
+        uint8_t* tile_ptr = ops + s * kOpStage + (is_a ? 0 : kATile);
+        expand_row<BITS>(cur, P, lut, tile_ptr, r);
+        fence_proxy_async_smem();
+        mbar_arrive(&tl->full[s]);
+        ++cf;
+      }
+      mbar_arrive(&tl->cempty[c]);
+      ++cc;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    qlinear_fast_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* stages = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  Tail* tl = reinterpret_cast<Tail*>(stages + kStages * kStageBytes);
+  uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* codes = ops + p.F * kOpStage;
+  Tail* tl = reinterpret_cast<Tail*>(codes + p.C * p.cstage_bytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntiles_m = (p.M + kBM - 1) / kBM, ntiles_n = (p.N + kBN - 1) / kBN;
   const int ntiles = ntiles_m * ntiles_n;
   const int KT = p.K / kBK;
+  const int KP = KT / 2;
 
   for (int i = tid; i < 256; i += kThreads) {
     tl->lut_a[i] = (i < (1 << p.bits_a)) ? p.lut_a[i] : 0;
     tl->lut_b[i] = (i < (1 << p.bits_b)) ? p.lut_b[i] : 0;
   }
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < p.F; ++s) {
       mbar_init(&tl->full[s], kExpandThreads);
       mbar_init(&tl->empty[s], 1);
+    }
+    for (int c = 0; c < p.C; ++c) {
+      mbar_init(&tl->cfull[c], 1);
+      mbar_init(&tl->cempty[c], kExpandThreads);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tl->acc_full[a], 1);
@@ -239,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
     tl->abort = 0u;
     mbar_fence_init();
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&tl->tmem_slot, 512);
     tmem_relinquish();
   }
@@ -248,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
   tc_fence_after();
   const uint32_t tmem = tl->tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, false);
@@ -260,10 +311,10 @@ __global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
         tc_fence_after();
         const uint32_t acc = tmem + a * kBN;
         for (int kb = 0; kb < KT; ++kb) {
-          const uint32_t s = cnt % kStages;
-          if (!wait_or_abort(&tl->full[s], (cnt / kStages) & 1, tl)) { ok = false; break; }
+          const uint32_t s = cnt % p.F;
+          if (!wait_or_abort(&tl->full[s], (cnt / p.F) & 1, tl)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(stages + s * kStageBytes);
+          const uint32_t a0 = smem_u32(ops + s * kOpStage);
           const uint32_t b0 = a0 + kATile;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
@@ -275,9 +326,45 @@ __global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
       }
       if (!ok) atomicOr(p.err, 2u);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp == kTmaWarp) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      uint32_t cnt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+        for (int kp = 0; kp < KP; ++kp) {
+          const uint32_t c = cnt % p.C;
+          if (cnt >= static_cast<uint32_t>(p.C) && !wait_or_abort(&tl->cempty[c], ((cnt / p.C) - 1) & 1, tl)) {
+            ok = false;
+            break;
+          }
+          uint8_t* stage = codes + c * p.cstage_bytes;
+          mbar_arrive_expect_tx(&tl->cfull[c], p.ga.bytes + p.gb.bytes);
+          if (p.ga.slice_bytes) {
+            tma_load_2d(stage + p.ga.offset, &tmA, (2 * kp) * 8 * p.ga.bits, mt * kBM, &tl->cfull[c]);
+            tma_load_2d(stage + p.ga.offset + p.ga.slice_bytes, &tmA, (2 * kp + 1) * 8 * p.ga.bits, mt * kBM,
+                        &tl->cfull[c]);
+          } else {
+            tma_load_2d(stage + p.ga.offset, &tmA, kp * 16 * p.ga.bits, mt * kBM, &tl->cfull[c]);
+          }
+          if (p.gb.slice_bytes) {
+            tma_load_2d(stage + p.gb.offset, &tmB, (2 * kp) * 8 * p.gb.bits, nt * kBN, &tl->cfull[c]);
+            tma_load_2d(stage + p.gb.offset + p.gb.slice_bytes, &tmB, (2 * kp + 1) * 8 * p.gb.bits, nt * kBN,
+                        &tl->cfull[c]);
+          } else {
+            tma_load_2d(stage + p.gb.offset, &tmB, kp * 16 * p.gb.bits, nt * kBN, &tl->cfull[c]);
+          }
+          ++cnt;
+        }
+      }
+      if (!ok) atomicOr(p.err, 16u);
+    }
+  } else if (warp < 4) {
     // ---------------- epilogue ----------------
-    const int q = warp & 3;                 // TMEM lane quadrant
+    const int q = warp;                     // TMEM lane quadrant
     const int r = 32 * q + lane;            // row within the tile
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
@@ -325,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
       tc_fence_before();
       mbar_arrive(&tl->acc_empty[a]);
     }
-  } else if (warp >= 8) {
+  } else {
     // ---------------- operand expansion ----------------
     const int e = tid - kExpandFirst;
     const bool is_a = e < kBM;
@@ -333,47 +420,112 @@ __global__ void __launch_bounds__(kThreads, 1) qlinear_fast_kernel(Params p) {
     const int bits = is_a ? p.bits_a : p.bits_b;
     const uint16_t* lut = is_a ? tl->lut_a : tl->lut_b;
     const Planes4 P = make_planes4(lut);
-    const uint8_t* base = is_a ? p.A : p.B;
-    const long long pitch = static_cast<long long>(p.K) * bits / 8;
-    const int rows_total = is_a ? p.M : p.N;
     switch (bits) {
-      case 2: expand_loop<2>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      case 3: expand_loop<3>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      case 4: expand_loop<4>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      case 5: expand_loop<5>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      case 6: expand_loop<6>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      case 7: expand_loop<7>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      case 8: expand_loop<8>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
-      default: expand_loop<1>(p, tl, stages, is_a, r, ntiles_m, ntiles, P, lut, base, pitch, rows_total); break;
+      case 1: expand_loop<1>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      case 2: expand_loop<2>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      case 3: expand_loop<3>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      case 4: expand_loop<4>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      case 5: expand_loop<5>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      case 6: expand_loop<6>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      case 7: expand_loop<7>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+      default: expand_loop<8>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
     }
     if (tl->abort && e == 0) atomicOr(p.err, 8u);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
+// ---- host side ------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// Geometry of one operand's share of a code stage, starting at `offset`.
+CodeGeo make_geo(uint32_t rows, uint32_t bits, uint32_t offset) {
+  CodeGeo g{};
+  g.rows = rows;
+  g.bits = bits;
+  g.offset = offset;
+  if ((bits & 1) == 0) {
+    const uint32_t sb = rows * 8 * bits;
+    g.slice_bytes = (sb + 1023u) & ~1023u;   // each slice buffer swizzle-aligned
+    g.bytes = 2 * sb;                        // bytes landing per stage
+    g.swz = bits == 4 ? 1 : bits == 8 ? 2 : 0;
+  } else {
+    g.slice_bytes = 0;
+    g.bytes = rows * 16 * bits;
+    g.swz = 0;
+  }
+  return g;
+}
+
+uint32_t geo_span(const CodeGeo& g) {
+  return g.slice_bytes ? 2 * g.slice_bytes : ((g.bytes + 1023u) & ~1023u);
+}
+
+int encode_map(CUtensorMap* map, const uint8_t* base, int rows, int bits, int K, const CodeGeo& g) {
+  auto fn = encode_fn();
+  if (!fn) return RBQ_ECUDA;
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(K) * bits / 8;
+  const cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {g.slice_bytes ? 8u * bits : 16u * bits, g.rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = g.swz == 1 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : g.swz == 2 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
+}
+
 }  // namespace qfast
 
-bool qlinear_fast_eligible(int M, int N, int K) {
-  return M >= 1 && N >= 1 && (N % 8) == 0 && (K % 64) == 0 && K >= 64;
+bool qlinear_fast_eligible(int M, int N, int K, int bits_a, int bits_w) {
+  if (M < 1 || N < 1 || (N % 8) != 0 || K < 128 || (K % 128) != 0) return false;
+  // TMA needs 16-byte row strides for both code tensors
+  return (static_cast<long long>(K) * bits_a / 8) % 16 == 0 && (static_cast<long long>(K) * bits_w / 8) % 16 == 0;
 }
 
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
                         const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st) {
-  qfast::Params p{};
-  p.A = a_codes;
-  p.B = w_codes;
+  using namespace qfast;
+  Params p{};
   p.M = M;
   p.N = N;
   p.K = K;
   p.bits_a = bits_a;
   p.bits_b = bits_w;
+  p.ga = make_geo(kBM, bits_a, 0);
+  p.gb = make_geo(kBN, bits_w, geo_span(p.ga));
+  p.cstage_bytes = geo_span(p.ga) + geo_span(p.gb);
+  const size_t tail = sizeof(Tail) + 64;
+  // as many operand stages (2..4) and code stages (2..4) as shared memory allows
+  int F = kMaxF, C = 2;
+  while (F > 2 && 1024 + F * kOpStage + C * p.cstage_bytes + tail > kSmemLimit) --F;
+  while (C < kMaxC && 1024 + F * kOpStage + (C + 1) * p.cstage_bytes + tail <= kSmemLimit) ++C;
+  const size_t smem = 1024 + static_cast<size_t>(F) * kOpStage + static_cast<size_t>(C) * p.cstage_bytes + tail;
+  if (smem > kSmemLimit) return RBQ_EINVAL;
+  p.F = F;
+  p.C = C;
   p.lut_a = ca->levels_f16;
   p.lut_b = cw->levels_f16;
   p.s = s;
@@ -381,16 +533,19 @@ int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, cons
   p.inv_k = ca->inv_d;
   p.Y = Y;
   p.err = err;
-  auto kern = qfast::qlinear_fast_kernel;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(qfast::kSmem));
+  CUtensorMap mA, mB;
+  int rc = encode_map(&mA, a_codes, M, bits_a, K, p.ga);
+  if (rc != RBQ_OK) return rc;
+  if ((rc = encode_map(&mB, w_codes, N, bits_w, K, p.gb)) != RBQ_OK) return rc;
+  auto kern = qlinear_fast_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int ntiles = ((M + qfast::kBM - 1) / qfast::kBM) * ((N + qfast::kBN - 1) / qfast::kBN);
+  const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
   const int grid = ntiles < sms ? ntiles : sms;
-  kern<<<grid, qfast::kThreads, qfast::kSmem, st>>>(p);
+  kern<<<grid, kThreads, smem, st>>>(mA, mB, p);
   e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }

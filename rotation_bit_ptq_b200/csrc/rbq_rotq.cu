@@ -266,8 +266,9 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) { return __ldcs(p); 
 
 template <int G>
 struct Layout {
-  // bytes: stage[2] (G*d*2 each) | off (4d) | mask (2d) | red (4*G*32) | grid
-  static __host__ __device__ size_t stage_bytes(int d) { return static_cast<size_t>(G) * d * 2; }
+  // bytes: stage[2] (G rows of 2d+16) | off (4d) | mask (2d) | red (4*G*32) | grid
+  static __host__ __device__ size_t row_pitch(int d) { return 2 * static_cast<size_t>(d) + 16; }
+  static __host__ __device__ size_t stage_bytes(int d) { return G * row_pitch(d); }
   static __host__ __device__ size_t off_at(int d) { return 2 * stage_bytes(d); }
   static __host__ __device__ size_t mask_at(int d) { return off_at(d) + 4 * static_cast<size_t>(d); }
   static __host__ __device__ size_t red_at(int d) { return mask_at(d) + 2 * static_cast<size_t>(d); }
@@ -293,6 +294,10 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
   constexpr bool kLloyd = (MODE == kAct || MODE == kWeightLM);
 
   // ---- per-CTA tables ------------------------------------------------------
+  // mask16[j]: 0x8000 where source position j is sign-flipped, i.e. D_k = -1
+  // for the output position k with pi(k) = j.  off[]: byte offset 2*pi(k) of
+  // the source of output position k inside a staged row, stored swizzled so
+  // that the threads of a warp read their 16-byte groups without conflicts.
   uint16_t* mask16 = reinterpret_cast<uint16_t*>(smem + L::mask_at(d));
   uint32_t* off = reinterpret_cast<uint32_t*>(smem + L::off_at(d));
   for (int k = tid; k < d; k += nthreads) {
@@ -300,37 +305,51 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
     mask16[j] = (__ldg(p.sign + k) < 0.f) ? 0x8000u : 0u;
     const int kb = k >> 6, ki = k & 63;
     const int slot = 64 * kb + 4 * ((ki >> 2) ^ (kb & 15)) + (ki & 3);
-    off[slot] = static_cast<uint32_t>((j >> 3) * (G * 16) + (j & 7) * 2);
+    off[slot] = static_cast<uint32_t>(2 * j);
   }
   if (kLloyd) {
     float2* gs = reinterpret_cast<float2*>(smem + L::grid_at(d));
     for (int n = tid; n < p.grid_n; n += nthreads) gs[n] = p.grid[n];
   }
+  __syncthreads();   // tables ready
 
-  // ---- staging helpers ------------------------------------------------------
-  const int sg = tid % G;              // staged token
-  const int sc0 = tid / G;             // first staged chunk; chunks sc0 + j*nblk
+  // ---- staging: 16-byte chunks, token-major rows, chunk index fastest ----
+  // Active thread t stages chunks L = t + i*nact (i = 0..7) of the G x (d/8)
+  // chunk grid, i.e. 8/G distinct chunk indices per thread; with G = 4 their
+  // sign masks stay in registers, otherwise they are read from shared memory.
+  // With nact = G*nblk and d/8 = 8*nblk, slot i is token (i*G)>>3, chunk
+  // t + ((i*G)&7)*nblk: compile-time in i.
+  constexpr bool kRegMasks = (G == 4);         // 2 chunks x 4 words per thread
+  constexpr int NM = kRegMasks ? 8 / G : 1;
+  uint4 msk[NM];
+  if (kRegMasks && active) {
+#pragma unroll
+    for (int i = 0; i < NM; ++i) msk[i] = lds128(mask_addr + 16 * (tid + ((i * G) & 7) * nblk));
+  }
   const long long ngroups = (p.T + G - 1) / G;
   uint4 pre[8];
   auto load_group = [&](long long gi) {
-    const long long row = gi * G + sg;
-    const bool valid = active && (gi < ngroups) && (row < p.T);
-    const uint4* src = reinterpret_cast<const uint4*>(p.X + (valid ? row : 0) * d);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) pre[j] = valid ? ldg_stream(src + sc0 + j * nblk) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < 8; ++i) {
+      const int sg = (i * G) >> 3, c = tid + ((i * G) & 7) * nblk;
+      const long long row = gi * G + sg;
+      const bool valid = active && (gi < ngroups) && (row < p.T);
+      pre[i] = valid ? ldg_stream(reinterpret_cast<const uint4*>(p.X + row * d) + c) : make_uint4(0, 0, 0, 0);
+    }
   };
   auto store_group = [&](int st) {
     if (!active) return;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = sc0 + j * nblk;
-      const uint4 m = lds128(mask_addr + 16 * c);
-      const uint4 v = make_uint4(pre[j].x ^ m.x, pre[j].y ^ m.y, pre[j].z ^ m.z, pre[j].w ^ m.w);
-      sts128(stage_addr[st] + 16 * (c * G + sg), v);
+    for (int i = 0; i < 8; ++i) {
+      const int sg = (i * G) >> 3, c = tid + ((i * G) & 7) * nblk;
+      uint4 m;
+      if constexpr (kRegMasks) m = msk[i % NM];
+      else m = lds128(mask_addr + 16 * c);
+      const uint4 v = make_uint4(pre[i].x ^ m.x, pre[i].y ^ m.y, pre[i].z ^ m.z, pre[i].w ^ m.w);
+      sts128(stage_addr[st] + static_cast<uint32_t>(sg * L::row_pitch(d)) + 16 * c, v);
     }
   };
 
-  __syncthreads();   // tables ready
   long long gi = blockIdx.x;
   load_group(gi);
   store_group(0);
@@ -344,7 +363,7 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
     // ---- gather (signs already applied) -> 32 fp32x2 pairs (y_2m, y_2m+1) ----
     unsigned long long P[32];
     if (active) {
-      const uint32_t base = stage_addr[st] + 16 * g;
+      const uint32_t base = stage_addr[st] + static_cast<uint32_t>(g * L::row_pitch(d));
 #pragma unroll
       for (int i4 = 0; i4 < 16; ++i4) {
         const uint4 o = lds128(off_addr + 4 * (64 * b + 4 * (i4 ^ (b & 15))));
@@ -405,9 +424,8 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
     for (int w = 0; w < nwarps; ++w)
       tot = (MODE == kInt8) ? fmaxf(tot, red[g * 32 + w]) : tot + red[g * 32 + w];
 
-    // ---- refill the other stage while this one is consumed ----
+    // ---- refill the other stage (its loads were issued one iteration ago) ----
     store_group(st ^ 1);
-    load_group(gi + 2 * static_cast<long long>(gridDim.x));
 
     const long long t = gi * G + g;
     if (active && t < p.T) {
@@ -428,11 +446,16 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
           const float u = fma_sat(z, A, 0.5f);
           const float qf = fmaf(u, p.grid_cells, 8388608.0f);   // 2^23: round(u*NC) in the low bits
           const float2 e = lds_f2(gbase + __float_as_uint(qf) * 8u);
-          const float diff = fmaf(z, inv, -e.x);
-          const uint32_t code = static_cast<uint32_t>(__float_as_int(e.y)) + ((__float_as_uint(diff) >> 31) ^ 1u);
+          // code = base + (v >= thr): the sign of z*inv - thr, as 0 / -1
+          const int below = __float_as_int(fmaf(z, inv, -e.x)) >> 31;
+          const uint32_t code = static_cast<uint32_t>(__float_as_int(e.y) + 1 + below);
           const int bit = r * BITS, wi = bit >> 5, sh = bit & 31;
-          w[wi] |= code << sh;
-          if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
+          if constexpr ((32 % BITS) == 0) {
+            w[wi] += code << sh;                   // disjoint fields: add = or
+          } else {
+            w[wi] |= code << sh;
+            if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
+          }
         }
         unsigned char* dst = static_cast<unsigned char*>(p.out) + t * (static_cast<long long>(d) * BITS / 8) +
                              static_cast<long long>(b) * 8 * BITS;
@@ -485,6 +508,9 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         if (b == 0 && p.aux) static_cast<float*>(p.aux)[t] = sqrtf(tot) * 0.125f;
       }
     }
+    // next group's loads: issued after the code phase so that the staging
+    // registers are not live while the codes are computed
+    load_group(gi + 2 * static_cast<long long>(gridDim.x));
     __syncthreads();   // stage st fully read and stage st^1 fully written
   }
 }
@@ -576,7 +602,9 @@ int launch_fast_bits(const fast::Params& p, cudaStream_t st) {
 
 template <int MODE>
 int launch_fast(int bits, const fast::Params& p, cudaStream_t st) {
-  if (MODE != kAct && MODE != kWeightLM) return launch_fast_bits<MODE, 8>(p, st);
+  if constexpr (MODE != kAct && MODE != kWeightLM) {
+    return launch_fast_bits<MODE, 8>(p, st);
+  } else {
   switch (bits) {
     case 1: return launch_fast_bits<MODE, 1>(p, st);
     case 2: return launch_fast_bits<MODE, 2>(p, st);
@@ -587,6 +615,7 @@ int launch_fast(int bits, const fast::Params& p, cudaStream_t st) {
     case 7: return launch_fast_bits<MODE, 7>(p, st);
     case 8: return launch_fast_bits<MODE, 8>(p, st);
     default: return RBQ_EINVAL;
+  }
   }
 }
 
