@@ -187,17 +187,21 @@ int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float* scale,
 /* ---- diagnostics ----------------------------------------------------------- */
 
 /*
- * rbq_code_grid -- the code-search table the kernels use for (d, bits), for
+ * rbq_code_grid -- a code-search table the kernels use for (d, bits), for
  * inspection and tests (host only).  A coordinate v gets
  *   n = round_to_nearest( clamp(v * scale + 0.5, 0, 1) * cells ),
  *   code = base[n] + (v >= thr[n]),
  * which equals #{ j : t_j <= v } outside a rounding band around each boundary.
+ *   variant  0: grid over [-R, R] just wider than the outermost boundary
+ *               (the kernels clamp); 1: grid over [-1, 1], the range of a unit
+ *               vector's coordinates (no clamp; RBQ_ECONVERGE when it would
+ *               exceed 5000 cells)
  *   thr    HOST float[cells + 1] (may be NULL)
  *   base   HOST int32[cells + 1] (may be NULL)
  *   cells, scale  receive the grid size and the factor 1/(2R)
  * Returns RBQ_OK, RBQ_EINVAL or RBQ_ECONVERGE.
  */
-int rbq_code_grid(int d, int bits, float* thr, int32_t* base, int* cells, float* scale);
+int rbq_code_grid(int d, int bits, int variant, float* thr, int32_t* base, int* cells, float* scale);
 
 /* Text for a return code (static storage). */
 const char* rbq_error_string(int code);

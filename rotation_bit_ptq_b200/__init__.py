@@ -36,7 +36,7 @@ SIGNATURES = {
     "qlinear_int8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
-    "rbq_code_grid": (_I, [_I, _I, _P, _P, _P, _P]),
+    "rbq_code_grid": (_I, [_I, _I, _I, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -251,15 +251,16 @@ def qlinear_int8(xrot, q, scale, out=None, stream=None):
     return out
 
 
-def code_grid(d, bits):
-    """The kernels' code-search table: (thr float32[n], base int32[n], cells, scale)."""
+def code_grid(d, bits, variant=0):
+    """A code-search table of the kernels: (thr float32[n], base int32[n], cells, scale).
+    variant 0: clamped grid just wider than the boundaries; 1: grid over [-1, 1]."""
     cells, scale = ctypes.c_int(), ctypes.c_float()
-    _check(lib().rbq_code_grid(int(d), int(bits), None, None, ctypes.byref(cells), ctypes.byref(scale)),
-           "rbq_code_grid")
+    _check(lib().rbq_code_grid(int(d), int(bits), int(variant), None, None, ctypes.byref(cells),
+                               ctypes.byref(scale)), "rbq_code_grid")
     thr = np.empty(cells.value + 1, dtype=np.float32)
     base = np.empty(cells.value + 1, dtype=np.int32)
-    _check(lib().rbq_code_grid(int(d), int(bits), thr.ctypes.data_as(_P), base.ctypes.data_as(_P), None, None),
-           "rbq_code_grid")
+    _check(lib().rbq_code_grid(int(d), int(bits), int(variant), thr.ctypes.data_as(_P), base.ctypes.data_as(_P),
+                               None, None), "rbq_code_grid")
     return thr, base, cells.value, np.float32(scale.value)
 
 

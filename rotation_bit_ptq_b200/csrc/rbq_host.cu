@@ -250,6 +250,21 @@ bool try_grid(const std::vector<double>& t, int nc, double R, Grid* g) {
   return true;
 }
 
+// Full-range variant: R = 1, the largest |v| a unit vector can have, so the
+// kernel needs no clamp.  Returns RBQ_ECONVERGE if it would need more than
+// `max_cells` cells.
+int build_grid_full(const std::vector<double>& bounds, int max_cells, Grid* g) {
+  double gap = INFINITY;
+  for (size_t j = 1; j < bounds.size(); ++j) gap = std::fmin(gap, bounds[j] - bounds[j - 1]);
+  if (bounds.size() == 1) gap = 1.0;
+  int nc = static_cast<int>(std::ceil(2.0 / (0.9 * gap)));
+  nc += nc & 1;
+  if (nc < 4) nc = 4;
+  for (; nc <= max_cells; nc += 2)
+    if (try_grid(bounds, nc, 1.0, g)) return RBQ_OK;
+  return RBQ_ECONVERGE;
+}
+
 int build_grid(const std::vector<double>& bounds, Grid* g) {
   double tmax = 0.0, gap = INFINITY;
   for (size_t j = 0; j < bounds.size(); ++j) {
@@ -348,12 +363,18 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
   cb->grid_cells = grid.cells;
   cb->grid_scale = static_cast<float>(1.0 / (2.0 * grid.R));
   if ((rc = upload(grid.lut.data(), grid.lut.size(), &cb->grid)) != RBQ_OK) { delete cb; return rc; }
+  Grid full;
+  if (build_grid_full(bounds, kMaxFullGridCells, &full) == RBQ_OK) {
+    cb->grid_full_cells = full.cells;
+    if ((rc = upload(full.lut.data(), full.lut.size(), &cb->grid_full)) != RBQ_OK) { delete cb; return rc; }
+  }
   std::lock_guard<std::mutex> lk(g_mu);
   auto ins = cb_cache().emplace(key, cb);
   if (!ins.second) {          // another thread won the race; keep its copy
     cudaFree(cb->bounds);
     cudaFree(cb->levels_f16);
     cudaFree(cb->grid);
+    cudaFree(cb->grid_full);
     delete cb;
   }
   *out = ins.first->second;
@@ -467,13 +488,15 @@ extern "C" int rbq_device_error(void* stream) {
   return RBQ_OK;
 }
 
-extern "C" int rbq_code_grid(int d, int bits, float* thr, int32_t* base, int* cells, float* scale) {
-  if (d <= 0 || bits < 1 || bits > 8) return RBQ_EINVAL;
+extern "C" int rbq_code_grid(int d, int bits, int variant, float* thr, int32_t* base, int* cells,
+                             float* scale) {
+  if (d <= 0 || bits < 1 || bits > 8 || (variant != 0 && variant != 1)) return RBQ_EINVAL;
   std::vector<double> levels, bounds;
   int rc = full_table(d, bits, levels, bounds);
   if (rc != RBQ_OK) return rc;
   Grid g;
-  if ((rc = build_grid(bounds, &g)) != RBQ_OK) return rc;
+  rc = variant ? build_grid_full(bounds, kMaxFullGridCells, &g) : build_grid(bounds, &g);
+  if (rc != RBQ_OK) return rc;
   for (size_t n = 0; n < g.lut.size(); ++n) {
     if (thr) thr[n] = g.lut[n].x;
     if (base) {

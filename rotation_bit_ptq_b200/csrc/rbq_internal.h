@@ -47,7 +47,13 @@ struct CodebookDevice {
   float2* grid = nullptr;
   int grid_cells = 0;
   float grid_scale = 0.f;         // 1 / (2R)
+  // The same over v in [-1, 1] (R = 1, no clamp needed); null when it would
+  // need more than kMaxFullGridCells cells.
+  float2* grid_full = nullptr;
+  int grid_full_cells = 0;
 };
+
+constexpr int kMaxFullGridCells = 5000;
 
 // Returns the device tables of `r` on the current device, uploading on first use.
 int rpbh_device(const rbq_rpbh* r, const RpbhDevice** out);

@@ -5,22 +5,32 @@
 //   the weights (§2.1) cancels the online one, so
 //   y[m,n] = s_m r'_n sum_k C_w[q_nk] C_a[p_mk].
 //
-// Each CTA (one per SM) walks a static list of 128 x 256 output tiles.
-//   warps 0..3   epilogue: TMEM lane quadrant w, one output row per thread;
-//                scale by s_m r'_n / K, round to BF16, store.
-//   warp 4       MMA issuer: one thread waits for a filled operand stage,
-//                issues four 128x256x16 kind::f16 MMAs into the tile's TMEM
-//                accumulator, commits them to the stage's "empty" barrier,
-//                and after the last K slice commits the accumulator.
-//   warp 5       TMA producer: one thread loads the packed codes of two K
-//                slices (64 codes each) for the tile's 128 A rows and 256 B
-//                rows into a ring of code stages (2D tiled bulk copies).
-//   warps 6..17  operand expansion, one row per thread (128 rows of A, 256 of
-//                B): read the row's codes of a K slice from the code stage,
-//                turn them into fp16 levels (x sqrt(K)), write the row into
-//                the operand stage's 128B-swizzled K-major tile.
-// Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i overlap
-// the MMAs of tile i+1.
+// Two kernels per call.
+//
+// 1. expand_weights_kernel: the weight codes are turned into fp16 levels
+//    (x sqrt(K)) once, into a stream-ordered workspace [N, K] -- an HBM-bound
+//    pass over N*K*(b/8 + 2) bytes.  Expanding each weight tile inside the
+//    GEMM instead would redo that work for every 128-row tile of tokens and
+//    saturate the SM's integer pipe.
+// 2. qlinear_fast_kernel: each CTA (one per SM) walks a static list of
+//    128 x 256 output tiles.
+//      warps 0..3  epilogue: TMEM lane quadrant w, one output row per thread;
+//                  scale by s_m r'_n / K, round to BF16, store.
+//      warp 4      MMA issuer: one thread waits for a filled operand stage,
+//                  issues four 128x256x16 kind::f16 MMAs into the tile's TMEM
+//                  accumulator, commits them to the stage's "empty" barrier,
+//                  and after the last K slice commits the accumulator.
+//      warp 5      TMA producer: one thread loads (a) the activation codes of
+//                  two K slices for the tile's 128 rows into a ring of code
+//                  stages and (b) the 256 x 64 fp16 weight tile of each K
+//                  slice straight into the operand stage, 128B-swizzled as the
+//                  tensor core reads it.
+//      warps 6..9  activation expansion, one row per thread: read the row's
+//                  codes of a K slice from the code stage, turn them into fp16
+//                  levels, write the row into the operand stage's swizzled
+//                  K-major tile.
+//    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
+//    overlap the MMAs of tile i+1.
 //
 // 4-bit codes are expanded in registers: by symmetry C[15-c] = -C[c], the
 // magnitude index m (0..7) selects the two bytes of |C| with byte permutes
@@ -28,7 +38,7 @@
 // eight positive fp16 levels, and the sign lands on the high byte.  Other
 // widths read a 2^b-entry fp16 table in shared memory.
 //
-// Code stages: an operand of even width b is loaded one K slice per box (rows
+// Activation code stages: an even width b is loaded one K slice per box (rows
 // of 8b bytes; 4- and 8-bit rows use the 32B / 64B TMA swizzle so that the
 // expansion threads, one row each, read them without bank conflicts); an odd
 // width is loaded two slices per box (rows of 16b bytes, an odd number of
@@ -58,15 +68,15 @@ constexpr int kATile = kBM * kBK * 2;          // 16 KB fp16
 constexpr int kBTile = kBN * kBK * 2;          // 32 KB fp16
 constexpr int kOpStage = kATile + kBTile;      // 48 KB
 constexpr int kMaxF = 4, kMaxC = 4;
-constexpr int kThreads = 576;                  // 18 warps
+constexpr int kThreads = 320;                  // 10 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
 constexpr int kExpandFirst = 192;              // warp 6
-constexpr int kExpandThreads = kBM + kBN;      // 384
+constexpr int kExpandThreads = kBM;            // 128 activation rows
 constexpr size_t kSmemLimit = 227 * 1024;
 
-// Code-stage geometry of one operand.
+// Code-stage geometry of the activation operand.
 struct CodeGeo {
-  uint32_t rows;         // 128 (A) or 256 (B)
+  uint32_t rows;         // 128
   uint32_t bits;
   uint32_t offset;       // byte offset of this operand inside a code stage
   uint32_t bytes;        // bytes of this operand landing per code stage (2 K slices)
@@ -76,12 +86,11 @@ struct CodeGeo {
 
 struct Params {
   int M, N, K;
-  int bits_a, bits_b;
+  int bits_a;
   int F, C;                          // operand stages, code stages
   uint32_t cstage_bytes;             // bytes per code stage (1024-aligned)
-  CodeGeo ga, gb;
+  CodeGeo ga;
   const uint16_t* lut_a;             // fp16 levels x sqrt(K), 2^bits entries
-  const uint16_t* lut_b;
   const float* s;
   const uint16_t* rnorm;
   float inv_k;
@@ -99,7 +108,6 @@ struct __align__(8) Tail {
   uint32_t tmem_slot;
   volatile uint32_t abort;
   uint16_t lut_a[256];
-  uint16_t lut_b[256];
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
@@ -228,9 +236,9 @@ __device__ __forceinline__ void read_slice(const uint8_t* part, const CodeGeo& g
 }
 
 template <int BITS>
-__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, bool is_a,
-                                            int r, int ntiles, Planes4 P, const uint16_t* lut) {
-  const CodeGeo& g = is_a ? p.ga : p.gb;
+__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, int r,
+                                            int ntiles, Planes4 P, const uint16_t* lut) {
+  const CodeGeo& g = p.ga;
   const int KP = p.K / (2 * kBK);
   uint32_t cf = 0, cc = 0;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
@@ -244,8 +252,7 @@ __device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* 
         read_slice<BITS>(part, g, r, h, cur);
         const uint32_t s = cf % p.F;
         if (cf >= static_cast<uint32_t>(p.F) && !wait_or_abort(&tl->empty[s], ((cf / p.F) - 1) & 1, tl)) return;
-        uint8_t* tile_ptr = ops + s * kOpStage + (is_a ? 0 : kATile);
-        expand_row<BITS>(cur, P, lut, tile_ptr, r);
+        expand_row<BITS>(cur, P, lut, ops + s * kOpStage, r);
         fence_proxy_async_smem();
         mbar_arrive(&tl->full[s]);
         ++cf;
@@ -270,13 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KT = p.K / kBK;
   const int KP = KT / 2;
 
-  for (int i = tid; i < 256; i += kThreads) {
-    tl->lut_a[i] = (i < (1 << p.bits_a)) ? p.lut_a[i] : 0;
-    tl->lut_b[i] = (i < (1 << p.bits_b)) ? p.lut_b[i] : 0;
-  }
+  for (int i = tid; i < 256; i += kThreads) tl->lut_a[i] = (i < (1 << p.bits_a)) ? p.lut_a[i] : 0;
   if (tid == 0) {
     for (int s = 0; s < p.F; ++s) {
-      mbar_init(&tl->full[s], kExpandThreads);
+      mbar_init(&tl->full[s], kExpandThreads + 1);   // + the producer's expect-tx arrival (weight tile)
       mbar_init(&tl->empty[s], 1);
     }
     for (int c = 0; c < p.C; ++c) {
@@ -331,18 +335,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      uint32_t cnt = 0;
+      uint32_t cc = 0, cf = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const int mt = tile % ntiles_m, nt = tile / ntiles_m;
-        for (int kp = 0; kp < KP; ++kp) {
-          const uint32_t c = cnt % p.C;
-          if (cnt >= static_cast<uint32_t>(p.C) && !wait_or_abort(&tl->cempty[c], ((cnt / p.C) - 1) & 1, tl)) {
+        for (int kp = 0; kp < KP && ok; ++kp) {
+          const uint32_t c = cc % p.C;
+          if (cc >= static_cast<uint32_t>(p.C) && !wait_or_abort(&tl->cempty[c], ((cc / p.C) - 1) & 1, tl)) {
             ok = false;
             break;
           }
           uint8_t* stage = codes + c * p.cstage_bytes;
-          mbar_arrive_expect_tx(&tl->cfull[c], p.ga.bytes + p.gb.bytes);
+          mbar_arrive_expect_tx(&tl->cfull[c], p.ga.bytes);
           if (p.ga.slice_bytes) {
             tma_load_2d(stage + p.ga.offset, &tmA, (2 * kp) * 8 * p.ga.bits, mt * kBM, &tl->cfull[c]);
             tma_load_2d(stage + p.ga.offset + p.ga.slice_bytes, &tmA, (2 * kp + 1) * 8 * p.ga.bits, mt * kBM,
@@ -350,14 +354,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(stage + p.ga.offset, &tmA, kp * 16 * p.ga.bits, mt * kBM, &tl->cfull[c]);
           }
-          if (p.gb.slice_bytes) {
-            tma_load_2d(stage + p.gb.offset, &tmB, (2 * kp) * 8 * p.gb.bits, nt * kBN, &tl->cfull[c]);
-            tma_load_2d(stage + p.gb.offset + p.gb.slice_bytes, &tmB, (2 * kp + 1) * 8 * p.gb.bits, nt * kBN,
-                        &tl->cfull[c]);
-          } else {
-            tma_load_2d(stage + p.gb.offset, &tmB, kp * 16 * p.gb.bits, nt * kBN, &tl->cfull[c]);
+          ++cc;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t s = cf % p.F;
+            if (cf >= static_cast<uint32_t>(p.F) && !wait_or_abort(&tl->empty[s], ((cf / p.F) - 1) & 1, tl)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&tl->full[s], kBTile);
+            tma_load_2d(ops + s * kOpStage + kATile, &tmB, (2 * kp + h) * kBK, nt * kBN, &tl->full[s]);
+            ++cf;
           }
-          ++cnt;
         }
       }
       if (!ok) atomicOr(p.err, 16u);
@@ -413,24 +421,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&tl->acc_empty[a]);
     }
   } else {
-    // ---------------- operand expansion ----------------
-    const int e = tid - kExpandFirst;
-    const bool is_a = e < kBM;
-    const int r = is_a ? e : e - kBM;
-    const int bits = is_a ? p.bits_a : p.bits_b;
-    const uint16_t* lut = is_a ? tl->lut_a : tl->lut_b;
+    // ---------------- activation expansion ----------------
+    const int r = tid - kExpandFirst;
+    const uint16_t* lut = tl->lut_a;
     const Planes4 P = make_planes4(lut);
-    switch (bits) {
-      case 1: expand_loop<1>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      case 2: expand_loop<2>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      case 3: expand_loop<3>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      case 4: expand_loop<4>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      case 5: expand_loop<5>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      case 6: expand_loop<6>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      case 7: expand_loop<7>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
-      default: expand_loop<8>(p, tl, ops, codes, is_a, r, ntiles, P, lut); break;
+    switch (p.bits_a) {
+      case 1: expand_loop<1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      case 2: expand_loop<2>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      case 3: expand_loop<3>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      case 4: expand_loop<4>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      case 5: expand_loop<5>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      case 6: expand_loop<6>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      case 7: expand_loop<7>(p, tl, ops, codes, r, ntiles, P, lut); break;
+      default: expand_loop<8>(p, tl, ops, codes, r, ntiles, P, lut); break;
     }
-    if (tl->abort && e == 0) atomicOr(p.err, 8u);
+    if (tl->abort && r == 0) atomicOr(p.err, 8u);
   }
 
   tc_fence_before();
@@ -438,6 +443,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Weight codes [N, K*b/8] -> fp16 levels (x sqrt(K)) [N, K], one 64-code slice
+// per thread: read 8b bytes, write 128 bytes (both contiguous across threads).
+template <int BITS>
+__global__ void __launch_bounds__(256) expand_weights_kernel(const uint8_t* codes, long long rows, int K,
+                                                            const uint16_t* lut_g, uint16_t* out) {
+  __shared__ uint16_t lut[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = (i < (1 << BITS)) ? lut_g[i] : 0;
+  __syncthreads();
+  const Planes4 P = make_planes4(lut);
+  const int slices = K / kBK;
+  const long long items = rows * slices;
+  for (long long it = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; it < items;
+       it += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint2* src = reinterpret_cast<const uint2*>(codes + it * (8 * BITS));
+    uint32_t w[slice_words<BITS>()];
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) {
+      const uint2 v = __ldcs(src + i);
+      w[2 * i] = v.x;
+      w[2 * i + 1] = v.y;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + it * kBK);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t o[4];
+      if constexpr (BITS == 4) {
+        expand8_4bit(w[c], P, o);
+      } else {
+        constexpr uint32_t mask = (1u << BITS) - 1u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pair = 0u;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int i = 8 * c + 2 * j + e;
+            const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
+            uint32_t code = w[wi] >> sh;
+            if (sh + BITS > 32) code |= w[wi + 1] << (32 - sh);
+            pair |= static_cast<uint32_t>(lut[code & mask]) << (16 * e);
+          }
+          o[j] = pair;
+        }
+      }
+      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
@@ -479,7 +532,7 @@ uint32_t geo_span(const CodeGeo& g) {
   return g.slice_bytes ? 2 * g.slice_bytes : ((g.bytes + 1023u) & ~1023u);
 }
 
-int encode_map(CUtensorMap* map, const uint8_t* base, int rows, int bits, int K, const CodeGeo& g) {
+int encode_codes_map(CUtensorMap* map, const uint8_t* base, int rows, int bits, int K, const CodeGeo& g) {
   auto fn = encode_fn();
   if (!fn) return RBQ_ECUDA;
   const cuuint64_t row_bytes = static_cast<cuuint64_t>(K) * bits / 8;
@@ -496,29 +549,88 @@ int encode_map(CUtensorMap* map, const uint8_t* base, int rows, int bits, int K,
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
 }
 
+// fp16 [rows, K] K-major, 256 x 64 tiles, 128B swizzle: the canonical K-major
+// operand layout of the tensor core.
+int encode_f16_map(CUtensorMap* map, const uint16_t* base, int rows, int K) {
+  auto fn = encode_fn();
+  if (!fn) return RBQ_ECUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBN)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
+}
+
+template <int BITS>
+int launch_expand(const uint8_t* codes, int rows, int K, const uint16_t* lut, uint16_t* out, cudaStream_t st,
+                  int sms) {
+  const long long items = static_cast<long long>(rows) * (K / kBK);
+  long long blocks = (items + 255) / 256;
+  if (blocks > 8LL * sms) blocks = 8LL * sms;
+  expand_weights_kernel<BITS><<<static_cast<int>(blocks), 256, 0, st>>>(codes, rows, K, lut, out);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+}
+
+int expand_weights(const uint8_t* codes, int bits, int rows, int K, const uint16_t* lut, uint16_t* out,
+                   cudaStream_t st, int sms) {
+  switch (bits) {
+    case 1: return launch_expand<1>(codes, rows, K, lut, out, st, sms);
+    case 2: return launch_expand<2>(codes, rows, K, lut, out, st, sms);
+    case 3: return launch_expand<3>(codes, rows, K, lut, out, st, sms);
+    case 4: return launch_expand<4>(codes, rows, K, lut, out, st, sms);
+    case 5: return launch_expand<5>(codes, rows, K, lut, out, st, sms);
+    case 6: return launch_expand<6>(codes, rows, K, lut, out, st, sms);
+    case 7: return launch_expand<7>(codes, rows, K, lut, out, st, sms);
+    default: return launch_expand<8>(codes, rows, K, lut, out, st, sms);
+  }
+}
+
+// A memory pool per device for the stream-ordered weight workspace; it keeps
+// freed blocks cached so repeated calls do not go back to the driver.
+cudaMemPool_t workspace_pool(int dev) {
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
 }  // namespace qfast
 
 bool qlinear_fast_eligible(int M, int N, int K, int bits_a, int bits_w) {
+  (void)bits_w;
   if (M < 1 || N < 1 || (N % 8) != 0 || K < 128 || (K % 128) != 0) return false;
-  // TMA needs 16-byte row strides for both code tensors
-  return (static_cast<long long>(K) * bits_a / 8) % 16 == 0 && (static_cast<long long>(K) * bits_w / 8) % 16 == 0;
+  // TMA needs 16-byte row strides for the activation codes
+  return (static_cast<long long>(K) * bits_a / 8) % 16 == 0;
 }
 
-int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
-                        const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
-                        const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st) {
+// The GEMM on already-expanded fp16 weights `wf16` [N, K].
+int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const uint16_t* wf16,
+                      const uint16_t* rnorm, int M, int N, int K, uint16_t* Y, const CodebookDevice* ca,
+                      unsigned int* err, cudaStream_t st, int sms) {
   using namespace qfast;
   Params p{};
   p.M = M;
   p.N = N;
   p.K = K;
   p.bits_a = bits_a;
-  p.bits_b = bits_w;
   p.ga = make_geo(kBM, bits_a, 0);
-  p.gb = make_geo(kBN, bits_w, geo_span(p.ga));
-  p.cstage_bytes = geo_span(p.ga) + geo_span(p.gb);
+  p.cstage_bytes = geo_span(p.ga);
   const size_t tail = sizeof(Tail) + 64;
-  // as many operand stages (2..4) and code stages (2..4) as shared memory allows
   int F = kMaxF, C = 2;
   while (F > 2 && 1024 + F * kOpStage + C * p.cstage_bytes + tail > kSmemLimit) --F;
   while (C < kMaxC && 1024 + F * kOpStage + (C + 1) * p.cstage_bytes + tail <= kSmemLimit) ++C;
@@ -527,27 +639,43 @@ int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, cons
   p.F = F;
   p.C = C;
   p.lut_a = ca->levels_f16;
-  p.lut_b = cw->levels_f16;
   p.s = s;
   p.rnorm = rnorm;
   p.inv_k = ca->inv_d;
   p.Y = Y;
   p.err = err;
   CUtensorMap mA, mB;
-  int rc = encode_map(&mA, a_codes, M, bits_a, K, p.ga);
+  int rc = encode_codes_map(&mA, a_codes, M, bits_a, K, p.ga);
   if (rc != RBQ_OK) return rc;
-  if ((rc = encode_map(&mB, w_codes, N, bits_w, K, p.gb)) != RBQ_OK) return rc;
+  if ((rc = encode_f16_map(&mB, wf16, N, K)) != RBQ_OK) return rc;
   auto kern = qlinear_fast_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
   const int grid = ntiles < sms ? ntiles : sms;
   kern<<<grid, kThreads, smem, st>>>(mA, mB, p);
   e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+}
+
+int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
+                        const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
+                        const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaMemPool_t pool = qfast::workspace_pool(dev);
+  if (!pool) return RBQ_ECUDA;
+  void* ws = nullptr;
+  e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K * 2, pool, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint16_t* wf16 = static_cast<uint16_t*>(ws);
+  int rc = qfast::expand_weights(w_codes, bits_w, N, K, cw->levels_f16, wf16, st, sms);
+  if (rc == RBQ_OK) rc = qlinear_fast_gemm(a_codes, s, bits_a, wf16, rnorm, M, N, K, Y, ca, err, st, sms);
+  e = cudaFreeAsync(ws, st);
+  if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
+  return rc;
 }
 
 }  // namespace rbq

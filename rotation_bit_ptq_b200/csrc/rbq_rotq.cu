@@ -23,6 +23,9 @@ namespace {
 
 enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
 
+// Widths up to this use the fast kernel's unclamped [-1, 1] code grid.
+constexpr int kFullGridBits = 6;
+
 struct RotqParams {
   const void* X;
   long long T;
@@ -238,6 +241,17 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// 0xFFFFFFFF if a >= b else 0 (IEEE compare: -0 >= -0, NaN never)
+__device__ __forceinline__ uint32_t set_ge(float a, float b) {
+  uint32_t d;
+  asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(d) : "f"(a), "f"(b));
+  return d;
+}
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float d;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -266,8 +280,10 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) { return __ldcs(p); 
 
 template <int G>
 struct Layout {
-  // bytes: stage[2] (G rows of 2d+16) | off (4d) | mask (2d) | red (4*G*32) | grid
-  static __host__ __device__ size_t row_pitch(int d) { return 2 * static_cast<size_t>(d) + 16; }
+  // bytes: stage[2] (G rows of 2d+32) | off (4d) | mask (2d) | red (4*G*32) | grid
+  // (the 32-byte pad puts token g's row 8g banks over, so the G threads of an
+  // output block read different banks)
+  static __host__ __device__ size_t row_pitch(int d) { return 2 * static_cast<size_t>(d) + 32; }
   static __host__ __device__ size_t stage_bytes(int d) { return G * row_pitch(d); }
   static __host__ __device__ size_t off_at(int d) { return 2 * stage_bytes(d); }
   static __host__ __device__ size_t mask_at(int d) { return off_at(d) + 4 * static_cast<size_t>(d); }
@@ -429,8 +445,59 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
 
     const long long t = gi * G + g;
     if (active && t < p.T) {
-      if constexpr (kLloyd) {
-        // z here is 8x the rotated value (H unnormalised): v = z / (||z|| + 8 eps)
+      if constexpr (kLloyd && BITS <= kFullGridBits) {
+        // z here is 8x the rotated value (H unnormalised): v = z / (||z|| + 8 eps).
+        // Grid over v in [-1, 1]: n = round((v + 1)/2 * NC) needs no clamp once
+        // z is finite, which holds for every coordinate when ||z|| is finite.
+        const float nrm = sqrtf(tot);
+        if (!(nrm < INFINITY)) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) P[j] = 0ull;
+        }
+        const float inv = 1.0f / (nrm + 8e-12f);
+        const float kq = inv * (0.5f * p.grid_cells);
+        const float cq = 0.5f * p.grid_cells + 8388608.0f;   // + 2^23: round(.) lands in the low bits
+        const unsigned long long kq2 = pk(kq, kq), cq2 = pk(cq, cq), inv2 = pk(inv, inv);
+        const uint32_t gbase = grid_addr - 0x4B000000u * 8u;
+        uint32_t w[2 * BITS];
+#pragma unroll
+        for (int i = 0; i < 2 * BITS; ++i) w[i] = 0u;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float q0, q1, v0, v1;
+          upk(fma2(P[j], kq2, cq2), q0, q1);
+          upk(mul2(P[j], inv2), v0, v1);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int r = 2 * j + e;
+            const float2 ent = lds_f2(gbase + __float_as_uint(e ? q1 : q0) * 8u);
+            const uint32_t code = static_cast<uint32_t>(__float_as_int(ent.y)) - set_ge(e ? v1 : v0, ent.x);
+            const int bit = r * BITS, wi = bit >> 5, sh = bit & 31;
+            if constexpr ((32 % BITS) == 0) {
+              w[wi] += code << sh;                 // disjoint fields: add = or
+            } else {
+              w[wi] |= code << sh;
+              if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
+            }
+          }
+        }
+        unsigned char* dst = static_cast<unsigned char*>(p.out) + t * (static_cast<long long>(d) * BITS / 8) +
+                             static_cast<long long>(b) * 8 * BITS;
+        if constexpr ((BITS % 2) == 0) {
+#pragma unroll
+          for (int i = 0; i < BITS / 2; ++i)
+            __stcs(reinterpret_cast<uint4*>(dst) + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < BITS; ++i) __stcs(reinterpret_cast<uint2*>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
+        }
+        if (b == 0) {
+          const float sn = nrm * 0.125f;
+          if (MODE == kAct) static_cast<float*>(p.aux)[t] = sn;
+          else static_cast<__nv_bfloat16*>(p.aux)[t] = __float2bfloat16_rn(sn);
+        }
+      } else if constexpr (kLloyd) {
+        // Clamped grid (wide codebooks): u = sat(v/(2R) + 1/2), n = round(u NC).
         const float nrm = sqrtf(tot);
         const float inv = 1.0f / (nrm + 8e-12f);
         const float A = inv * p.grid_scale;
@@ -636,10 +703,18 @@ int run_fast(const rbq_rpbh* r, int mode, int bits, long long rows, const void* 
   if (mode == kAct || mode == kWeightLM) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
-    p.grid = cb->grid;
-    p.grid_n = cb->grid_cells + 1;
-    p.grid_cells = static_cast<float>(cb->grid_cells);
-    p.grid_scale = cb->grid_scale;
+    if (bits <= kFullGridBits) {
+      if (!cb->grid_full) return RBQ_ECONVERGE;   // caller falls back to the general kernel
+      p.grid = cb->grid_full;
+      p.grid_n = cb->grid_full_cells + 1;
+      p.grid_cells = static_cast<float>(cb->grid_full_cells);
+      p.grid_scale = 0.5f;
+    } else {
+      p.grid = cb->grid;
+      p.grid_n = cb->grid_cells + 1;
+      p.grid_cells = static_cast<float>(cb->grid_cells);
+      p.grid_scale = cb->grid_scale;
+    }
   }
   switch (mode) {
     case kAct: return launch_fast<kAct>(bits, p, st);
@@ -694,8 +769,10 @@ extern "C" int rotate_quantize_act(const rbq_rpbh* r, const void* X, int dtype, 
   if (!aligned(X, 16) || !aligned(codes_out, 16) || (norms_out && !aligned(norms_out, 4)))
     return RBQ_EALIGN;
   const int mode = rot ? kRotate : kAct;
-  if (fast_eligible(dtype, r->d))
-    return run_fast(r, mode, bits, T, X, codes_out, norms_out, static_cast<cudaStream_t>(stream));
+  if (fast_eligible(dtype, r->d)) {
+    const int frc = run_fast(r, mode, bits, T, X, codes_out, norms_out, static_cast<cudaStream_t>(stream));
+    if (frc != RBQ_ECONVERGE) return frc;
+  }
   RotqParams p;
   int rc = prepare(r, mode, bits, T, X, codes_out, norms_out, &p);
   if (rc != RBQ_OK) return rc;
@@ -718,8 +795,10 @@ extern "C" int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int
   if (!aligned(W, 16) || !aligned(codes_or_q, 16) || !aligned(rownorm_or_scale, 4))
     return RBQ_EALIGN;
   const int m = (mode == RBQ_LLOYDMAX) ? kWeightLM : kInt8;
-  if (fast_eligible(dtype, r->d))
-    return run_fast(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, static_cast<cudaStream_t>(stream));
+  if (fast_eligible(dtype, r->d)) {
+    const int frc = run_fast(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, static_cast<cudaStream_t>(stream));
+    if (frc != RBQ_ECONVERGE) return frc;
+  }
   RotqParams p;
   int rc = prepare(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, &p);
   if (rc != RBQ_OK) return rc;
