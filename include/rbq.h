@@ -53,6 +53,7 @@ extern "C" {
 #define RBQ_ENOMEM     (-4)  /* host allocation failed                          */
 #define RBQ_ECONVERGE  (-5)  /* Lloyd-Max solver did not converge               */
 #define RBQ_EDEVICE    (-6)  /* kernel reported an internal error (see below)   */
+#define RBQ_ESCRATCH   (-7)  /* problem larger than a fixed scratch area        */
 
 /* ---- element types and modes --------------------------------------------- */
 #define RBQ_F32    0
@@ -183,6 +184,41 @@ int qlinear(const uint8_t* a_codes, const float* s, int bits_a,
  */
 int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float* scale,
                  int M, int N, int K, uint16_t* Y, void* stream);
+
+/*
+ * qlinear_noalloc -- the same result as qlinear, for callers that cannot
+ * allocate device memory.  (The pages have no counterpart: this is a
+ * deployment variant of the library, not a step of the method.)
+ *
+ * qlinear expands the weight codes into an fp16 workspace of N*K*2 bytes taken
+ * from a stream-ordered memory pool on every call.  Callers that own all device
+ * memory through their own allocator, forbid allocation on their inference
+ * thread, or run inside a process whose allocator is not CUDA's cannot accept
+ * that.  This entry point allocates nothing: its workspace, its two level
+ * tables and a fallback error word live in one fixed __device__ array of
+ * 32 MiB + 1280 bytes inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   Arguments as qlinear, plus
+ *   err   device uint32 the kernels OR a non-zero value into when a bounded
+ *         pipeline wait runs out (Y is then invalid); caller-owned, the caller
+ *         clears it; NULL = record in the array's own word (not reported).
+ * Limits: N*K <= 16,777,216 (else RBQ_ESCRATCH, nothing launched); K a
+ * multiple of 128, N a multiple of 8, K*bits_a/8 a multiple of 16 (else
+ * RBQ_EINVAL).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call uses the same array and the array
+ * keeps the last call's contents, so calls whose work overlaps on the GPU (on
+ * different streams, or from several host threads) race and corrupt each
+ * other's results; serialise them on one stream.  Nothing in the array needs
+ * to start at zero: each call rewrites the tables and every workspace element
+ * it reads.
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ESCRATCH, RBQ_ECONVERGE, RBQ_ECUDA.
+ */
+int qlinear_noalloc(const uint8_t* a_codes, const float* s, int bits_a,
+                    const uint8_t* w_codes, const uint16_t* rnorm, int bits_w,
+                    int M, int N, int K, uint16_t* Y, unsigned int* err,
+                    void* stream);
 
 /* ---- diagnostics ----------------------------------------------------------- */
 

@@ -21,6 +21,7 @@ RBQ_F32, RBQ_BF16 = 0, 1
 RBQ_LLOYDMAX, RBQ_INT8_SYM = 0, 1
 RBQ_ROTATE_ONLY = 16
 RBQ_OK, RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA, RBQ_ENOMEM, RBQ_ECONVERGE, RBQ_EDEVICE = 0, -1, -2, -3, -4, -5, -6
+RBQ_ESCRATCH = -7
 
 # name -> (restype, argtypes); mirrors include/rbq.h
 _P, _I, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
@@ -34,6 +35,7 @@ SIGNATURES = {
     "quantize_weights": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "qlinear": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
     "qlinear_int8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "qlinear_noalloc": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
     "rbq_code_grid": (_I, [_I, _I, _I, _P, _P, _P, _P]),
@@ -230,6 +232,28 @@ def qlinear(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, stream=None
     _need_cuda(out, "out", torch.bfloat16)
     _check(lib().qlinear(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M, N,
                          int(K), _ptr(out), _stream(stream)), "qlinear")
+    return out
+
+
+def qlinear_noalloc(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out, err=None, stream=None):
+    """qlinear without any device allocation inside the library (its workspace
+    is a fixed array in the library, N*K <= 2**24).  `out` (bfloat16 [M, N])
+    and the optional error word `err` (int32 [1], OR-ed non-zero on a pipeline
+    time-out) are the caller's.  Calls that overlap on the GPU race."""
+    import torch
+    for t, n, dt in ((a_codes, "a_codes", torch.uint8), (s, "s", torch.float32),
+                     (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16),
+                     (out, "out", torch.bfloat16)):
+        _need_cuda(t, n, dt)
+    if err is not None:
+        _need_cuda(err, "err", torch.int32)
+    M, N = a_codes.shape[0], w_codes.shape[0]
+    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
+        raise ValueError("code row widths do not match K and the bit widths")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    _check(lib().qlinear_noalloc(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M,
+                                 N, int(K), _ptr(out), _ptr(err), _stream(stream)), "qlinear_noalloc")
     return out
 
 

@@ -467,6 +467,7 @@ extern "C" const char* rbq_error_string(int code) {
     case RBQ_ENOMEM: return "out of host memory";
     case RBQ_ECONVERGE: return "Lloyd-Max solver did not converge";
     case RBQ_EDEVICE: return "kernel reported an internal error (bounded wait expired)";
+    case RBQ_ESCRATCH: return "problem exceeds the fixed scratch area (qlinear_noalloc: N*K <= 16777216)";
     default: return "unknown error code";
   }
 }
