@@ -333,6 +333,28 @@ int rpbh_device(const rbq_rpbh* r, const RpbhDevice** out) {
   return RBQ_OK;
 }
 
+int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out) {
+  const RpbhDevice* rd = nullptr;
+  int rc = rpbh_device(r, &rd);
+  if (rc != RBQ_OK) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto* D = const_cast<RpbhDevice*>(rd);
+  if (!D->pair_tab) {
+    const int d = r->d;
+    std::vector<uint32_t> tab(2 * static_cast<size_t>(d));
+    for (int k = 0; k < d; ++k) {
+      const uint32_t slot = pair_tab_slot(k / kH, k % kH);
+      tab[slot] = 2u * static_cast<uint32_t>(r->perm[k]);
+      tab[d + slot] = r->sign[k] < 0 ? 0x80000000u : 0u;
+    }
+    uint32_t* dev = nullptr;
+    if ((rc = upload(tab.data(), tab.size(), &dev)) != RBQ_OK) return rc;
+    D->pair_tab = dev;
+  }
+  *out = D->pair_tab;
+  return RBQ_OK;
+}
+
 int codebook_device(int d, int bits, const CodebookDevice** out) {
   int dev;
   int rc = current_device(&dev);
@@ -435,6 +457,7 @@ extern "C" void rpbh_free(rbq_rpbh* r) {
     if (!D.ready) continue;
     cudaFree(D.perm);
     cudaFree(D.sign);
+    cudaFree(D.pair_tab);
   }
   delete r;
 }

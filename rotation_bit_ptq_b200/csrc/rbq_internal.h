@@ -21,7 +21,18 @@ struct RpbhDevice {
   bool ready = false;
   int32_t* perm = nullptr;        // pi(k), destination order
   float* sign = nullptr;          // D_k as +-1.0f, destination order
+  // Gather tables of the token-pair kernel (built on first use): d byte
+  // offsets 2 pi(k), then d sign words (0 or 0x80000000), both at
+  // pair_tab_slot(k / 64, k % 64).
+  uint32_t* pair_tab = nullptr;
 };
+
+// Slot of output position (block b, index i) in the token-pair kernel's
+// tables: the 16-byte chunk index inside the block is XORed with b & 7 so that
+// the four blocks a warp reads hit four different bank quads.
+__host__ __device__ inline uint32_t pair_tab_slot(int b, int i) {
+  return 64u * b + 4u * ((static_cast<uint32_t>(i) >> 2) ^ (static_cast<uint32_t>(b) & 7u)) + (i & 3);
+}
 
 }  // namespace rbq
 
@@ -57,6 +68,9 @@ constexpr int kMaxFullGridCells = 5000;
 
 // Returns the device tables of `r` on the current device, uploading on first use.
 int rpbh_device(const rbq_rpbh* r, const RpbhDevice** out);
+// Returns the token-pair kernel's gather tables of `r` on the current device
+// (2 d words, see RpbhDevice::pair_tab), building them on first use.
+int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out);
 // Returns the codebook of (d, bits) on the current device, computing and
 // uploading it on first use.
 int codebook_device(int d, int bits, const CodebookDevice** out);

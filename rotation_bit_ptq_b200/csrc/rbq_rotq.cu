@@ -755,6 +755,13 @@ int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X
 }
 
 }  // namespace
+
+// The token-pair kernel (rbq_rotq_pair.cu): BF16 rows, d = 1024..3072 in
+// steps of 256.  RBQ_ECONVERGE from the launch means "not this kernel".
+bool rotq_pair_eligible(int dtype, int d);
+int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
+                     cudaStream_t st);
+
 }  // namespace rbq
 
 using namespace rbq;
@@ -769,6 +776,11 @@ extern "C" int rotate_quantize_act(const rbq_rpbh* r, const void* X, int dtype, 
   if (!aligned(X, 16) || !aligned(codes_out, 16) || (norms_out && !aligned(norms_out, 4)))
     return RBQ_EALIGN;
   const int mode = rot ? kRotate : kAct;
+  if (rotq_pair_eligible(dtype, r->d)) {
+    const int prc = rotq_pair_launch(r, mode, rot ? 8 : bits, T, X, codes_out, norms_out,
+                                     static_cast<cudaStream_t>(stream));
+    if (prc != RBQ_ECONVERGE) return prc;
+  }
   if (fast_eligible(dtype, r->d)) {
     const int frc = run_fast(r, mode, bits, T, X, codes_out, norms_out, static_cast<cudaStream_t>(stream));
     if (frc != RBQ_ECONVERGE) return frc;
@@ -795,6 +807,11 @@ extern "C" int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int
   if (!aligned(W, 16) || !aligned(codes_or_q, 16) || !aligned(rownorm_or_scale, 4))
     return RBQ_EALIGN;
   const int m = (mode == RBQ_LLOYDMAX) ? kWeightLM : kInt8;
+  if (rotq_pair_eligible(dtype, r->d)) {
+    const int prc = rotq_pair_launch(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale,
+                                     static_cast<cudaStream_t>(stream));
+    if (prc != RBQ_ECONVERGE) return prc;
+  }
   if (fast_eligible(dtype, r->d)) {
     const int frc = run_fast(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, static_cast<cudaStream_t>(stream));
     if (frc != RBQ_ECONVERGE) return frc;

@@ -1,0 +1,744 @@
+// Rotate-then-quantise for BF16 rows of width 1024..3072 (d a multiple of
+// 256): the token-pair kernel.
+//
+//   OrbitQuant (hotelren.com/news/3376620) §2.2 / §2.1: x' = Pi_d x, s = ||x'||,
+//   codes of x'/(s + eps) in the Lloyd-Max codebook of N(0, 1/d); weights the
+//   same with BF16 row norms.  INT8-convrot (cloud.baidu.com/article/9430339)
+//   §4: rotate, scale = max|w'|/127, round.  Rotate-only: x' in BF16.
+//   Pi_d = blkdiag(H_64 D_1, ..., H_64 D_{d/64}) · P_pi (OrbitQuant §2.3).
+//
+// Work unit: a tile of 16 token rows.  Thread (p, b) owns output block b of
+// the token pair (p, p+8), p = 0..7, holding the pair's values as packed
+// fp32x2 registers, so every butterfly stage is one packed add/sub per pair.
+// It gathers and transforms one 32-position half-block at a time (strides
+// 1..16), parks both halves in its own lane of tensor memory, and runs the
+// last stage (stride 32) inside the encoding loop as it reads them back; the
+// smaller live register set leaves room for many loads in flight.  A warp covers 8 pairs x 4 blocks; the 8 lanes that share
+// a block read the same source position of 8 different rows, which a 16-byte
+// row padding puts in 8 different banks.
+//
+// Data movement: one producer warp streams whole rows with bulk asynchronous
+// copies (TMA, no tensor map needed for contiguous rows) into a ring of tile
+// slots, each completion counted on the slot's mbarrier.  Consumers release a
+// slot as soon as they have gathered from it, so the next tile streams in
+// while the current one is transformed and encoded.
+//
+// Norm: the rotation is orthogonal, so ||Pi x|| = ||x||; every thread sums the
+// squares of the 64 inputs it gathered (each input lands in exactly one
+// block), the partial sums meet in shared memory, and the wait for them is
+// split from the arrival so the butterfly overlaps it.  (INT8 needs max|w'|,
+// which exists only after the butterfly, so there the arrival follows it.)
+//
+// Codes: z (8x the rotated value, H unnormalised) -> v = z / (||z|| + 8 eps).
+// A uniform grid over v in [-1, 1] (|v| <= 1 for a unit vector) gives a cell
+// n = round((v + 1)/2 * cells) whose entry holds the count of boundaries below
+// the cell and the boundary inside it (or +inf): code = base + (v >= thr).
+// Wide codebooks whose full-range grid does not fit use a grid over [-R, R]
+// with a saturating clamp.
+
+#include <cuda_bf16.h>
+
+#include "rbq_internal.h"
+#include "rbq_sm100.cuh"
+
+namespace rbq {
+namespace pairk {
+
+using namespace sm100;
+
+enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
+
+constexpr int kRows = 16;            // tokens per tile
+constexpr int kMaxWarps = 12;        // consumer warps (d <= 3072)
+constexpr int kGuard = 2;            // grid entries past each end
+constexpr size_t kSmemLimit = 227 * 1024;
+
+struct Params {
+  const __nv_bfloat16* X;
+  long long T;
+  int d, nblk, nwarps;               // consumer warps = nblk / 4
+  int ntiles;                        // ceil(T / 16)
+  int NS;                            // ring slots
+  uint32_t pitch;                    // bytes per staged row (2d + 16)
+  const uint32_t* tab;               // 2 d words: offsets, then sign words (pair_tab_slot order)
+  const float2* grid;                // Lloyd-Max modes: cells + 1 entries
+  int grid_n;
+  float grid_cells, grid_scale;      // full grid: scale unused
+  void* out;
+  void* aux;
+  unsigned int* err;
+};
+
+// Shared-memory layout (bytes from the 128-aligned base).
+struct Layout {
+  uint32_t ring, off, sgn, grid, part, bars, total;
+};
+
+__host__ __device__ inline Layout layout(int d, int NS, int grid_n) {
+  Layout L{};
+  const uint32_t pitch = 2u * d + 16u;
+  L.ring = 0;
+  L.off = L.ring + NS * kRows * pitch;
+  L.sgn = L.off + 4u * d;
+  L.grid = L.sgn + 4u * d;
+  L.part = (L.grid + 8u * (grid_n + 2 * kGuard) + 15u) & ~15u;
+  L.bars = L.part + 4u * (2 * NS) * kRows * kMaxWarps;   // [2NS][16 tokens][12 warps]
+  L.bars = (L.bars + 7u) & ~7u;
+  // full[NS], red[2NS], tab | cnt[NS], issued[NS], TMEM base
+  L.total = L.bars + 8u * (NS + 2 * NS + 1) + 8u * NS + 8u;
+  return L;
+}
+
+__device__ __forceinline__ unsigned long long pk(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk(unsigned long long r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// 0xFFFFFFFF if a >= b else 0 (IEEE: -0 >= -0; NaN never)
+__device__ __forceinline__ uint32_t set_ge(float a, float b) {
+  uint32_t d;
+  asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// Whole contiguous row, global -> shared, completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+// bf16 bits (low 16 of u) -> fp32 with the sign word S (0 or 0x80000000)
+// folded in: (u << 16) + S flips the sign bit exactly when S is set.
+__device__ __forceinline__ float bf16_signed(uint32_t u, uint32_t S) { return __uint_as_float(u * 65536u + S); }
+
+
+__device__ __forceinline__ unsigned long long pk_u(uint32_t a, uint32_t b) {
+  return pk(__uint_as_float(a), __uint_as_float(b));
+}
+__device__ __forceinline__ void upk_u(unsigned long long r, uint32_t& a, uint32_t& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(r));
+}
+__device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Code of each half of a packed pair z (two tokens) from the shared-memory
+// grid.  Full-range grid: n = round((v + 1)/2 * cells) through the +2^23
+// trick, code = base + (v >= thr).  Clamped grid over [-R, R]: u = sat(v/(2R)
+// + 1/2), n = round(u * cells), code = base + 1 + sign(z * inv - thr).
+template <bool FULL>
+struct Enc;
+
+template <>
+struct Enc<true> {
+  unsigned long long kq2, cq2, inv2;
+  uint32_t gbase;
+  __device__ __forceinline__ Enc(float inv0, float inv1, float cells, float, uint32_t gb) : gbase(gb) {
+    const float hc = 0.5f * cells;
+    kq2 = pk(inv0 * hc, inv1 * hc);
+    cq2 = pk(hc + 8388608.0f, hc + 8388608.0f);
+    inv2 = pk(inv0, inv1);
+  }
+  __device__ __forceinline__ void codes(unsigned long long z, uint32_t& c0, uint32_t& c1) const {
+    float q0, q1, v0, v1;
+    upk(fma2(z, kq2, cq2), q0, q1);
+    upk(mul2(z, inv2), v0, v1);
+    const float2 e0 = lds_f2(gbase + __float_as_uint(q0) * 8u);
+    const float2 e1 = lds_f2(gbase + __float_as_uint(q1) * 8u);
+    c0 = __float_as_uint(e0.y) - set_ge(v0, e0.x);
+    c1 = __float_as_uint(e1.y) - set_ge(v1, e1.x);
+  }
+};
+
+template <>
+struct Enc<false> {
+  float A0, A1, inv0, inv1, cells;
+  uint32_t gbase;
+  __device__ __forceinline__ Enc(float i0, float i1, float nc, float scale, uint32_t gb)
+      : A0(i0 * scale), A1(i1 * scale), inv0(i0), inv1(i1), cells(nc), gbase(gb) {}
+  __device__ __forceinline__ void codes(unsigned long long z, uint32_t& c0, uint32_t& c1) const {
+    float z0, z1;
+    upk(z, z0, z1);
+    const float qf0 = fmaf(fma_sat(z0, A0, 0.5f), cells, 8388608.0f);
+    const float qf1 = fmaf(fma_sat(z1, A1, 0.5f), cells, 8388608.0f);
+    const float2 e0 = lds_f2(gbase + __float_as_uint(qf0) * 8u);
+    const float2 e1 = lds_f2(gbase + __float_as_uint(qf1) * 8u);
+    const int below0 = __float_as_int(fmaf(z0, inv0, -e0.x)) >> 31;
+    const int below1 = __float_as_int(fmaf(z1, inv1, -e1.x)) >> 31;
+    c0 = static_cast<uint32_t>(__float_as_int(e0.y) + 1 + below0);
+    c1 = static_cast<uint32_t>(__float_as_int(e1.y) + 1 + below1);
+  }
+};
+
+// Packs `code` (already < 2^BITS) into bit i*BITS of the word array w.
+template <int BITS>
+__device__ __forceinline__ void put_code(uint32_t* w, int i, uint32_t code) {
+  const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
+  if constexpr ((32 % BITS) == 0) {
+    w[wi] += code << sh;                     // disjoint fields: add = or
+  } else {
+    w[wi] |= code << sh;
+    if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void store_codes(unsigned char* dst, const uint32_t* w) {
+  if constexpr ((BITS % 2) == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS / 2; ++i)
+      __stcs(reinterpret_cast<uint4*>(dst) + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) __stcs(reinterpret_cast<uint2*>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
+  }
+}
+
+
+// Codes of one block for both tokens: the last butterfly stage (stride 32)
+// runs here, on half-blocks read back from tensor memory 16 positions at a
+// time.  SAN: the token(s) flagged bad are encoded as the zero vector.
+template <int BITS, bool FULL, bool SAN>
+__device__ __forceinline__ void encode_block(const Enc<FULL>& enc, uint32_t tA, uint32_t tB, bool bad0, bool bad1,
+                                             uint32_t* w0, uint32_t* w1) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t va[32], vb[32];
+    __syncwarp();
+    tmem_ld32(tA + 32u * c, va);
+    tmem_ld32(tB + 32u * c, vb);
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const unsigned long long a = pk_u(va[2 * k], va[2 * k + 1]), bb = pk_u(vb[2 * k], vb[2 * k + 1]);
+      unsigned long long z = add2(a, bb), y = sub2(a, bb);
+      if constexpr (SAN) {
+        float z0, z1, y0, y1;
+        upk(z, z0, z1);
+        upk(y, y0, y1);
+        z = pk(bad0 ? 0.f : z0, bad1 ? 0.f : z1);
+        y = pk(bad0 ? 0.f : y0, bad1 ? 0.f : y1);
+      }
+      uint32_t c0, c1, d0, d1;
+      enc.codes(z, c0, c1);
+      enc.codes(y, d0, d1);
+      const int i = 16 * c + k;
+      put_code<BITS>(w0, i, c0);
+      put_code<BITS>(w1, i, c1);
+      put_code<BITS>(w0, i + 32, d0);
+      put_code<BITS>(w1, i + 32, d1);
+    }
+  }
+}
+
+template <int MODE, int BITS, bool FULL>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 127u) & ~127u;
+  unsigned char* sm = smem_raw + (sbase - sraw);
+  const Layout L = layout(p.d, p.NS, p.grid_n);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint64_t* red = full + p.NS;
+  uint64_t* tabbar = red + 2 * p.NS;
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(tabbar + 1);        // readers done, per slot
+  uint32_t* issued = cnt + p.NS;                                   // tiles issued, per slot
+  uint32_t* tmem_slot = issued + p.NS;                             // TMEM base address
+  constexpr bool kLloyd = (MODE == kAct || MODE == kWeightLM);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nthreads_c = p.nwarps * 32;
+  const int NS = p.NS;
+
+  const uint32_t pitch = p.pitch;
+  const uint32_t slot_bytes = kRows * pitch;
+  const uint32_t ring = sbase + L.ring;
+
+  // Bulk-copies tile `tile` into slot `slot`; counted on full[slot].
+  auto issue = [&](int tile, int slot) {
+    const size_t row_bytes = 2 * static_cast<size_t>(p.d);
+    const long long r0 = static_cast<long long>(tile) * kRows;
+    const int rows = static_cast<int>(min(static_cast<long long>(kRows), p.T - r0));
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    ++issued[slot];
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(rows * row_bytes));
+    for (int r = 0; r < rows; ++r)
+      bulk_load(ring + slot * slot_bytes + r * pitch, p.X + (r0 + r) * p.d, static_cast<uint32_t>(row_bytes),
+                &full[slot]);
+  };
+
+  // ---- prologue: the first tiles and the gather tables start streaming at
+  //      once; the code grid and the partial sums are set up meanwhile ----
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      cnt[s] = 0u;
+      issued[s] = 0u;
+    }
+    for (int r = 0; r < 2 * NS; ++r) mbar_init(&red[r], nthreads_c);
+    mbar_init(tabbar, 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(tabbar, 8u * p.d);
+    bulk_load(sbase + L.off, p.tab, 8u * p.d, tabbar);
+    for (int s = 0; s < NS; ++s)
+      if (blockIdx.x + s * static_cast<int>(gridDim.x) < p.ntiles) issue(blockIdx.x + s * gridDim.x, s);
+  }
+  if (kLloyd) {
+    float2* g = reinterpret_cast<float2*>(sm + L.grid);
+    const int n = p.grid_n + 2 * kGuard;
+#pragma unroll 4
+    for (int i = tid; i < n; i += blockDim.x) {
+      const int src = min(max(i - kGuard, 0), p.grid_n - 1);
+      g[i] = p.grid[src];
+    }
+  }
+  {
+    float* part = reinterpret_cast<float*>(sm + L.part);
+    for (int i = tid; i < (2 * NS) * kRows * kMaxWarps; i += blockDim.x) part[i] = 0.f;
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (!mbar_wait(tabbar, 0)) atomicOr(p.err, 256u);
+
+  // ---------------- consumers ----------------
+  const int j = lane >> 3, pp = lane & 7;          // lane = 8 j + p
+  const int b = 4 * warp + j;                      // output block of this thread
+  const int bx = b & 7;
+  const uint32_t off_addr = sbase + L.off + 256u * b;
+  const uint32_t sgn_addr = sbase + L.sgn + 256u * b;
+  const uint32_t part_addr = sbase + L.part;
+  const uint32_t gbase = sbase + L.grid + 8u * kGuard - 0x4B000000u * 8u;
+  const uint32_t pitch8 = 8u * pitch;
+  // Tensor memory: each thread parks its pair's two half-blocks (2 x 64 words)
+  // in its own lane; warps w, w+4, w+8 share a lane quarter, 128 columns each.
+  const uint32_t tA = *tmem_slot + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 128u * (warp >> 2);
+  const uint32_t tB = tA + 64u;
+  int it = 0;
+  for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++it) {
+    const int s = it % NS, rb = it % (2 * NS);
+    // A timed-out wait ends the whole warp's loop together: the tensor-memory
+    // accesses below are warp-collective (.sync.aligned).
+    if (__any_sync(0xffffffffu, !mbar_wait(&full[s], (it / NS) & 1))) { atomicOr(p.err, 64u); break; }
+
+    // ---- gather x[pi(k)] with D_k folded in (tokens p, p+8), one half-block
+    //      at a time; butterfly strides 1..16 inside each half; park in TMEM ----
+    const uint32_t rowA = ring + s * slot_bytes + pp * pitch;
+    unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      unsigned long long R[32];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const uint32_t c = 16u * (static_cast<uint32_t>(8 * h + q4) ^ static_cast<uint32_t>(bx));
+        const uint4 o = lds128(off_addr + c);
+        const uint4 sg = lds128(sgn_addr + c);
+        const uint32_t oo[4] = {o.x, o.y, o.z, o.w};
+        const uint32_t ss[4] = {sg.x, sg.y, sg.z, sg.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t a = rowA + oo[e];
+          const float y0 = bf16_signed(lds_u16(a), ss[e]);
+          const float y1 = bf16_signed(lds_u16(a + pitch8), ss[e]);
+          R[4 * q4 + e] = pk(y0, y1);
+          acc[e] = fma2(R[4 * q4 + e], R[4 * q4 + e], acc[e]);
+        }
+      }
+      if (h == 1) {
+        // The last thread done with the slot's rows refills it with the tile
+        // NS steps ahead (release/acquire through the counter orders every
+        // read before the asynchronous overwrite).
+        uint32_t prev;
+        asm volatile("atom.release.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(prev) : "r"(smem_u32(&cnt[s]))
+                     : "memory");
+        if (prev == static_cast<uint32_t>(nthreads_c - 1)) {
+          asm volatile("fence.acq_rel.cta;" ::: "memory");
+          cnt[s] = 0u;
+          const int nxt = tile + NS * static_cast<int>(gridDim.x);
+          if (nxt < p.ntiles) issue(nxt, s);
+        }
+        if constexpr (MODE != kInt8) {
+          // ||x||^2 partials of both tokens (||Pi x|| = ||x||): 4 lanes share a pair
+          float a0, a1;
+          upk(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), a0, a1);
+          a0 += __shfl_xor_sync(0xffffffffu, a0, 8);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, 8);
+          a0 += __shfl_xor_sync(0xffffffffu, a0, 16);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, 16);
+          if (j == 0) {
+            sts_f32(part_addr + 4u * ((rb * kRows + pp) * kMaxWarps + warp), a0);
+            sts_f32(part_addr + 4u * ((rb * kRows + pp + 8) * kMaxWarps + warp), a1);
+          }
+          mbar_arrive(&red[rb]);
+        }
+      }
+#pragma unroll
+      for (int st = 1; st < 32; st <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if ((i & st) == 0) {
+            const unsigned long long a = R[i], c = R[i + st];
+            R[i] = add2(a, c);
+            R[i + st] = sub2(a, c);
+          }
+        }
+      }
+      uint32_t v0[32], v1[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        upk_u(R[i], v0[2 * i], v0[2 * i + 1]);
+        upk_u(R[16 + i], v1[2 * i], v1[2 * i + 1]);
+      }
+      __syncwarp();
+      tmem_st32((h ? tB : tA), v0);
+      tmem_st32((h ? tB : tA) + 32u, v1);
+    }
+    tmem_wait_st();
+
+    if constexpr (MODE == kInt8) {
+      // max |z| needs the last butterfly stage: z_i = A_i + B_i, z_{i+32} = A_i - B_i
+      float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t va[32], vb[32];
+        __syncwarp();
+        tmem_ld32(tA + 32u * c, va);
+        tmem_ld32(tB + 32u * c, vb);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const unsigned long long a = pk_u(va[2 * k], va[2 * k + 1]), bb = pk_u(vb[2 * k], vb[2 * k + 1]);
+          float z0, z1, y0, y1;
+          upk(add2(a, bb), z0, z1);
+          upk(sub2(a, bb), y0, y1);
+          m0 = fmaxf(m0, fmaxf(fabsf(z0), fabsf(y0)));
+          m1 = fmaxf(m1, fmaxf(fabsf(z1), fabsf(y1)));
+        }
+      }
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 8));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 8));
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 16));
+      if (j == 0) {
+        sts_f32(part_addr + 4u * ((rb * kRows + pp) * kMaxWarps + warp), m0);
+        sts_f32(part_addr + 4u * ((rb * kRows + pp + 8) * kMaxWarps + warp), m1);
+      }
+      mbar_arrive(&red[rb]);
+    }
+
+    // ---- per-token totals: fixed summation order, identical in every thread ----
+    if (__any_sync(0xffffffffu, !mbar_wait(&red[rb], (it / (2 * NS)) & 1))) { atomicOr(p.err, 64u); break; }
+    float tot[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t pa = part_addr + 4u * ((rb * kRows + pp + 8 * h) * kMaxWarps);
+      const uint4 q0 = lds128(pa), q1 = lds128(pa + 16), q2 = lds128(pa + 32);
+      const float v[12] = {__uint_as_float(q0.x), __uint_as_float(q0.y), __uint_as_float(q0.z),
+                           __uint_as_float(q0.w), __uint_as_float(q1.x), __uint_as_float(q1.y),
+                           __uint_as_float(q1.z), __uint_as_float(q1.w), __uint_as_float(q2.x),
+                           __uint_as_float(q2.y), __uint_as_float(q2.z), __uint_as_float(q2.w)};
+      if constexpr (MODE == kInt8) {
+        float m = v[0];
+#pragma unroll
+        for (int w = 1; w < 12; ++w) m = fmaxf(m, v[w]);
+        tot[h] = m;
+      } else {
+        tot[h] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7])) + ((v[8] + v[9]) + (v[10] + v[11]));
+      }
+    }
+
+    const long long t0 = static_cast<long long>(tile) * kRows + pp, t1 = t0 + 8;
+    const bool ok0 = t0 < p.T, ok1 = t1 < p.T;
+
+    if constexpr (kLloyd) {
+      const float s0 = sqrtf(tot[0]), s1 = sqrtf(tot[1]);      // ||x|| = ||Pi x||
+      // A non-finite row (or a padding row past T) is encoded as the zero
+      // vector, which also keeps every grid index inside the table.
+      const bool bad0 = !(tot[0] < INFINITY) || !ok0, bad1 = !(tot[1] < INFINITY) || !ok1;
+      // z is 8x the rotated value: v = z / (8 s + 8 eps)
+      const float inv0 = 1.0f / (8.0f * s0 + 8e-12f), inv1 = 1.0f / (8.0f * s1 + 8e-12f);
+      uint32_t w0[2 * BITS], w1[2 * BITS];
+#pragma unroll
+      for (int i = 0; i < 2 * BITS; ++i) w0[i] = w1[i] = 0u;
+      const Enc<FULL> enc(inv0, inv1, p.grid_cells, p.grid_scale, gbase);
+      // warp-uniform choice: encode_block reads tensor memory collectively
+      if (__any_sync(0xffffffffu, bad0 || bad1)) {
+        encode_block<BITS, FULL, true>(enc, tA, tB, bad0, bad1, w0, w1);
+      } else {
+        encode_block<BITS, FULL, false>(enc, tA, tB, false, false, w0, w1);
+      }
+      const long long cp = static_cast<long long>(p.d) * BITS / 8;
+      unsigned char* out = static_cast<unsigned char*>(p.out) + static_cast<long long>(b) * 8 * BITS;
+      if (ok0) store_codes<BITS>(out + t0 * cp, w0);
+      if (ok1) store_codes<BITS>(out + t1 * cp, w1);
+      if (b == 0) {
+        if (MODE == kAct) {
+          if (ok0) static_cast<float*>(p.aux)[t0] = s0;
+          if (ok1) static_cast<float*>(p.aux)[t1] = s1;
+        } else {
+          if (ok0) static_cast<__nv_bfloat16*>(p.aux)[t0] = __float2bfloat16_rn(s0);
+          if (ok1) static_cast<__nv_bfloat16*>(p.aux)[t1] = __float2bfloat16_rn(s1);
+        }
+      }
+    } else if constexpr (MODE == kInt8) {
+      // scale = max|w'| / 127 with w' = z / 8; q = clamp(round(w' / scale), +-127)
+      const float sc0 = (tot[0] * 0.125f) / 127.0f, sc1 = (tot[1] * 0.125f) / 127.0f;
+      const float r0 = (sc0 > 0.f) ? 1.0f / sc0 : 0.f, r1 = (sc1 > 0.f) ? 1.0f / sc1 : 0.f;
+      int8_t* out = static_cast<int8_t*>(p.out) + 64 * b;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t va[32], vb[32];
+        __syncwarp();
+        tmem_ld32(tA + 32u * c, va);
+        tmem_ld32(tB + 32u * c, vb);
+        tmem_wait_ld();
+        uint32_t qa0[4] = {0u, 0u, 0u, 0u}, qa1[4] = {0u, 0u, 0u, 0u};   // positions 16c + k
+        uint32_t qb0[4] = {0u, 0u, 0u, 0u}, qb1[4] = {0u, 0u, 0u, 0u};   // positions 32 + 16c + k
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const unsigned long long a = pk_u(va[2 * k], va[2 * k + 1]), bb = pk_u(vb[2 * k], vb[2 * k + 1]);
+          float z0, z1, y0, y1;
+          upk(add2(a, bb), z0, z1);
+          upk(sub2(a, bb), y0, y1);
+          const int sh = 8 * (k & 3);
+          qa0[k >> 2] |= (static_cast<uint32_t>(max(-127, min(127, __float2int_rn(z0 * 0.125f * r0)))) & 0xFFu) << sh;
+          qa1[k >> 2] |= (static_cast<uint32_t>(max(-127, min(127, __float2int_rn(z1 * 0.125f * r1)))) & 0xFFu) << sh;
+          qb0[k >> 2] |= (static_cast<uint32_t>(max(-127, min(127, __float2int_rn(y0 * 0.125f * r0)))) & 0xFFu) << sh;
+          qb1[k >> 2] |= (static_cast<uint32_t>(max(-127, min(127, __float2int_rn(y1 * 0.125f * r1)))) & 0xFFu) << sh;
+        }
+        if (ok0) {
+          __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 16 * c), make_uint4(qa0[0], qa0[1], qa0[2], qa0[3]));
+          __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 32 + 16 * c), make_uint4(qb0[0], qb0[1], qb0[2], qb0[3]));
+        }
+        if (ok1) {
+          __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 16 * c), make_uint4(qa1[0], qa1[1], qa1[2], qa1[3]));
+          __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 32 + 16 * c), make_uint4(qb1[0], qb1[1], qb1[2], qb1[3]));
+        }
+      }
+      if (b == 0) {
+        if (ok0) static_cast<float*>(p.aux)[t0] = sc0;
+        if (ok1) static_cast<float*>(p.aux)[t1] = sc1;
+      }
+    } else {   // kRotate: x' = z / 8 in BF16
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + 64 * b;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t va[32], vb[32];
+        __syncwarp();
+        tmem_ld32(tA + 32u * c, va);
+        tmem_ld32(tB + 32u * c, vb);
+        tmem_wait_ld();
+        uint32_t ua0[8], ua1[8], ub0[8], ub1[8];
+#pragma unroll
+        for (int k2 = 0; k2 < 8; ++k2) {
+          float z[2][2], y[2][2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int k = 2 * k2 + e;
+            const unsigned long long a = pk_u(va[2 * k], va[2 * k + 1]), bb = pk_u(vb[2 * k], vb[2 * k + 1]);
+            upk(add2(a, bb), z[e][0], z[e][1]);
+            upk(sub2(a, bb), y[e][0], y[e][1]);
+          }
+          ua0[k2] = bf2_bits(z[0][0] * 0.125f, z[1][0] * 0.125f);
+          ua1[k2] = bf2_bits(z[0][1] * 0.125f, z[1][1] * 0.125f);
+          ub0[k2] = bf2_bits(y[0][0] * 0.125f, y[1][0] * 0.125f);
+          ub1[k2] = bf2_bits(y[0][1] * 0.125f, y[1][1] * 0.125f);
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (ok0) {
+            __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 16 * c) + q,
+                   make_uint4(ua0[4 * q], ua0[4 * q + 1], ua0[4 * q + 2], ua0[4 * q + 3]));
+            __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 32 + 16 * c) + q,
+                   make_uint4(ub0[4 * q], ub0[4 * q + 1], ub0[4 * q + 2], ub0[4 * q + 3]));
+          }
+          if (ok1) {
+            __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 16 * c) + q,
+                   make_uint4(ua1[4 * q], ua1[4 * q + 1], ua1[4 * q + 2], ua1[4 * q + 3]));
+            __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 32 + 16 * c) + q,
+                   make_uint4(ub1[4 * q], ub1[4 * q + 1], ub1[4 * q + 2], ub1[4 * q + 3]));
+          }
+        }
+      }
+      if (b == 0 && p.aux) {
+        if (ok0) static_cast<float*>(p.aux)[t0] = sqrtf(tot[0]);
+        if (ok1) static_cast<float*>(p.aux)[t1] = sqrtf(tot[1]);
+      }
+    }
+  }
+
+  // Every bulk copy this CTA issued has landed before it exits (they all have
+  // on the normal path; after a timed-out wait this bounds the exit).
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
+    bool ok = true;
+    for (int s = 0; s < NS; ++s)
+      if (issued[s] && !mbar_wait(&full[s], (issued[s] - 1) & 1)) ok = false;
+    if (!ok) atomicOr(p.err, 128u);
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(*tmem_slot, 512);
+  }
+}
+
+}  // namespace pairk
+
+// ---- host side ------------------------------------------------------------
+
+namespace {
+
+int sm_count_pair() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// Most ring slots that fit next to the tables (at least 2, at most 6), or 0.
+int slots_that_fit(int d, int grid_n) {
+  int best = 0;
+  for (int ns = 2; ns <= 6; ++ns)
+    if (pairk::layout(d, ns, grid_n).total + 128 <= pairk::kSmemLimit) best = ns;
+  return best;
+}
+
+template <int MODE, int BITS, bool FULL>
+int launch_pair(const pairk::Params& p, cudaStream_t st) {
+  auto kern = pairk::rotq_pair_kernel<MODE, BITS, FULL>;
+  const size_t smem = pairk::layout(p.d, p.NS, p.grid_n).total + 128;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int sms = sm_count_pair();
+  const int grid = p.ntiles < sms ? p.ntiles : sms;
+  kern<<<grid, p.nwarps * 32, smem, st>>>(p);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+}
+
+template <int MODE, bool FULL>
+int launch_pair_bits(int bits, const pairk::Params& p, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_pair<MODE, 1, FULL>(p, st);
+    case 2: return launch_pair<MODE, 2, FULL>(p, st);
+    case 3: return launch_pair<MODE, 3, FULL>(p, st);
+    case 4: return launch_pair<MODE, 4, FULL>(p, st);
+    case 5: return launch_pair<MODE, 5, FULL>(p, st);
+    case 6: return launch_pair<MODE, 6, FULL>(p, st);
+    case 7: if constexpr (!FULL) return launch_pair<MODE, 7, FULL>(p, st); else return RBQ_ECONVERGE;
+    case 8: if constexpr (!FULL) return launch_pair<MODE, 8, FULL>(p, st); else return RBQ_ECONVERGE;
+    default: return RBQ_EINVAL;
+  }
+}
+
+}  // namespace
+
+bool rotq_pair_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d % 256 == 0 && d >= 1024 && d <= 3072; }
+
+// Returns RBQ_ECONVERGE when the tables do not fit (the caller then uses
+// another kernel); any other code is the call's result.
+int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
+                     cudaStream_t st) {
+  using namespace pairk;
+  const uint32_t* tab = nullptr;
+  int rc = rpbh_pair_tables(r, &tab);
+  if (rc != RBQ_OK) return rc;
+  Params p{};
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.T = rows;
+  p.d = r->d;
+  p.nblk = r->d / kH;
+  p.nwarps = p.nblk / 4;
+  p.ntiles = static_cast<int>((rows + kRows - 1) / kRows);
+  p.pitch = 2u * static_cast<uint32_t>(r->d) + 16u;
+  p.tab = tab;
+  p.out = out;
+  p.aux = aux;
+  if ((rc = device_error_word_ptr(&p.err)) != RBQ_OK) return rc;
+  const bool lloyd = (mode == kAct || mode == kWeightLM);
+  bool full = false;
+  if (lloyd) {
+    const CodebookDevice* cb = nullptr;
+    if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
+    if (bits <= 6 && cb->grid_full && slots_that_fit(r->d, cb->grid_full_cells + 1) >= 2) {
+      full = true;
+      p.grid = cb->grid_full;
+      p.grid_n = cb->grid_full_cells + 1;
+      p.grid_cells = static_cast<float>(cb->grid_full_cells);
+      p.grid_scale = 0.5f;
+    } else {
+      p.grid = cb->grid;
+      p.grid_n = cb->grid_cells + 1;
+      p.grid_cells = static_cast<float>(cb->grid_cells);
+      p.grid_scale = cb->grid_scale;
+    }
+  }
+  p.NS = slots_that_fit(r->d, p.grid_n);
+  if (p.NS < 2) return RBQ_ECONVERGE;
+  switch (mode) {
+    case kAct: return full ? launch_pair_bits<kAct, true>(bits, p, st) : launch_pair_bits<kAct, false>(bits, p, st);
+    case kWeightLM:
+      return full ? launch_pair_bits<kWeightLM, true>(bits, p, st) : launch_pair_bits<kWeightLM, false>(bits, p, st);
+    case kInt8: return launch_pair<kInt8, 8, false>(p, st);
+    default: return launch_pair<kRotate, 8, false>(p, st);
+  }
+}
+
+}  // namespace rbq

@@ -140,6 +140,72 @@ def test_video_w4a6_activations_sampled_frames(d):
 
 
 # --------------------------------------------------------------------------
+# token-pair kernel (BF16, d = 1024..3072 in steps of 256): every mode, ragged
+# tiles of 16 tokens, and enough tiles per CTA to wrap its ring of slots and
+# its norm barriers several times
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_pair_kernel_all_bit_widths(bits):
+    # d = 1280: 5 warps per CTA; 37 tokens = 2 full tiles + 5 rows
+    X, _ = synth.student_t_act(37, 1280, seed=40 + bits)
+    _act_parity(X, 1280, bits, seed=bits)
+
+
+@pytest.mark.parametrize("d,T,bits", [(3072, 1, 4), (3072, 17, 6), (3072, 33, 8), (1024, 16, 2), (2816, 31, 3)])
+def test_pair_kernel_shapes(d, T, bits):
+    X, _ = synth.student_t_act(T, d, seed=d + T)
+    _act_parity(X, d, bits, seed=d)
+
+
+@pytest.mark.parametrize("d,T,bits", [(1024, 148 * 16 * 14 + 5, 4), (3072, 148 * 16 * 6 + 9, 4)])
+def test_pair_kernel_many_tiles_per_cta(d, T, bits):
+    X, _ = synth.student_t_act(T, d, seed=7)
+    rows = np.unique(np.concatenate([[0, 15, 16, T - 1, T - 6],
+                                     np.random.default_rng(d).choice(T, 60, replace=False)]))
+    _act_parity(X, d, bits, seed=3, rows=rows)
+
+
+@pytest.mark.parametrize("d", [1280, 3072])
+def test_pair_kernel_rotate_only(d):
+    X, _ = synth.student_t_act(41, d, seed=d)
+    r, Pi = _rpbh(d, 6)
+    nr = torch.empty((41,), dtype=torch.float32, device="cuda")
+    xr = rbq.rotate_act(r, torch_bf16(X), norms=nr)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.rotate_only(X.astype(np.float64), Pi)
+    check_bf16_rounding(bf16_to_numpy(xr), ora["xr"], "rotate-only")
+    check_rel(nr.cpu().numpy(), np.linalg.norm(ora["xr"], axis=1), NORM_RTOL, "rotate-only norms")
+
+
+@pytest.mark.parametrize("d,n", [(1024, 33), (3072, 50)])
+def test_pair_kernel_weights_int8(d, n):
+    W = synth.to_bf16(synth.gaussian_weights(synth.rng(12, d), n, d, outlier_frac=0.01).astype(np.float32))
+    W[3] = 0.0
+    r, Pi = _rpbh(d, 9)
+    q, sc = rbq.quantize_weights(r, torch_bf16(W), 8, mode="int8")
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi)
+    check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
+
+
+@pytest.mark.parametrize("bits", [6, 8])
+def test_pair_kernel_weights_wide_codebooks(bits):
+    d = 3072
+    W = synth.attn_proj()["W"][:40].copy()
+    W[2] = 0.0
+    r, Pi = _rpbh(d, 0)
+    codes, rn = rbq.quantize_weights(r, torch_bf16(W), bits)
+    torch.cuda.synchronize()
+    _, bounds = oracle.lloydmax_table(d, bits)
+    ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
+    check_codes(_unpack(codes, bits, d), ora["codes"], ora["v"], bounds, d)
+    check_bf16_rounding(bf16_to_numpy(rn), ora["rnorm"], "row norms")
+
+
+# --------------------------------------------------------------------------
 # rotate-only (BF16 x') and offline weights
 # --------------------------------------------------------------------------
 
