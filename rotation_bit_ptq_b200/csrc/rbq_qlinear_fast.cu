@@ -7,31 +7,38 @@
 //
 // Two kernels per call.
 //
-// 1. expand_weights_kernel: the weight codes are turned into fp16 levels
+// 1. expand_weights_kernel(8): the weight codes are turned into fp16 levels
 //    (x sqrt(K)) once, into a stream-ordered workspace [N, K] -- an HBM-bound
 //    pass over N*K*(b/8 + 2) bytes.  Expanding each weight tile inside the
 //    GEMM instead would redo that work for every 128-row tile of tokens and
 //    saturate the SM's integer pipe.
 // 2. qlinear_fast_kernel: each CTA (one per SM) walks a static list of
-//    128 x 256 output tiles.
+//    128 x 192 output tiles.
 //      warps 0..3  epilogue: TMEM lane quadrant w, one output row per thread;
 //                  scale by s_m r'_n / K, round to BF16, store.
 //      warp 4      MMA issuer: one thread waits for a filled operand stage,
-//                  issues four 128x256x16 kind::f16 MMAs into the tile's TMEM
+//                  issues four 128x192x16 kind::f16 MMAs (A from tensor
+//                  memory, B from shared memory) into the tile's TMEM
 //                  accumulator, commits them to the stage's "empty" barrier,
 //                  and after the last K slice commits the accumulator.
 //      warp 5      TMA producer: one thread loads (a) the activation codes of
 //                  two K slices for the tile's 128 rows into a ring of code
-//                  stages and (b) the 256 x 64 fp16 weight tile of each K
+//                  stages and (b) the 192 x 64 fp16 weight tile of each K
 //                  slice straight into the operand stage, 128B-swizzled as the
 //                  tensor core reads it.
-//      warps 6..9  activation expansion, one row per thread: read the row's
-//                  codes of a K slice from the code stage, turn them into fp16
-//                  levels, write the row into the operand stage's swizzled
-//                  K-major tile.
-//    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
-//    overlap the MMAs of tile i+1.
-//
+//      warps 6..13 activation expansion, two threads per row (row = the
+//                  thread's TMEM lane; warps w and w+4 take the two halves of
+//                  the row's 64 codes): read the codes of a K slice from the
+//                  code stage, turn them into fp16 levels before waiting for
+//                  the stage, then store them into 16 of the stage's 32 TMEM
+//                  columns with one tcgen05.st.
+//    Tensor memory: two accumulators (2 x 192 columns, so the epilogue of
+//    tile i overlaps the MMAs of tile i+1) and four A stages (4 x 32).
+//    Keeping A out of shared memory matters: per K slice the weight tile is
+//    written by TMA and read by the MMA (48 KB), and an A tile in shared
+//    memory would add another 32 KB of stores and reads to a port that
+//    moves 128 bytes per cycle.
+
 // 4-bit codes are expanded in registers: by symmetry C[15-c] = -C[c], the
 // magnitude index m (0..7) selects the two bytes of |C| with byte permutes
 // (prmt) from four registers holding the low and high byte planes of the
@@ -63,15 +70,19 @@ namespace qfast {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kATile = kBM * kBK * 2;          // 16 KB fp16
-constexpr int kBTile = kBN * kBK * 2;          // 32 KB fp16
-constexpr int kOpStage = kATile + kBTile;      // 48 KB
-constexpr int kMaxF = 4, kMaxC = 4;
-constexpr int kThreads = 320;                  // 10 warps
+constexpr int kBM = 128, kBN = 192, kBK = 64;
+constexpr int kBTile = kBN * kBK * 2;          // 24 KB fp16 (weights, shared memory)
+constexpr int kOpStage = kBTile;
+// Tensor memory (512 columns): two fp32 accumulators of kBN columns, then
+// the activation operand stages, 32 columns (64 fp16 of K) each.
+constexpr uint32_t kACol = 2 * kBN;            // 384
+constexpr uint32_t kAStageCols = kBK / 2;      // 32
+constexpr int kAStages = 4;                    // kACol + kAStages * kAStageCols == 512
+constexpr int kMaxF = 8, kMaxC = 4;            // weight stages (shared memory), code stages
+constexpr int kThreads = 448;                  // 14 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
 constexpr int kExpandFirst = 192;              // warp 6
-constexpr int kExpandThreads = kBM;            // 128 activation rows
+constexpr int kExpandThreads = 2 * kBM;        // two threads per activation row (32 codes each)
 constexpr size_t kSmemLimit = 227 * 1024;
 
 // Code-stage geometry of the activation operand.
@@ -99,8 +110,10 @@ struct Params {
 };
 
 struct __align__(8) Tail {
-  uint64_t full[kMaxF];
-  uint64_t empty[kMaxF];
+  uint64_t full[kMaxF];          // weight stage landed (TMA bytes)
+  uint64_t empty[kMaxF];         // weight stage consumed (MMA commit)
+  uint64_t afull[kAStages];      // activation stage stored in TMEM (128 threads)
+  uint64_t aempty[kAStages];     // activation stage consumed (MMA commit)
   uint64_t cfull[kMaxC];
   uint64_t cempty[kMaxC];
   uint64_t acc_full[2];
@@ -171,21 +184,24 @@ __device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint3
 template <int BITS>
 constexpr int slice_words() { return 2 * BITS; }
 
-// One row's 64 codes of a K slice -> 8 swizzled 16-byte chunks of fp16.
-template <int BITS>
+// Half HF (codes 32 HF .. 32 HF + 31) of one row's 64 codes of a K slice ->
+// 16 words of fp16 pairs (k even in the low half), 16 of the row's operand
+// columns in tensor memory.
+template <int BITS, int HF>
 __device__ __forceinline__ void expand_row(const uint32_t (&src)[slice_words<BITS>()], const Planes4& P,
-                                           const uint16_t* lut, uint8_t* tile, int r) {
+                                           const uint16_t* lut, uint32_t (&out)[16]) {
   if constexpr (BITS == 4) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 4 * HF; c < 4 * HF + 4; ++c) {
       uint32_t w[4];
       expand8_4bit(src[c], P, w);
-      *reinterpret_cast<uint4*>(tile + sw128_offset(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[4 * (c - 4 * HF) + j] = w[j];
     }
   } else {
     constexpr uint32_t mask = (1u << BITS) - 1u;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 4 * HF; c < 4 * HF + 4; ++c) {
       uint32_t w[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -200,7 +216,8 @@ __device__ __forceinline__ void expand_row(const uint32_t (&src)[slice_words<BIT
         }
         w[j] = pair;
       }
-      *reinterpret_cast<uint4*>(tile + sw128_offset(r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[4 * (c - 4 * HF) + j] = w[j];
     }
   }
 }
@@ -235,30 +252,42 @@ __device__ __forceinline__ void read_slice(const uint8_t* part, const CodeGeo& g
   }
 }
 
-template <int BITS>
-__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, int r,
+// Waits on a barrier for the whole warp: every lane returns the same answer,
+// so the warp-collective tensor-memory stores that follow run converged.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* tl) {
+  return !__any_sync(0xffffffffu, !wait_or_abort(bar, parity, tl));
+}
+
+// Row r = 32 (warp % 4) + lane of every activation tile: the thread's own
+// tensor-memory lane, which `tA` addresses.
+template <int BITS, int HF>
+__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* codes, int r, uint32_t tA,
                                             int ntiles, Planes4 P, const uint16_t* lut) {
   const CodeGeo& g = p.ga;
   const int KP = p.K / (2 * kBK);
-  uint32_t cf = 0, cc = 0;
+  const uint32_t C = static_cast<uint32_t>(p.C);
+  uint32_t c = 0, cph = 0, s = 0, aph = 0;       // code stage / A stage and their phases
+  bool a_first = true;                           // first round of A stages: nothing to wait for
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     for (int kp = 0; kp < KP; ++kp) {
-      const uint32_t c = cc % p.C;
-      if (!wait_or_abort(&tl->cfull[c], (cc / p.C) & 1, tl)) return;
+      if (!warp_wait(&tl->cfull[c], cph, tl)) return;
       const uint8_t* part = codes + c * p.cstage_bytes + g.offset;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t cur[slice_words<BITS>()];
         read_slice<BITS>(part, g, r, h, cur);
-        const uint32_t s = cf % p.F;
-        if (cf >= static_cast<uint32_t>(p.F) && !wait_or_abort(&tl->empty[s], ((cf / p.F) - 1) & 1, tl)) return;
-        expand_row<BITS>(cur, P, lut, ops + s * kOpStage, r);
-        fence_proxy_async_smem();
-        mbar_arrive(&tl->full[s]);
-        ++cf;
+        uint32_t w[16];
+        expand_row<BITS, HF>(cur, P, lut, w);          // before the wait: off the critical path
+        if (!a_first && !warp_wait(&tl->aempty[s], aph ^ 1u, tl)) return;
+        tc_fence_after();
+        tmem_st16(tA + s * kAStageCols + 16 * HF, w);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&tl->afull[s]);
+        if (++s == kAStages) { s = 0; aph ^= 1u; a_first = false; }
       }
       mbar_arrive(&tl->cempty[c]);
-      ++cc;
+      if (++c == C) { c = 0; cph ^= 1u; }
     }
   }
 }
@@ -280,8 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = tid; i < 256; i += kThreads) tl->lut_a[i] = (i < (1 << p.bits_a)) ? p.lut_a[i] : 0;
   if (tid == 0) {
     for (int s = 0; s < p.F; ++s) {
-      mbar_init(&tl->full[s], kExpandThreads + 1);   // + the producer's expect-tx arrival (weight tile)
+      mbar_init(&tl->full[s], 1);                    // the producer's expect-tx arrival
       mbar_init(&tl->empty[s], 1);
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&tl->afull[s], kExpandThreads);
+      mbar_init(&tl->aempty[s], 1);
     }
     for (int c = 0; c < p.C; ++c) {
       mbar_init(&tl->cfull[c], 1);
@@ -305,9 +338,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
+    // One thread feeds the tensor core, so its own instruction latency sets
+    // the pace: stage indices and phases advance incrementally, a barrier
+    // that is already complete costs one try_wait, and the operand
+    // descriptors step by constants.
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, false);
-      uint32_t cnt = 0, it = 0;
+      const uint64_t bdesc0 = sdesc_k_sw128(smem_u32(ops));
+      const uint32_t F = static_cast<uint32_t>(p.F);
+      uint32_t s = 0, ph = 0, sa = 0, pha = 0, it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const uint32_t a = it & 1u, use = it >> 1;
@@ -315,16 +354,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t acc = tmem + a * kBN;
         for (int kb = 0; kb < KT; ++kb) {
-          const uint32_t s = cnt % p.F;
-          if (!wait_or_abort(&tl->full[s], (cnt / p.F) & 1, tl)) { ok = false; break; }
+          if ((!mbar_try_wait(&tl->full[s], ph) && !wait_or_abort(&tl->full[s], ph, tl)) ||
+              (!mbar_try_wait(&tl->afull[sa], pha) && !wait_or_abort(&tl->afull[sa], pha, tl))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(ops + s * kOpStage);
-          const uint32_t b0 = a0 + kATile;
-#pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_f16(acc, sdesc_k_sw128(a0 + 32 * k), sdesc_k_sw128(b0 + 32 * k), kIdesc, (kb | k) != 0);
+          const uint32_t a0 = tmem + kACol + sa * kAStageCols;            // A: tensor memory
+          const uint64_t b0 = bdesc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);   // B: shared memory
+          umma_f16_ta(acc, a0, b0, kIdesc, kb != 0);
+          umma_f16_ta(acc, a0 + 8, b0 + 2, kIdesc, 1u);                  // +32 bytes of K per step
+          umma_f16_ta(acc, a0 + 16, b0 + 4, kIdesc, 1u);
+          umma_f16_ta(acc, a0 + 24, b0 + 6, kIdesc, 1u);
           umma_commit(&tl->empty[s]);
-          ++cnt;
+          umma_commit(&tl->aempty[sa]);
+          if (++s == F) { s = 0; ph ^= 1u; }
+          if (++sa == kAStages) { sa = 0; pha ^= 1u; }
         }
         if (ok) umma_commit(&tl->acc_full[a]);
       }
@@ -335,13 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      uint32_t cc = 0, cf = 0;
+      const uint32_t C = static_cast<uint32_t>(p.C), F = static_cast<uint32_t>(p.F);
+      uint32_t c = 0, cph = 0, s = 0, ph = 0;     // code / weight stage and their phases
+      bool c_first = true, b_first = true;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const int mt = tile % ntiles_m, nt = tile / ntiles_m;
         for (int kp = 0; kp < KP && ok; ++kp) {
-          const uint32_t c = cc % p.C;
-          if (cc >= static_cast<uint32_t>(p.C) && !wait_or_abort(&tl->cempty[c], ((cc / p.C) - 1) & 1, tl)) {
+          if (!c_first && !wait_or_abort(&tl->cempty[c], cph ^ 1u, tl)) {
             ok = false;
             break;
           }
@@ -354,17 +400,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(stage + p.ga.offset, &tmA, kp * 16 * p.ga.bits, mt * kBM, &tl->cfull[c]);
           }
-          ++cc;
+          if (++c == C) { c = 0; cph ^= 1u; c_first = false; }
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {
-            const uint32_t s = cf % p.F;
-            if (cf >= static_cast<uint32_t>(p.F) && !wait_or_abort(&tl->empty[s], ((cf / p.F) - 1) & 1, tl)) {
+            if (!b_first && !wait_or_abort(&tl->empty[s], ph ^ 1u, tl)) {
               ok = false;
               break;
             }
             mbar_arrive_expect_tx(&tl->full[s], kBTile);
-            tma_load_2d(ops + s * kOpStage + kATile, &tmB, (2 * kp + h) * kBK, nt * kBN, &tl->full[s]);
-            ++cf;
+            tma_load_2d(ops + s * kOpStage, &tmB, (2 * kp + h) * kBK, nt * kBN, &tl->full[s]);
+            if (++s == F) { s = 0; ph ^= 1u; b_first = false; }
           }
         }
       }
@@ -377,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const uint32_t a = it & 1u, use = it >> 1;
-      if (!wait_or_abort(&tl->acc_full[a], use & 1, tl)) {
+      if (!warp_wait(&tl->acc_full[a], use & 1, tl)) {   // warp-uniform: tmem loads follow
         if (lane == 0) atomicOr(p.err, 4u);
         break;
       }
@@ -422,20 +467,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- activation expansion ----------------
-    const int r = tid - kExpandFirst;
+    // warps 6..13: lane quarter warp % 4, code half (warp - 6) / 4
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t tA = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kACol;
     const uint16_t* lut = tl->lut_a;
     const Planes4 P = make_planes4(lut);
-    switch (p.bits_a) {
-      case 1: expand_loop<1>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      case 2: expand_loop<2>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      case 3: expand_loop<3>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      case 4: expand_loop<4>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      case 5: expand_loop<5>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      case 6: expand_loop<6>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      case 7: expand_loop<7>(p, tl, ops, codes, r, ntiles, P, lut); break;
-      default: expand_loop<8>(p, tl, ops, codes, r, ntiles, P, lut); break;
+    if (warp < 10) {
+      switch (p.bits_a) {
+        case 1: expand_loop<1, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 2: expand_loop<2, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 3: expand_loop<3, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 4: expand_loop<4, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 5: expand_loop<5, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 6: expand_loop<6, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 7: expand_loop<7, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        default: expand_loop<8, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+      }
+    } else {
+      switch (p.bits_a) {
+        case 1: expand_loop<1, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 2: expand_loop<2, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 3: expand_loop<3, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 4: expand_loop<4, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 5: expand_loop<5, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 6: expand_loop<6, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 7: expand_loop<7, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        default: expand_loop<8, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+      }
     }
-    if (tl->abort && r == 0) atomicOr(p.err, 8u);
+    if (tl->abort && r == 0 && warp < 10) atomicOr(p.err, 8u);
   }
 
   tc_fence_before();
@@ -564,13 +624,49 @@ int encode_f16_map(CUtensorMap* map, const uint16_t* base, int rows, int K) {
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
 }
 
+// Widths that divide 8 bits: one thread per 8 codes (BITS bytes in, 16 bytes
+// out), so a warp reads 32*BITS and writes 512 contiguous bytes.
+template <int BITS>
+__global__ void __launch_bounds__(256) expand_weights_kernel8(const uint8_t* codes, long long groups,
+                                                             const uint16_t* lut_g, uint16_t* out) {
+  __shared__ uint16_t lut[256];
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = (i < (1 << BITS)) ? lut_g[i] : 0;
+  __syncthreads();
+  const Planes4 P = make_planes4(lut);
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    uint32_t w[4];
+    if constexpr (BITS == 4) {
+      expand8_4bit(__ldcs(reinterpret_cast<const uint32_t*>(codes) + g), P, w);
+    } else {
+      uint64_t x;
+      if constexpr (BITS == 8) x = __ldcs(reinterpret_cast<const unsigned long long*>(codes) + g);
+      else if constexpr (BITS == 2) x = __ldcs(reinterpret_cast<const unsigned short*>(codes) + g);
+      else x = codes[g];
+      constexpr uint32_t mask = (1u << BITS) - 1u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = static_cast<uint32_t>(lut[(x >> (2 * j * BITS)) & mask]) |
+               (static_cast<uint32_t>(lut[(x >> ((2 * j + 1) * BITS)) & mask]) << 16);
+    }
+    __stcg(reinterpret_cast<uint4*>(out) + g, make_uint4(w[0], w[1], w[2], w[3]));
+  }
+}
+
 template <int BITS>
 int launch_expand(const uint8_t* codes, int rows, int K, const uint16_t* lut, uint16_t* out, cudaStream_t st,
                   int sms) {
-  const long long items = static_cast<long long>(rows) * (K / kBK);
-  long long blocks = (items + 255) / 256;
-  if (blocks > 8LL * sms) blocks = 8LL * sms;
-  expand_weights_kernel<BITS><<<static_cast<int>(blocks), 256, 0, st>>>(codes, rows, K, lut, out);
+  if constexpr (8 % BITS == 0) {
+    const long long groups = static_cast<long long>(rows) * (K / 8);
+    long long blocks = (groups + 255) / 256;
+    if (blocks > 16LL * sms) blocks = 16LL * sms;
+    expand_weights_kernel8<BITS><<<static_cast<int>(blocks), 256, 0, st>>>(codes, groups, lut, out);
+  } else {
+    const long long items = static_cast<long long>(rows) * (K / kBK);
+    long long blocks = (items + 255) / 256;
+    if (blocks > 8LL * sms) blocks = 8LL * sms;
+    expand_weights_kernel<BITS><<<static_cast<int>(blocks), 256, 0, st>>>(codes, rows, K, lut, out);
+  }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }
