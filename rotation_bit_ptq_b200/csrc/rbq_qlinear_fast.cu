@@ -78,7 +78,7 @@ constexpr int kOpStage = kBTile;
 constexpr uint32_t kACol = 2 * kBN;            // 384
 constexpr uint32_t kAStageCols = kBK / 2;      // 32
 constexpr int kAStages = 4;                    // kACol + kAStages * kAStageCols == 512
-constexpr int kMaxF = 8, kMaxC = 4;            // weight stages (shared memory), code stages
+constexpr int kMaxF = kAStages, kMaxC = 8;     // operand stages (A in TMEM, B in smem), code stages
 constexpr int kThreads = 448;                  // 14 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
 constexpr int kExpandFirst = 192;              // warp 6
@@ -110,10 +110,8 @@ struct Params {
 };
 
 struct __align__(8) Tail {
-  uint64_t full[kMaxF];          // weight stage landed (TMA bytes)
-  uint64_t empty[kMaxF];         // weight stage consumed (MMA commit)
-  uint64_t afull[kAStages];      // activation stage stored in TMEM (128 threads)
-  uint64_t aempty[kAStages];     // activation stage consumed (MMA commit)
+  uint64_t full[kMaxF];          // weight tile landed (TMA bytes) and activation tile stored (expansion threads)
+  uint64_t empty[kMaxF];         // stage consumed (MMA commit)
   uint64_t cfull[kMaxC];
   uint64_t cempty[kMaxC];
   uint64_t acc_full[2];
@@ -278,12 +276,12 @@ __device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* 
         read_slice<BITS>(part, g, r, h, cur);
         uint32_t w[16];
         expand_row<BITS, HF>(cur, P, lut, w);          // before the wait: off the critical path
-        if (!a_first && !warp_wait(&tl->aempty[s], aph ^ 1u, tl)) return;
+        if (!a_first && !warp_wait(&tl->empty[s], aph ^ 1u, tl)) return;
         tc_fence_after();
         tmem_st16(tA + s * kAStageCols + 16 * HF, w);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&tl->afull[s]);
+        mbar_arrive(&tl->full[s]);
         if (++s == kAStages) { s = 0; aph ^= 1u; a_first = false; }
       }
       mbar_arrive(&tl->cempty[c]);
@@ -308,13 +306,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   for (int i = tid; i < 256; i += kThreads) tl->lut_a[i] = (i < (1 << p.bits_a)) ? p.lut_a[i] : 0;
   if (tid == 0) {
-    for (int s = 0; s < p.F; ++s) {
-      mbar_init(&tl->full[s], 1);                    // the producer's expect-tx arrival
+    for (int s = 0; s < kMaxF; ++s) {
+      mbar_init(&tl->full[s], kExpandThreads + 1);   // + the producer's expect-tx arrival
       mbar_init(&tl->empty[s], 1);
-    }
-    for (int s = 0; s < kAStages; ++s) {
-      mbar_init(&tl->afull[s], kExpandThreads);
-      mbar_init(&tl->aempty[s], 1);
     }
     for (int c = 0; c < p.C; ++c) {
       mbar_init(&tl->cfull[c], 1);
@@ -345,8 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, false);
       const uint64_t bdesc0 = sdesc_k_sw128(smem_u32(ops));
-      const uint32_t F = static_cast<uint32_t>(p.F);
-      uint32_t s = 0, ph = 0, sa = 0, pha = 0, it = 0;
+      constexpr uint32_t F = kMaxF;
+      uint32_t s = 0, ph = 0, it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const uint32_t a = it & 1u, use = it >> 1;
@@ -354,22 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t acc = tmem + a * kBN;
         for (int kb = 0; kb < KT; ++kb) {
-          if ((!mbar_try_wait(&tl->full[s], ph) && !wait_or_abort(&tl->full[s], ph, tl)) ||
-              (!mbar_try_wait(&tl->afull[sa], pha) && !wait_or_abort(&tl->afull[sa], pha, tl))) {
+          if (!mbar_try_wait(&tl->full[s], ph) && !wait_or_abort(&tl->full[s], ph, tl)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = tmem + kACol + sa * kAStageCols;            // A: tensor memory
+          const uint32_t a0 = tmem + kACol + s * kAStageCols;             // A: tensor memory
           const uint64_t b0 = bdesc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);   // B: shared memory
           umma_f16_ta(acc, a0, b0, kIdesc, kb != 0);
           umma_f16_ta(acc, a0 + 8, b0 + 2, kIdesc, 1u);                  // +32 bytes of K per step
           umma_f16_ta(acc, a0 + 16, b0 + 4, kIdesc, 1u);
           umma_f16_ta(acc, a0 + 24, b0 + 6, kIdesc, 1u);
           umma_commit(&tl->empty[s]);
-          umma_commit(&tl->aempty[sa]);
           if (++s == F) { s = 0; ph ^= 1u; }
-          if (++sa == kAStages) { sa = 0; pha ^= 1u; }
         }
         if (ok) umma_commit(&tl->acc_full[a]);
       }
@@ -727,8 +718,10 @@ int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const 
   p.ga = make_geo(kBM, bits_a, 0);
   p.cstage_bytes = geo_span(p.ga);
   const size_t tail = sizeof(Tail) + 64;
-  int F = kMaxF, C = 2;
-  while (F > 2 && 1024 + F * kOpStage + C * p.cstage_bytes + tail > kSmemLimit) --F;
+  // The operand ring is fixed at kMaxF stages (their A halves fill the rest of
+  // tensor memory); the code ring takes what shared memory is left.
+  const int F = kMaxF;
+  int C = 2;
   while (C < kMaxC && 1024 + F * kOpStage + (C + 1) * p.cstage_bytes + tail <= kSmemLimit) ++C;
   const size_t smem = 1024 + static_cast<size_t>(F) * kOpStage + static_cast<size_t>(C) * p.cstage_bytes + tail;
   if (smem > kSmemLimit) return RBQ_EINVAL;
