@@ -35,6 +35,14 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
+
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel as
+# it stands (profiles/qlinear_W4A4_4608x3072x3072.md,
+# profiles/rotate_quantize_act_d3072_T32768_A4.md).  The rotate-quantize
+# capture ran 32768 tokens; its bytes are scaled to this workload's 4608 by
+# the token count (its traffic grows in proportion to the tokens).
+QLINEAR_DRAM_BYTES = 26_066_944 + 83_968
+ROTQ_DRAM_BYTES = round((201_669_632 + 29_559_296) * 4608 / 32768)
 METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
 
@@ -252,12 +260,14 @@ def run_ours(args, rank, world):
                     "avg_us": round(k2_avg_s * 1e6, 3)},
         "roofline": {"kernel": "qlinear", "bound": "tensor", "achieved": round(flops / k2_avg_s / 1e12, 2),
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": None,
-                     "peak_source": pk["source"] + " bf16 burst"},
+                     "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": QLINEAR_DRAM_BYTES,
+                     "peak_source": pk["source"] + " bf16 burst",
+                     "note": "achieved includes the per-call weight-code expansion launch"},
         "roofline_rotate_quantize": {"kernel": "rotate_quantize_act", "bound": "hbm",
                                      "achieved": round(act_bytes / k1_avg_s / 1e9, 2), "peak": pk["hbm_gbs"],
                                      "unit": "GB/s", "frac": round(act_bytes / k1_avg_s / 1e9 / pk["hbm_gbs"], 4),
-                                     "traffic": None, "peak_source": pk["source"]},
+                                     "traffic": ROTQ_DRAM_BYTES, "algorithmic_bytes": act_bytes,
+                                     "peak_source": pk["source"]},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
         "e2e": e2e,
@@ -296,6 +306,153 @@ def run_e2e(r, X_host, dev, stream, args):
     torch.cuda.synchronize()
     return a.elapsed_time(b), int(xh.numel() * 2), int(ch.numel() + nh.numel() * 4)
 
+
+
+# ---------------------------------------------------------------------------
+# the other workloads of the pages (kernel timings; inputs reused across
+# iterations -- every case except the INT8 4096-wide ones exceeds L2)
+# ---------------------------------------------------------------------------
+
+def _time_us(fn, stream, warmup=3, iters=10):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters * 1e3
+
+
+def _tile_rows(X, T):
+    reps = -(-T // X.shape[0])
+    return np.ascontiguousarray(np.tile(X, (reps, 1))[:T])
+
+
+def run_suite(dev, stream, pk):
+    """Every kernel of the path on the MLP pair (W2A4, W3A3), the INT8 W8A16
+    single-stream DiT block and the video-DiT layers (W4A6)."""
+    import torch
+    import rotation_bit_ptq_b200 as rbq
+
+    hbm, tc = pk["hbm_gbs"], pk["bf16_tflops"]
+    out = {}
+
+    def rotq_entry(us, T, d, bits):
+        gbs = T * (2 * d + d * bits // 8 + 4) / (us * 1e-6) / 1e9
+        return {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+
+    def gemm_entry(us, M, N, K):
+        tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+        return {"us": round(us, 2), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / tc, 4)}
+
+    # MLP pair: up 3072 -> 12288, down 12288 -> 3072, 4608 tokens
+    m = synth.mlp()
+    T = 4608
+    Xu, Xd = to_bf16_tensor(m["X_up"], dev), to_bf16_tensor(m["X_dn"], dev)
+    Wu, Wd = to_bf16_tensor(m["W_up"], dev), to_bf16_tensor(m["W_dn"], dev)
+    ru, rd = rbq.RPBH(3072, 11), rbq.RPBH(12288, 12)
+    mlp = {}
+    for ba, bw in ((4, 2), (3, 3)):
+        e = {}
+        au, su = rbq.rotate_quantize_act(ru, Xu, ba)
+        ad, sd = rbq.rotate_quantize_act(rd, Xd, ba)
+        e["rotate_quantize d=3072"] = rotq_entry(_time_us(lambda: rbq.rotate_quantize_act(ru, Xu, ba, au, su, stream=stream), stream), T, 3072, ba)
+        e["rotate_quantize d=12288"] = rotq_entry(_time_us(lambda: rbq.rotate_quantize_act(rd, Xd, ba, ad, sd, stream=stream), stream), T, 12288, ba)
+        wu, nu = rbq.quantize_weights(ru, Wu, bw)
+        wd, nd = rbq.quantize_weights(rd, Wd, bw)
+        yu = torch.empty((T, 12288), dtype=torch.bfloat16, device=dev)
+        yd = torch.empty((T, 3072), dtype=torch.bfloat16, device=dev)
+        e["qlinear up 4608x12288x3072"] = gemm_entry(
+            _time_us(lambda: rbq.qlinear(au, su, ba, wu, nu, bw, 3072, yu, stream=stream), stream), T, 12288, 3072)
+        e["qlinear down 4608x3072x12288"] = gemm_entry(
+            _time_us(lambda: rbq.qlinear(ad, sd, ba, wd, nd, bw, 12288, yd, stream=stream), stream), T, 3072, 12288)
+        mlp[f"W{bw}A{ba}"] = e
+    out["mlp_pair"] = mlp
+    ru.close()
+    rd.close()
+    del Xu, Xd, Wu, Wd, yu, yd
+
+    # INT8 rotate-then-quantize, W8A16, 4096 tokens; one block of the
+    # 32-block single-stream DiT (the per-block work is the same in every block)
+    int8 = {}
+    params = sum(o * i for _, o, i in synth.INT8_DIT_SHAPES)
+    rows = sum(o for _, o, _ in synth.INT8_DIT_SHAPES)
+    block_quant_us = 0.0
+    for name, n_out, d_in in synth.INT8_DIT_SHAPES:
+        if name in ("k", "v", "o"):          # same shape as q
+            block_quant_us += int8["q 4096->4096"]["quantize_weights_int8"]["us"]
+            continue
+        W = to_bf16_tensor(synth.int8_dit_weight(0, name), dev)
+        X = to_bf16_tensor(synth.int8_dit_act(d_in), dev)
+        r = rbq.RPBH(d_in, 100 + d_in)
+        q, sc = rbq.quantize_weights(r, W, 8, mode="int8")
+        xr = rbq.rotate_act(r, X)
+        y = torch.empty((4096, n_out), dtype=torch.bfloat16, device=dev)
+        e = {}
+        us = _time_us(lambda: rbq.quantize_weights(r, W, 8, "int8", q, sc, stream=stream), stream)
+        block_quant_us += us
+        gbs = n_out * (3 * d_in + 4) / (us * 1e-6) / 1e9
+        e["quantize_weights_int8"] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+        us = _time_us(lambda: rbq.rotate_act(r, X, xr, stream=stream), stream)
+        gbs = 4096 * 4 * d_in / (us * 1e-6) / 1e9
+        e["rotate_only"] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+        e["qlinear_int8"] = gemm_entry(_time_us(lambda: rbq.qlinear_int8(xr, q, sc, y, stream=stream), stream),
+                                       4096, n_out, d_in)
+        # output error on 64 tokens, against the dense layer (fp32 reference
+        # matmul, a report only): rotated INT8 vs naive per-channel INT8
+        with torch.no_grad():
+            xs, Wf = X[:64].float(), W.float()
+            dense = xs @ Wf.t()
+            scale_n = Wf.abs().amax(dim=1, keepdim=True) / 127.0
+            Wn = torch.clamp(torch.round(Wf / torch.where(scale_n > 0, scale_n, torch.ones_like(scale_n))), -127, 127) * scale_n
+            naive = xs @ Wn.t()
+            err_rot = (y[:64].float() - dense).norm() / dense.norm()
+            err_naive = (naive - dense).norm() / dense.norm()
+        e["rel_error_rotated_int8"] = round(err_rot.item(), 5)
+        e["rel_error_naive_int8"] = round(err_naive.item(), 5)
+        int8[f"{name} {d_in}->{n_out}"] = e
+        r.close()
+        del W, X, q, sc, xr, y
+    int8["model"] = {
+        "blocks": 32, "params": 32 * params,
+        "bf16_bytes": 2 * 32 * params, "int8_bytes": 32 * params + 4 * 32 * rows,
+        "ratio": round((32 * params + 4 * 32 * rows) / (2 * 32 * params), 4),
+        "pages_ratio": round(6.76 / 13.25, 4),
+        "quantize_weights_int8_ms_all_blocks": round(32 * block_quant_us * 1e-3, 3),
+    }
+    out["int8_dit"] = int8
+
+    # video DiT W4A6: 32760 tokens (21 frames x 1560), hidden 1536, MLP 8960
+    T = 32760
+    vid = {}
+    acts = {}
+    for d in (1536, 8960):
+        X = to_bf16_tensor(_tile_rows(synth.video_act(d, 0, frames=[0, 1, 2, 3]), T), dev)
+        r = rbq.RPBH(d, 1000 + d)
+        a, sv = rbq.rotate_quantize_act(r, X, 6)
+        vid[f"rotate_quantize d={d} A6"] = rotq_entry(
+            _time_us(lambda: rbq.rotate_quantize_act(r, X, 6, a, sv, stream=stream), stream), T, d, 6)
+        acts[d] = (a, sv, r)
+        del X
+    for n_out, d_in in ((1536, 1536), (8960, 1536), (1536, 8960)):
+        a, sv, r = acts[d_in]
+        W = to_bf16_tensor(synth.video_weight(n_out, d_in, 0), dev)
+        wc, wn = rbq.quantize_weights(r, W, 4)
+        y = torch.empty((T, n_out), dtype=torch.bfloat16, device=dev)
+        vid[f"qlinear {T}x{n_out}x{d_in} W4A6"] = gemm_entry(
+            _time_us(lambda: rbq.qlinear(a, sv, 6, wc, wn, 4, d_in, y, stream=stream), stream), T, n_out, d_in)
+        del W, wc, wn, y
+    for a, sv, r in acts.values():
+        r.close()
+    out["video_w4a6"] = vid
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    return out
 
 # ---------------------------------------------------------------------------
 # oracle (CPU) timings
@@ -390,6 +547,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-suite", action="store_true", help="skip the other workloads' kernel timings")
     ap.add_argument("--kernel-only", choices=["rotate_quantize", "rotate_only", "quantize_weights", "qlinear"],
                     help="run one kernel on a profiling-sized case (for ncu) instead of the benchmark")
     ap.add_argument("--tokens", type=int, default=0)
@@ -414,6 +572,10 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_ours(args, rank, world)
+    if rank == 0 and not args.no_suite:
+        import torch
+        res["suite"] = run_suite(torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))),
+                                 torch.cuda.current_stream(), peaks())
     if rank == 0:
         if not args.no_cpu_baseline:
             gbs, el, reps = oracle_rotq_gbs(T, 10.0)
