@@ -247,6 +247,9 @@ int launch_qgemm(const QParams& p, cudaStream_t st) {
 }  // namespace rbq
 
 namespace rbq {
+bool qlinear_int8_fast_eligible(int M, int N, int K);
+int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float* scale, int M, int N, int K,
+                             uint16_t* Y, unsigned int* err, cudaStream_t st);
 bool qlinear_fast_eligible(int M, int N, int K, int bits_a, int bits_w);
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
@@ -305,6 +308,8 @@ extern "C" int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float*
   unsigned int* err = nullptr;
   int rc = device_error_word_ptr(&err);
   if (rc != RBQ_OK) return rc;
+  if (qlinear_int8_fast_eligible(M, N, K))
+    return qlinear_int8_fast_launch(Xrot, Wq, scale, M, N, K, Y, err, static_cast<cudaStream_t>(stream));
   QParams p{};
   p.A = reinterpret_cast<const uint8_t*>(Xrot);
   p.B = reinterpret_cast<const uint8_t*>(Wq);

@@ -1,0 +1,335 @@
+// qlinear_int8, throughput version: the W8A16 linear of the INT8 path.
+//
+//   INT8-convrot (cloud.baidu.com/article/9430339) §4: rotate, quantise to
+//   INT8 per output channel, then run the layer through an INT8-aware operator:
+//     Y[m, n] = bf16( scale[n] * sum_k q[n, k] * x'[m, k] ),  x' = bf16(Pi x).
+//
+// Two kernels per call.
+//
+// 1. widen_int8_kernel: q [N, K] int8 -> bf16 [N, K] in a stream-ordered
+//    workspace.  Integers up to 127 are exact in bf16, so the tensor core sees
+//    the same values; an HBM pass over 3 N K bytes.
+// 2. qlinear_bf16_kernel: persistent tcgen05 GEMM, one CTA per SM, 128 x 256
+//    output tiles, K slices of 64.
+//      warps 0..3  epilogue: TMEM lane quadrant w, one output row per thread;
+//                  multiply by scale[n], round to BF16, store.
+//      warp 4      MMA issuer: one thread, four 128x256x16 kind::f16 (bf16)
+//                  MMAs per slice from shared memory, one commit per slice.
+//      warp 5      TMA producer: x' tile (128 x 64) and weight tile
+//                  (256 x 64) of each slice into a 4-stage ring, both
+//                  128B-swizzled K-major.
+//    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
+//    overlap the MMAs of tile i+1.
+//
+// Every mbarrier wait is bounded (see qlinear_fast); a thread whose wait runs
+// out raises the shared abort flag and records an error bit.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "rbq_internal.h"
+#include "rbq_sm100.cuh"
+
+namespace rbq {
+namespace q8fast {
+
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kATile = kBM * kBK * 2;          // 16 KB
+constexpr int kBTile = kBN * kBK * 2;          // 32 KB
+constexpr int kStage = kATile + kBTile;        // 48 KB
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kMmaWarp = 4, kTmaWarp = 5;
+
+struct Params {
+  int M, N, K;
+  const float* scale;
+  uint16_t* Y;
+  unsigned int* err;
+};
+
+struct __align__(8) Tail {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_slot;
+  volatile uint32_t abort;
+};
+
+constexpr size_t kSmem = 1024 + kStages * kStage + sizeof(Tail) + 64;
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (tl->abort) return false;
+    if (clock64() - t0 > (1ll << 31) || i > (1u << 26)) {
+      tl->abort = 1u;
+      return false;
+    }
+  }
+}
+
+// The same for a whole warp: every lane returns the same answer, so the
+// warp-collective tensor-memory loads that follow run converged.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* tl) {
+  return !__any_sync(0xffffffffu, !wait_or_abort(bar, parity, tl));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    qlinear_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  Tail* tl = reinterpret_cast<Tail*>(ops + kStages * kStage);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ntiles_m = (p.M + kBM - 1) / kBM, ntiles_n = (p.N + kBN - 1) / kBN;
+  const int ntiles = ntiles_m * ntiles_n;
+  const int KT = p.K / kBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&tl->full[s], 1);
+      mbar_init(&tl->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tl->acc_full[a], 1);
+      mbar_init(&tl->acc_empty[a], 128);
+    }
+    tl->abort = 0u;
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&tl->tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tl->tmem_slot;
+
+  if (warp == kMmaWarp) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, true);
+      const uint64_t desc0 = sdesc_k_sw128(smem_u32(ops));
+      uint32_t s = 0, ph = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+        const uint32_t a = it & 1u, use = it >> 1;
+        if (use >= 1 && !wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, tl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t acc = tmem + a * kBN;
+        for (int kb = 0; kb < KT; ++kb) {
+          if (!wait_or_abort(&tl->full[s], ph, tl)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(kStage)) >> 4);
+          const uint64_t bd = ad + (kATile >> 4);
+          umma_f16(acc, ad, bd, kIdesc, kb != 0);
+          umma_f16(acc, ad + 2, bd + 2, kIdesc, 1u);           // +32 bytes of K per step
+          umma_f16(acc, ad + 4, bd + 4, kIdesc, 1u);
+          umma_f16(acc, ad + 6, bd + 6, kIdesc, 1u);
+          umma_commit(&tl->empty[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        if (ok) umma_commit(&tl->acc_full[a]);
+      }
+      if (!ok) atomicOr(p.err, 2u);
+    }
+  } else if (warp == kTmaWarp) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      uint32_t s = 0, ph = 0;
+      bool first = true, ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+        for (int kb = 0; kb < KT; ++kb) {
+          if (!first && !wait_or_abort(&tl->empty[s], ph ^ 1u, tl)) { ok = false; break; }
+          uint8_t* st = ops + s * kStage;
+          mbar_arrive_expect_tx(&tl->full[s], kStage);
+          tma_load_2d(st, &tmA, kb * kBK, mt * kBM, &tl->full[s]);
+          tma_load_2d(st + kATile, &tmB, kb * kBK, nt * kBN, &tl->full[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; first = false; }
+        }
+      }
+      if (!ok) atomicOr(p.err, 16u);
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int q = warp;                     // TMEM lane quadrant
+    const int r = 32 * q + lane;            // row within the tile
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const uint32_t a = it & 1u, use = it >> 1;
+      if (!warp_wait(&tl->acc_full[a], use & 1, tl)) {
+        if (lane == 0) atomicOr(p.err, 4u);
+        break;
+      }
+      tc_fence_after();
+      const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+      const int m = mt * kBM + r;
+#pragma unroll 1
+      for (int cc = 0; cc < kBN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + a * kBN + 32 * cc, v);
+        tmem_wait_ld();
+        const int nb = nt * kBN + 32 * cc;
+        if (m >= p.M || nb >= p.N) continue;
+        uint16_t* dst = p.Y + static_cast<long long>(m) * p.N + nb;
+        if (nb + 32 <= p.N) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * __ldg(p.scale + nb + 2 * j),
+                                                           __uint_as_float(v[2 * j + 1]) * __ldg(p.scale + nb + 2 * j + 1));
+            packed[j] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (nb + j < p.N)
+              dst[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * p.scale[nb + j]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tl->acc_empty[a]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// int8 [n] -> bf16 [n], 16 values per thread (16 bytes in, 32 bytes out).
+__global__ void __launch_bounds__(256) widen_int8_kernel(const int8_t* q, long long groups, uint16_t* out) {
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(q) + g);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float f0 = static_cast<float>(static_cast<int8_t>((w[i] >> (16 * h)) & 0xFFu));
+        const float f1 = static_cast<float>(static_cast<int8_t>((w[i] >> (16 * h + 8)) & 0xFFu));
+        const __nv_bfloat162 b = __floats2bfloat162_rn(f0, f1);
+        o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out) + 2 * g;
+    __stcg(dst, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcg(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 [rows, K] K-major, box = 64 x box_rows, 128B swizzle.
+int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return RBQ_ECUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
+}
+
+cudaMemPool_t workspace_pool(int dev) {
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
+}  // namespace q8fast
+
+bool qlinear_int8_fast_eligible(int M, int N, int K) {
+  return M >= 1 && N >= 8 && (N % 8) == 0 && K >= 64 && (K % 64) == 0;
+}
+
+int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float* scale, int M, int N, int K,
+                             uint16_t* Y, unsigned int* err, cudaStream_t st) {
+  using namespace q8fast;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return RBQ_EINVAL;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaMemPool_t pool = workspace_pool(dev);
+  if (!pool) return RBQ_ECUDA;
+  void* ws = nullptr;
+  e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K * 2, pool, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint16_t* wb = static_cast<uint16_t*>(ws);
+  const long long groups = static_cast<long long>(N) * K / 16;
+  long long blocks = (groups + 255) / 256;
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  widen_int8_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(Wq, groups, wb);
+  int rc = RBQ_OK;
+  if ((e = cudaGetLastError()) != cudaSuccess) rc = cuda_fail(e);
+  CUtensorMap mA, mB;
+  if (rc == RBQ_OK) rc = encode_bf16_map(&mA, Xrot, M, K, kBM);
+  if (rc == RBQ_OK) rc = encode_bf16_map(&mB, wb, N, K, kBN);
+  if (rc == RBQ_OK) {
+    Params p{M, N, K, scale, Y, err};
+    auto kern = qlinear_bf16_kernel;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    if (e != cudaSuccess) {
+      rc = cuda_fail(e);
+    } else {
+      const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+      kern<<<ntiles < sms ? ntiles : sms, kThreads, kSmem, st>>>(mA, mB, p);
+      if ((e = cudaGetLastError()) != cudaSuccess) rc = cuda_fail(e);
+    }
+  }
+  e = cudaFreeAsync(ws, st);
+  if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
+  return rc;
+}
+
+}  // namespace rbq
