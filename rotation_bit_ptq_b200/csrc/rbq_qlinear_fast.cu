@@ -13,31 +13,30 @@
 //    GEMM instead would redo that work for every 128-row tile of tokens and
 //    saturate the SM's integer pipe.
 // 2. qlinear_fast_kernel: each CTA (one per SM) walks a static list of
-//    128 x 192 output tiles.
+//    128 x 256 output tiles.
 //      warps 0..3  epilogue: TMEM lane quadrant w, one output row per thread;
 //                  scale by s_m r'_n / K, round to BF16, store.
 //      warp 4      MMA issuer: one thread waits for a filled operand stage,
-//                  issues four 128x192x16 kind::f16 MMAs (A from tensor
-//                  memory, B from shared memory) into the tile's TMEM
-//                  accumulator, commits them to the stage's "empty" barrier,
-//                  and after the last K slice commits the accumulator.
+//                  issues four 128x256x16 kind::f16 MMAs (both operands from
+//                  shared memory) into the tile's TMEM accumulator, commits
+//                  them to the stage's "empty" barrier, and after the last K
+//                  slice commits the accumulator.  Its own instruction latency
+//                  sets the pace, so stage indices and phases advance
+//                  incrementally and a completed barrier costs one try_wait.
 //      warp 5      TMA producer: one thread loads (a) the activation codes of
 //                  two K slices for the tile's 128 rows into a ring of code
-//                  stages and (b) the 192 x 64 fp16 weight tile of each K
+//                  stages and (b) the 256 x 64 fp16 weight tile of each K
 //                  slice straight into the operand stage, 128B-swizzled as the
 //                  tensor core reads it.
-//      warps 6..13 activation expansion, two threads per row (row = the
-//                  thread's TMEM lane; warps w and w+4 take the two halves of
-//                  the row's 64 codes): read the codes of a K slice from the
-//                  code stage, turn them into fp16 levels before waiting for
-//                  the stage, then store them into 16 of the stage's 32 TMEM
-//                  columns with one tcgen05.st.
-//    Tensor memory: two accumulators (2 x 192 columns, so the epilogue of
-//    tile i overlaps the MMAs of tile i+1) and four A stages (4 x 32).
-//    Keeping A out of shared memory matters: per K slice the weight tile is
-//    written by TMA and read by the MMA (48 KB), and an A tile in shared
-//    memory would add another 32 KB of stores and reads to a port that
-//    moves 128 bytes per cycle.
+//      warps 6..13 activation expansion, two threads per row (warps w and
+//                  w+4 take the two halves of the row's 64 codes): read the
+//                  codes of a K slice from the code stage, turn them into
+//                  fp16 levels before waiting for the stage, then write them
+//                  into the stage's swizzled K-major A tile.
+//    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
+//    overlap the MMAs of tile i+1.  (A variant that kept the activation tile
+//    in tensor memory, written with tcgen05.st, measured slower: the stores
+//    cost more than the shared-memory traffic they save.)
 
 // 4-bit codes are expanded in registers: by symmetry C[15-c] = -C[c], the
 // magnitude index m (0..7) selects the two bytes of |C| with byte permutes
@@ -70,15 +69,13 @@ namespace qfast {
 
 using namespace sm100;
 
-constexpr int kBM = 128, kBN = 192, kBK = 64;
-constexpr int kBTile = kBN * kBK * 2;          // 24 KB fp16 (weights, shared memory)
-constexpr int kOpStage = kBTile;
-// Tensor memory (512 columns): two fp32 accumulators of kBN columns, then
-// the activation operand stages, 32 columns (64 fp16 of K) each.
-constexpr uint32_t kACol = 2 * kBN;            // 384
-constexpr uint32_t kAStageCols = kBK / 2;      // 32
-constexpr int kAStages = 4;                    // kACol + kAStages * kAStageCols == 512
-constexpr int kMaxF = kAStages, kMaxC = 8;     // operand stages (A in TMEM, B in smem), code stages
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kATile = kBM * kBK * 2;          // 16 KB fp16 activation tile
+constexpr int kBTile = kBN * kBK * 2;          // 32 KB fp16 weight tile
+constexpr int kOpStage = kATile + kBTile;      // 48 KB per operand stage (shared memory)
+constexpr int kAStages = 4;
+constexpr int kMaxF = kAStages, kMaxC = 8;     // operand stages, code stages
+// Tensor memory: two fp32 accumulators of kBN columns (512 columns).
 constexpr int kThreads = 448;                  // 14 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
 constexpr int kExpandFirst = 192;              // warp 6
@@ -251,15 +248,15 @@ __device__ __forceinline__ void read_slice(const uint8_t* part, const CodeGeo& g
 }
 
 // Waits on a barrier for the whole warp: every lane returns the same answer,
-// so the warp-collective tensor-memory stores that follow run converged.
+// so a warp leaves its loop together (the epilogue's warp-collective
+// tensor-memory loads rely on this).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* tl) {
   return !__any_sync(0xffffffffu, !wait_or_abort(bar, parity, tl));
 }
 
-// Row r = 32 (warp % 4) + lane of every activation tile: the thread's own
-// tensor-memory lane, which `tA` addresses.
+// Row r = 32 (warp % 4) + lane of every activation tile, code half HF.
 template <int BITS, int HF>
-__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* codes, int r, uint32_t tA,
+__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, int r,
                                             int ntiles, Planes4 P, const uint16_t* lut) {
   const CodeGeo& g = p.ga;
   const int KP = p.K / (2 * kBK);
@@ -277,10 +274,12 @@ __device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* 
         uint32_t w[16];
         expand_row<BITS, HF>(cur, P, lut, w);          // before the wait: off the critical path
         if (!a_first && !warp_wait(&tl->empty[s], aph ^ 1u, tl)) return;
-        tc_fence_after();
-        tmem_st16(tA + s * kAStageCols + 16 * HF, w);
-        tmem_wait_st();
-        tc_fence_before();
+        uint8_t* tile = ops + s * kOpStage;            // the stage's A tile, 128B-swizzled K-major
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(tile + sw128_offset(r, 4 * HF + c)) =
+              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        fence_proxy_async_smem();                      // visible to the tensor core
         mbar_arrive(&tl->full[s]);
         if (++s == kAStages) { s = 0; aph ^= 1u; a_first = false; }
       }
@@ -353,12 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = tmem + kACol + s * kAStageCols;             // A: tensor memory
-          const uint64_t b0 = bdesc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);   // B: shared memory
-          umma_f16_ta(acc, a0, b0, kIdesc, kb != 0);
-          umma_f16_ta(acc, a0 + 8, b0 + 2, kIdesc, 1u);                  // +32 bytes of K per step
-          umma_f16_ta(acc, a0 + 16, b0 + 4, kIdesc, 1u);
-          umma_f16_ta(acc, a0 + 24, b0 + 6, kIdesc, 1u);
+          const uint64_t a0 = bdesc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);   // A, then B
+          const uint64_t b0 = a0 + (kATile >> 4);
+          umma_f16(acc, a0, b0, kIdesc, kb != 0);
+          umma_f16(acc, a0 + 2, b0 + 2, kIdesc, 1u);                      // +32 bytes of K per step
+          umma_f16(acc, a0 + 4, b0 + 4, kIdesc, 1u);
+          umma_f16(acc, a0 + 6, b0 + 6, kIdesc, 1u);
           umma_commit(&tl->empty[s]);
           if (++s == F) { s = 0; ph ^= 1u; }
         }
@@ -399,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&tl->full[s], kBTile);
-            tma_load_2d(ops + s * kOpStage, &tmB, (2 * kp + h) * kBK, nt * kBN, &tl->full[s]);
+            tma_load_2d(ops + s * kOpStage + kATile, &tmB, (2 * kp + h) * kBK, nt * kBN, &tl->full[s]);
             if (++s == F) { s = 0; ph ^= 1u; b_first = false; }
           }
         }
@@ -460,30 +459,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- activation expansion ----------------
     // warps 6..13: lane quarter warp % 4, code half (warp - 6) / 4
     const int r = 32 * (warp & 3) + lane;
-    const uint32_t tA = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kACol;
     const uint16_t* lut = tl->lut_a;
     const Planes4 P = make_planes4(lut);
     if (warp < 10) {
       switch (p.bits_a) {
-        case 1: expand_loop<1, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 2: expand_loop<2, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 3: expand_loop<3, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 4: expand_loop<4, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 5: expand_loop<5, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 6: expand_loop<6, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 7: expand_loop<7, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        default: expand_loop<8, 0>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 1: expand_loop<1, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 2: expand_loop<2, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 3: expand_loop<3, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 4: expand_loop<4, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 5: expand_loop<5, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 6: expand_loop<6, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 7: expand_loop<7, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        default: expand_loop<8, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
       }
     } else {
       switch (p.bits_a) {
-        case 1: expand_loop<1, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 2: expand_loop<2, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 3: expand_loop<3, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 4: expand_loop<4, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 5: expand_loop<5, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 6: expand_loop<6, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        case 7: expand_loop<7, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
-        default: expand_loop<8, 1>(p, tl, codes, r, tA, ntiles, P, lut); break;
+        case 1: expand_loop<1, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 2: expand_loop<2, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 3: expand_loop<3, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 4: expand_loop<4, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 5: expand_loop<5, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 6: expand_loop<6, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        case 7: expand_loop<7, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
+        default: expand_loop<8, 1>(p, tl, ops, codes, r, ntiles, P, lut); break;
       }
     }
     if (tl->abort && r == 0 && warp < 10) atomicOr(p.err, 8u);
