@@ -78,7 +78,6 @@ constexpr int kMaxF = kAStages, kMaxC = 8;     // operand stages, code stages
 // Tensor memory: two fp32 accumulators of kBN columns (512 columns).
 constexpr int kThreads = 448;                  // 14 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
-constexpr int kExpandFirst = 192;              // warp 6
 constexpr int kExpandThreads = 2 * kBM;        // two threads per activation row (32 codes each)
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -642,10 +641,40 @@ __global__ void __launch_bounds__(256) expand_weights_kernel8(const uint8_t* cod
   }
 }
 
+// 4-bit codes: one thread per 32 codes (16 bytes in, 64 bytes out).
+__global__ void __launch_bounds__(256) expand_weights_kernel4x32(const uint4* codes, long long groups,
+                                                                const uint16_t* lut_g, uint4* out) {
+  Planes4 P;
+  {
+    uint16_t lut[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) lut[i] = __ldg(lut_g + i);
+    P = make_planes4(lut);
+  }
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldcs(codes + g);
+    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t w[4];
+      expand8_4bit(x[i], P, w);
+      __stcg(out + 4 * g + i, make_uint4(w[0], w[1], w[2], w[3]));
+    }
+  }
+}
+
 template <int BITS>
 int launch_expand(const uint8_t* codes, int rows, int K, const uint16_t* lut, uint16_t* out, cudaStream_t st,
                   int sms) {
-  if constexpr (8 % BITS == 0) {
+  if constexpr (BITS == 4) {
+    // K is a multiple of 128, so every row holds whole 32-code groups
+    const long long groups = static_cast<long long>(rows) * (K / 32);
+    long long blocks = (groups + 255) / 256;
+    if (blocks > 16LL * sms) blocks = 16LL * sms;
+    expand_weights_kernel4x32<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint4*>(codes),
+                                                                         groups, lut, reinterpret_cast<uint4*>(out));
+  } else if constexpr (8 % BITS == 0) {
     const long long groups = static_cast<long long>(rows) * (K / 8);
     long long blocks = (groups + 255) / 256;
     if (blocks > 16LL * sms) blocks = 16LL * sms;
