@@ -252,6 +252,22 @@ const char* rbq_error_string(int code);
  */
 int rbq_device_error(void* stream);
 
+/*
+ * rbq_selftest_wait_limit -- launch, on `stream`, one CTA whose shared-memory
+ * barriers nothing ever arrives at, so that each of the library's three
+ * bounded-wait forms runs out: bit 0 of *out = a single thread's wait gave up,
+ * bit 1 = a wait sharing the CTA's give-up flag gave up, bit 2 = a whole
+ * warp's uniform wait gave up, bit 3 = the give-up flag was raised.  A clean
+ * run leaves *out == 15 and the device error word set, so the next
+ * rbq_device_error() returns RBQ_EDEVICE (and clears it).  The kernel ends by
+ * itself after about a second of waiting; no other state is touched.
+ * (Not a step of the method: it checks the failure handling of the kernels.)
+ *
+ * out: DEVICE pointer to one caller-allocated unsigned int, 4-byte aligned.
+ * Errors: RBQ_EINVAL (NULL), RBQ_EALIGN, RBQ_ECUDA.
+ */
+int rbq_selftest_wait_limit(unsigned int* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

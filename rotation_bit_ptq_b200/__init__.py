@@ -38,6 +38,7 @@ SIGNATURES = {
     "qlinear_noalloc": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
+    "rbq_selftest_wait_limit": (_I, [_P, _P]),
     "rbq_code_grid": (_I, [_I, _I, _I, _P, _P, _P, _P]),
 }
 
@@ -291,3 +292,13 @@ def code_grid(d, bits, variant=0):
 def device_error(stream=None):
     """Synchronise and read/clear the library's device error word (0 = clean)."""
     return lib().rbq_device_error(_stream(stream))
+
+
+def selftest_wait_limit(out, stream=None):
+    """Launch the kernel whose barriers nothing arrives at, so that every
+    bounded-wait form gives up (about a second); ``out`` is a CUDA int32[1]
+    that receives the bit mask of the waits that gave up (15 when all did)."""
+    import torch
+    if not (out.is_cuda and out.dtype == torch.int32 and out.numel() >= 1):
+        raise ValueError("out must be a CUDA int32 tensor with at least one element")
+    _check(lib().rbq_selftest_wait_limit(_P(out.data_ptr()), _stream(stream)), "rbq_selftest_wait_limit")

@@ -118,15 +118,7 @@ struct __align__(8) Tail {
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
-  const long long t0 = clock64();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (tl->abort) return false;
-    if (clock64() - t0 > (1ll << 31) || i > (1u << 26)) {
-      tl->abort = 1u;
-      return false;
-    }
-  }
+  return mbar_wait_or_abort(bar, parity, &tl->abort);
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -250,7 +242,7 @@ __device__ __forceinline__ void read_slice(const uint8_t* part, const CodeGeo& g
 // so a warp leaves its loop together (the epilogue's warp-collective
 // tensor-memory loads rely on this).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* tl) {
-  return !__any_sync(0xffffffffu, !wait_or_abort(bar, parity, tl));
+  return mbar_warp_wait(bar, parity, &tl->abort);
 }
 
 // Row r = 32 (warp % 4) + lane of every activation tile, code half HF.

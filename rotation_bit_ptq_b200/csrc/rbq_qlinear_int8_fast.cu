@@ -65,22 +65,10 @@ struct __align__(8) Tail {
 constexpr size_t kSmem = 1024 + kStages * kStage + sizeof(Tail) + 64;
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (tl->abort) return false;
-    if (clock64() - t0 > (1ll << 31) || i > (1u << 26)) {
-      tl->abort = 1u;
-      return false;
-    }
-  }
+  return mbar_wait_or_abort(bar, parity, &tl->abort);
 }
-
-// The same for a whole warp: every lane returns the same answer, so the
-// warp-collective tensor-memory loads that follow run converged.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* tl) {
-  return !__any_sync(0xffffffffu, !wait_or_abort(bar, parity, tl));
+  return mbar_warp_wait(bar, parity, &tl->abort);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

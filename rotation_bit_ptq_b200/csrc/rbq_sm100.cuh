@@ -40,6 +40,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
   return false;
 }
+// Bounded wait for the warps of one CTA that share a give-up flag: returns
+// false as soon as another waiter has raised `*abort`, or after the same limits
+// as mbar_wait, raising `*abort` itself so that the CTA's other waiters leave
+// too instead of each spending its own second.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity, volatile uint32_t* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > (1ll << 31) || i > (1u << 26)) {
+      *abort = 1u;
+      return false;
+    }
+  }
+}
+// The same for a whole warp: every lane returns the same answer, so the
+// warp-collective tensor-memory operations after it run converged.
+__device__ __forceinline__ bool mbar_warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort) {
+  return !__any_sync(0xffffffffu, !mbar_wait_or_abort(bar, parity, abort));
+}
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
