@@ -5,6 +5,7 @@
 // structure and §6.3 for reproducible random draws; §1 and §4.2 for the
 // per-d Lloyd-Max codebook of N(0, 1/d).
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -355,6 +356,15 @@ int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out) {
   return RBQ_OK;
 }
 
+// The grid with kGridGuard copies of each end entry outside it, padded with
+// one more copy of the last entry to an even count.
+std::vector<float2> guarded(const std::vector<float2>& lut) {
+  const int n = static_cast<int>(lut.size());
+  std::vector<float2> g(guarded_grid_entries(n));
+  for (int i = 0; i < static_cast<int>(g.size()); ++i) g[i] = lut[std::min(std::max(i - kGridGuard, 0), n - 1)];
+  return g;
+}
+
 int codebook_device(int d, int bits, const CodebookDevice** out) {
   int dev;
   int rc = current_device(&dev);
@@ -385,10 +395,14 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
   cb->grid_cells = grid.cells;
   cb->grid_scale = static_cast<float>(1.0 / (2.0 * grid.R));
   if ((rc = upload(grid.lut.data(), grid.lut.size(), &cb->grid)) != RBQ_OK) { delete cb; return rc; }
+  std::vector<float2> pad = guarded(grid.lut);
+  if ((rc = upload(pad.data(), pad.size(), &cb->grid_pad)) != RBQ_OK) { delete cb; return rc; }
   Grid full;
   if (build_grid_full(bounds, kMaxFullGridCells, &full) == RBQ_OK) {
     cb->grid_full_cells = full.cells;
     if ((rc = upload(full.lut.data(), full.lut.size(), &cb->grid_full)) != RBQ_OK) { delete cb; return rc; }
+    pad = guarded(full.lut);
+    if ((rc = upload(pad.data(), pad.size(), &cb->grid_full_pad)) != RBQ_OK) { delete cb; return rc; }
   }
   std::lock_guard<std::mutex> lk(g_mu);
   auto ins = cb_cache().emplace(key, cb);
@@ -397,6 +411,8 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
     cudaFree(cb->levels_f16);
     cudaFree(cb->grid);
     cudaFree(cb->grid_full);
+    cudaFree(cb->grid_pad);
+    cudaFree(cb->grid_full_pad);
     delete cb;
   }
   *out = ins.first->second;

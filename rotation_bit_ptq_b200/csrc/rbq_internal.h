@@ -62,7 +62,16 @@ struct CodebookDevice {
   // need more than kMaxFullGridCells cells.
   float2* grid_full = nullptr;
   int grid_full_cells = 0;
+  // Both grids again with kGridGuard copies of the end entries before and
+  // after, padded to an even entry count, so that one bulk copy (16-byte
+  // multiple) brings a guarded grid into shared memory.
+  float2* grid_pad = nullptr;
+  float2* grid_full_pad = nullptr;
 };
+
+constexpr int kGridGuard = 2;
+// Entries of a guarded grid of n entries (see CodebookDevice::grid_pad).
+__host__ __device__ inline int guarded_grid_entries(int n) { return (n + 2 * kGridGuard + 1) & ~1; }
 
 constexpr int kMaxFullGridCells = 5000;
 

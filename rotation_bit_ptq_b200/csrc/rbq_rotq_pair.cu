@@ -17,11 +17,13 @@
 // a block read the same source position of 8 different rows, which a 16-byte
 // row padding puts in 8 different banks.
 //
-// Data movement: one producer warp streams whole rows with bulk asynchronous
-// copies (TMA, no tensor map needed for contiguous rows) into a ring of tile
-// slots, each completion counted on the slot's mbarrier.  Consumers release a
-// slot as soon as they have gathered from it, so the next tile streams in
-// while the current one is transformed and encoded.
+// Data movement: whole rows arrive by bulk asynchronous copies (TMA, no
+// tensor map needed for contiguous rows), one row per lane of an issuing
+// warp, into a ring of tile slots, each completion counted on the slot's
+// mbarrier.  The gather tables and the code grid are copied first, so they are
+// not queued behind the tiles.  The last warp done gathering from a slot
+// refills it with a later tile, so the next tiles stream in while the current
+// one is transformed and encoded.
 //
 // Norm: the rotation is orthogonal, so ||Pi x|| = ||x||; every thread sums the
 // squares of the 64 inputs it gathered (each input lands in exactly one
@@ -50,7 +52,6 @@ enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
 
 constexpr int kRows = 16;            // tokens per tile
 constexpr int kMaxWarps = 12;        // consumer warps (d <= 3072)
-constexpr int kGuard = 2;            // grid entries past each end
 constexpr size_t kSmemLimit = 227 * 1024;
 
 struct Params {
@@ -61,8 +62,8 @@ struct Params {
   int NS;                            // ring slots
   uint32_t pitch;                    // bytes per staged row (2d + 16)
   const uint32_t* tab;               // 2 d words: offsets, then sign words (pair_tab_slot order)
-  const float2* grid;                // Lloyd-Max modes: cells + 1 entries
-  int grid_n;
+  const float2* grid;                // Lloyd-Max modes: guarded grid (kGridGuard entries each side)
+  int grid_n;                        // entries of the unguarded grid (cells + 1)
   float grid_cells, grid_scale;      // full grid: scale unused
   void* out;
   void* aux;
@@ -81,11 +82,11 @@ __host__ __device__ inline Layout layout(int d, int NS, int grid_n) {
   L.off = L.ring + NS * kRows * pitch;
   L.sgn = L.off + 4u * d;
   L.grid = L.sgn + 4u * d;
-  L.part = (L.grid + 8u * (grid_n + 2 * kGuard) + 15u) & ~15u;
+  L.part = (L.grid + 8u * guarded_grid_entries(grid_n) + 15u) & ~15u;
   L.bars = L.part + 4u * (2 * NS) * kRows * kMaxWarps;   // [2NS][16 tokens][12 warps]
   L.bars = (L.bars + 7u) & ~7u;
-  // full[NS], red[2NS], tab | cnt[NS], issued[NS], TMEM base
-  L.total = L.bars + 8u * (NS + 2 * NS + 1) + 8u * NS + 8u;
+  // full[NS], red[2NS], tab | TMEM base
+  L.total = L.bars + 8u * (NS + 2 * NS + 1) + 8u;
   return L;
 }
 
@@ -292,9 +293,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* red = full + p.NS;
   uint64_t* tabbar = red + 2 * p.NS;
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(tabbar + 1);        // readers done, per slot
-  uint32_t* issued = cnt + p.NS;                                   // tiles issued, per slot
-  uint32_t* tmem_slot = issued + p.NS;                             // TMEM base address
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tabbar + 1);  // TMEM base address
   constexpr bool kLloyd = (MODE == kAct || MODE == kWeightLM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nthreads_c = p.nwarps * 32;
@@ -304,43 +303,37 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   const uint32_t slot_bytes = kRows * pitch;
   const uint32_t ring = sbase + L.ring;
 
-  // Bulk-copies tile `tile` into slot `slot`; counted on full[slot].
-  auto issue = [&](int tile, int slot) {
-    const size_t row_bytes = 2 * static_cast<size_t>(p.d);
+  // The bulk copies of tile `tile` into slot `slot`, shared out over the
+  // CTA: row r is copied by lane r / nwarps of warp r % nwarps (at most a few
+  // copies per warp, so no warp stalls long on the copy engine), and thread 0
+  // posts the expected bytes.  Every thread calls it at the same points, in
+  // slot order 0, 1, ..., NS-1, 0, ..., and counts the calls.
+  int n_issued = 0;
+  auto issue_rows = [&](int tile, int slot) {
+    const uint32_t row_bytes = 2u * static_cast<uint32_t>(p.d);
     const long long r0 = static_cast<long long>(tile) * kRows;
     const int rows = static_cast<int>(min(static_cast<long long>(kRows), p.T - r0));
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    ++issued[slot];
-    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(rows * row_bytes));
-    for (int r = 0; r < rows; ++r)
-      bulk_load(ring + slot * slot_bytes + r * pitch, p.X + (r0 + r) * p.d, static_cast<uint32_t>(row_bytes),
-                &full[slot]);
+    ++n_issued;
+    if (tid == 0) mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(rows) * row_bytes);
+    for (int r = warp + p.nwarps * lane; r < rows; r += 32 * p.nwarps) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      bulk_load(ring + slot * slot_bytes + r * pitch, p.X + (r0 + r) * p.d, row_bytes, &full[slot]);
+    }
   };
 
-  // ---- prologue: the first tiles and the gather tables start streaming at
-  //      once; the code grid and the partial sums are set up meanwhile ----
+  // ---- prologue: the gather tables and the guarded code grid start streaming
+  //      first; the first tile follows once the barriers are visible to all
+  //      (the other slots fill after it has landed, so that it is not slowed
+  //      by them) ----
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      cnt[s] = 0u;
-      issued[s] = 0u;
-    }
+    for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1);
     for (int r = 0; r < 2 * NS; ++r) mbar_init(&red[r], nthreads_c);
     mbar_init(tabbar, 1);
     mbar_fence_init();
-    mbar_arrive_expect_tx(tabbar, 8u * p.d);
+    const uint32_t gbytes = kLloyd ? 8u * static_cast<uint32_t>(guarded_grid_entries(p.grid_n)) : 0u;
+    mbar_arrive_expect_tx(tabbar, 8u * p.d + gbytes);
     bulk_load(sbase + L.off, p.tab, 8u * p.d, tabbar);
-    for (int s = 0; s < NS; ++s)
-      if (blockIdx.x + s * static_cast<int>(gridDim.x) < p.ntiles) issue(blockIdx.x + s * gridDim.x, s);
-  }
-  if (kLloyd) {
-    float2* g = reinterpret_cast<float2*>(sm + L.grid);
-    const int n = p.grid_n + 2 * kGuard;
-#pragma unroll 4
-    for (int i = tid; i < n; i += blockDim.x) {
-      const int src = min(max(i - kGuard, 0), p.grid_n - 1);
-      g[i] = p.grid[src];
-    }
+    if (kLloyd) bulk_load(sbase + L.grid, p.grid, gbytes, tabbar);
   }
   {
     float* part = reinterpret_cast<float*>(sm + L.part);
@@ -354,6 +347,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (blockIdx.x < p.ntiles) issue_rows(blockIdx.x, 0);
   if (!mbar_wait(tabbar, 0)) atomicOr(p.err, 256u);
 
   // ---------------- consumers ----------------
@@ -363,7 +357,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   const uint32_t off_addr = sbase + L.off + 256u * b;
   const uint32_t sgn_addr = sbase + L.sgn + 256u * b;
   const uint32_t part_addr = sbase + L.part;
-  const uint32_t gbase = sbase + L.grid + 8u * kGuard - 0x4B000000u * 8u;
+  const uint32_t gbase = sbase + L.grid + 8u * kGridGuard - 0x4B000000u * 8u;
   const uint32_t pitch8 = 8u * pitch;
   // Tensor memory: each thread parks its pair's two half-blocks (2 x 64 words)
   // in its own lane; warps w, w+4, w+8 share a lane quarter, 128 columns each.
@@ -375,6 +369,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     // A timed-out wait ends the whole warp's loop together: the tensor-memory
     // accesses below are warp-collective (.sync.aligned).
     if (__any_sync(0xffffffffu, !mbar_wait(&full[s], (it / NS) & 1))) { atomicOr(p.err, 64u); break; }
+    if (it == 0)
+      for (int s2 = 1; s2 < NS; ++s2)
+        if (blockIdx.x + s2 * static_cast<int>(gridDim.x) < p.ntiles) issue_rows(blockIdx.x + s2 * gridDim.x, s2);
 
     // ---- gather x[pi(k)] with D_k folded in (tokens p, p+8), one half-block
     //      at a time; butterfly strides 1..16 inside each half; park in TMEM ----
@@ -400,18 +397,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
         }
       }
       if (h == 1) {
-        // The last thread done with the slot's rows refills it with the tile
-        // NS steps ahead (release/acquire through the counter orders every
-        // read before the asynchronous overwrite).
-        uint32_t prev;
-        asm volatile("atom.release.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(prev) : "r"(smem_u32(&cnt[s]))
-                     : "memory");
-        if (prev == static_cast<uint32_t>(nthreads_c - 1)) {
-          asm volatile("fence.acq_rel.cta;" ::: "memory");
-          cnt[s] = 0u;
-          const int nxt = tile + NS * static_cast<int>(gridDim.x);
-          if (nxt < p.ntiles) issue(nxt, s);
-        }
         if constexpr (MODE != kInt8) {
           // ||x||^2 partials of both tokens (||Pi x|| = ||x||): 4 lanes share a pair
           float a0, a1;
@@ -483,6 +468,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
 
     // ---- per-token totals: fixed summation order, identical in every thread ----
     if (__any_sync(0xffffffffu, !mbar_wait(&red[rb], (it / (2 * NS)) & 1))) { atomicOr(p.err, 64u); break; }
+    // Every thread arrived on red[rb] after its last read of slot s, so the
+    // slot can take the tile NS steps ahead (the barrier's release/acquire
+    // orders those reads before the asynchronous overwrite).
+    if (tile + NS * static_cast<int>(gridDim.x) < p.ntiles) issue_rows(tile + NS * gridDim.x, s);
     float tot[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -622,14 +611,18 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     }
   }
 
-  // Every bulk copy this CTA issued has landed before it exits (they all have
-  // on the normal path; after a timed-out wait this bounds the exit).
+  // Every bulk copy this CTA issued has landed before it exits: each thread
+  // that copies rows waits for the last phase of every slot it wrote (they
+  // all have landed on the normal path; after a timed-out wait, when the
+  // threads may have left the loop at different tiles, this bounds the exit).
   tc_fence_before();
   __syncthreads();
-  if (tid == 0) {
+  if (warp + p.nwarps * lane < kRows) {
     bool ok = true;
-    for (int s = 0; s < NS; ++s)
-      if (issued[s] && !mbar_wait(&full[s], (issued[s] - 1) & 1)) ok = false;
+    for (int s = 0; s < NS; ++s) {
+      const int uses = n_issued > s ? (n_issued - 1 - s) / NS + 1 : 0;
+      if (uses && !mbar_wait(&full[s], (uses - 1) & 1)) ok = false;
+    }
     if (!ok) atomicOr(p.err, 128u);
   }
   __syncwarp();
@@ -719,12 +712,12 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
     if (bits <= 6 && cb->grid_full && slots_that_fit(r->d, cb->grid_full_cells + 1) >= 2) {
       full = true;
-      p.grid = cb->grid_full;
+      p.grid = cb->grid_full_pad;
       p.grid_n = cb->grid_full_cells + 1;
       p.grid_cells = static_cast<float>(cb->grid_full_cells);
       p.grid_scale = 0.5f;
     } else {
-      p.grid = cb->grid;
+      p.grid = cb->grid_pad;
       p.grid_n = cb->grid_cells + 1;
       p.grid_cells = static_cast<float>(cb->grid_cells);
       p.grid_scale = cb->grid_scale;
