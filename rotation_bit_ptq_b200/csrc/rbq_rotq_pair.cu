@@ -42,210 +42,13 @@
 
 #include "rbq_internal.h"
 #include "rbq_sm100.cuh"
+#include "rbq_rowtile.cuh"
 
 namespace rbq {
 namespace pairk {
 
 using namespace sm100;
-
-enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
-
-constexpr int kRows = 16;            // tokens per tile
-constexpr int kMaxWarps = 12;        // consumer warps (d <= 3072)
-constexpr size_t kSmemLimit = 227 * 1024;
-
-struct Params {
-  const __nv_bfloat16* X;
-  long long T;
-  int d, nblk, nwarps;               // consumer warps = nblk / 4
-  int ntiles;                        // ceil(T / 16)
-  int NS;                            // ring slots
-  uint32_t pitch;                    // bytes per staged row (2d + 16)
-  const uint32_t* tab;               // 2 d words: offsets, then sign words (pair_tab_slot order)
-  const float2* grid;                // Lloyd-Max modes: guarded grid (kGridGuard entries each side)
-  int grid_n;                        // entries of the unguarded grid (cells + 1)
-  float grid_cells, grid_scale;      // full grid: scale unused
-  void* out;
-  void* aux;
-  unsigned int* err;
-};
-
-// Shared-memory layout (bytes from the 128-aligned base).
-struct Layout {
-  uint32_t ring, off, sgn, grid, part, bars, total;
-};
-
-__host__ __device__ inline Layout layout(int d, int NS, int grid_n) {
-  Layout L{};
-  const uint32_t pitch = 2u * d + 16u;
-  L.ring = 0;
-  L.off = L.ring + NS * kRows * pitch;
-  L.sgn = L.off + 4u * d;
-  L.grid = L.sgn + 4u * d;
-  L.part = (L.grid + 8u * guarded_grid_entries(grid_n) + 15u) & ~15u;
-  L.bars = L.part + 4u * (2 * NS) * kRows * kMaxWarps;   // [2NS][16 tokens][12 warps]
-  L.bars = (L.bars + 7u) & ~7u;
-  // full[NS], red[2NS], tab | TMEM base
-  L.total = L.bars + 8u * (NS + 2 * NS + 1) + 8u;
-  return L;
-}
-
-__device__ __forceinline__ unsigned long long pk(float a, float b) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void upk(unsigned long long r, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
-}
-__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-// 0xFFFFFFFF if a >= b else 0 (IEEE: -0 >= -0; NaN never)
-__device__ __forceinline__ uint32_t set_ge(float a, float b) {
-  uint32_t d;
-  asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(d) : "f"(a), "f"(b));
-  return d;
-}
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
-  float d;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// Whole contiguous row, global -> shared, completion counted in bytes on `bar`.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-// bf16 bits (low 16 of u) -> fp32 with the sign word S (0 or 0x80000000)
-// folded in: (u << 16) + S flips the sign bit exactly when S is set.
-__device__ __forceinline__ float bf16_signed(uint32_t u, uint32_t S) { return __uint_as_float(u * 65536u + S); }
-
-
-__device__ __forceinline__ unsigned long long pk_u(uint32_t a, uint32_t b) {
-  return pk(__uint_as_float(a), __uint_as_float(b));
-}
-__device__ __forceinline__ void upk_u(unsigned long long r, uint32_t& a, uint32_t& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(r));
-}
-__device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Code of each half of a packed pair z (two tokens) from the shared-memory
-// grid.  Full-range grid: n = round((v + 1)/2 * cells) through the +2^23
-// trick, code = base + (v >= thr).  Clamped grid over [-R, R]: u = sat(v/(2R)
-// + 1/2), n = round(u * cells), code = base + 1 + sign(z * inv - thr).
-template <bool FULL>
-struct Enc;
-
-template <>
-struct Enc<true> {
-  unsigned long long kq2, cq2, inv2;
-  uint32_t gbase;
-  __device__ __forceinline__ Enc(float inv0, float inv1, float cells, float, uint32_t gb) : gbase(gb) {
-    const float hc = 0.5f * cells;
-    kq2 = pk(inv0 * hc, inv1 * hc);
-    cq2 = pk(hc + 8388608.0f, hc + 8388608.0f);
-    inv2 = pk(inv0, inv1);
-  }
-  __device__ __forceinline__ void codes(unsigned long long z, uint32_t& c0, uint32_t& c1) const {
-    float q0, q1, v0, v1;
-    upk(fma2(z, kq2, cq2), q0, q1);
-    upk(mul2(z, inv2), v0, v1);
-    const float2 e0 = lds_f2(gbase + __float_as_uint(q0) * 8u);
-    const float2 e1 = lds_f2(gbase + __float_as_uint(q1) * 8u);
-    c0 = __float_as_uint(e0.y) - set_ge(v0, e0.x);
-    c1 = __float_as_uint(e1.y) - set_ge(v1, e1.x);
-  }
-};
-
-template <>
-struct Enc<false> {
-  float A0, A1, inv0, inv1, cells;
-  uint32_t gbase;
-  __device__ __forceinline__ Enc(float i0, float i1, float nc, float scale, uint32_t gb)
-      : A0(i0 * scale), A1(i1 * scale), inv0(i0), inv1(i1), cells(nc), gbase(gb) {}
-  __device__ __forceinline__ void codes(unsigned long long z, uint32_t& c0, uint32_t& c1) const {
-    float z0, z1;
-    upk(z, z0, z1);
-    const float qf0 = fmaf(fma_sat(z0, A0, 0.5f), cells, 8388608.0f);
-    const float qf1 = fmaf(fma_sat(z1, A1, 0.5f), cells, 8388608.0f);
-    const float2 e0 = lds_f2(gbase + __float_as_uint(qf0) * 8u);
-    const float2 e1 = lds_f2(gbase + __float_as_uint(qf1) * 8u);
-    const int below0 = __float_as_int(fmaf(z0, inv0, -e0.x)) >> 31;
-    const int below1 = __float_as_int(fmaf(z1, inv1, -e1.x)) >> 31;
-    c0 = static_cast<uint32_t>(__float_as_int(e0.y) + 1 + below0);
-    c1 = static_cast<uint32_t>(__float_as_int(e1.y) + 1 + below1);
-  }
-};
-
-// Packs `code` (already < 2^BITS) into bit i*BITS of the word array w.
-template <int BITS>
-__device__ __forceinline__ void put_code(uint32_t* w, int i, uint32_t code) {
-  const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
-  if constexpr ((32 % BITS) == 0) {
-    w[wi] += code << sh;                     // disjoint fields: add = or
-  } else {
-    w[wi] |= code << sh;
-    if (sh + BITS > 32) w[wi + 1] |= code >> (32 - sh);
-  }
-}
-
-template <int BITS>
-__device__ __forceinline__ void store_codes(unsigned char* dst, const uint32_t* w) {
-  if constexpr ((BITS % 2) == 0) {
-#pragma unroll
-    for (int i = 0; i < BITS / 2; ++i)
-      __stcs(reinterpret_cast<uint4*>(dst) + i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
-  } else {
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) __stcs(reinterpret_cast<uint2*>(dst) + i, make_uint2(w[2 * i], w[2 * i + 1]));
-  }
-}
-
+using namespace rowtile;
 
 // Codes of one block for both tokens: the last butterfly stage (stride 32)
 // runs here, on half-blocks read back from tensor memory 16 positions at a
@@ -296,7 +99,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tabbar + 1);  // TMEM base address
   constexpr bool kLloyd = (MODE == kAct || MODE == kWeightLM);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nthreads_c = p.nwarps * 32;
   const int NS = p.NS;
 
   const uint32_t pitch = p.pitch;
@@ -327,7 +129,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   //      by them) ----
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) mbar_init(&full[s], 1);
-    for (int r = 0; r < 2 * NS; ++r) mbar_init(&red[r], nthreads_c);
+    for (int r = 0; r < 2 * NS; ++r) mbar_init(&red[r], p.nwarps);   // one arrival per warp
     mbar_init(tabbar, 1);
     mbar_fence_init();
     const uint32_t gbytes = kLloyd ? 8u * static_cast<uint32_t>(guarded_grid_entries(p.grid_n)) : 0u;
@@ -409,7 +211,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
             sts_f32(part_addr + 4u * ((rb * kRows + pp) * kMaxWarps + warp), a0);
             sts_f32(part_addr + 4u * ((rb * kRows + pp + 8) * kMaxWarps + warp), a1);
           }
-          mbar_arrive(&red[rb]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&red[rb]);
         }
       }
 #pragma unroll
@@ -463,7 +266,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
         sts_f32(part_addr + 4u * ((rb * kRows + pp) * kMaxWarps + warp), m0);
         sts_f32(part_addr + 4u * ((rb * kRows + pp + 8) * kMaxWarps + warp), m1);
       }
-      mbar_arrive(&red[rb]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&red[rb]);
     }
 
     // ---- per-token totals: fixed summation order, identical in every thread ----
@@ -638,28 +442,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
 
 namespace {
 
-int sm_count_pair() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
-// Most ring slots that fit next to the tables (at least 2, at most 6), or 0.
-int slots_that_fit(int d, int grid_n) {
-  int best = 0;
-  for (int ns = 2; ns <= 6; ++ns)
-    if (pairk::layout(d, ns, grid_n).total + 128 <= pairk::kSmemLimit) best = ns;
-  return best;
-}
-
 template <int MODE, int BITS, bool FULL>
 int launch_pair(const pairk::Params& p, cudaStream_t st) {
   auto kern = pairk::rotq_pair_kernel<MODE, BITS, FULL>;
-  const size_t smem = pairk::layout(p.d, p.NS, p.grid_n).total + 128;
+  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_n).total + 128;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
-  const int sms = sm_count_pair();
+  const int sms = rowtile::sm_count();
   const int grid = p.ntiles < sms ? p.ntiles : sms;
   kern<<<grid, p.nwarps * 32, smem, st>>>(p);
   e = cudaGetLastError();
