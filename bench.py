@@ -42,7 +42,7 @@ D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
 # capture ran 32768 tokens; its bytes are scaled to this workload's 4608 by
 # the token count (its traffic grows in proportion to the tokens).
 QLINEAR_DRAM_BYTES = 26_065_920 + 85_248
-ROTQ_DRAM_BYTES = round((201_669_632 + 29_559_296) * 4608 / 32768)
+ROTQ_DRAM_BYTES = round((201_796_864 + 29_309_696) * 4608 / 32768)
 METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
 
