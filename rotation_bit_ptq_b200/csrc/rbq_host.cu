@@ -395,14 +395,12 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
   cb->grid_cells = grid.cells;
   cb->grid_scale = static_cast<float>(1.0 / (2.0 * grid.R));
   if ((rc = upload(grid.lut.data(), grid.lut.size(), &cb->grid)) != RBQ_OK) { delete cb; return rc; }
-  std::vector<float2> pad = guarded(grid.lut);
+  const std::vector<float2> pad = guarded(grid.lut);
   if ((rc = upload(pad.data(), pad.size(), &cb->grid_pad)) != RBQ_OK) { delete cb; return rc; }
   Grid full;
   if (build_grid_full(bounds, kMaxFullGridCells, &full) == RBQ_OK) {
     cb->grid_full_cells = full.cells;
     if ((rc = upload(full.lut.data(), full.lut.size(), &cb->grid_full)) != RBQ_OK) { delete cb; return rc; }
-    pad = guarded(full.lut);
-    if ((rc = upload(pad.data(), pad.size(), &cb->grid_full_pad)) != RBQ_OK) { delete cb; return rc; }
   }
   std::lock_guard<std::mutex> lk(g_mu);
   auto ins = cb_cache().emplace(key, cb);
@@ -412,7 +410,6 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
     cudaFree(cb->grid);
     cudaFree(cb->grid_full);
     cudaFree(cb->grid_pad);
-    cudaFree(cb->grid_full_pad);
     delete cb;
   }
   *out = ins.first->second;

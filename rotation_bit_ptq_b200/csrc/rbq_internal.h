@@ -62,11 +62,10 @@ struct CodebookDevice {
   // need more than kMaxFullGridCells cells.
   float2* grid_full = nullptr;
   int grid_full_cells = 0;
-  // Both grids again with kGridGuard copies of the end entries before and
-  // after, padded to an even entry count, so that one bulk copy (16-byte
+  // The [-R, R] grid again with kGridGuard copies of the end entries before
+  // and after, padded to an even entry count, so that one bulk copy (16-byte
   // multiple) brings a guarded grid into shared memory.
   float2* grid_pad = nullptr;
-  float2* grid_full_pad = nullptr;
 };
 
 constexpr int kGridGuard = 2;

@@ -32,11 +32,9 @@
 // which exists only after the butterfly, so there the arrival follows it.)
 //
 // Codes: z (8x the rotated value, H unnormalised) -> v = z / (||z|| + 8 eps).
-// A uniform grid over v in [-1, 1] (|v| <= 1 for a unit vector) gives a cell
-// n = round((v + 1)/2 * cells) whose entry holds the count of boundaries below
-// the cell and the boundary inside it (or +inf): code = base + (v >= thr).
-// Wide codebooks whose full-range grid does not fit use a grid over [-R, R]
-// with a saturating clamp.
+// A small uniform grid over [-R, R], v clamped into it, gives a cell n whose
+// entry holds the count of boundaries below the cell and the boundary inside
+// it (or +inf): code = base + (v >= thr) (see rowtile::Enc).
 
 #include <cuda_bf16.h>
 
@@ -53,8 +51,8 @@ using namespace rowtile;
 // Codes of one block for both tokens: the last butterfly stage (stride 32)
 // runs here, on half-blocks read back from tensor memory 16 positions at a
 // time.  SAN: the token(s) flagged bad are encoded as the zero vector.
-template <int BITS, bool FULL, bool SAN>
-__device__ __forceinline__ void encode_block(const Enc<FULL>& enc, uint32_t tA, uint32_t tB, bool bad0, bool bad1,
+template <int BITS, bool SAN>
+__device__ __forceinline__ void encode_block(const Enc& enc, uint32_t tA, uint32_t tB, bool bad0, bool bad1,
                                              uint32_t* w0, uint32_t* w1) {
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
@@ -86,7 +84,7 @@ __device__ __forceinline__ void encode_block(const Enc<FULL>& enc, uint32_t tA, 
   }
 }
 
-template <int MODE, int BITS, bool FULL>
+template <int MODE, int BITS>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) {
   extern __shared__ unsigned char smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -308,12 +306,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       uint32_t w0[2 * BITS], w1[2 * BITS];
 #pragma unroll
       for (int i = 0; i < 2 * BITS; ++i) w0[i] = w1[i] = 0u;
-      const Enc<FULL> enc(inv0, inv1, p.grid_cells, p.grid_scale, gbase);
+      const Enc enc(inv0, inv1, p.grid_cells, p.grid_scale, gbase);
       // warp-uniform choice: encode_block reads tensor memory collectively
       if (__any_sync(0xffffffffu, bad0 || bad1)) {
-        encode_block<BITS, FULL, true>(enc, tA, tB, bad0, bad1, w0, w1);
+        encode_block<BITS, true>(enc, tA, tB, bad0, bad1, w0, w1);
       } else {
-        encode_block<BITS, FULL, false>(enc, tA, tB, false, false, w0, w1);
+        encode_block<BITS, false>(enc, tA, tB, false, false, w0, w1);
       }
       const long long cp = static_cast<long long>(p.d) * BITS / 8;
       unsigned char* out = static_cast<unsigned char*>(p.out) + static_cast<long long>(b) * 8 * BITS;
@@ -442,9 +440,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
 
 namespace {
 
-template <int MODE, int BITS, bool FULL>
+template <int MODE, int BITS>
 int launch_pair(const pairk::Params& p, cudaStream_t st) {
-  auto kern = pairk::rotq_pair_kernel<MODE, BITS, FULL>;
+  auto kern = pairk::rotq_pair_kernel<MODE, BITS>;
   const size_t smem = rowtile::layout(p.d, p.NS, p.grid_n).total + 128;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
@@ -455,17 +453,17 @@ int launch_pair(const pairk::Params& p, cudaStream_t st) {
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }
 
-template <int MODE, bool FULL>
+template <int MODE>
 int launch_pair_bits(int bits, const pairk::Params& p, cudaStream_t st) {
   switch (bits) {
-    case 1: return launch_pair<MODE, 1, FULL>(p, st);
-    case 2: return launch_pair<MODE, 2, FULL>(p, st);
-    case 3: return launch_pair<MODE, 3, FULL>(p, st);
-    case 4: return launch_pair<MODE, 4, FULL>(p, st);
-    case 5: return launch_pair<MODE, 5, FULL>(p, st);
-    case 6: return launch_pair<MODE, 6, FULL>(p, st);
-    case 7: if constexpr (!FULL) return launch_pair<MODE, 7, FULL>(p, st); else return RBQ_ECONVERGE;
-    case 8: if constexpr (!FULL) return launch_pair<MODE, 8, FULL>(p, st); else return RBQ_ECONVERGE;
+    case 1: return launch_pair<MODE, 1>(p, st);
+    case 2: return launch_pair<MODE, 2>(p, st);
+    case 3: return launch_pair<MODE, 3>(p, st);
+    case 4: return launch_pair<MODE, 4>(p, st);
+    case 5: return launch_pair<MODE, 5>(p, st);
+    case 6: return launch_pair<MODE, 6>(p, st);
+    case 7: return launch_pair<MODE, 7>(p, st);
+    case 8: return launch_pair<MODE, 8>(p, st);
     default: return RBQ_EINVAL;
   }
 }
@@ -495,31 +493,21 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
   p.aux = aux;
   if ((rc = device_error_word_ptr(&p.err)) != RBQ_OK) return rc;
   const bool lloyd = (mode == kAct || mode == kWeightLM);
-  bool full = false;
   if (lloyd) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
-    if (bits <= 6 && cb->grid_full && slots_that_fit(r->d, cb->grid_full_cells + 1) >= 2) {
-      full = true;
-      p.grid = cb->grid_full_pad;
-      p.grid_n = cb->grid_full_cells + 1;
-      p.grid_cells = static_cast<float>(cb->grid_full_cells);
-      p.grid_scale = 0.5f;
-    } else {
-      p.grid = cb->grid_pad;
-      p.grid_n = cb->grid_cells + 1;
-      p.grid_cells = static_cast<float>(cb->grid_cells);
-      p.grid_scale = cb->grid_scale;
-    }
+    p.grid = cb->grid_pad;
+    p.grid_n = cb->grid_cells + 1;
+    p.grid_cells = static_cast<float>(cb->grid_cells);
+    p.grid_scale = cb->grid_scale;
   }
   p.NS = slots_that_fit(r->d, p.grid_n);
   if (p.NS < 2) return RBQ_ECONVERGE;
   switch (mode) {
-    case kAct: return full ? launch_pair_bits<kAct, true>(bits, p, st) : launch_pair_bits<kAct, false>(bits, p, st);
-    case kWeightLM:
-      return full ? launch_pair_bits<kWeightLM, true>(bits, p, st) : launch_pair_bits<kWeightLM, false>(bits, p, st);
-    case kInt8: return launch_pair<kInt8, 8, false>(p, st);
-    default: return launch_pair<kRotate, 8, false>(p, st);
+    case kAct: return launch_pair_bits<kAct>(bits, p, st);
+    case kWeightLM: return launch_pair_bits<kWeightLM>(bits, p, st);
+    case kInt8: return launch_pair<kInt8, 8>(p, st);
+    default: return launch_pair<kRotate, 8>(p, st);
   }
 }
 
