@@ -498,6 +498,39 @@ def run_suite(dev, stream, pk):
     for a, sv, r in acts.values():
         r.close()
     out["video_w4a6"] = vid
+
+    # Transform ablation (OrbitQuant §2.3 and §3.3): RPBH against the block
+    # Hadamard transform without the permutation (the same kernels with
+    # pi = identity) and against a dense d x d rotation, which is a plain GEMM
+    # x' = X R^T -- timed here as a cuBLAS BF16 matmul (the comparator only;
+    # the pages report structured transforms > 25x faster than dense ones).
+    # 4608 tokens of the attention-projection recipe, d = 3072 and 12288.
+    abl = {}
+    for d in (3072, 12288):
+        T = 4608
+        X = to_bf16_tensor(_tile_rows(synth.student_t_act(512, d, seed=31)[0], T), dev)
+        e = {}
+        xr = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+        codes = torch.empty((T, d // 2), dtype=torch.uint8, device=dev)
+        norms = torch.empty((T,), dtype=torch.float32, device=dev)
+        for label, r in (("RPBH", rbq.RPBH(d, 41)), ("block Hadamard (no permutation)", rbq.RPBH(d, 41, permute=False))):
+            rbq.rotate_act(r, X, xr)
+            rbq.rotate_quantize_act(r, X, 4, codes, norms)
+            us = _time_us(lambda: rbq.rotate_act(r, X, xr, stream=stream), stream)
+            e[f"rotate_only {label}"] = {"us": round(us, 2), "GB/s": round(T * 4 * d / (us * 1e-6) / 1e9, 1)}
+            e[f"rotate_quantize A4 {label}"] = rotq_entry(
+                _time_us(lambda: rbq.rotate_quantize_act(r, X, 4, codes, norms, stream=stream), stream), T, d, 4)
+            r.close()
+        R = (torch.randn((d, d), device=dev) / d ** 0.5).to(torch.bfloat16)
+        with torch.no_grad():
+            us = _time_us(lambda: torch.matmul(X, R.t(), out=xr), stream)
+        e["dense rotation (cuBLAS BF16 GEMM)"] = {"us": round(us, 2), "TFLOP/s": round(2.0 * T * d * d / (us * 1e-6) / 1e12, 1)}
+        e["dense / RPBH rotate_only time"] = round(us / e["rotate_only RPBH"]["us"], 2)
+        e["RPBH / block Hadamard rotate_only time"] = round(
+            e["rotate_only RPBH"]["us"] / e["rotate_only block Hadamard (no permutation)"]["us"], 3)
+        abl[f"d={d}, {T} tokens"] = e
+        del X, xr, codes, norms, R
+    out["transform_ablation"] = abl
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     return out

@@ -85,6 +85,22 @@ typedef struct rbq_rpbh rbq_rpbh;
  */
 int rpbh_make(int d, int h, uint64_t seed, rbq_rpbh** out);
 
+/*
+ * rpbh_make_ablation -- the same draw with parts of Pi_d switched off, for the
+ * ablations the OrbitQuant write-up reports (§3.3; §2.3 gives the reason for
+ * P_pi: without it outliers can stay concentrated in some blocks, with it
+ * every coordinate's variance is close to 1/d).  The random stream is consumed exactly
+ * as by rpbh_make, so with flags = 0 the result equals rpbh_make's and the
+ * signs of an RBQ_RPBH_NO_PERMUTATION handle equal the full draw's.
+ *   flags  RBQ_RPBH_NO_PERMUTATION: pi = identity (block Hadamard with D)
+ *          RBQ_RPBH_NO_SIGNS:       D = +1
+ * The handle is used like any other (every kernel takes it).
+ * Host only.  Errors: RBQ_EINVAL (also for unknown flag bits), RBQ_ENOMEM.
+ */
+#define RBQ_RPBH_NO_PERMUTATION 1
+#define RBQ_RPBH_NO_SIGNS       2
+int rpbh_make_ablation(int d, int h, uint64_t seed, int flags, rbq_rpbh** out);
+
 /* rpbh_free -- release a handle and its device copies (NULL is a no-op).
  * The caller must ensure no launched kernel still uses it. */
 void rpbh_free(rbq_rpbh* r);

@@ -22,11 +22,13 @@ RBQ_LLOYDMAX, RBQ_INT8_SYM = 0, 1
 RBQ_ROTATE_ONLY = 16
 RBQ_OK, RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA, RBQ_ENOMEM, RBQ_ECONVERGE, RBQ_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 RBQ_ESCRATCH = -7
+RBQ_RPBH_NO_PERMUTATION, RBQ_RPBH_NO_SIGNS = 1, 2
 
 # name -> (restype, argtypes); mirrors include/rbq.h
 _P, _I, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
 SIGNATURES = {
     "rpbh_make": (_I, [_I, _I, _U64, ctypes.POINTER(_P)]),
+    "rpbh_make_ablation": (_I, [_I, _I, _U64, _I, ctypes.POINTER(_P)]),
     "rpbh_free": (None, [_P]),
     "rpbh_export": (_I, [_P, _P, _P]),
     "rpbh_dim": (_I, [_P]),
@@ -107,12 +109,20 @@ def _dtype_code(t):
 # ---------------------------------------------------------------------------
 
 class RPBH:
-    """Pi_d = blkdiag(H_64 D_1, ..., H_64 D_{d/64}) · P_pi drawn from `seed`."""
+    """Pi_d = blkdiag(H_64 D_1, ..., H_64 D_{d/64}) · P_pi drawn from `seed`.
 
-    def __init__(self, d, seed, h=64):
+    permute=False gives pi = identity and signs=False gives D = +1 (the
+    ablations of OrbitQuant §3.3, through rpbh_make_ablation)."""
+
+    def __init__(self, d, seed, h=64, permute=True, signs=True):
         out = ctypes.c_void_p()
-        _check(lib().rpbh_make(int(d), int(h), ctypes.c_uint64(seed & (2 ** 64 - 1)), ctypes.byref(out)),
-               "rpbh_make")
+        flags = (0 if permute else RBQ_RPBH_NO_PERMUTATION) | (0 if signs else RBQ_RPBH_NO_SIGNS)
+        if flags:
+            _check(lib().rpbh_make_ablation(int(d), int(h), ctypes.c_uint64(seed & (2 ** 64 - 1)), flags,
+                                            ctypes.byref(out)), "rpbh_make_ablation")
+        else:
+            _check(lib().rpbh_make(int(d), int(h), ctypes.c_uint64(seed & (2 ** 64 - 1)), ctypes.byref(out)),
+                   "rpbh_make")
         self._h = out
         self.d = int(d)
         self.seed = int(seed)

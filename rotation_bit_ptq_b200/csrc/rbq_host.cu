@@ -464,6 +464,21 @@ extern "C" int rpbh_make(int d, int h, uint64_t seed, rbq_rpbh** out) {
   return RBQ_OK;
 }
 
+extern "C" int rpbh_make_ablation(int d, int h, uint64_t seed, int flags, rbq_rpbh** out) {
+  if (flags & ~(RBQ_RPBH_NO_PERMUTATION | RBQ_RPBH_NO_SIGNS)) {
+    if (out) *out = nullptr;
+    return RBQ_EINVAL;
+  }
+  const int rc = rpbh_make(d, h, seed, out);
+  if (rc != RBQ_OK) return rc;
+  rbq_rpbh* r = *out;
+  if (flags & RBQ_RPBH_NO_PERMUTATION)
+    for (int k = 0; k < d; ++k) r->perm[k] = k;
+  if (flags & RBQ_RPBH_NO_SIGNS)
+    for (int k = 0; k < d; ++k) r->sign[k] = 1;
+  return RBQ_OK;
+}
+
 extern "C" void rpbh_free(rbq_rpbh* r) {
   if (!r) return;
   for (auto& D : r->dev) {

@@ -82,6 +82,30 @@ def test_rpbh_make_rejects_bad_arguments(lib):
     lib.rpbh_free(None)
 
 
+@pytest.mark.parametrize("flags", [0, 1, 2, 3])
+def test_rpbh_make_ablation_flags(lib, flags):
+    d, seed = 1024, 99
+    out = ctypes.c_void_p()
+    assert lib.rpbh_make_ablation(d, 64, seed, flags, ctypes.byref(out)) == rbq.RBQ_OK
+    perm = np.empty(d, dtype=np.int32)
+    signs = np.empty(d, dtype=np.int8)
+    assert lib.rpbh_export(out, perm.ctypes.data_as(ctypes.c_void_p), signs.ctypes.data_as(ctypes.c_void_p)) == 0
+    lib.rpbh_free(out)
+    op, os_ = oracle.rpbh_draw(d, seed)
+    # the draw is consumed as by rpbh_make, then the switched-off parts reset
+    expect_perm = np.arange(d) if flags & rbq.RBQ_RPBH_NO_PERMUTATION else op
+    expect_signs = np.ones(d) if flags & rbq.RBQ_RPBH_NO_SIGNS else os_
+    assert np.array_equal(perm, expect_perm)
+    assert np.array_equal(signs, expect_signs)
+
+
+def test_rpbh_make_ablation_rejects_unknown_flags(lib):
+    out = ctypes.c_void_p(1234)
+    assert lib.rpbh_make_ablation(256, 64, 0, 4, ctypes.byref(out)) == rbq.RBQ_EINVAL
+    assert out.value is None
+    assert lib.rpbh_make_ablation(100, 64, 0, 1, ctypes.byref(out)) == rbq.RBQ_EINVAL
+
+
 def test_lloydmax_rejects_bad_arguments(lib):
     for d, b in ((0, 4), (64, 0), (64, 9), (-1, 2)):
         assert lib.lloydmax_table(d, b, None, None) == rbq.RBQ_EINVAL

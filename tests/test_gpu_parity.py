@@ -206,6 +206,38 @@ def test_pair_kernel_weights_wide_codebooks(bits):
 
 
 # --------------------------------------------------------------------------
+# ablation handles (OrbitQuant §3.3): block Hadamard without the permutation,
+# and without the signs; the same kernels, checked against the oracle's
+# dense matrix built from the same pi and D
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,T,bits,permute,signs", [(3072, 37, 4, False, True), (1024, 20, 2, False, True),
+                                                    (3072, 19, 3, True, False), (512, 33, 4, False, False)])
+def test_ablation_handles_quantize(d, T, bits, permute, signs):
+    X, _ = synth.student_t_act(T, d, seed=d + bits)
+    r = rbq.RPBH(d, 21, permute=permute, signs=signs)
+    perm, sg = r.export()
+    op, os_ = oracle.rpbh_draw(d, 21)
+    assert np.array_equal(perm, np.arange(d) if not permute else op)
+    assert np.array_equal(sg, np.ones(d) if not signs else os_)
+    Pi = oracle.rpbh_matrix(perm.astype(np.int64), sg.astype(np.int64))
+    _act_parity(X, d, bits, Pi=Pi, r=r)
+
+
+@pytest.mark.parametrize("d", [1024, 3072])
+def test_ablation_handle_rotate_only(d):
+    X, _ = synth.student_t_act(40, d, seed=d)
+    r = rbq.RPBH(d, 8, permute=False)
+    perm, sg = r.export()
+    Pi = oracle.rpbh_matrix(perm.astype(np.int64), sg.astype(np.int64))
+    xr = rbq.rotate_act(r, torch_bf16(X))
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.rotate_only(X.astype(np.float64), Pi)
+    check_bf16_rounding(bf16_to_numpy(xr), ora["xr"], "block-Hadamard rotate-only")
+
+
+# --------------------------------------------------------------------------
 # rotate-only (BF16 x') and offline weights
 # --------------------------------------------------------------------------
 
