@@ -319,6 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tl->tmem_slot;
+  // The prologue above reads only constant tables; the operands (written by
+  // the kernels before this one on the stream) wait for them.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
@@ -761,8 +765,19 @@ int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const 
   if (e != cudaSuccess) return cuda_fail(e);
   const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
   const int grid = ntiles < sms ? ntiles : sms;
-  kern<<<grid, kThreads, smem, st>>>(mA, mB, p);
-  e = cudaGetLastError();
+  // programmatic dependent launch: the prologue overlaps the weight expansion's tail
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }
 

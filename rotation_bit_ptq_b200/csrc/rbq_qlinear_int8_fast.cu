@@ -103,6 +103,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tl->tmem_slot;
+  // The prologue above reads only constant tables; the operands (written by
+  // the kernels before this one on the stream) wait for them.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
@@ -311,8 +315,20 @@ int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float
       rc = cuda_fail(e);
     } else {
       const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
-      kern<<<ntiles < sms ? ntiles : sms, kThreads, kSmem, st>>>(mA, mB, p);
-      if ((e = cudaGetLastError()) != cudaSuccess) rc = cuda_fail(e);
+      // programmatic dependent launch: the prologue overlaps the widening kernel's tail
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kSmem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+      if (e == cudaSuccess) e = cudaGetLastError();
+      if (e != cudaSuccess) rc = cuda_fail(e);
     }
   }
   e = cudaFreeAsync(ws, st);

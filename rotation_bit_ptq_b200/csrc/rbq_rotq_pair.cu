@@ -147,6 +147,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Everything above touches only this launch's own shared memory and the
+  // handle's constant tables; the rows and every output wait for the kernels
+  // this launch depends on (launched with programmatic dependent launch, the
+  // prologue overlaps their tail).
+  griddep_wait();
+  griddep_launch_dependents();
   if (blockIdx.x < p.ntiles) issue_rows(blockIdx.x, 0);
   if (!mbar_wait(tabbar, 0)) atomicOr(p.err, 256u);
 
@@ -448,9 +454,7 @@ int launch_pair(const pairk::Params& p, cudaStream_t st) {
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = rowtile::sm_count();
   const int grid = p.ntiles < sms ? p.ntiles : sms;
-  kern<<<grid, p.nwarps * 32, smem, st>>>(p);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+  return rowtile::launch_pdl(kern, grid, p.nwarps * 32, smem, st, p);
 }
 
 template <int MODE>

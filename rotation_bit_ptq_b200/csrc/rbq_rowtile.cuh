@@ -212,5 +212,25 @@ inline int slots_that_fit(int d, int grid_n) {
   return best;
 }
 
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous launch on the stream finishes; it calls griddep_wait()
+// before reading anything that launch may have written.
+template <typename Kern>
+inline int launch_pdl(Kern kern, int grid, int threads, size_t smem, cudaStream_t st, const Params& p) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+}
+
 }  // namespace rowtile
 }  // namespace rbq

@@ -84,6 +84,16 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+// Wait until the grids this launch depends on have completed and their writes
+// are visible (returns at once for a launch without a programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next launch on the stream to be scheduled before this grid ends
+// (it still waits for this grid's completion before reading its results).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- proxies and tcgen05 ordering ------------------------------------------
 // Make generic-proxy shared-memory writes visible to the async proxy (the
 // tensor core reads operands through it).
