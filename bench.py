@@ -463,6 +463,14 @@ def run_suite(dev, stream, pk):
             err_naive = (naive - dense).norm() / dense.norm()
         e["rel_error_rotated_int8"] = round(err_rot.item(), 5)
         e["rel_error_naive_int8"] = round(err_naive.item(), 5)
+        # one scale for the whole tensor (two passes over W), same layer kernel
+        qt, st_ = rbq.quantize_weights(r, W, 8, "int8_tensor")
+        us = _time_us(lambda: rbq.quantize_weights(r, W, 8, "int8_tensor", qt, st_, stream=stream), stream)
+        e["quantize_weights_int8_per_tensor"] = {"us": round(us, 2)}
+        yt = rbq.qlinear_int8(xr[:64].contiguous(), qt, st_)
+        with torch.no_grad():
+            e["rel_error_rotated_int8_per_tensor"] = round(((yt.float() - dense).norm() / dense.norm()).item(), 5)
+        del qt, st_, yt
         int8[f"{name} {d_in}->{n_out}"] = e
         r.close()
         del W, X, q, sc, xr, y

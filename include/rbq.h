@@ -61,6 +61,7 @@ extern "C" {
 
 #define RBQ_LLOYDMAX   0   /* OrbitQuant direction codes + BF16 row norms     */
 #define RBQ_INT8_SYM   1   /* symmetric per-output-channel INT8 + fp32 scales */
+#define RBQ_INT8_TENSOR 2  /* symmetric INT8, one scale for the whole tensor   */
 
 #define RBQ_ROTATE_ONLY 16 /* `bits` value of rotate_quantize_act: x' only  */
 
@@ -161,6 +162,12 @@ int rotate_quantize_act(const rbq_rpbh* r, const void* X, int dtype, int T,
  *        `rownorm_or_scale` = float scale_i = max_k |w'_ik| / 127;
  *        q = clamp(round_half_even(w' / scale), -127, 127); a zero row gives
  *        scale 0 and q 0 (INT8-convrot §4; the zero point is 0).
+ *   mode RBQ_INT8_TENSOR: as RBQ_INT8_SYM with one scale for the whole
+ *        tensor, S = max_ik |w'_ik| / 127 (the INT8 image-text model page,
+ *        cloud.baidu.com/article/9432337, "how it works": one scale per
+ *        tensor), written to every entry of `rownorm_or_scale` so that
+ *        qlinear_int8 takes it unchanged.  Two passes over W: per-row maxima
+ *        (then their maximum), then the rows quantised with S.
  *   W  device, d_out x d, dtype RBQ_BF16 or RBQ_F32, 16-byte aligned.
  *   Output pointers 16-byte (codes/q) and 4-byte (norms/scales) aligned.
  * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.

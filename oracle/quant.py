@@ -87,13 +87,18 @@ def quantize_weights_lloydmax(W, Pi, bounds, eps=EPS):
             "v": V, "wr": Wr}
 
 
-def quantize_weights_int8(W, Pi=None):
-    """Symmetric per-output-channel INT8 of the rotated rows (Pi=None: naive).
+def quantize_weights_int8(W, Pi=None, per_tensor=False):
+    """Symmetric INT8 of the rotated rows (Pi=None: naive), one scale per
+    output channel (INT8-convrot §4), or with per_tensor=True one scale for
+    the whole tensor (INT8 image-text model page, "how it works"), repeated
+    per row.
 
     Returns dict(q int64[N,d], scale fp32-valued fp64[N], ratio w'/scale, wr).
     """
     Wr = np.asarray(W, dtype=np.float64) if Pi is None else rpbh_apply(Pi, W)
     amax = np.max(np.abs(Wr), axis=1)
+    if per_tensor:
+        amax = np.full_like(amax, np.max(amax))
     scale = (amax / 127.0).astype(np.float32).astype(np.float64)
     safe = np.where(scale > 0, scale, 1.0)
     ratio = Wr / safe[:, None]

@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librbq.so")
 
 RBQ_F32, RBQ_BF16 = 0, 1
-RBQ_LLOYDMAX, RBQ_INT8_SYM = 0, 1
+RBQ_LLOYDMAX, RBQ_INT8_SYM, RBQ_INT8_TENSOR = 0, 1, 2
 RBQ_ROTATE_ONLY = 16
 RBQ_OK, RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA, RBQ_ENOMEM, RBQ_ECONVERGE, RBQ_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 RBQ_ESCRATCH = -7
@@ -200,7 +200,8 @@ def rotate_act(rpbh, X, out=None, norms=None, stream=None):
 
 def quantize_weights(rpbh, W, bits, mode="lloydmax", out=None, aux=None, stream=None):
     """Offline weights.  mode='lloydmax': (codes uint8, r' bfloat16[N]);
-    mode='int8': (q int8[N, d], scale float32[N])."""
+    mode='int8': (q int8[N, d], scale float32[N]) with one scale per row;
+    mode='int8_tensor': the same with one scale for the tensor (repeated)."""
     import torch
     _need_cuda(W, "W")
     N, d = W.shape
@@ -214,8 +215,8 @@ def quantize_weights(rpbh, W, bits, mode="lloydmax", out=None, aux=None, stream=
             aux = torch.empty((N,), dtype=torch.bfloat16, device=W.device)
         _need_cuda(out, "codes", torch.uint8)
         _need_cuda(aux, "rnorm", torch.bfloat16)
-    elif mode == "int8":
-        code, bits = RBQ_INT8_SYM, 8
+    elif mode in ("int8", "int8_tensor"):
+        code, bits = (RBQ_INT8_SYM if mode == "int8" else RBQ_INT8_TENSOR), 8
         if out is None:
             out = torch.empty((N, d), dtype=torch.int8, device=W.device)
         if aux is None:
@@ -223,7 +224,7 @@ def quantize_weights(rpbh, W, bits, mode="lloydmax", out=None, aux=None, stream=
         _need_cuda(out, "q", torch.int8)
         _need_cuda(aux, "scale", torch.float32)
     else:
-        raise ValueError("mode must be 'lloydmax' or 'int8'")
+        raise ValueError("mode must be 'lloydmax', 'int8' or 'int8_tensor'")
     _check(lib().quantize_weights(rpbh.handle, _ptr(W), _dtype_code(W), N, code, int(bits), _ptr(out),
                                   _ptr(aux), _stream(stream)), "quantize_weights")
     return out, aux

@@ -35,6 +35,7 @@ struct RotqParams {
   const float* bounds;   // 2^bits - 1 Lloyd-Max boundaries (Lloyd-Max modes)
   void* out;             // packed codes | int8 q | bf16 x'
   void* aux;             // float norms | bf16 row norms | float scales | float norms (optional)
+  const float* fixed_scale;   // INT8: one scale for every row (not written back), else null
 };
 
 template <typename Tin> __device__ __forceinline__ float to_f32(Tin v);
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
         else static_cast<__nv_bfloat16*>(p.aux)[t] = __float2bfloat16_rn(s);
       }
     } else if constexpr (MODE == kInt8) {
-      const float scale = s / 127.0f;
+      const float scale = p.fixed_scale ? __ldg(p.fixed_scale) : s / 127.0f;
       int8_t* dst = static_cast<int8_t*>(p.out) + static_cast<size_t>(t) * d + 64 * b;
       uint32_t packed[16];
 #pragma unroll
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-      if (b == 0) static_cast<float*>(p.aux)[t] = scale;
+      if (b == 0 && !p.fixed_scale) static_cast<float*>(p.aux)[t] = scale;
     } else {   // kRotate
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(t) * d + 64 * b;
       uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -215,6 +216,7 @@ struct Params {
   float grid_cells, grid_scale;
   void* out;
   void* aux;
+  const float* fixed_scale;  // INT8: one scale for every row (not written back), else null
 };
 
 __device__ __forceinline__ unsigned long long pk(float a, float b) {
@@ -540,7 +542,7 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
           else static_cast<__nv_bfloat16*>(p.aux)[t] = __float2bfloat16_rn(sn);
         }
       } else if constexpr (MODE == kInt8) {
-        const float scale = (tot * 0.125f) / 127.0f;
+        const float scale = p.fixed_scale ? __ldg(p.fixed_scale) : (tot * 0.125f) / 127.0f;
         const float rcp = (scale > 0.f) ? 1.0f / scale : 0.f;
         uint32_t q4[16];
 #pragma unroll
@@ -557,7 +559,7 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         uint4* dst = reinterpret_cast<uint4*>(static_cast<int8_t*>(p.out) + t * d + 64 * b);
 #pragma unroll
         for (int i = 0; i < 4; ++i) __stcs(dst + i, make_uint4(q4[4 * i], q4[4 * i + 1], q4[4 * i + 2], q4[4 * i + 3]));
-        if (b == 0) static_cast<float*>(p.aux)[t] = scale;
+        if (b == 0 && !p.fixed_scale) static_cast<float*>(p.aux)[t] = scale;
       } else {   // kRotate
         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + t * d + 64 * b);
 #pragma unroll
@@ -687,7 +689,7 @@ int launch_fast(int bits, const fast::Params& p, cudaStream_t st) {
 }
 
 int run_fast(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
-             cudaStream_t st) {
+             cudaStream_t st, const float* fixed_scale = nullptr) {
   const RpbhDevice* rd = nullptr;
   int rc = rpbh_device(r, &rd);
   if (rc != RBQ_OK) return rc;
@@ -700,6 +702,7 @@ int run_fast(const rbq_rpbh* r, int mode, int bits, long long rows, const void* 
   p.sign = rd->sign;
   p.out = out;
   p.aux = aux;
+  p.fixed_scale = fixed_scale;
   if (mode == kAct || mode == kWeightLM) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
@@ -732,7 +735,7 @@ int tokens_per_cta(int nblk) {
 }
 
 int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out,
-            void* aux, RotqParams* p) {
+            void* aux, RotqParams* p, const float* fixed_scale = nullptr) {
   const RpbhDevice* rd = nullptr;
   int rc = rpbh_device(r, &rd);
   if (rc != RBQ_OK) return rc;
@@ -746,6 +749,7 @@ int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X
   p->bounds = nullptr;
   p->out = out;
   p->aux = aux;
+  p->fixed_scale = fixed_scale;
   if (mode == kAct || mode == kWeightLM) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
@@ -760,7 +764,30 @@ int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X
 // steps of 256.  RBQ_ECONVERGE from the launch means "not this kernel".
 bool rotq_pair_eligible(int dtype, int d);
 int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
-                     cudaStream_t st);
+                     cudaStream_t st, const float* fixed_scale = nullptr);
+
+namespace {
+
+// Per-tensor INT8: the largest per-row scale, written to every entry of the
+// row-scale array (one block; rows are few compared with the weight bytes).
+__global__ void __launch_bounds__(1024) max_broadcast_kernel(float* scale, int n) {
+  __shared__ float part[32];
+  float m = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, scale[i]);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = (threadIdx.x < (blockDim.x >> 5)) ? part[threadIdx.x] : 0.f;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) part[0] = m;
+  }
+  __syncthreads();
+  m = part[0];
+  for (int i = threadIdx.x; i < n; i += blockDim.x) scale[i] = m;
+}
+
+}  // namespace
 
 }  // namespace rbq
 
@@ -792,12 +819,34 @@ extern "C" int rotate_quantize_act(const rbq_rpbh* r, const void* X, int dtype, 
   return rot ? launch_mode<kRotate>(dtype, 8, p, st) : launch_mode<kAct>(dtype, bits, p, st);
 }
 
+namespace {
+
+// One rotate-then-quantise pass over the weight rows through the first
+// kernel that takes this width (fixed_scale: INT8 with one given scale).
+int weights_pass(const rbq_rpbh* r, const void* W, int dtype, int d_out, int m, int bits, void* out, void* aux,
+                 cudaStream_t st, const float* fixed_scale) {
+  if (rotq_pair_eligible(dtype, r->d)) {
+    const int prc = rotq_pair_launch(r, m, bits, d_out, W, out, aux, st, fixed_scale);
+    if (prc != RBQ_ECONVERGE) return prc;
+  }
+  if (fast_eligible(dtype, r->d)) {
+    const int frc = run_fast(r, m, bits, d_out, W, out, aux, st, fixed_scale);
+    if (frc != RBQ_ECONVERGE) return frc;
+  }
+  RotqParams p;
+  int rc = prepare(r, m, bits, d_out, W, out, aux, &p, fixed_scale);
+  if (rc != RBQ_OK) return rc;
+  return (m == kWeightLM) ? launch_mode<kWeightLM>(dtype, bits, p, st) : launch_mode<kInt8>(dtype, 8, p, st);
+}
+
+}  // namespace
+
 extern "C" int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int d_out, int mode,
                                 int bits, void* codes_or_q, void* rownorm_or_scale, void* stream) {
   if (!r || d_out < 0 || (dtype != RBQ_F32 && dtype != RBQ_BF16)) return RBQ_EINVAL;
   if (mode == RBQ_LLOYDMAX) {
     if (bits < 1 || bits > 8) return RBQ_EINVAL;
-  } else if (mode == RBQ_INT8_SYM) {
+  } else if (mode == RBQ_INT8_SYM || mode == RBQ_INT8_TENSOR) {
     if (bits != 8) return RBQ_EINVAL;
   } else {
     return RBQ_EINVAL;
@@ -806,20 +855,14 @@ extern "C" int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int
   if (!W || !codes_or_q || !rownorm_or_scale) return RBQ_EINVAL;
   if (!aligned(W, 16) || !aligned(codes_or_q, 16) || !aligned(rownorm_or_scale, 4))
     return RBQ_EALIGN;
-  const int m = (mode == RBQ_LLOYDMAX) ? kWeightLM : kInt8;
-  if (rotq_pair_eligible(dtype, r->d)) {
-    const int prc = rotq_pair_launch(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale,
-                                     static_cast<cudaStream_t>(stream));
-    if (prc != RBQ_ECONVERGE) return prc;
-  }
-  if (fast_eligible(dtype, r->d)) {
-    const int frc = run_fast(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, static_cast<cudaStream_t>(stream));
-    if (frc != RBQ_ECONVERGE) return frc;
-  }
-  RotqParams p;
-  int rc = prepare(r, m, bits, d_out, W, codes_or_q, rownorm_or_scale, &p);
-  if (rc != RBQ_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return (m == kWeightLM) ? launch_mode<kWeightLM>(dtype, bits, p, st)
-                          : launch_mode<kInt8>(dtype, 8, p, st);
+  const int m = (mode == RBQ_LLOYDMAX) ? kWeightLM : kInt8;
+  int rc = weights_pass(r, W, dtype, d_out, m, bits, codes_or_q, rownorm_or_scale, st, nullptr);
+  if (rc != RBQ_OK || mode != RBQ_INT8_TENSOR) return rc;
+  // per tensor: the largest row scale, then the rows again with that scale
+  float* scale = static_cast<float*>(rownorm_or_scale);
+  max_broadcast_kernel<<<1, 1024, 0, st>>>(scale, d_out);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return weights_pass(r, W, dtype, d_out, kInt8, 8, codes_or_q, rownorm_or_scale, st, scale);
 }

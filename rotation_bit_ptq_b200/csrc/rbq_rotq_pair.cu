@@ -334,7 +334,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       }
     } else if constexpr (MODE == kInt8) {
       // scale = max|w'| / 127 with w' = z / 8; q = clamp(round(w' / scale), +-127)
-      const float sc0 = (tot[0] * 0.125f) / 127.0f, sc1 = (tot[1] * 0.125f) / 127.0f;
+      const float sc0 = p.fixed_scale ? *p.fixed_scale : (tot[0] * 0.125f) / 127.0f;
+      const float sc1 = p.fixed_scale ? *p.fixed_scale : (tot[1] * 0.125f) / 127.0f;
       const float r0 = (sc0 > 0.f) ? 1.0f / sc0 : 0.f, r1 = (sc1 > 0.f) ? 1.0f / sc1 : 0.f;
       int8_t* out = static_cast<int8_t*>(p.out) + 64 * b;
 #pragma unroll
@@ -368,8 +369,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
         }
       }
       if (b == 0) {
-        if (ok0) static_cast<float*>(p.aux)[t0] = sc0;
-        if (ok1) static_cast<float*>(p.aux)[t1] = sc1;
+        if (ok0 && !p.fixed_scale) static_cast<float*>(p.aux)[t0] = sc0;
+        if (ok1 && !p.fixed_scale) static_cast<float*>(p.aux)[t1] = sc1;
       }
     } else {   // kRotate: x' = z / 8 in BF16
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + 64 * b;
@@ -479,7 +480,7 @@ bool rotq_pair_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d % 256 
 // Returns RBQ_ECONVERGE when the tables do not fit (the caller then uses
 // another kernel); any other code is the call's result.
 int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
-                     cudaStream_t st) {
+                     cudaStream_t st, const float* fixed_scale) {
   using namespace pairk;
   const uint32_t* tab = nullptr;
   int rc = rpbh_pair_tables(r, &tab);
@@ -495,6 +496,7 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
   p.tab = tab;
   p.out = out;
   p.aux = aux;
+  p.fixed_scale = fixed_scale;
   if ((rc = device_error_word_ptr(&p.err)) != RBQ_OK) return rc;
   const bool lloyd = (mode == kAct || mode == kWeightLM);
   if (lloyd) {

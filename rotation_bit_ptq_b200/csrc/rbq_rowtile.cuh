@@ -37,6 +37,7 @@ struct Params {
   void* out;
   void* aux;
   unsigned int* err;
+  const float* fixed_scale;          // INT8: one scale for every row (not written back), else null
 };
 
 // Shared-memory layout (bytes from the 128-aligned base).

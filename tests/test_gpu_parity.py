@@ -191,6 +191,29 @@ def test_pair_kernel_weights_int8(d, n):
     check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
 
 
+@pytest.mark.parametrize("d,n,dtype", [(1024, 40, "bf16"), (3072, 56, "bf16"),    # token-pair kernel
+                                       (4096, 40, "bf16"),                         # register-staged kernel
+                                       (512, 37, "f32")])                          # general kernel
+def test_weights_int8_per_tensor(d, n, dtype):
+    W = synth.to_bf16(synth.gaussian_weights(synth.rng(13, d), n, d, outlier_frac=0.01).astype(np.float32))
+    W[4] = 0.0
+    r, Pi = _rpbh(d, 10)
+    q, sc = rbq.quantize_weights(r, _dense(W, dtype), 8, mode="int8_tensor")
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi, per_tensor=True)
+    check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
+    # and the layer runs unchanged on it
+    X = synth.to_bf16(np.random.default_rng(d).standard_normal((20, d)).astype(np.float32))
+    xr = rbq.rotate_act(r, torch_bf16(X)) if dtype == "bf16" else None
+    if xr is not None:
+        y = rbq.qlinear_int8(xr, q, sc)
+        torch.cuda.synchronize()
+        ref = oracle.qlinear_int8(bf16_to_numpy(xr), q.cpu().numpy().astype(np.float64),
+                                  sc.cpu().numpy().astype(np.float64))
+        assert rel_frobenius(bf16_to_numpy(y), ref) < QLINEAR8_RTOL
+
+
 @pytest.mark.parametrize("bits", [6, 8])
 def test_pair_kernel_weights_wide_codebooks(bits):
     d = 3072

@@ -119,6 +119,26 @@ def test_rotation_spreads_outliers():
     assert abs(stats.kurtosis(vy.ravel(), fisher=False) - 3) < 0.1
 
 
+def test_int8_per_tensor_bounds():
+    # one scale for the tensor: exactly one |q| = 127 in the row holding the
+    # tensor's largest |w'|, the dequantisation error bound, and the scale
+    # equals the largest per-row scale (max commutes with the monotone /127)
+    data, Pi, _, _ = _tiny_setup()
+    W = data["W"].astype(np.float64)
+    W[3] = 0.0
+    t = oracle.quantize_weights_int8(W, Pi, per_tensor=True)
+    c = oracle.quantize_weights_int8(W, Pi)
+    q, scale, wr = t["q"], t["scale"], t["wr"]
+    assert np.all(scale == scale[0]) and scale[0] == np.max(c["scale"])
+    assert np.all(np.abs(q) <= 127)
+    i, _ = np.unravel_index(np.argmax(np.abs(wr)), wr.shape)
+    assert np.max(np.abs(q[i])) == 127
+    assert np.all(q[3] == 0)
+    assert np.all(np.abs(wr - scale[0] * q) <= scale[0] * (0.5 + 1e-6))
+    # with a coarser grid the per-tensor error is at least the per-channel one
+    assert np.linalg.norm(wr - scale[0] * q) >= np.linalg.norm(wr - c["scale"][:, None] * c["q"])
+
+
 def test_int8_bounds_and_rotation_helps():
     data, Pi, _, _ = _tiny_setup()
     W = data["W"].astype(np.float64)
