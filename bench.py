@@ -471,6 +471,16 @@ def run_suite(dev, stream, pk):
         with torch.no_grad():
             e["rel_error_rotated_int8_per_tensor"] = round(((yt.float() - dense).norm() / dense.norm()).item(), 5)
         del qt, st_, yt
+        # zero point per channel (asymmetric), same layer GEMM on (q - z)
+        qa, sa, za = rbq.quantize_weights_int8_asym(r, W)
+        us = _time_us(lambda: rbq.quantize_weights_int8_asym(r, W, qa, sa, za, stream=stream), stream)
+        e["quantize_weights_int8_asym"] = {"us": round(us, 2)}
+        e["qlinear_int8_asym"] = gemm_entry(_time_us(lambda: rbq.qlinear_int8_asym(xr, qa, sa, za, y, stream=stream),
+                                                     stream), 4096, n_out, d_in)
+        ya = rbq.qlinear_int8_asym(xr[:64].contiguous(), qa, sa, za)
+        with torch.no_grad():
+            e["rel_error_rotated_int8_asym"] = round(((ya.float() - dense).norm() / dense.norm()).item(), 5)
+        del qa, sa, za, ya
         int8[f"{name} {d_in}->{n_out}"] = e
         r.close()
         del W, X, q, sc, xr, y
@@ -539,6 +549,33 @@ def run_suite(dev, stream, pk):
         abl[f"d={d}, {T} tokens"] = e
         del X, xr, codes, norms, R
     out["transform_ablation"] = abl
+
+    # Bit-width sweep (mixed per-layer widths): the
+    # attention projection (4608 x 3072 x 3072) at every activation width
+    # with 4-bit weights and every weight width with 4-bit activations.
+    data = synth.attn_proj(seed=5)
+    X = to_bf16_tensor(data["X"], dev)
+    W = to_bf16_tensor(data["W"], dev)
+    r = rbq.RPBH(3072, 77)
+    y = torch.empty((4608, 3072), dtype=torch.bfloat16, device=dev)
+    sweep = {}
+    wc4, wn4 = rbq.quantize_weights(r, W, 4)
+    a4, s4 = rbq.rotate_quantize_act(r, X, 4)
+    for b in (2, 3, 4, 5, 6, 8):
+        a, sa = rbq.rotate_quantize_act(r, X, b)
+        wc, wn = rbq.quantize_weights(r, W, b)
+        sweep[f"A{b}"] = {
+            "rotate_quantize": rotq_entry(
+                _time_us(lambda: rbq.rotate_quantize_act(r, X, b, a, sa, stream=stream), stream), 4608, 3072, b),
+            "qlinear W4A%d" % b: gemm_entry(
+                _time_us(lambda: rbq.qlinear(a, sa, b, wc4, wn4, 4, 3072, y, stream=stream), stream), 4608, 3072, 3072),
+            "qlinear W%dA4" % b: gemm_entry(
+                _time_us(lambda: rbq.qlinear(a4, s4, 4, wc, wn, b, 3072, y, stream=stream), stream), 4608, 3072, 3072),
+        }
+        del a, sa, wc, wn
+    out["bit_width_sweep_attn_proj"] = sweep
+    r.close()
+    del X, W, y, wc4, wn4, a4, s4
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     return out

@@ -176,6 +176,25 @@ int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int d_out,
                      int mode, int bits, void* codes_or_q,
                      void* rownorm_or_scale, void* stream);
 
+/*
+ * quantize_weights_int8_asym -- asymmetric per-output-channel INT8 with a zero
+ * point (INT8-convrot, "the quantized model file": scale and zero point per
+ * layer/channel; the INT8 image-text model page, "how it works").  For each
+ * row w'_i = Pi_d w_i:
+ *   hi = max(max_k w'_ik, 0), lo = min(min_k w'_ik, 0), scale_i = (hi - lo)/255,
+ *   z_i = clamp(round_half_even(-lo / scale_i), 0, 255),
+ *   q_ik = clamp(round_half_even(w'_ik / scale_i) + z_i, 0, 255);
+ *   w'_ik ~ scale_i (q_ik - z_i); a zero row gives scale 0, z 0, q 0.
+ *   W           device, d_out x d, RBQ_BF16 or RBQ_F32, 16-byte aligned
+ *   q           device uint8 [d_out, d], 16-byte aligned
+ *   scale       device float [d_out], 4-byte aligned
+ *   zero_point  device uint8 [d_out]
+ * Offline weights: runs the general rotation kernel (any width).
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int quantize_weights_int8_asym(const rbq_rpbh* r, const void* W, int dtype, int d_out, uint8_t* q, float* scale,
+                               uint8_t* zero_point, void* stream);
+
 /* ---- quantised linear layers --------------------------------------------- */
 
 /*
@@ -263,6 +282,19 @@ int qlinear_noalloc(const uint8_t* a_codes, const float* s, int bits_a,
 int rbq_code_grid(int d, int bits, int variant, float* thr, int32_t* base, int* cells, float* scale);
 
 /* Text for a return code (static storage). */
+/*
+ * qlinear_int8_asym -- the W8A16 layer on asymmetric INT8 weights:
+ *   Y[m, n] = bf16( scale[n] * sum_k (q[n,k] - z[n]) * Xrot[m,k] ),
+ * fp32 accumulation.  The weights are widened once per call to bf16 (q - z),
+ * which is exact, and run through the same tensor-core GEMM as qlinear_int8.
+ *   Xrot        device BF16 [M, K] from rotate_quantize_act(bits=RBQ_ROTATE_ONLY)
+ *   q, scale, zero_point  from quantize_weights_int8_asym
+ *   N a multiple of 8, K a multiple of 64 (else RBQ_EINVAL); Y BF16 [M, N].
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int qlinear_int8_asym(const uint16_t* Xrot, const uint8_t* Wq, const float* scale, const uint8_t* zero_point,
+                      int M, int N, int K, uint16_t* Y, void* stream);
+
 const char* rbq_error_string(int code);
 
 /*

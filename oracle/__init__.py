@@ -39,7 +39,8 @@ lloydmax.*             closed form at 1 bit; J. Max (1960) Gaussian tables;
                        1-D k-means on samples
 quant.assign_codes     brute-force nearest level on tiny inputs
 quant.pack/unpack      hand-made bit-layout fixture (tests/golden)
-quant.quantize_*       invariants (norm, cancellation, INT8 bounds)
+quant.quantize_*       invariants (norm, cancellation, INT8 bounds; per-tensor
+                       and zero-point variants: range, bound and code-of-0 pins)
 qlinear.*              pure-Python triple loop; equal-code closed form
 =====================  ===================================================
 """
@@ -50,13 +51,14 @@ from .lloydmax import lloydmax_unit, lloydmax_table, lloydmax_distortion_unit
 from .bf16 import round_to_bf16
 from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
                     quantize_weights_lloydmax, quantize_weights_int8,
-                    rotate_only, EPS)
-from .qlinear import qlinear, qlinear_int8
+                    quantize_weights_int8_asym, rotate_only, EPS)
+from .qlinear import qlinear, qlinear_int8, qlinear_int8_asym
 
 __all__ = [
     "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_rows", "rpbh_apply",
     "lloydmax_unit", "lloydmax_table", "lloydmax_distortion_unit",
     "round_to_bf16", "assign_codes", "pack_codes", "unpack_codes",
     "quantize_act", "quantize_weights_lloydmax", "quantize_weights_int8",
-    "rotate_only", "EPS", "qlinear", "qlinear_int8",
+    "quantize_weights_int8_asym", "rotate_only", "EPS", "qlinear", "qlinear_int8",
+    "qlinear_int8_asym",
 ]

@@ -29,3 +29,10 @@ def qlinear_int8(xr, q, scale):
     xr = np.asarray(xr, dtype=np.float64)
     q = np.asarray(q, dtype=np.float64)
     return (xr @ q.T) * np.asarray(scale, dtype=np.float64)[None, :]
+
+
+def qlinear_int8_asym(xr, q, scale, z):
+    """y = scale_n * sum_k (q_nk - z_n) x'_mk in fp64 (asymmetric INT8 layer)."""
+    xr = np.asarray(xr, dtype=np.float64)
+    qz = np.asarray(q, dtype=np.float64) - np.asarray(z, dtype=np.float64)[:, None]
+    return (xr @ qz.T) * np.asarray(scale, dtype=np.float64)[None, :]

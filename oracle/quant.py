@@ -108,6 +108,29 @@ def quantize_weights_int8(W, Pi=None, per_tensor=False):
     return {"q": q, "scale": scale, "ratio": ratio, "wr": Wr}
 
 
+def quantize_weights_int8_asym(W, Pi=None):
+    """Asymmetric per-output-channel INT8 with a zero point (INT8-convrot,
+    "the quantized model file": a scale and a zero point per channel).  The
+    row's range is widened to contain 0 and cut into 255 steps:
+    scale = (hi - lo)/255, z = clip(round(-lo/scale), 0, 255),
+    q = clip(round(w'/scale) + z, 0, 255), w' ~ scale (q - z).
+
+    Returns dict(q int64[N,d] in 0..255, scale fp32-valued fp64[N], z int64[N],
+    ratio w'/scale, zratio -lo/scale, wr).
+    """
+    Wr = np.asarray(W, dtype=np.float64) if Pi is None else rpbh_apply(Pi, W)
+    hi = np.maximum(np.max(Wr, axis=1), 0.0)
+    lo = np.minimum(np.min(Wr, axis=1), 0.0)
+    scale = ((hi - lo) / 255.0).astype(np.float32).astype(np.float64)
+    safe = np.where(scale > 0, scale, 1.0)
+    zratio = np.where(scale > 0, -lo / safe, 0.0)
+    z = np.clip(np.rint(zratio), 0, 255).astype(np.int64)
+    ratio = np.where(scale[:, None] > 0, Wr / safe[:, None], 0.0)
+    q = np.clip(np.rint(ratio) + z[:, None], 0, 255).astype(np.int64)
+    q[scale == 0] = 0
+    return {"q": q, "scale": scale, "z": z, "ratio": ratio, "zratio": zratio, "wr": Wr}
+
+
 def rotate_only(X, Pi):
     """x' = Pi x rounded to BF16: the activation operand of the INT8 path
     (INT8-convrot §3/§4: the transform information is used at inference)."""

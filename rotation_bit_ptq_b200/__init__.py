@@ -37,6 +37,8 @@ SIGNATURES = {
     "quantize_weights": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "qlinear": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
     "qlinear_int8": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "quantize_weights_int8_asym": (_I, [_P, _P, _I, _I, _P, _P, _P, _P]),
+    "qlinear_int8_asym": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "qlinear_noalloc": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
@@ -284,6 +286,42 @@ def qlinear_int8(xrot, q, scale, out=None, stream=None):
     _need_cuda(out, "out", torch.bfloat16)
     _check(lib().qlinear_int8(_ptr(xrot), _ptr(q), _ptr(scale), M, N, K, _ptr(out), _stream(stream)),
            "qlinear_int8")
+    return out
+
+
+def quantize_weights_int8_asym(rpbh, W, q=None, scale=None, zero_point=None, stream=None):
+    """Asymmetric per-channel INT8 of the rotated rows: (q uint8[N, d],
+    scale float32[N], zero_point uint8[N]); w' ~ scale (q - z)."""
+    import torch
+    _need_cuda(W, "W")
+    N, d = W.shape
+    if d != rpbh.d:
+        raise ValueError("W width does not match the RPBH handle")
+    q = torch.empty((N, d), dtype=torch.uint8, device=W.device) if q is None else q
+    scale = torch.empty((N,), dtype=torch.float32, device=W.device) if scale is None else scale
+    zero_point = torch.empty((N,), dtype=torch.uint8, device=W.device) if zero_point is None else zero_point
+    _need_cuda(q, "q", torch.uint8)
+    _need_cuda(scale, "scale", torch.float32)
+    _need_cuda(zero_point, "zero_point", torch.uint8)
+    _check(lib().quantize_weights_int8_asym(rpbh.handle, _ptr(W), _dtype_code(W), N, _ptr(q), _ptr(scale),
+                                            _ptr(zero_point), _stream(stream)), "quantize_weights_int8_asym")
+    return q, scale, zero_point
+
+
+def qlinear_int8_asym(xrot, q, scale, zero_point, out=None, stream=None):
+    """Y = bf16(scale[n] * sum_k (q[n,k] - z[n]) * x'[m,k]) on asymmetric INT8 weights."""
+    import torch
+    _need_cuda(xrot, "xrot", torch.bfloat16)
+    _need_cuda(q, "q", torch.uint8)
+    _need_cuda(scale, "scale", torch.float32)
+    _need_cuda(zero_point, "zero_point", torch.uint8)
+    M, K = xrot.shape
+    N = q.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xrot.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _check(lib().qlinear_int8_asym(_ptr(xrot), _ptr(q), _ptr(scale), _ptr(zero_point), M, N, K, _ptr(out),
+                                   _stream(stream)), "qlinear_int8_asym")
     return out
 
 

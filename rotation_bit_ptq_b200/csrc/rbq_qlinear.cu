@@ -249,7 +249,7 @@ int launch_qgemm(const QParams& p, cudaStream_t st) {
 namespace rbq {
 bool qlinear_int8_fast_eligible(int M, int N, int K);
 int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float* scale, int M, int N, int K,
-                             uint16_t* Y, unsigned int* err, cudaStream_t st);
+                             uint16_t* Y, unsigned int* err, cudaStream_t st, const uint8_t* zero_point = nullptr);
 bool qlinear_fast_eligible(int M, int N, int K, int bits_a, int bits_w);
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
@@ -322,4 +322,18 @@ extern "C" int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float*
   p.Y = Y;
   p.err = err;
   return launch_qgemm<true>(p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int qlinear_int8_asym(const uint16_t* Xrot, const uint8_t* Wq, const float* scale,
+                                 const uint8_t* zero_point, int M, int N, int K, uint16_t* Y, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % kH || K > kMaxD) return RBQ_EINVAL;
+  if (M == 0 || N == 0) return RBQ_OK;
+  if (!Xrot || !Wq || !scale || !zero_point || !Y) return RBQ_EINVAL;
+  if (!qlinear_int8_fast_eligible(M, N, K)) return RBQ_EINVAL;
+  if (!aligned(Xrot, 16) || !aligned(Wq, 16) || !aligned(Y, 16) || !aligned(scale, 4)) return RBQ_EALIGN;
+  unsigned int* err = nullptr;
+  const int rc = device_error_word_ptr(&err);
+  if (rc != RBQ_OK) return rc;
+  return qlinear_int8_fast_launch(Xrot, reinterpret_cast<const int8_t*>(Wq), scale, M, N, K, Y, err,
+                                  static_cast<cudaStream_t>(stream), zero_point);
 }

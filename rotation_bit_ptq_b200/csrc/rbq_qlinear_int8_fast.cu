@@ -210,6 +210,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// uint8 q [N, K] with a zero point per row -> bf16 (q - z) [N, K], 16 values
+// per thread; |q - z| <= 255 is exact in bf16, so the layer needs no extra
+// epilogue term (the asymmetric variant of INT8-convrot's "quantized model
+// file": scale and zero point per channel).  K % 16 == 0: a group never
+// straddles two rows.
+__global__ void __launch_bounds__(256) widen_u8_zp_kernel(const uint8_t* q, const uint8_t* zp, int K,
+                                                          long long groups, uint16_t* out) {
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int z = zp[(g * 16) / K];
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(q) + g);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int a = static_cast<int>((w[i] >> (16 * h)) & 0xFFu) - z;
+        const int b = static_cast<int>((w[i] >> (16 * h + 8)) & 0xFFu) - z;
+        const __nv_bfloat162 pr = __floats2bfloat162_rn(static_cast<float>(a), static_cast<float>(b));
+        o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&pr);
+      }
+    }
+    __stcg(reinterpret_cast<uint4*>(out) + 2 * g, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcg(reinterpret_cast<uint4*>(out) + 2 * g + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  }
+}
+
 // int8 [n] -> bf16 [n], 16 values per thread (16 bytes in, 32 bytes out).
 __global__ void __launch_bounds__(256) widen_int8_kernel(const int8_t* q, long long groups, uint16_t* out) {
   for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
@@ -285,7 +313,7 @@ bool qlinear_int8_fast_eligible(int M, int N, int K) {
 }
 
 int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float* scale, int M, int N, int K,
-                             uint16_t* Y, unsigned int* err, cudaStream_t st) {
+                             uint16_t* Y, unsigned int* err, cudaStream_t st, const uint8_t* zero_point) {
   using namespace q8fast;
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
@@ -301,7 +329,11 @@ int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float
   const long long groups = static_cast<long long>(N) * K / 16;
   long long blocks = (groups + 255) / 256;
   if (blocks > 16LL * sms) blocks = 16LL * sms;
-  widen_int8_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(Wq, groups, wb);
+  if (zero_point)
+    widen_u8_zp_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint8_t*>(Wq), zero_point, K,
+                                                                 groups, wb);
+  else
+    widen_int8_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(Wq, groups, wb);
   int rc = RBQ_OK;
   if ((e = cudaGetLastError()) != cudaSuccess) rc = cuda_fail(e);
   CUtensorMap mA, mB;

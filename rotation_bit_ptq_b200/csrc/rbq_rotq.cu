@@ -21,7 +21,7 @@
 namespace rbq {
 namespace {
 
-enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
+enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3, kInt8Asym = 4 };
 
 // Widths up to this use the fast kernel's unclamped [-1, 1] code grid.
 constexpr int kFullGridBits = 6;
@@ -36,6 +36,7 @@ struct RotqParams {
   void* out;             // packed codes | int8 q | bf16 x'
   void* aux;             // float norms | bf16 row norms | float scales | float norms (optional)
   const float* fixed_scale;   // INT8: one scale for every row (not written back), else null
+  uint8_t* zero_point;        // asymmetric INT8: uint8 zero point per row
 };
 
 template <typename Tin> __device__ __forceinline__ float to_f32(Tin v);
@@ -77,7 +78,9 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
   float* rows = reinterpret_cast<float*>(smem_raw);     // [G][d]
   float* red = rows + static_cast<size_t>(G) * d;       // [G][nblk]
   float* tok = red + G * nblk;                           // [G]
-  float* bnd = tok + G;                                  // [2^BITS - 1]
+  float* bnd = tok + G;                                  // [2^BITS - 1] (256 reserved)
+  float* red2 = bnd + 256;                               // [G][nblk] minima (asymmetric INT8)
+  float* tok2 = red2 + G * nblk;                         // [G]
 
   constexpr bool kLloyd = (MODE == kAct || MODE == kWeightLM);
   if (kLloyd) {
@@ -105,19 +108,35 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
       y[i] = p.sign[k] * rows[g * d + p.perm[k]];
     }
     fwht64(y);
-    float acc = 0.f;
+    float acc = (MODE == kInt8Asym) ? -INFINITY : 0.f, acc2 = INFINITY;
 #pragma unroll
     for (int i = 0; i < 64; ++i) {
       y[i] *= 0.125f;                                    // 1/sqrt(64): orthonormal H
-      acc = (MODE == kInt8) ? fmaxf(acc, fabsf(y[i])) : fmaf(y[i], y[i], acc);
+      if constexpr (MODE == kInt8Asym) {
+        acc = fmaxf(acc, y[i]);
+        acc2 = fminf(acc2, y[i]);
+      } else {
+        acc = (MODE == kInt8) ? fmaxf(acc, fabsf(y[i])) : fmaf(y[i], y[i], acc);
+      }
     }
     red[g * nblk + b] = acc;
+    if constexpr (MODE == kInt8Asym) red2[g * nblk + b] = acc2;
     __syncthreads();
     if (b == 0) {
-      float tot = 0.f;
-      for (int j = 0; j < nblk; ++j)
-        tot = (MODE == kInt8) ? fmaxf(tot, red[g * nblk + j]) : tot + red[g * nblk + j];
-      tok[g] = (MODE == kInt8) ? tot : sqrtf(tot);
+      if constexpr (MODE == kInt8Asym) {
+        float hi = -INFINITY, lo = INFINITY;
+        for (int j = 0; j < nblk; ++j) {
+          hi = fmaxf(hi, red[g * nblk + j]);
+          lo = fminf(lo, red2[g * nblk + j]);
+        }
+        tok[g] = hi;
+        tok2[g] = lo;
+      } else {
+        float tot = 0.f;
+        for (int j = 0; j < nblk; ++j)
+          tot = (MODE == kInt8) ? fmaxf(tot, red[g * nblk + j]) : tot + red[g * nblk + j];
+        tok[g] = (MODE == kInt8) ? tot : sqrtf(tot);
+      }
     }
     __syncthreads();
     if (t >= p.T) continue;
@@ -164,6 +183,31 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
       for (int i = 0; i < 4; ++i)
         d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
       if (b == 0 && !p.fixed_scale) static_cast<float*>(p.aux)[t] = scale;
+    } else if constexpr (MODE == kInt8Asym) {
+      // the range [min(w'), max(w')] widened to contain 0, 255 steps; the
+      // zero point is the code of 0
+      const float hi = fmaxf(s, 0.f), lo = fminf(tok2[g], 0.f);
+      const float scale = (hi - lo) / 255.0f;
+      int z = 0;
+      if (scale > 0.f) z = min(255, max(0, __float2int_rn(__fdiv_rn(-lo, scale))));
+      uint8_t* dst = static_cast<uint8_t*>(p.out) + static_cast<size_t>(t) * d + 64 * b;
+      uint32_t packed[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) packed[i] = 0u;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        int q = 0;
+        if (scale > 0.f) q = min(255, max(0, __float2int_rn(__fdiv_rn(y[i], scale)) + z));
+        packed[i >> 2] |= static_cast<uint32_t>(q) << (8 * (i & 3));
+      }
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+      if (b == 0) {
+        static_cast<float*>(p.aux)[t] = scale;
+        p.zero_point[t] = static_cast<uint8_t>(z);
+      }
     } else {   // kRotate
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(t) * d + 64 * b;
       uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -600,7 +644,7 @@ int sm_count() {
 template <int MODE, int BITS, typename Tin>
 int launch_one(const RotqParams& p, cudaStream_t st) {
   const int threads = p.G * p.nblk;
-  const size_t smem = sizeof(float) * (static_cast<size_t>(p.G) * p.d + p.G * p.nblk + p.G + 256);
+  const size_t smem = sizeof(float) * (static_cast<size_t>(p.G) * p.d + 2 * (p.G * p.nblk + p.G) + 256);
   auto kern = rotq_kernel<MODE, BITS, Tin>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -750,6 +794,7 @@ int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X
   p->out = out;
   p->aux = aux;
   p->fixed_scale = fixed_scale;
+  p->zero_point = nullptr;
   if (mode == kAct || mode == kWeightLM) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
@@ -865,4 +910,17 @@ extern "C" int quantize_weights(const rbq_rpbh* r, const void* W, int dtype, int
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return weights_pass(r, W, dtype, d_out, kInt8, 8, codes_or_q, rownorm_or_scale, st, scale);
+}
+
+extern "C" int quantize_weights_int8_asym(const rbq_rpbh* r, const void* W, int dtype, int d_out, uint8_t* q,
+                                          float* scale, uint8_t* zero_point, void* stream) {
+  if (!r || d_out < 0 || (dtype != RBQ_F32 && dtype != RBQ_BF16)) return RBQ_EINVAL;
+  if (d_out == 0) return RBQ_OK;
+  if (!W || !q || !scale || !zero_point) return RBQ_EINVAL;
+  if (!aligned(W, 16) || !aligned(q, 16) || !aligned(scale, 4)) return RBQ_EALIGN;
+  RotqParams p;
+  int rc = prepare(r, kInt8Asym, 8, d_out, W, q, scale, &p);
+  if (rc != RBQ_OK) return rc;
+  p.zero_point = zero_point;
+  return launch_mode<kInt8Asym>(dtype, 8, p, static_cast<cudaStream_t>(stream));
 }

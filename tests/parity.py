@@ -106,6 +106,32 @@ def check_int8(gpu_q, gpu_scale, ora):
     return int(mism.sum())
 
 
+def check_int8_asym(gpu_q, gpu_scale, gpu_z, ora):
+    """Asymmetric INT8 rows: scales to 1e-6 relative; the zero point and every
+    code exact except where the deciding ratio (-lo/scale, w'/scale) lies within
+    the half-integer band, by one step (a row whose zero point moved is then
+    allowed to move as a whole)."""
+    scale_ref, z_ref = ora["scale"], ora["z"]
+    assert np.all((gpu_scale == 0) == (scale_ref == 0))
+    check_rel(gpu_scale[scale_ref > 0], scale_ref[scale_ref > 0], 1e-6, "int8 asym scale")
+    zr = ora["zratio"]
+    zk = np.floor(zr)
+    z_near = np.abs(zr - (zk + 0.5)) <= BAND * np.maximum(np.abs(zk + 0.5), 1.0)
+    zmis = gpu_z != z_ref
+    assert not np.any(zmis & ~z_near), "zero points differ outside the band"
+    assert np.all(np.abs(gpu_z[zmis].astype(np.int64) - z_ref[zmis]) <= 1)
+    q_ref = ora["q"] + (gpu_z.astype(np.int64) - z_ref)[:, None]
+    q_ref = np.clip(q_ref, 0, 255)
+    mism = gpu_q != q_ref
+    ratio = ora["ratio"]
+    k = np.floor(ratio)
+    near = np.abs(ratio - (k + 0.5)) <= BAND * np.maximum(np.abs(k + 0.5), 1.0)
+    bad = mism & ~near
+    assert not np.any(bad), f"{int(bad.sum())} asymmetric int8 values differ outside the band"
+    assert np.all(np.abs(gpu_q[mism].astype(np.int64) - q_ref[mism]) == 1)
+    return int(mism.sum())
+
+
 def rel_frobenius(y, ref):
     y = np.asarray(y, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

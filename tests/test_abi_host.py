@@ -138,6 +138,17 @@ def test_kernel_entry_points_validate_before_launch(lib):
     assert lib.qlinear(odd, fake, 4, fake, fake, 4, 8, 8, 64, fake, None) == rbq.RBQ_EALIGN
     assert lib.qlinear_int8(fake, fake, fake, 8, 8, 96, fake, None) == rbq.RBQ_EINVAL
     assert lib.qlinear_int8(fake, odd, fake, 8, 8, 64, fake, None) == rbq.RBQ_EALIGN
+    # per-tensor INT8 takes bits 8 only; the zero-point variants
+    assert lib.quantize_weights(h, fake, rbq.RBQ_BF16, 4, rbq.RBQ_INT8_TENSOR, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_weights(h, odd, rbq.RBQ_BF16, 4, rbq.RBQ_INT8_TENSOR, 8, fake, fake, None) == rbq.RBQ_EALIGN
+    assert lib.quantize_weights_int8_asym(h, None, rbq.RBQ_BF16, 0, None, None, None, None) == rbq.RBQ_OK
+    assert lib.quantize_weights_int8_asym(h, fake, rbq.RBQ_BF16, 4, fake, fake, None, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_weights_int8_asym(h, fake, 3, 4, fake, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_weights_int8_asym(h, fake, rbq.RBQ_BF16, 4, odd, fake, fake, None) == rbq.RBQ_EALIGN
+    assert lib.qlinear_int8_asym(fake, fake, fake, fake, 8, 12, 64, fake, None) == rbq.RBQ_EINVAL   # N % 8
+    assert lib.qlinear_int8_asym(fake, fake, fake, fake, 8, 8, 96, fake, None) == rbq.RBQ_EINVAL    # K % 64
+    assert lib.qlinear_int8_asym(fake, fake, fake, None, 8, 8, 64, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_asym(odd, fake, fake, fake, 8, 8, 64, fake, None) == rbq.RBQ_EALIGN
     r.close()
 
 

@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 import synth
-from parity import (bf16_to_numpy, check_bf16_rounding, check_codes, check_int8, check_rel,
+from parity import (bf16_to_numpy, check_bf16_rounding, check_codes, check_int8, check_int8_asym, check_rel,
                     rel_frobenius, torch_bf16)
 
 pytestmark = pytest.mark.gpu
@@ -211,6 +211,30 @@ def test_weights_int8_per_tensor(d, n, dtype):
         torch.cuda.synchronize()
         ref = oracle.qlinear_int8(bf16_to_numpy(xr), q.cpu().numpy().astype(np.float64),
                                   sc.cpu().numpy().astype(np.float64))
+        assert rel_frobenius(bf16_to_numpy(y), ref) < QLINEAR8_RTOL
+
+
+@pytest.mark.parametrize("d,n,dtype", [(1024, 40, "bf16"), (4096, 24, "bf16"), (512, 37, "f32")])
+def test_weights_int8_asymmetric(d, n, dtype):
+    W = synth.gaussian_weights(synth.rng(14, d), n, d, outlier_frac=0.01).astype(np.float32)
+    W[: n // 2] += 0.01                      # some rows skewed, so zero points vary
+    W = synth.to_bf16(W)
+    W[2] = 0.0
+    r, Pi = _rpbh(d, 12)
+    q, sc, z = rbq.quantize_weights_int8_asym(r, _dense(W, dtype))
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.quantize_weights_int8_asym(W.astype(np.float64), Pi)
+    check_int8_asym(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64),
+                    z.cpu().numpy().astype(np.int64), ora)
+    if n % 8 == 0 and dtype == "bf16":
+        X = synth.to_bf16(np.random.default_rng(d + 1).standard_normal((24, d)).astype(np.float32))
+        xr = rbq.rotate_act(r, torch_bf16(X))
+        y = rbq.qlinear_int8_asym(xr, q, sc, z)
+        torch.cuda.synchronize()
+        assert rbq.device_error() == 0
+        ref = oracle.qlinear_int8_asym(bf16_to_numpy(xr), q.cpu().numpy(), sc.cpu().numpy().astype(np.float64),
+                                       z.cpu().numpy())
         assert rel_frobenius(bf16_to_numpy(y), ref) < QLINEAR8_RTOL
 
 

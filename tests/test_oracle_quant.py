@@ -139,6 +139,37 @@ def test_int8_per_tensor_bounds():
     assert np.linalg.norm(wr - scale[0] * q) >= np.linalg.norm(wr - c["scale"][:, None] * c["q"])
 
 
+def test_int8_asymmetric_zero_point_pins():
+    # the range [min, max] (widened to hold 0) is cut into 255 steps: codes
+    # stay in 0..255, 0 maps to exactly the zero point, every value is within
+    # half a step (one step where the top code clips), and on rows whose
+    # values are mostly positive the zero point beats the symmetric scheme
+    data, Pi, _, _ = _tiny_setup()
+    W = data["W"].astype(np.float64)
+    W[3] = 0.0
+    a = oracle.quantize_weights_int8_asym(W, Pi)
+    q, scale, z, wr = a["q"], a["scale"], a["z"], a["wr"]
+    assert q.min() >= 0 and q.max() <= 255
+    assert np.all(q[3] == 0) and scale[3] == 0 and z[3] == 0
+    nz = scale > 0
+    deq = scale[:, None] * (q - z[:, None])
+    err = np.abs(wr - deq)
+    inner = (q > 0) & (q < 255)
+    half = 0.5 * scale[:, None] * (1 + 1e-9)
+    assert np.all((err <= half)[nz & inner.any(axis=1)][inner[nz & inner.any(axis=1)]])
+    assert np.all(err[nz] <= 2 * half[nz])
+    # zero is representable: the code of 0 is z
+    zero_codes = np.clip(np.rint(0.0 / np.where(scale > 0, scale, 1.0)) + z, 0, 255)
+    assert np.array_equal(zero_codes, z)
+    # skewed rows (shifted up): the zero point uses the whole range
+    Ws = oracle.rpbh_apply(Pi.T, np.abs(oracle.rpbh_apply(Pi, W)) + 0.01)   # rotated rows all positive
+    asym = oracle.quantize_weights_int8_asym(Ws, Pi)
+    sym = oracle.quantize_weights_int8(Ws, Pi)
+    e_asym = np.linalg.norm(asym["wr"] - asym["scale"][:, None] * (asym["q"] - asym["z"][:, None]))
+    e_sym = np.linalg.norm(sym["wr"] - sym["scale"][:, None] * sym["q"])
+    assert e_asym < 0.6 * e_sym
+
+
 def test_int8_bounds_and_rotation_helps():
     data, Pi, _, _ = _tiny_setup()
     W = data["W"].astype(np.float64)
