@@ -54,6 +54,7 @@ extern "C" {
 #define RBQ_ECONVERGE  (-5)  /* Lloyd-Max solver did not converge               */
 #define RBQ_EDEVICE    (-6)  /* kernel reported an internal error (see below)   */
 #define RBQ_ESCRATCH   (-7)  /* problem larger than a fixed scratch area        */
+#define RBQ_EIO        (-8)  /* layer file: open/read/write failed or not valid */
 
 /* ---- element types and modes --------------------------------------------- */
 #define RBQ_F32    0
@@ -109,6 +110,11 @@ void rpbh_free(rbq_rpbh* r);
 /* rpbh_export -- copy pi (int32[d]) and D (int8[d], +-1) to HOST buffers.
  * Either pointer may be NULL.  Errors: RBQ_EINVAL. */
 int rpbh_export(const rbq_rpbh* r, int32_t* perm_host, int8_t* signs_host);
+
+/* rpbh_describe -- the transform info that rebuilds the handle exactly:
+ * rpbh_make_ablation(d, h, seed, flags) draws the same pi and D.  Any output
+ * pointer may be NULL.  Errors: RBQ_EINVAL. */
+int rpbh_describe(const rbq_rpbh* r, int* d, int* h, uint64_t* seed, int* flags);
 
 /* rpbh_dim -- d of a handle, or RBQ_EINVAL for NULL. */
 int rpbh_dim(const rbq_rpbh* r);
@@ -294,6 +300,50 @@ int rbq_code_grid(int d, int bits, int variant, float* thr, int32_t* base, int* 
  */
 int qlinear_int8_asym(const uint16_t* Xrot, const uint8_t* Wq, const float* scale, const uint8_t* zero_point,
                       int M, int N, int K, uint16_t* Y, void* stream);
+
+/* ---- quantised layer files ------------------------------------------------
+ * The pages' "quantized model file" (INT8-convrot, section 1): the quantised
+ * weights, their quantisation parameters (scale, zero point or row norms) and
+ * the transform info that reproduces the rotation at inference.  One file per
+ * linear layer; the transform is stored as the RPBH draw (d, h, seed, flags),
+ * from which rpbh_make_ablation rebuilds pi and D exactly.  Host buffers only
+ * (the caller moves them to and from the device).
+ *
+ * Layout (little-endian): 64-byte header -- "RBQLAYER", version u32 = 1,
+ * header size u32 = 64, d, h, rpbh_flags, mode, bits, rows (i32 each),
+ * seed u64, FNV-1a-64 checksum of the payload u64, zero padding -- then the
+ * payload: codes, aux, zero points, back to back.
+ */
+#define RBQ_LAYER_LLOYDMAX    0   /* packed codes [rows, d*bits/8] + BF16 r' [rows]       */
+#define RBQ_LAYER_INT8_SYM    1   /* int8 q [rows, d] + fp32 scale [rows]                  */
+#define RBQ_LAYER_INT8_TENSOR 2   /* int8 q [rows, d] + fp32 scale [rows] (one value)      */
+#define RBQ_LAYER_INT8_ASYM   3   /* uint8 q [rows, d] + fp32 scale + uint8 zero point [rows] */
+
+typedef struct rbq_layer_info {
+  int32_t d;           /* input width (a multiple of h)            */
+  int32_t h;           /* Hadamard block size (64)                 */
+  uint64_t seed;       /* RPBH seed                                */
+  int32_t rpbh_flags;  /* RBQ_RPBH_NO_* of the draw                */
+  int32_t mode;        /* RBQ_LAYER_*                              */
+  int32_t bits;        /* code width; 8 for the INT8 modes         */
+  int32_t rows;        /* output channels                          */
+} rbq_layer_info;
+
+/* rbq_layer_sizes -- payload sizes in bytes for `info` (any output may be
+ * NULL).  Errors: RBQ_EINVAL for an inconsistent info. */
+int rbq_layer_sizes(const rbq_layer_info* info, uint64_t* codes_bytes, uint64_t* aux_bytes, uint64_t* zp_bytes);
+
+/* rbq_layer_write -- write a layer file.  `codes`, `aux` and (RBQ_LAYER_INT8_ASYM
+ * only) `zero_point` are HOST buffers of the sizes rbq_layer_sizes gives.
+ * Errors: RBQ_EINVAL, RBQ_EIO. */
+int rbq_layer_write(const char* path, const rbq_layer_info* info, const void* codes, const void* aux,
+                    const void* zero_point);
+
+/* rbq_layer_read -- read a layer file's info and, when the buffer pointers are
+ * not NULL, its payload into HOST buffers sized by rbq_layer_sizes(info).
+ * The checksum is verified whenever the payload is read.
+ * Errors: RBQ_EINVAL, RBQ_EIO (missing, short, corrupt or foreign file). */
+int rbq_layer_read(const char* path, rbq_layer_info* info, void* codes, void* aux, void* zero_point);
 
 const char* rbq_error_string(int code);
 

@@ -23,6 +23,17 @@ RBQ_ROTATE_ONLY = 16
 RBQ_OK, RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA, RBQ_ENOMEM, RBQ_ECONVERGE, RBQ_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 RBQ_ESCRATCH = -7
 RBQ_RPBH_NO_PERMUTATION, RBQ_RPBH_NO_SIGNS = 1, 2
+RBQ_EIO = -8
+RBQ_LAYER_LLOYDMAX, RBQ_LAYER_INT8_SYM, RBQ_LAYER_INT8_TENSOR, RBQ_LAYER_INT8_ASYM = 0, 1, 2, 3
+_LAYER_KINDS = {"lloydmax": RBQ_LAYER_LLOYDMAX, "int8": RBQ_LAYER_INT8_SYM, "int8_tensor": RBQ_LAYER_INT8_TENSOR,
+                "int8_asym": RBQ_LAYER_INT8_ASYM}
+
+
+class LayerInfo(ctypes.Structure):
+    """rbq_layer_info of include/rbq.h."""
+    _fields_ = [("d", ctypes.c_int32), ("h", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("rpbh_flags", ctypes.c_int32), ("mode", ctypes.c_int32), ("bits", ctypes.c_int32),
+                ("rows", ctypes.c_int32)]
 
 # name -> (restype, argtypes); mirrors include/rbq.h
 _P, _I, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64
@@ -32,6 +43,10 @@ SIGNATURES = {
     "rpbh_free": (None, [_P]),
     "rpbh_export": (_I, [_P, _P, _P]),
     "rpbh_dim": (_I, [_P]),
+    "rpbh_describe": (_I, [_P, _P, _P, _P, _P]),
+    "rbq_layer_sizes": (_I, [_P, _P, _P, _P]),
+    "rbq_layer_write": (_I, [ctypes.c_char_p, _P, _P, _P, _P]),
+    "rbq_layer_read": (_I, [ctypes.c_char_p, _P, _P, _P, _P]),
     "lloydmax_table": (_I, [_I, _I, _P, _P]),
     "rotate_quantize_act": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "quantize_weights": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
@@ -134,6 +149,19 @@ class RPBH:
         if self._h is None:
             raise ValueError("RPBH handle already freed")
         return self._h
+
+    @classmethod
+    def from_description(cls, d, seed, flags, h=64):
+        return cls(d, seed, h=h, permute=not (flags & RBQ_RPBH_NO_PERMUTATION),
+                   signs=not (flags & RBQ_RPBH_NO_SIGNS))
+
+    def describe(self):
+        """(d, h, seed, flags): the transform info that rebuilds this handle."""
+        d, h, flags = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        seed = ctypes.c_uint64()
+        _check(lib().rpbh_describe(self.handle, ctypes.byref(d), ctypes.byref(h), ctypes.byref(seed),
+                                   ctypes.byref(flags)), "rpbh_describe")
+        return d.value, h.value, seed.value, flags.value
 
     def export(self):
         perm = np.empty(self.d, dtype=np.int32)
@@ -322,6 +350,68 @@ def qlinear_int8_asym(xrot, q, scale, zero_point, out=None, stream=None):
     _need_cuda(out, "out", torch.bfloat16)
     _check(lib().qlinear_int8_asym(_ptr(xrot), _ptr(q), _ptr(scale), _ptr(zero_point), M, N, K, _ptr(out),
                                    _stream(stream)), "qlinear_int8_asym")
+    return out
+
+
+def _host_bytes(t):
+    """A contiguous host numpy copy of a torch tensor or array (bytes only)."""
+    if hasattr(t, "detach"):
+        t = t.detach().contiguous().cpu()
+        import torch
+        return np.ascontiguousarray(t.view(torch.uint8).numpy()) if t.dtype != torch.uint8 else \
+            np.ascontiguousarray(t.numpy())
+    return np.ascontiguousarray(t)
+
+
+def save_layer(path, rpbh, kind, codes, aux, zero_point=None, bits=None):
+    """Write one quantised linear layer (weights, quantisation parameters and
+    the transform info) to `path`: kind 'lloydmax' (codes + BF16 r', give
+    bits), 'int8', 'int8_tensor' or 'int8_asym' (+ zero_point)."""
+    d, h, seed, flags = rpbh.describe()
+    mode = _LAYER_KINDS[kind]
+    rows = codes.shape[0]
+    info = LayerInfo(d, h, seed, flags, mode, int(bits) if mode == RBQ_LAYER_LLOYDMAX else 8, rows)
+    c, a = _host_bytes(codes), _host_bytes(aux)
+    z = _host_bytes(zero_point) if zero_point is not None else None
+    nc, na, nz = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check(lib().rbq_layer_sizes(ctypes.byref(info), ctypes.byref(nc), ctypes.byref(na), ctypes.byref(nz)),
+           "rbq_layer_sizes")
+    if c.nbytes != nc.value or a.nbytes != na.value or (nz.value and (z is None or z.nbytes != nz.value)):
+        raise ValueError("array sizes do not match the layer description")
+    _check(lib().rbq_layer_write(os.fsencode(path), ctypes.byref(info), c.ctypes.data_as(_P), a.ctypes.data_as(_P),
+                                 z.ctypes.data_as(_P) if z is not None else None), "rbq_layer_write")
+
+
+def load_layer(path, device=None):
+    """Read a layer file: dict(kind, bits, rpbh (rebuilt from the transform
+    info), codes, aux, zero_point) -- numpy arrays, or torch tensors on
+    `device` when given."""
+    info = LayerInfo()
+    _check(lib().rbq_layer_read(os.fsencode(path), ctypes.byref(info), None, None, None), "rbq_layer_read")
+    nc, na, nz = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check(lib().rbq_layer_sizes(ctypes.byref(info), ctypes.byref(nc), ctypes.byref(na), ctypes.byref(nz)),
+           "rbq_layer_sizes")
+    c = np.empty(nc.value, dtype=np.uint8)
+    a = np.empty(na.value, dtype=np.uint8)
+    z = np.empty(nz.value, dtype=np.uint8) if nz.value else None
+    _check(lib().rbq_layer_read(os.fsencode(path), ctypes.byref(info), c.ctypes.data_as(_P), a.ctypes.data_as(_P),
+                                z.ctypes.data_as(_P) if z is not None else None), "rbq_layer_read")
+    kind = {v: k for k, v in _LAYER_KINDS.items()}[info.mode]
+    rows, d = info.rows, info.d
+    if kind == "lloydmax":
+        codes, aux = c.reshape(rows, d * info.bits // 8), a.view(np.uint16)
+    else:
+        codes = c.reshape(rows, d).view(np.int8 if kind != "int8_asym" else np.uint8)
+        aux = a.view(np.float32)
+    out = {"kind": kind, "bits": info.bits, "d": d, "rows": rows,
+           "rpbh": RPBH.from_description(d, info.seed, info.rpbh_flags, h=info.h),
+           "codes": codes, "aux": aux, "zero_point": z}
+    if device is not None:
+        import torch
+        out["codes"] = torch.from_numpy(np.ascontiguousarray(codes)).to(device)
+        aux_t = torch.from_numpy(np.ascontiguousarray(aux))
+        out["aux"] = (aux_t.view(torch.bfloat16) if kind == "lloydmax" else aux_t).to(device)
+        out["zero_point"] = torch.from_numpy(z).to(device) if z is not None else None
     return out
 
 

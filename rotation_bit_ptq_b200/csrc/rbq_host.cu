@@ -472,6 +472,7 @@ extern "C" int rpbh_make_ablation(int d, int h, uint64_t seed, int flags, rbq_rp
   const int rc = rpbh_make(d, h, seed, out);
   if (rc != RBQ_OK) return rc;
   rbq_rpbh* r = *out;
+  r->flags = flags;
   if (flags & RBQ_RPBH_NO_PERMUTATION)
     for (int k = 0; k < d; ++k) r->perm[k] = k;
   if (flags & RBQ_RPBH_NO_SIGNS)
@@ -488,6 +489,15 @@ extern "C" void rpbh_free(rbq_rpbh* r) {
     cudaFree(D.pair_tab);
   }
   delete r;
+}
+
+extern "C" int rpbh_describe(const rbq_rpbh* r, int* d, int* h, uint64_t* seed, int* flags) {
+  if (!r) return RBQ_EINVAL;
+  if (d) *d = r->d;
+  if (h) *h = kH;
+  if (seed) *seed = r->seed;
+  if (flags) *flags = r->flags;
+  return RBQ_OK;
 }
 
 extern "C" int rpbh_export(const rbq_rpbh* r, int32_t* perm_host, int8_t* signs_host) {
@@ -519,6 +529,7 @@ extern "C" const char* rbq_error_string(int code) {
     case RBQ_ECONVERGE: return "Lloyd-Max solver did not converge";
     case RBQ_EDEVICE: return "kernel reported an internal error (bounded wait expired)";
     case RBQ_ESCRATCH: return "problem exceeds the fixed scratch area (qlinear_noalloc: N*K <= 16777216)";
+    case RBQ_EIO: return "layer file could not be opened, read or written, or is not a valid layer file";
     default: return "unknown error code";
   }
 }

@@ -39,6 +39,7 @@ __host__ __device__ inline uint32_t pair_tab_slot(int b, int i) {
 struct rbq_rpbh {
   int d = 0;
   uint64_t seed = 0;
+  int flags = 0;                  // RBQ_RPBH_NO_* ablation flags of the draw
   std::vector<int32_t> perm;      // pi
   std::vector<int8_t> sign;       // D
   rbq::RpbhDevice dev[rbq::kMaxDevices];
