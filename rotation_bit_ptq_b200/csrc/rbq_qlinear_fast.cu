@@ -127,16 +127,17 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Byte planes of the eight positive fp16 levels C[8..15].
+// Byte planes of the positive fp16 levels C[half + m], m < half <= 8 (the
+// codebooks are antisymmetric: C[L-1-c] = -C[c], exactly, also in fp16).
 struct Planes4 {
   uint32_t lo0, lo1, hi0, hi1;
 };
 
-__device__ __forceinline__ Planes4 make_planes4(const uint16_t* lut) {
+__device__ __forceinline__ Planes4 make_planes_sym(const uint16_t* lut, int half) {
   Planes4 p{0, 0, 0, 0};
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
-    const uint32_t v = lut[8 + m];
+    const uint32_t v = (m < half) ? lut[half + m] : 0u;
     const uint32_t lo = v & 0xFFu, hi = v >> 8;
     if (m < 4) {
       p.lo0 |= lo << (8 * m);
@@ -149,10 +150,17 @@ __device__ __forceinline__ Planes4 make_planes4(const uint16_t* lut) {
   return p;
 }
 
-// Eight 4-bit codes (x, LSB first) -> eight fp16 levels in four words.
-__device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint32_t (&w)[4]) {
-  const uint32_t neg = (~x >> 3) & 0x11111111u;           // 1 where c < 8
-  const uint32_t m = (x ^ (neg * 7u)) & 0x77777777u;      // c<8: 7-c, else c-8
+__device__ __forceinline__ Planes4 make_planes4(const uint16_t* lut) { return make_planes_sym(lut, 8); }
+
+// Eight codes of width B <= 4, one per nibble (x, LSB first) -> eight fp16
+// levels in four words: the top bit of a code picks the half, the rest
+// (mirrored in the lower half) indexes the positive levels through byte
+// permutes, and the sign lands on the high byte.
+template <int B>
+__device__ __forceinline__ void expand8_sym(uint32_t x, const Planes4& P, uint32_t (&w)[4]) {
+  constexpr uint32_t kMag = (1u << (B - 1)) - 1u;
+  const uint32_t neg = (~x >> (B - 1)) & 0x11111111u;     // 1 where c < half
+  const uint32_t m = (x ^ (neg * kMag)) & (0x11111111u * kMag);   // c<half: half-1-c, else c-half
   const uint32_t a7 = neg << 7, a3 = neg << 3;            // 0xFF bytes where negative
   const uint32_t s_lo = prmt(a7, a3, 0xD9C8u);
   const uint32_t s_hi = prmt(a7, a3, 0xFBEAu);
@@ -165,6 +173,29 @@ __device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint3
   w[1] = prmt(lo0, hi0, 0x7362u);
   w[2] = prmt(lo1, hi1, 0x5140u);
   w[3] = prmt(lo1, hi1, 0x7362u);
+}
+__device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint32_t (&w)[4]) {
+  expand8_sym<4>(x, P, w);
+}
+
+// Codes 8c .. 8c+7 of a row's LSB-first bitstream of B-bit codes (B = 2, 3),
+// one per nibble.
+template <int B>
+__device__ __forceinline__ uint32_t spread8(const uint32_t* src, int c) {
+  if constexpr (B == 2) {
+    uint32_t x = (src[c >> 1] >> (16 * (c & 1))) & 0xFFFFu;
+    x = (x | (x << 8)) & 0x00FF00FFu;
+    x = (x | (x << 4)) & 0x0F0F0F0Fu;
+    return (x | (x << 2)) & 0x33333333u;
+  } else {
+    const int bit = 24 * c, wi = bit >> 5, sh = bit & 31;
+    uint32_t u = src[wi] >> sh;
+    if (sh > 8) u |= src[wi + 1] << (32 - sh);
+    uint32_t x = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x |= ((u >> (3 * k)) & 7u) << (4 * k);
+    return x;
+  }
 }
 
 template <int BITS>
@@ -181,6 +212,14 @@ __device__ __forceinline__ void expand_row(const uint32_t (&src)[slice_words<BIT
     for (int c = 4 * HF; c < 4 * HF + 4; ++c) {
       uint32_t w[4];
       expand8_4bit(src[c], P, w);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[4 * (c - 4 * HF) + j] = w[j];
+    }
+  } else if constexpr (BITS == 2 || BITS == 3) {
+#pragma unroll
+    for (int c = 4 * HF; c < 4 * HF + 4; ++c) {
+      uint32_t w[4];
+      expand8_sym<BITS>(spread8<BITS>(src, c), P, w);
 #pragma unroll
       for (int j = 0; j < 4; ++j) out[4 * (c - 4 * HF) + j] = w[j];
     }
@@ -455,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warps 6..13: lane quarter warp % 4, code half (warp - 6) / 4
     const int r = 32 * (warp & 3) + lane;
     const uint16_t* lut = tl->lut_a;
-    const Planes4 P = make_planes4(lut);
+    const Planes4 P = make_planes_sym(lut, p.bits_a <= 4 ? (1 << (p.bits_a - 1)) : 8);
     if (warp < 10) {
       switch (p.bits_a) {
         case 1: expand_loop<1, 0>(p, tl, ops, codes, r, ntiles, P, lut); break;
