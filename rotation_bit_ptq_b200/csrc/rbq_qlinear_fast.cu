@@ -28,11 +28,12 @@
 //                  stages and (b) the 256 x 64 fp16 weight tile of each K
 //                  slice straight into the operand stage, 128B-swizzled as the
 //                  tensor core reads it.
-//      warps 6..13 activation expansion, two threads per row (warps w and
-//                  w+4 take the two halves of the row's 64 codes): read the
-//                  codes of a K slice from the code stage, turn them into
-//                  fp16 levels before waiting for the stage, then write them
-//                  into the stage's swizzled K-major A tile.
+//      warps 6..13 activation expansion, a thread per row, two warp groups
+//                  taking alternate K slices (warps 6..9 the even ones, 10..13
+//                  the odd ones), so two slices are in flight in this stage:
+//                  read the row's 64 codes of the slice from the code stage,
+//                  turn them into fp16 levels before waiting for the stage,
+//                  then write them into the stage's swizzled K-major A tile.
 //    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
 //    overlap the MMAs of tile i+1.  (A variant that kept the activation tile
 //    in tensor memory, written with tcgen05.st, measured slower: the stores
@@ -284,37 +285,42 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* 
   return mbar_warp_wait(bar, parity, &tl->abort);
 }
 
-// Row r = 32 (warp % 4) + lane of every activation tile, code half HF.
-template <int BITS, int HF>
+// Row r = 32 (warp % 4) + lane of every activation tile, whole rows of the K
+// slices of parity G (2 kp + G): the two warp groups expand alternate slices,
+// so two slices are in flight in the expansion stage.
+template <int BITS, int G>
 __device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, int r,
                                             int ntiles, Planes4 P, const uint16_t* lut) {
   const CodeGeo& g = p.ga;
   const int KP = p.K / (2 * kBK);
   const uint32_t C = static_cast<uint32_t>(p.C);
-  uint32_t c = 0, cph = 0, s = 0, aph = 0;       // code stage / A stage and their phases
+  uint32_t c = 0, cph = 0, s = G, aph = 0;       // code stage / A stage and their phases
   bool a_first = true;                           // first round of A stages: nothing to wait for
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     for (int kp = 0; kp < KP; ++kp) {
       if (!warp_wait(&tl->cfull[c], cph, tl)) return;
       const uint8_t* part = codes + c * p.cstage_bytes + g.offset;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t cur[slice_words<BITS>()];
-        read_slice<BITS>(part, g, r, h, cur);
-        uint32_t w[16];
-        expand_row<BITS, HF>(cur, P, lut, w);          // before the wait: off the critical path
-        if (!a_first && !warp_wait(&tl->empty[s], aph ^ 1u, tl)) return;
-        uint8_t* tile = ops + s * kOpStage;            // the stage's A tile, 128B-swizzled K-major
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(tile + sw128_offset(r, 4 * HF + c)) =
-              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-        fence_proxy_async_smem();                      // visible to the tensor core
-        mbar_arrive(&tl->full[s]);
-        if (++s == kAStages) { s = 0; aph ^= 1u; a_first = false; }
-      }
-      mbar_arrive(&tl->cempty[c]);
+      uint32_t cur[slice_words<BITS>()];
+      read_slice<BITS>(part, g, r, G, cur);
+      uint32_t w0[16], w1[16];
+      expand_row<BITS, 0>(cur, P, lut, w0);          // before the wait: off the critical path
+      expand_row<BITS, 1>(cur, P, lut, w1);
+      mbar_arrive(&tl->cempty[c]);                     // the codes are in registers now
       if (++c == C) { c = 0; cph ^= 1u; }
+      if (!a_first && !warp_wait(&tl->empty[s], aph ^ 1u, tl)) return;
+      uint8_t* tile = ops + s * kOpStage;              // the stage's A tile, 128B-swizzled K-major
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(tile + sw128_offset(r, q)) =
+            make_uint4(w0[4 * q], w0[4 * q + 1], w0[4 * q + 2], w0[4 * q + 3]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(tile + sw128_offset(r, 4 + q)) =
+            make_uint4(w1[4 * q], w1[4 * q + 1], w1[4 * q + 2], w1[4 * q + 3]);
+      fence_proxy_async_smem();                        // visible to the tensor core
+      mbar_arrive(&tl->full[s]);
+      s += 2;                                          // this group's next slice
+      if (s >= kAStages) { s -= kAStages; aph ^= 1u; a_first = false; }
     }
   }
 }
@@ -336,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = tid; i < 256; i += kThreads) tl->lut_a[i] = (i < (1 << p.bits_a)) ? p.lut_a[i] : 0;
   if (tid == 0) {
     for (int s = 0; s < kMaxF; ++s) {
-      mbar_init(&tl->full[s], kExpandThreads + 1);   // + the producer's expect-tx arrival
+      mbar_init(&tl->full[s], kBM + 1);   // one warp group (a thread per row) + the producer's expect-tx arrival
       mbar_init(&tl->empty[s], 1);
     }
     for (int c = 0; c < p.C; ++c) {
@@ -491,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- activation expansion ----------------
-    // warps 6..13: lane quarter warp % 4, code half (warp - 6) / 4
+    // warps 6..13: lane quarter warp % 4, slice parity (warp - 6) / 4
     const int r = 32 * (warp & 3) + lane;
     const uint16_t* lut = tl->lut_a;
     const Planes4 P = make_planes_sym(lut, p.bits_a <= 4 ? (1 << (p.bits_a - 1)) : 8);
