@@ -79,7 +79,7 @@ constexpr int kMaxF = kAStages, kMaxC = 8;     // operand stages, code stages
 // Tensor memory: two fp32 accumulators of kBN columns (512 columns).
 constexpr int kThreads = 448;                  // 14 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
-constexpr int kExpandThreads = 2 * kBM;        // two threads per activation row (32 codes each)
+constexpr int kExpandThreads = 2 * kBM;        // two warp groups of a thread per activation row
 constexpr size_t kSmemLimit = 227 * 1024;
 
 // Code-stage geometry of the activation operand.
