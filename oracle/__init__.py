@@ -42,6 +42,9 @@ quant.pack/unpack      hand-made bit-layout fixture (tests/golden)
 quant.quantize_*       invariants (norm, cancellation, INT8 bounds; per-tensor
                        and zero-point variants: range, bound and code-of-0 pins)
 qlinear.*              pure-Python triple loop; equal-code closed form
+qlinear.int8_levels    J. Max (1960) 16-level table rounded by hand
+                       (tests/golden); grid bounds and antisymmetry; the
+                       layer within its rounding bound of the exact one
 =====================  ===================================================
 """
 
@@ -52,7 +55,7 @@ from .bf16 import round_to_bf16
 from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
                     quantize_weights_lloydmax, quantize_weights_int8,
                     quantize_weights_int8_asym, rotate_only, EPS)
-from .qlinear import qlinear, qlinear_int8, qlinear_int8_asym
+from .qlinear import qlinear, qlinear_int8, qlinear_int8_asym, int8_levels, qlinear_int8_levels
 
 __all__ = [
     "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_rows", "rpbh_apply",
@@ -60,5 +63,5 @@ __all__ = [
     "round_to_bf16", "assign_codes", "pack_codes", "unpack_codes",
     "quantize_act", "quantize_weights_lloydmax", "quantize_weights_int8",
     "quantize_weights_int8_asym", "rotate_only", "EPS", "qlinear", "qlinear_int8",
-    "qlinear_int8_asym",
+    "qlinear_int8_asym", "int8_levels", "qlinear_int8_levels",
 ]

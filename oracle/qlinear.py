@@ -11,7 +11,17 @@ INT8 path (INT8-convrot §4: "load W_int8, dequantise or use an INT8 operator"):
 
     y[m, n] = scale_n · sum_k q_nk · x'_mk,   x' = bf16(Pi x).
 
-Both are plain definitions; the oracle evaluates them with one fp64 matmul.
+8-bit integer-level variant (a deployment form of the first layer for INT8
+tensor cores, in the spirit of OrbitQuant §4.2-§4.4: start from W8A8, lower
+the widths; the pages do not define it, so its definition is ours): every
+codebook's levels c_j are put on a signed 8-bit grid,
+
+    alpha = 127 / max_j |c_j|,   l_j = round_half_even(alpha · c_j),
+
+and y[m, n] = s_m · r'_n · (sum_k l_w[q_nk] · l_a[p_mk]) / (alpha_w · alpha_a),
+the sum an exact integer.
+
+All are plain definitions; the oracle evaluates them with one matmul.
 """
 
 import numpy as np
@@ -36,3 +46,22 @@ def qlinear_int8_asym(xr, q, scale, z):
     xr = np.asarray(xr, dtype=np.float64)
     qz = np.asarray(q, dtype=np.float64) - np.asarray(z, dtype=np.float64)[:, None]
     return (xr @ qz.T) * np.asarray(scale, dtype=np.float64)[None, :]
+
+
+def int8_levels(levels):
+    """(l int64[L], alpha): levels on the signed 8-bit grid, l = RNE(alpha c)
+    with alpha = 127 / max |c| (np.rint rounds halves to even); fp64 throughout."""
+    c = np.asarray(levels, dtype=np.float64)
+    alpha = 127.0 / np.max(np.abs(c))
+    return np.rint(alpha * c).astype(np.int64), alpha
+
+
+def qlinear_int8_levels(a_codes, s, levels_a, w_codes, rnorm, levels_w):
+    """y = s_m r'_n (sum_k l_w[q_nk] l_a[p_mk]) / (alpha_w alpha_a); the integer
+    sum is exact (int64), the scaling fp64."""
+    la, alpha_a = int8_levels(levels_a)
+    lw, alpha_w = int8_levels(levels_w)
+    acc = la[np.asarray(a_codes)] @ lw[np.asarray(w_codes)].T
+    s = np.asarray(s, dtype=np.float64)
+    r = np.asarray(rnorm, dtype=np.float64)
+    return acc.astype(np.float64) * s[:, None] * r[None, :] / (alpha_a * alpha_w)
