@@ -234,6 +234,36 @@ int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float* scale,
                  int M, int N, int K, uint16_t* Y, void* stream);
 
 /*
+ * qlinear_int8_levels -- the quantised linear layer with each codebook's
+ * levels rounded onto a signed 8-bit grid, run on the INT8 tensor cores
+ * (tcgen05 kind::i8) with exact int32 accumulation.  A deployment variant of
+ * qlinear (OrbitQuant §2.2, "Online inference": the same codes, norms and
+ * cancellation) for 8-bit integer tensor cores, the kind of low-precision
+ * operator OrbitQuant §4.2-§4.4 points deployments to (start from W8A8, then
+ * lower the widths); the pages do not define it, so its result is its own:
+ *   l_b[j] = RNE(alpha_b * c_j),  alpha_b = 127 / max_j |c_j|   (int8 levels)
+ *   Y[m, n] = bf16( s[m] * r'[n] * (sum_k l_w[q_nk] * l_a[p_mk]) / (alpha_w * alpha_a) )
+ * with c_j the N(0, 1/K) Lloyd-Max levels of lloydmax_table(K, bits); the
+ * integer sum is exact, the scaling is fp32.  rbq_int8_levels returns l and
+ * alpha.  Arguments, layouts and ownership as qlinear.
+ * Limits: K a multiple of 128, N a multiple of 8, K*bits_a/8 a multiple of
+ * 16 (else RBQ_EINVAL; there is no fallback kernel).
+ * The weight codes are expanded once per call into an int8 workspace of N*K
+ * bytes from a stream-ordered memory pool.
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECONVERGE, RBQ_ECUDA.
+ */
+int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int bits_a,
+                        const uint8_t* w_codes, const uint16_t* rnorm, int bits_w,
+                        int M, int N, int K, uint16_t* Y, void* stream);
+
+/*
+ * rbq_int8_levels -- the integer levels qlinear_int8_levels uses for (d, bits)
+ * (host only): levels HOST int8[2^bits] (may be NULL), alpha HOST double
+ * (may be NULL).  Returns RBQ_OK, RBQ_EINVAL or RBQ_ECONVERGE.
+ */
+int rbq_int8_levels(int d, int bits, int8_t* levels, double* alpha);
+
+/*
  * qlinear_noalloc -- the same result as qlinear, for callers that cannot
  * allocate device memory.  (The pages have no counterpart: this is a
  * deployment variant of the library, not a step of the method.)
@@ -287,7 +317,6 @@ int qlinear_noalloc(const uint8_t* a_codes, const float* s, int bits_a,
  */
 int rbq_code_grid(int d, int bits, int variant, float* thr, int32_t* base, int* cells, float* scale);
 
-/* Text for a return code (static storage). */
 /*
  * qlinear_int8_asym -- the W8A16 layer on asymmetric INT8 weights:
  *   Y[m, n] = bf16( scale[n] * sum_k (q[n,k] - z[n]) * Xrot[m,k] ),
@@ -345,6 +374,7 @@ int rbq_layer_write(const char* path, const rbq_layer_info* info, const void* co
  * Errors: RBQ_EINVAL, RBQ_EIO (missing, short, corrupt or foreign file). */
 int rbq_layer_read(const char* path, rbq_layer_info* info, void* codes, void* aux, void* zero_point);
 
+/* Text for a return code (static storage). */
 const char* rbq_error_string(int code);
 
 /*

@@ -55,6 +55,8 @@ SIGNATURES = {
     "quantize_weights_int8_asym": (_I, [_P, _P, _I, _I, _P, _P, _P, _P]),
     "qlinear_int8_asym": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "qlinear_noalloc": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "qlinear_int8_levels": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "rbq_int8_levels": (_I, [_I, _I, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
     "rbq_selftest_wait_limit": (_I, [_P, _P]),
@@ -275,6 +277,35 @@ def qlinear(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, stream=None
     _check(lib().qlinear(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M, N,
                          int(K), _ptr(out), _stream(stream)), "qlinear")
     return out
+
+
+def qlinear_int8_levels(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, stream=None):
+    """qlinear with each codebook's levels rounded onto a signed 8-bit grid and
+    the sum taken exactly on the INT8 tensor cores:
+    y[m, n] = s_m r'_n sum_k l_w[q_nk] l_a[p_mk] / (alpha_w alpha_a), bfloat16 [M, N]
+    (see int8_levels).  K a multiple of 128, N of 8."""
+    import torch
+    for t, n, dt in ((a_codes, "a_codes", torch.uint8), (s, "s", torch.float32),
+                     (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16)):
+        _need_cuda(t, n, dt)
+    M, N = a_codes.shape[0], w_codes.shape[0]
+    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
+        raise ValueError("code row widths do not match K and the bit widths")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _check(lib().qlinear_int8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w),
+                                     M, N, int(K), _ptr(out), _stream(stream)), "qlinear_int8_levels")
+    return out
+
+
+def int8_levels(d, bits):
+    """(levels int8[2^bits], alpha) that qlinear_int8_levels uses for (d, bits):
+    levels = RNE(alpha * c), alpha = 127 / max |c|, c the Lloyd-Max levels."""
+    lv = np.empty(2 ** int(bits), dtype=np.int8)
+    alpha = ctypes.c_double(0.0)
+    _check(lib().rbq_int8_levels(int(d), int(bits), lv.ctypes.data_as(_P), ctypes.byref(alpha)), "rbq_int8_levels")
+    return lv, alpha.value
 
 
 def qlinear_noalloc(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out, err=None, stream=None):

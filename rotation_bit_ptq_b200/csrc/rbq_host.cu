@@ -365,6 +365,15 @@ std::vector<float2> guarded(const std::vector<float2>& lut) {
   return g;
 }
 
+void int8_levels(const std::vector<double>& levels, std::vector<int8_t>& out, double* alpha) {
+  double cmax = 0.0;
+  for (double c : levels) cmax = std::max(cmax, std::fabs(c));
+  const double a = 127.0 / cmax;
+  out.assign(levels.size(), 0);
+  for (size_t j = 0; j < levels.size(); ++j) out[j] = static_cast<int8_t>(std::nearbyint(a * levels[j]));
+  *alpha = a;
+}
+
 int codebook_device(int d, int bits, const CodebookDevice** out) {
   int dev;
   int rc = current_device(&dev);
@@ -390,6 +399,12 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
   for (int j = 0; j < L; ++j) lh[j] = f32_to_f16_bits(static_cast<float>(levels[j] * sd));
   if ((rc = upload(bf.data(), bf.size(), &cb->bounds)) != RBQ_OK) { delete cb; return rc; }
   if ((rc = upload(lh.data(), lh.size(), &cb->levels_f16)) != RBQ_OK) { delete cb; return rc; }
+  {
+    std::vector<int8_t> li;
+    int8_levels(levels, li, &cb->alpha);
+    li.resize(256, 0);
+    if ((rc = upload(li.data(), li.size(), &cb->levels_i8)) != RBQ_OK) { delete cb; return rc; }
+  }
   Grid grid;
   if ((rc = build_grid(bounds, &grid)) != RBQ_OK) { delete cb; return rc; }
   cb->grid_cells = grid.cells;
@@ -407,6 +422,7 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
   if (!ins.second) {          // another thread won the race; keep its copy
     cudaFree(cb->bounds);
     cudaFree(cb->levels_f16);
+    cudaFree(cb->levels_i8);
     cudaFree(cb->grid);
     cudaFree(cb->grid_full);
     cudaFree(cb->grid_pad);
@@ -516,6 +532,19 @@ extern "C" int lloydmax_table(int d, int bits, double* levels, double* bounds) {
   if (rc != RBQ_OK) return rc;
   if (levels) std::memcpy(levels, lv.data(), lv.size() * sizeof(double));
   if (bounds) std::memcpy(bounds, bd.data(), bd.size() * sizeof(double));
+  return RBQ_OK;
+}
+
+extern "C" int rbq_int8_levels(int d, int bits, int8_t* levels, double* alpha) {
+  if (d <= 0 || bits < 1 || bits > 8) return RBQ_EINVAL;
+  std::vector<double> lv, bd;
+  const int rc = full_table(d, bits, lv, bd);
+  if (rc != RBQ_OK) return rc;
+  std::vector<int8_t> li;
+  double a = 0.0;
+  int8_levels(lv, li, &a);
+  if (levels) std::memcpy(levels, li.data(), li.size());
+  if (alpha) *alpha = a;
   return RBQ_OK;
 }
 

@@ -53,6 +53,10 @@ struct CodebookDevice {
   float* bounds = nullptr;        // fp32[2^bits - 1], increasing
   uint16_t* levels_f16 = nullptr; // fp16[2^bits]: levels times sqrt(d) (unit scale)
   float inv_d = 0.f;              // 1/d: undoes the two sqrt(d) factors in qlinear
+  // qlinear_int8_levels: levels rounded onto a signed 8-bit grid,
+  // RNE(alpha * level), alpha = 127 / max |level| (int8[256], zero padded).
+  int8_t* levels_i8 = nullptr;
+  double alpha = 0.0;
   // Code-search grid: `grid_cells` + 1 cells centred at -R + n*2R/cells;
   // entry n = {boundary inside cell n or +inf, number of boundaries below
   // that cell}.  See build_grid() in rbq_host.cu.
@@ -83,6 +87,9 @@ int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out);
 // Returns the codebook of (d, bits) on the current device, computing and
 // uploading it on first use.
 int codebook_device(int d, int bits, const CodebookDevice** out);
+
+// The 8-bit integer levels of a codebook (see CodebookDevice::levels_i8).
+void int8_levels(const std::vector<double>& levels, std::vector<int8_t>& out, double* alpha);
 
 // Records a CUDA error (for rbq_error_string) and maps it to RBQ_ECUDA.
 int cuda_fail(cudaError_t e);

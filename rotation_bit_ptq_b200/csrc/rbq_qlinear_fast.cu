@@ -64,6 +64,7 @@
 
 #include "rbq_internal.h"
 #include "rbq_sm100.cuh"
+#include "rbq_qcodes.cuh"
 
 namespace rbq {
 namespace qfast {
@@ -81,16 +82,6 @@ constexpr int kThreads = 448;                  // 14 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
 constexpr int kExpandThreads = 2 * kBM;        // two warp groups of a thread per activation row
 constexpr size_t kSmemLimit = 227 * 1024;
-
-// Code-stage geometry of the activation operand.
-struct CodeGeo {
-  uint32_t rows;         // 128
-  uint32_t bits;
-  uint32_t offset;       // byte offset of this operand inside a code stage
-  uint32_t bytes;        // bytes of this operand landing per code stage (2 K slices)
-  uint32_t slice_bytes;  // per-slice sub-buffer stride (even widths), else 0
-  uint32_t swz;          // 0 none, 1 = 32B swizzle (4-bit), 2 = 64B swizzle (8-bit)
-};
 
 struct Params {
   int M, N, K;
@@ -120,12 +111,6 @@ struct __align__(8) Tail {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
   return mbar_wait_or_abort(bar, parity, &tl->abort);
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
 }
 
 // Byte planes of the positive fp16 levels C[half + m], m < half <= 8 (the
@@ -179,29 +164,6 @@ __device__ __forceinline__ void expand8_4bit(uint32_t x, const Planes4& P, uint3
   expand8_sym<4>(x, P, w);
 }
 
-// Codes 8c .. 8c+7 of a row's LSB-first bitstream of B-bit codes (B = 2, 3),
-// one per nibble.
-template <int B>
-__device__ __forceinline__ uint32_t spread8(const uint32_t* src, int c) {
-  if constexpr (B == 2) {
-    uint32_t x = (src[c >> 1] >> (16 * (c & 1))) & 0xFFFFu;
-    x = (x | (x << 8)) & 0x00FF00FFu;
-    x = (x | (x << 4)) & 0x0F0F0F0Fu;
-    return (x | (x << 2)) & 0x33333333u;
-  } else {
-    const int bit = 24 * c, wi = bit >> 5, sh = bit & 31;
-    uint32_t u = src[wi] >> sh;
-    if (sh > 8) u |= src[wi + 1] << (32 - sh);
-    uint32_t x = 0u;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) x |= ((u >> (3 * k)) & 7u) << (4 * k);
-    return x;
-  }
-}
-
-template <int BITS>
-constexpr int slice_words() { return 2 * BITS; }
-
 // Half HF (codes 32 HF .. 32 HF + 31) of one row's 64 codes of a K slice ->
 // 16 words of fp16 pairs (k even in the low half), 16 of the row's operand
 // columns in tensor memory.
@@ -244,36 +206,6 @@ __device__ __forceinline__ void expand_row(const uint32_t (&src)[slice_words<BIT
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) out[4 * (c - 4 * HF) + j] = w[j];
-    }
-  }
-}
-
-// Row r's codes of K slice h (0/1) of a code stage -> 2*BITS words.
-template <int BITS>
-__device__ __forceinline__ void read_slice(const uint8_t* part, const CodeGeo& g, int r, int h,
-                                           uint32_t (&dst)[slice_words<BITS>()]) {
-  if constexpr ((BITS & 1) == 0) {
-    // even width: sub-buffer per slice, rows of 8*BITS bytes, maybe swizzled
-    const uint8_t* row = part + h * g.slice_bytes + r * (8 * BITS);
-#pragma unroll
-    for (int c = 0; c < BITS / 2; ++c) {
-      uint32_t pc = c;
-      if constexpr (BITS == 4) pc ^= (r >> 2) & 1;   // 32B swizzle
-      if constexpr (BITS == 8) pc ^= (r >> 1) & 3;   // 64B swizzle
-      const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * pc);
-      dst[4 * c] = v.x;
-      dst[4 * c + 1] = v.y;
-      dst[4 * c + 2] = v.z;
-      dst[4 * c + 3] = v.w;
-    }
-  } else {
-    // odd width: one box of two slices, rows of 16*BITS bytes
-    const uint2* row = reinterpret_cast<const uint2*>(part + r * (16 * BITS) + h * (8 * BITS));
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) {
-      const uint2 v = row[i];
-      dst[2 * i] = v.x;
-      dst[2 * i + 1] = v.y;
     }
   }
 }

@@ -149,7 +149,28 @@ def test_kernel_entry_points_validate_before_launch(lib):
     assert lib.qlinear_int8_asym(fake, fake, fake, fake, 8, 8, 96, fake, None) == rbq.RBQ_EINVAL    # K % 64
     assert lib.qlinear_int8_asym(fake, fake, fake, None, 8, 8, 64, fake, None) == rbq.RBQ_EINVAL
     assert lib.qlinear_int8_asym(odd, fake, fake, fake, 8, 8, 64, fake, None) == rbq.RBQ_EALIGN
+    # integer-level layer: K % 128, N % 8, 16-byte code rows, bit widths, pointers
+    assert lib.qlinear_int8_levels(None, None, 4, None, None, 4, 0, 8, 128, None, None) == rbq.RBQ_OK
+    assert lib.qlinear_int8_levels(fake, fake, 4, fake, fake, 4, 8, 8, 64, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_levels(fake, fake, 4, fake, fake, 4, 8, 12, 128, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_levels(fake, fake, 9, fake, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_levels(fake, fake, 4, fake, fake, 0, 8, 8, 128, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_levels(fake, fake, 4, fake, fake, 4, 8, 8, 32896, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_levels(fake, None, 4, fake, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_int8_levels(odd, fake, 4, fake, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EALIGN
     r.close()
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+def test_int8_levels_match_oracle(lib, bits):
+    for d in (64, 3072, 12288):
+        lv, alpha = rbq.int8_levels(d, bits)
+        olv, oalpha = oracle.int8_levels(oracle.lloydmax_table(d, bits)[0])
+        assert np.array_equal(lv.astype(np.int64), olv)
+        # the two solvers' 8-bit tables agree to ~3e-11 (see the test above)
+        assert abs(alpha / oalpha - 1) < (1e-12 if bits <= 7 else 1e-10)
+    assert lib.rbq_int8_levels(64, 0, None, None) == rbq.RBQ_EINVAL
+    assert lib.rbq_int8_levels(0, 4, None, None) == rbq.RBQ_EINVAL
 
 
 def test_error_strings(lib):

@@ -400,6 +400,57 @@ def test_qlinear_mlp_full_size_sampled(ba, bw):
     assert err_up < QLINEAR_RTOL and err_dn < QLINEAR_RTOL, (err_up, err_dn)
 
 
+def _qlinear_i8_case(X, W, d, bits_a, bits_w, seed=0, rows=None):
+    """qlinear_int8_levels on the library's own codes vs the oracle's integer
+    layer on the same codes: BF16 outputs bit-exact outside the rounding band
+    (the integer sum is exact on both sides, only the fp32 scaling differs)."""
+    r, _ = _rpbh(d, seed)
+    a_codes, s = rbq.rotate_quantize_act(r, _dense(X, "bf16"), bits_a)
+    w_codes, rn = rbq.quantize_weights(r, _dense(W, "bf16"), bits_w)
+    y = rbq.qlinear_int8_levels(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    y_fp16 = rbq.qlinear(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
+    idx = torch.as_tensor(rows).cuda()
+    la, _ = oracle.lloydmax_table(d, bits_a)
+    lw, _ = oracle.lloydmax_table(d, bits_w)
+    pa = _unpack(a_codes[idx], bits_a, d)
+    pw = _unpack(w_codes, bits_w, d)
+    exact = oracle.qlinear_int8_levels(pa, s.cpu().numpy()[rows], la, pw, bf16_to_numpy(rn), lw)
+    got = bf16_to_numpy(y[idx])
+    n_band = check_bf16_rounding(got, exact, "qlinear_int8_levels")
+    # and against the exact-level layer: the levels' rounding only
+    return n_band, rel_frobenius(got, bf16_to_numpy(y_fp16[idx]))
+
+
+@pytest.mark.parametrize("M,N,K,ba,bw", [(1, 8, 128, 4, 4), (130, 136, 128, 4, 2), (257, 264, 384, 3, 3),
+                                         (64, 512, 256, 6, 4), (200, 128, 256, 8, 8), (77, 72, 256, 2, 6),
+                                         (300, 520, 256, 5, 7), (129, 512, 1024, 4, 4), (513, 1032, 512, 3, 1),
+                                         (260, 256, 640, 1, 5), (128, 256, 128, 7, 3)])
+def test_qlinear_int8_levels_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
+    g = np.random.default_rng(M * N + 1)
+    X = synth.to_bf16(g.standard_t(3, (M, K)).astype(np.float32))
+    W = synth.to_bf16((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    n_band, dev = _qlinear_i8_case(X, W, K, ba, bw, seed=M)
+    print(f"int8-level qlinear {M}x{N}x{K} W{bw}A{ba}: {n_band} in-band roundings, {dev:.2e} from exact levels")
+
+
+def test_qlinear_int8_levels_attention_projection_sampled():
+    data = synth.attn_proj()
+    rows = np.random.default_rng(5).choice(4608, 32, replace=False)
+    n_band, dev = _qlinear_i8_case(data["X"], data["W"], 3072, 4, 4, rows=rows)
+    print(f"int8-level qlinear attn_proj W4A4: {n_band} in-band, {dev:.2e} from exact levels")
+    assert dev < 2e-2
+
+
+def test_qlinear_int8_levels_mlp_down_sampled():
+    m = synth.mlp()
+    rows = np.random.default_rng(6).choice(4608, 8, replace=False)
+    n_band, dev = _qlinear_i8_case(m["X_dn"], m["W_dn"], 12288, 4, 2, seed=5, rows=rows)
+    assert dev < 2e-2
+
+
 def _int8_case(X, W, d, seed=0, rows=None):
     r, Pi = _rpbh(d, seed)
     xr = rbq.rotate_act(r, torch_bf16(X))
