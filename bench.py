@@ -686,7 +686,8 @@ def run_reference(args):
 def run_kernel_only(args):
     """One kernel on a profiling-sized case (for ncu): a few launches, no
     timing.  rotate_quantize: 32768 tokens x 3072 (201 MB of BF16 input,
-    larger than L2); qlinear: the attention-projection GEMM 4608x3072x3072."""
+    larger than L2); qlinear (and its integer-level variant): the
+    attention-projection GEMM 4608x3072x3072."""
     import torch
     import rotation_bit_ptq_b200 as rbq
     dev = torch.device("cuda", 0)
@@ -707,8 +708,9 @@ def run_kernel_only(args):
         data = synth.attn_proj(seed=SEED)
         a_codes, s = rbq.rotate_quantize_act(r, to_bf16_tensor(data["X"], dev), BITS_A)
         w_codes, rn = rbq.quantize_weights(r, to_bf16_tensor(data["W"], dev), BITS_W)
+        fn = rbq.qlinear_int8_levels if args.kernel_only == "qlinear_int8_levels" else rbq.qlinear
         for _ in range(args.launches):
-            rbq.qlinear(a_codes, s, BITS_A, w_codes, rn, BITS_W, D)
+            fn(a_codes, s, BITS_A, w_codes, rn, BITS_W, D)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     print(json.dumps({"kernel_only": args.kernel_only, "launches": args.launches, "ok": True}))
@@ -723,7 +725,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-suite", action="store_true", help="skip the other workloads' kernel timings")
     ap.add_argument("--no-graphs", action="store_true", help="time direct API calls instead of graph replays")
-    ap.add_argument("--kernel-only", choices=["rotate_quantize", "rotate_only", "quantize_weights", "qlinear"],
+    ap.add_argument("--kernel-only", choices=["rotate_quantize", "rotate_only", "quantize_weights", "qlinear",
+                                                   "qlinear_int8_levels"],
                     help="run one kernel on a profiling-sized case (for ncu) instead of the benchmark")
     ap.add_argument("--tokens", type=int, default=0)
     ap.add_argument("--launches", type=int, default=3)
