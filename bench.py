@@ -687,7 +687,8 @@ def run_kernel_only(args):
     """One kernel on a profiling-sized case (for ncu): a few launches, no
     timing.  rotate_quantize: 32768 tokens x 3072 (201 MB of BF16 input,
     larger than L2); qlinear (and its integer-level variant): the
-    attention-projection GEMM 4608x3072x3072."""
+    attention-projection GEMM 4608x3072x3072; qlinear_int8 and
+    quantize_weights_int8: the DiT block's q projection, 4096 x 4096 x 4096."""
     import torch
     import rotation_bit_ptq_b200 as rbq
     dev = torch.device("cuda", 0)
@@ -704,6 +705,18 @@ def run_kernel_only(args):
         W = to_bf16_tensor(synth.attn_proj(seed=SEED)["W"], dev)
         for _ in range(args.launches):
             rbq.quantize_weights(r, W, BITS_W)
+    elif args.kernel_only in ("qlinear_int8", "quantize_weights_int8"):
+        # the single-stream DiT block's q projection: 4096 tokens, 4096 -> 4096
+        r4 = rbq.RPBH(4096, 100 + 4096)
+        W = to_bf16_tensor(synth.int8_dit_weight(0, "q"), dev)
+        q, sc = rbq.quantize_weights(r4, W, 8, mode="int8")
+        if args.kernel_only == "quantize_weights_int8":
+            for _ in range(args.launches):
+                rbq.quantize_weights(r4, W, 8, "int8", q, sc)
+        else:
+            xr = rbq.rotate_act(r4, to_bf16_tensor(synth.int8_dit_act(4096), dev))
+            for _ in range(args.launches):
+                rbq.qlinear_int8(xr, q, sc)
     else:
         data = synth.attn_proj(seed=SEED)
         a_codes, s = rbq.rotate_quantize_act(r, to_bf16_tensor(data["X"], dev), BITS_A)
@@ -726,7 +739,7 @@ def main():
     ap.add_argument("--no-suite", action="store_true", help="skip the other workloads' kernel timings")
     ap.add_argument("--no-graphs", action="store_true", help="time direct API calls instead of graph replays")
     ap.add_argument("--kernel-only", choices=["rotate_quantize", "rotate_only", "quantize_weights", "qlinear",
-                                                   "qlinear_int8_levels"],
+                                                   "qlinear_int8_levels", "qlinear_int8", "quantize_weights_int8"],
                     help="run one kernel on a profiling-sized case (for ncu) instead of the benchmark")
     ap.add_argument("--tokens", type=int, default=0)
     ap.add_argument("--launches", type=int, default=3)
