@@ -248,8 +248,8 @@ int qlinear_int8(const uint16_t* Xrot, const int8_t* Wq, const float* scale,
  * alpha.  Arguments, layouts and ownership as qlinear.
  * Limits: K a multiple of 128, N a multiple of 8, K*bits_a/8 a multiple of
  * 16 (else RBQ_EINVAL; there is no fallback kernel).
- * The weight codes are expanded once per call into an int8 workspace of N*K
- * bytes from a stream-ordered memory pool.
+ * The weight and activation codes are expanded once per call into an int8
+ * workspace of (N + M)*K bytes from a stream-ordered memory pool.
  * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECONVERGE, RBQ_ECUDA.
  */
 int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int bits_a,

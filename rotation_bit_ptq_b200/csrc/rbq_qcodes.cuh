@@ -1,8 +1,9 @@
 // Packed-code operands of the tcgen05 GEMMs on Lloyd-Max codes: the layout of
 // a row's codes in a code stage (as the TMA producer lands them), reading one
 // row's codes back, byte-permute helpers, and the host calls that build the
-// tensor maps and the weight workspace pool.  Shared by the fp16-operand
-// qlinear kernel and the 8-bit-operand variant.
+// tensor maps and the weight workspace pool.  Used by the fp16-operand
+// qlinear kernel; the 8-bit-operand variant takes the byte permute, the
+// tensor-map encoder and the workspace pool.
 #pragma once
 
 #include <cuda.h>

@@ -8,24 +8,26 @@
 //   the sum exact in int32 (|sum| <= K 127^2 < 2^31 for K <= 32768), on
 //   tcgen05 kind::i8: twice the fp16 tensor rate and half the operand bytes.
 //
-// The kernel is the fp16 qlinear kernel (rbq_qlinear_fast.cu) with 128-wide K
-// slices: a K-major row of 128 int8 values is one 128-byte swizzle row, so the
-// operand stages (128 x 128 activation bytes + 256 x 128 weight bytes = 48 KB),
-// their descriptors and the MMA steps (+32 bytes = 32 values of K per
-// tcgen05.mma) keep the same byte geometry, and each stage carries twice the K.
-//   warps 0..3  epilogue: TMEM lane quadrant, one output row per thread; the
-//               int32 sums to fp32, times s_m r'_n / (alpha_w alpha_a), BF16.
-//   warp 4      MMA issuer (one thread): four 128x256x32 kind::i8 MMAs per
-//               slice into one of two TMEM accumulators.
-//   warp 5      TMA producer (one thread): per slice, the 128 rows' activation
-//               codes (one code stage = the slice's two 64-code halves) and
-//               the 256 x 128 int8 weight tile (128B swizzle).
-//   warps 6..13 activation expansion, a thread per row, the two warp groups
-//               taking alternate slices: codes to level bytes (2-, 3- and
-//               4-bit codes by byte permutes over register-held level bytes,
-//               other widths from a byte table in shared memory), written
-//               into the stage's swizzled K-major A tile.
-// The weight codes are expanded once per call into an int8 workspace [N, K].
+// Three kernels per call.
+// 1./2. expand_weights_i8_*: the weight codes [N, K*b/8] and the activation
+//    codes [M, K*b/8] become int8 levels [N, K] and [M, K] in one
+//    stream-ordered workspace (4-bit codes by byte permutes over a 16-byte
+//    register table, other widths through a byte table in shared memory).
+//    The activation part (M*K bytes) stays in L2 for the GEMM.
+// 3. qlinear_i8_kernel: persistent, one CTA per SM, 128 x 256 output
+//    tiles, K slices of 128 int8 values (one 128-byte swizzle row per operand
+//    row, so a stage is 16 KB of activations + 32 KB of weights):
+//      warps 0..3  epilogue: TMEM lane quadrant, one output row per thread;
+//                  int32 -> fp32, times s_m r'_n / (alpha_w alpha_a), BF16.
+//      warp 4      MMA issuer (one thread): four 128x256x32 kind::i8 MMAs
+//                  per slice (+32 bytes of K per step) into one of two int32
+//                  TMEM accumulators, so the epilogue of tile i overlaps the
+//                  MMAs of tile i+1.
+//      warp 5      TMA producer (one thread): both operand tiles of each slice
+//                  into a 4-stage ring, 128B-swizzled K-major.
+// (Expanding the activation codes inside the GEMM, as the fp16 qlinear kernel
+// does, measured slower here: at twice the tensor rate the expansion warps
+// set the pace, 57.3 vs 51.4 us at 4608 x 3072 x 3072 W4A4.)
 //
 // Every mbarrier wait is bounded; a thread whose wait runs out raises a shared
 // abort flag, records an error in the library's device error word, and the
@@ -43,47 +45,15 @@ namespace rbq {
 namespace qi8 {
 
 using namespace sm100;
-using qfast::CodeGeo;
 using qfast::prmt;
-using qfast::read_slice;
-using qfast::slice_words;
-using qfast::spread8;
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;  // K values per slice (= bytes per operand row)
 constexpr int kATile = kBM * kBK;               // 16 KB int8 activation tile
 constexpr int kBTile = kBN * kBK;               // 32 KB int8 weight tile
 constexpr int kOpStage = kATile + kBTile;       // 48 KB per operand stage
-constexpr int kAStages = 4;
-constexpr int kMaxF = kAStages, kMaxC = 8;      // operand stages, code stages
-constexpr int kThreads = 448;                   // 14 warps
+constexpr int kAStages = 4;                     // operand stages
+constexpr int kThreads = 192;                   // 6 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
-constexpr size_t kSmemLimit = 227 * 1024;
-
-struct Params {
-  int M, N, K;
-  int bits_a;
-  int F, C;                   // operand stages, code stages
-  uint32_t cstage_bytes;      // bytes per code stage (1024-aligned)
-  CodeGeo ga;
-  const int8_t* lut_a;        // int8 activation levels, 256 entries (zero padded)
-  const float* s;
-  const uint16_t* rnorm;
-  float inv_scale;            // 1 / (alpha_w alpha_a)
-  uint16_t* Y;
-  unsigned int* err;
-};
-
-struct __align__(8) Tail {
-  uint64_t full[kMaxF];       // weight tile landed (TMA bytes) + activation tile stored (one warp group)
-  uint64_t empty[kMaxF];      // stage consumed (MMA commit)
-  uint64_t cfull[kMaxC];
-  uint64_t cempty[kMaxC];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint32_t tmem_slot;
-  volatile uint32_t abort;
-  uint8_t lut_a[256];
-};
 
 // Instruction descriptor of kind::i8: s32 accumulator (D format 2), signed
 // 8-bit A and B (format 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
@@ -127,129 +97,44 @@ __device__ __forceinline__ uint2 expand8_4bit_i8(uint32_t x, const Tab16& T) {
   return make_uint2((hi0 & m0) | (lo0 & ~m0), (hi1 & m1) | (lo1 & ~m1));
 }
 
-// 64 codes of width BITS (one half of a slice) -> 64 level bytes in
-// out[16 H .. 16 H + 15].
-template <int BITS, int H>
-__device__ __forceinline__ void expand64_i8(const uint32_t (&src)[slice_words<BITS>()], const Tab16& T,
-                                            const uint8_t* lut, uint32_t (&out)[32]) {
-  if constexpr (BITS == 4) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint2 w = expand8_4bit_i8(src[c], T);
-      out[16 * H + 2 * c] = w.x;
-      out[16 * H + 2 * c + 1] = w.y;
-    }
-  } else if constexpr (BITS == 2 || BITS == 3) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint32_t x = spread8<BITS>(src, c);     // codes < 8: the low table words only
-      out[16 * H + 2 * c] = prmt(T.t0, T.t1, x);
-      out[16 * H + 2 * c + 1] = prmt(T.t0, T.t1, x >> 16);
-    }
-  } else {
-    constexpr uint32_t mask = (1u << BITS) - 1u;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      uint32_t word = 0u;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * j + e;
-        const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
-        uint32_t code = src[wi] >> sh;
-        if (sh + BITS > 32) code |= src[wi + 1] << (32 - sh);
-        word |= static_cast<uint32_t>(lut[code & mask]) << (8 * e);
-      }
-      out[16 * H + j] = word;
-    }
-  }
-}
+// ---- the GEMM: both int8 operands by TMA ------------------------------------
+struct Params {
+  int M, N, K;
+  const float* s;
+  const uint16_t* rnorm;
+  float inv_scale;
+  uint16_t* Y;
+  unsigned int* err;
+};
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
-  return mbar_wait_or_abort(bar, parity, &tl->abort);
-}
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* tl) {
-  return mbar_warp_wait(bar, parity, &tl->abort);
-}
+struct __align__(8) Tail {
+  uint64_t full[kAStages];
+  uint64_t empty[kAStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_slot;
+  volatile uint32_t abort;
+};
 
-// Row r = 32 (warp % 4) + lane of every activation tile, for the slices of
-// parity G in the CTA's running slice count: the two warp groups expand
-// alternate slices, so two are in flight in this stage.  Slice n sits in code
-// stage n mod C and operand stage n mod F; the group steps both by two.
-template <int BITS, int G>
-__device__ __forceinline__ void expand_loop(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, int r,
-                                            int ntiles, const Tab16 T, const uint8_t* lut) {
-  const CodeGeo& g = p.ga;
-  const int KS = p.K / kBK;
-  const uint32_t C = static_cast<uint32_t>(p.C), F = static_cast<uint32_t>(p.F);
-  uint32_t c = G, cph = 0, s = G, aph = 0, n = 0;
-  bool a_first = true;                           // first round of operand stages: nothing to wait for
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    for (int ks = 0; ks < KS; ++ks, ++n) {
-      if ((n & 1u) != static_cast<uint32_t>(G)) continue;
-      if (!warp_wait(&tl->cfull[c], cph, tl)) return;
-      const uint8_t* part = codes + c * p.cstage_bytes + g.offset;
-      uint32_t w[32];
-      {
-        uint32_t h0[slice_words<BITS>()], h1[slice_words<BITS>()];
-        read_slice<BITS>(part, g, r, 0, h0);
-        read_slice<BITS>(part, g, r, 1, h1);
-        expand64_i8<BITS, 0>(h0, T, lut, w);       // before the stage wait: off the critical path
-        expand64_i8<BITS, 1>(h1, T, lut, w);
-      }
-      mbar_arrive(&tl->cempty[c]);                 // the codes are consumed
-      c += 2;
-      if (c >= C) { c -= C; cph ^= 1u; }
-      if (!a_first && !warp_wait(&tl->empty[s], aph ^ 1u, tl)) return;
-      uint8_t* tile_a = ops + s * kOpStage;          // the stage's A tile, 128B-swizzled K-major
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<uint4*>(tile_a + sw128_offset(r, q)) =
-            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-      fence_proxy_async_smem();                      // visible to the tensor core
-      mbar_arrive(&tl->full[s]);
-      s += 2;
-      if (s >= F) { s -= F; aph ^= 1u; a_first = false; }
-    }
-  }
-}
-
-template <int G>
-__device__ __forceinline__ void expand_dispatch(const Params& p, Tail* tl, uint8_t* ops, uint8_t* codes, int r,
-                                                int ntiles, const Tab16 T, const uint8_t* lut) {
-  switch (p.bits_a) {
-    case 1: expand_loop<1, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    case 2: expand_loop<2, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    case 3: expand_loop<3, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    case 4: expand_loop<4, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    case 5: expand_loop<5, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    case 6: expand_loop<6, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    case 7: expand_loop<7, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-    default: expand_loop<8, G>(p, tl, ops, codes, r, ntiles, T, lut); break;
-  }
-}
+constexpr size_t kSmem = 1024 + kAStages * kOpStage + sizeof(Tail) + 64;
 
 __global__ void __launch_bounds__(kThreads, 1)
     qlinear_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const Params p) {
+                          const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* codes = ops + p.F * kOpStage;
-  Tail* tl = reinterpret_cast<Tail*>(codes + p.C * p.cstage_bytes);
+  Tail* tl = reinterpret_cast<Tail*>(ops + kAStages * kOpStage);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntiles_m = (p.M + kBM - 1) / kBM, ntiles_n = (p.N + kBN - 1) / kBN;
   const int ntiles = ntiles_m * ntiles_n;
   const int KS = p.K / kBK;
+  volatile uint32_t* abort = &tl->abort;
 
-  for (int i = tid; i < 256; i += kThreads) tl->lut_a[i] = static_cast<uint8_t>(p.lut_a[i]);
   if (tid == 0) {
-    for (int s = 0; s < kMaxF; ++s) {
-      mbar_init(&tl->full[s], kBM + 1);   // one warp group (a thread per row) + the producer's expect-tx arrival
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&tl->full[s], 1);
       mbar_init(&tl->empty[s], 1);
-    }
-    for (int c = 0; c < p.C; ++c) {
-      mbar_init(&tl->cfull[c], 1);
-      mbar_init(&tl->cempty[c], kBM);      // the one warp group that expands the slice
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tl->acc_full[a], 1);
@@ -266,8 +151,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tl->tmem_slot;
-  // The prologue reads only constant tables; the operands wait for the
-  // kernels before this one on the stream.
   griddep_wait();
   griddep_launch_dependents();
 
@@ -276,28 +159,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_i8(kBM, kBN);
       const uint64_t desc0 = sdesc_k_sw128(smem_u32(ops));
-      const uint32_t F = static_cast<uint32_t>(p.F);
       uint32_t s = 0, ph = 0, it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
         const uint32_t a = it & 1u, use = it >> 1;
-        if (use >= 1 && !wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, tl)) { ok = false; break; }
+        if (use >= 1 && !mbar_wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc = tmem + a * kBN;
         for (int ks = 0; ks < KS; ++ks) {
-          if (!mbar_try_wait(&tl->full[s], ph) && !wait_or_abort(&tl->full[s], ph, tl)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait_or_abort(&tl->full[s], ph, abort)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t a0 = desc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);   // A, then B
-          const uint64_t b0 = a0 + (kATile >> 4);
-          umma_i8(acc, a0, b0, kIdesc, ks != 0);
-          umma_i8(acc, a0 + 2, b0 + 2, kIdesc, 1u);                       // +32 bytes = 32 values of K
-          umma_i8(acc, a0 + 4, b0 + 4, kIdesc, 1u);
-          umma_i8(acc, a0 + 6, b0 + 6, kIdesc, 1u);
+          const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);
+          const uint64_t bd = ad + (kATile >> 4);
+          umma_i8(acc, ad, bd, kIdesc, ks != 0);
+          umma_i8(acc, ad + 2, bd + 2, kIdesc, 1u);            // +32 bytes = 32 values of K
+          umma_i8(acc, ad + 4, bd + 4, kIdesc, 1u);
+          umma_i8(acc, ad + 6, bd + 6, kIdesc, 1u);
           umma_commit(&tl->empty[s]);
-          if (++s == F) { s = 0; ph ^= 1u; }
+          if (++s == kAStages) { s = 0; ph ^= 1u; }
         }
         if (ok) umma_commit(&tl->acc_full[a]);
       }
@@ -308,40 +187,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      const uint32_t C = static_cast<uint32_t>(p.C), F = static_cast<uint32_t>(p.F);
-      uint32_t c = 0, cph = 0, s = 0, ph = 0;     // code / operand stage and their phases
-      bool c_first = true, b_first = true;
-      bool ok = true;
+      uint32_t s = 0, ph = 0;
+      bool first = true, ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const int mt = tile % ntiles_m, nt = tile / ntiles_m;
         for (int ks = 0; ks < KS; ++ks) {
-          if (!c_first && !wait_or_abort(&tl->cempty[c], cph ^ 1u, tl)) { ok = false; break; }
-          uint8_t* stage = codes + c * p.cstage_bytes;
-          mbar_arrive_expect_tx(&tl->cfull[c], p.ga.bytes);
-          if (p.ga.slice_bytes) {
-            tma_load_2d(stage + p.ga.offset, &tmA, (2 * ks) * 8 * p.ga.bits, mt * kBM, &tl->cfull[c]);
-            tma_load_2d(stage + p.ga.offset + p.ga.slice_bytes, &tmA, (2 * ks + 1) * 8 * p.ga.bits, mt * kBM,
-                        &tl->cfull[c]);
-          } else {
-            tma_load_2d(stage + p.ga.offset, &tmA, ks * 16 * p.ga.bits, mt * kBM, &tl->cfull[c]);
-          }
-          if (++c == C) { c = 0; cph ^= 1u; c_first = false; }
-          if (!b_first && !wait_or_abort(&tl->empty[s], ph ^ 1u, tl)) { ok = false; break; }
-          mbar_arrive_expect_tx(&tl->full[s], kBTile);
-          tma_load_2d(ops + s * kOpStage + kATile, &tmB, ks * kBK, nt * kBN, &tl->full[s]);
-          if (++s == F) { s = 0; ph ^= 1u; b_first = false; }
+          if (!first && !mbar_wait_or_abort(&tl->empty[s], ph ^ 1u, abort)) { ok = false; break; }
+          uint8_t* st = ops + s * kOpStage;
+          mbar_arrive_expect_tx(&tl->full[s], kOpStage);
+          tma_load_2d(st, &tmA, ks * kBK, mt * kBM, &tl->full[s]);
+          tma_load_2d(st + kATile, &tmB, ks * kBK, nt * kBN, &tl->full[s]);
+          if (++s == kAStages) { s = 0; ph ^= 1u; first = false; }
         }
       }
       if (!ok) atomicOr(p.err, 16u);
     }
-  } else if (warp < 4) {
+  } else {
     // ---------------- epilogue ----------------
     const int q = warp;                     // TMEM lane quadrant
     const int r = 32 * q + lane;            // row within the tile
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const uint32_t a = it & 1u, use = it >> 1;
-      if (!warp_wait(&tl->acc_full[a], use & 1, tl)) {   // warp-uniform: tmem loads follow
+      if (!mbar_warp_wait(&tl->acc_full[a], use & 1, abort)) {   // warp-uniform: tmem loads follow
         if (lane == 0) atomicOr(p.err, 4u);
         break;
       }
@@ -386,15 +254,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&tl->acc_empty[a]);
     }
-  } else {
-    // ---------------- activation expansion ----------------
-    // warps 6..13: row quarter warp % 4, slice parity (warp - 6) / 4
-    const int r = 32 * (warp & 3) + lane;
-    const uint8_t* lut = tl->lut_a;
-    const Tab16 T = make_tab16(lut);
-    if (warp < 10) expand_dispatch<0>(p, tl, ops, codes, r, ntiles, T, lut);
-    else expand_dispatch<1>(p, tl, ops, codes, r, ntiles, T, lut);
-    if (tl->abort && r == 0 && warp < 10) atomicOr(p.err, 8u);
   }
 
   tc_fence_before();
@@ -481,12 +340,12 @@ int expand_weights(const uint8_t* codes, int bits, int rows, int K, const int8_t
 }
 
 // int8 [rows, K] K-major, 256 x 128 boxes, 128B swizzle.
-int encode_i8_map(CUtensorMap* map, const int8_t* base, int rows, int K) {
+int encode_i8_map(CUtensorMap* map, const int8_t* base, int rows, int K, int box_rows = kBN) {
   auto fn = qfast::encode_fn();
   if (!fn) return RBQ_ECUDA;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBN)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -494,44 +353,31 @@ int encode_i8_map(CUtensorMap* map, const int8_t* base, int rows, int K) {
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
 }
 
-int gemm(const uint8_t* a_codes, const float* s, int bits_a, const int8_t* wi8, const uint16_t* rnorm, int M, int N,
-         int K, uint16_t* Y, const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st,
-         int sms) {
+// The GEMM on expanded int8 operands: activations `ai8` [M, K], weights `wi8` [N, K].
+int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* rnorm, int M, int N, int K,
+             uint16_t* Y, const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st,
+             int sms) {
   Params p{};
   p.M = M;
   p.N = N;
   p.K = K;
-  p.bits_a = bits_a;
-  p.ga = qfast::make_geo(kBM, bits_a, 0);
-  p.cstage_bytes = qfast::geo_span(p.ga);
-  const size_t tail = sizeof(Tail) + 64;
-  const int F = kMaxF;
-  int C = 2;
-  while (C < kMaxC && 1024 + F * kOpStage + (C + 1) * p.cstage_bytes + tail <= kSmemLimit) ++C;
-  const size_t smem = 1024 + static_cast<size_t>(F) * kOpStage + static_cast<size_t>(C) * p.cstage_bytes + tail;
-  if (smem > kSmemLimit) return RBQ_EINVAL;
-  p.F = F;
-  p.C = C;
-  p.lut_a = ca->levels_i8;
   p.s = s;
   p.rnorm = rnorm;
   p.inv_scale = static_cast<float>(1.0 / (ca->alpha * cw->alpha));
   p.Y = Y;
   p.err = err;
   CUtensorMap mA, mB;
-  int rc = qfast::encode_codes_map(&mA, a_codes, M, bits_a, K, p.ga);
+  int rc = encode_i8_map(&mA, ai8, M, K, kBM);
   if (rc != RBQ_OK) return rc;
-  if ((rc = encode_i8_map(&mB, wi8, N, K)) != RBQ_OK) return rc;
+  if ((rc = encode_i8_map(&mB, wi8, N, K, kBN)) != RBQ_OK) return rc;
   auto kern = qlinear_i8_kernel;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
-  const int grid = ntiles < sms ? ntiles : sms;
-  // programmatic dependent launch: the prologue overlaps the weight expansion's tail
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -572,11 +418,13 @@ extern "C" int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int b
   cudaMemPool_t pool = qfast::workspace_pool(dev);
   if (!pool) return RBQ_ECUDA;
   void* ws = nullptr;
-  e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K, pool, st);
+  e = cudaMallocFromPoolAsync(&ws, (static_cast<size_t>(N) + M) * K, pool, st);
   if (e != cudaSuccess) return cuda_fail(e);
   int8_t* wi8 = static_cast<int8_t*>(ws);
+  int8_t* ai8 = wi8 + static_cast<size_t>(N) * K;
   rc = qi8::expand_weights(w_codes, bits_w, N, K, cw->levels_i8, wi8, st, sms);
-  if (rc == RBQ_OK) rc = qi8::gemm(a_codes, s, bits_a, wi8, rnorm, M, N, K, Y, ca, cw, err, st, sms);
+  if (rc == RBQ_OK) rc = qi8::expand_weights(a_codes, bits_a, M, K, ca->levels_i8, ai8, st, sms);
+  if (rc == RBQ_OK) rc = qi8::gemm(ai8, s, wi8, rnorm, M, N, K, Y, ca, cw, err, st, sms);
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
   return rc;
