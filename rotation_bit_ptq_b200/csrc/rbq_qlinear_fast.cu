@@ -95,6 +95,7 @@ struct Params {
   float inv_k;
   uint16_t* Y;
   unsigned int* err;
+  int n_fast;                 // tile order: N fastest (the activation operand is the larger)
 };
 
 struct __align__(8) Tail {
@@ -347,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool c_first = true, b_first = true;
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+        const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
+        const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
         for (int kp = 0; kp < KP && ok; ++kp) {
           if (!c_first && !wait_or_abort(&tl->cempty[c], cph ^ 1u, tl)) {
             ok = false;
@@ -389,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+      const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
+      const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
       const int m = mt * kBM + r;
       const float rs = (m < p.M) ? p.s[m] * p.inv_k : 0.f;
 #pragma unroll 1
@@ -733,6 +736,8 @@ int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const 
   p.inv_k = ca->inv_d;
   p.Y = Y;
   p.err = err;
+  // walk N fastest when the activation codes outweigh the fp16 weights
+  p.n_fast = static_cast<long long>(M) * bits_a > 16LL * N;
   CUtensorMap mA, mB;
   int rc = encode_codes_map(&mA, a_codes, M, bits_a, K, p.ga);
   if (rc != RBQ_OK) return rc;

@@ -105,6 +105,7 @@ struct Params {
   float inv_scale;
   uint16_t* Y;
   unsigned int* err;
+  int n_fast;                 // tile order: N fastest (the activation operand is the larger)
 };
 
 struct __align__(8) Tail {
@@ -190,7 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t s = 0, ph = 0;
       bool first = true, ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+        const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
+        const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
         for (int ks = 0; ks < KS; ++ks) {
           if (!first && !mbar_wait_or_abort(&tl->empty[s], ph ^ 1u, abort)) { ok = false; break; }
           uint8_t* st = ops + s * kOpStage;
@@ -214,7 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+      const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
+      const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
       const int m = mt * kBM + r;
       const float rs = (m < p.M) ? p.s[m] * p.inv_scale : 0.f;
 #pragma unroll 1
@@ -366,6 +369,7 @@ int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* r
   p.inv_scale = static_cast<float>(1.0 / (ca->alpha * cw->alpha));
   p.Y = Y;
   p.err = err;
+  p.n_fast = M > N;
   CUtensorMap mA, mB;
   int rc = encode_i8_map(&mA, ai8, M, K, kBM);
   if (rc != RBQ_OK) return rc;

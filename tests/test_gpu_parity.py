@@ -374,7 +374,9 @@ def test_qlinear_tiny_w4a4():
                                          (64, 512, 256, 6, 4), (200, 128, 192, 8, 8), (77, 72, 64, 2, 6),
                                          # TMA-fed kernel (K % 128 == 0): every code-stage kind
                                          (130, 256, 384, 8, 8), (64, 264, 256, 2, 6), (300, 520, 256, 5, 7),
-                                         (129, 512, 1024, 4, 4), (513, 1032, 512, 3, 1), (1, 256, 128, 4, 4)])
+                                         (129, 512, 1024, 4, 4), (513, 1032, 512, 3, 1), (1, 256, 128, 4, 4),
+                                         # activation codes outweigh the weights: tiles walked N-fastest
+                                         (1030, 64, 256, 4, 4), (700, 136, 384, 6, 3)])
 def test_qlinear_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
     g = np.random.default_rng(M * N)
     X = synth.to_bf16(g.standard_t(3, (M, K)).astype(np.float32))
