@@ -736,8 +736,10 @@ int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const 
   p.inv_k = ca->inv_d;
   p.Y = Y;
   p.err = err;
-  // walk N fastest when the activation codes outweigh the fp16 weights
-  p.n_fast = static_cast<long long>(M) * bits_a > 16LL * N;
+  // walk N fastest when the activation codes outweigh the fp16 weights and
+  // would not stay in L2 between waves of CTAs (more than half of its 126 MB)
+  const long long a_bytes = static_cast<long long>(M) * K * bits_a / 8;
+  p.n_fast = a_bytes > 2LL * N * K && a_bytes > (64LL << 20);
   CUtensorMap mA, mB;
   int rc = encode_codes_map(&mA, a_codes, M, bits_a, K, p.ga);
   if (rc != RBQ_OK) return rc;

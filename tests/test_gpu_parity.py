@@ -374,9 +374,7 @@ def test_qlinear_tiny_w4a4():
                                          (64, 512, 256, 6, 4), (200, 128, 192, 8, 8), (77, 72, 64, 2, 6),
                                          # TMA-fed kernel (K % 128 == 0): every code-stage kind
                                          (130, 256, 384, 8, 8), (64, 264, 256, 2, 6), (300, 520, 256, 5, 7),
-                                         (129, 512, 1024, 4, 4), (513, 1032, 512, 3, 1), (1, 256, 128, 4, 4),
-                                         # activation codes outweigh the weights: tiles walked N-fastest
-                                         (1030, 64, 256, 4, 4), (700, 136, 384, 6, 3)])
+                                         (129, 512, 1024, 4, 4), (513, 1032, 512, 3, 1), (1, 256, 128, 4, 4)])
 def test_qlinear_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
     g = np.random.default_rng(M * N)
     X = synth.to_bf16(g.standard_t(3, (M, K)).astype(np.float32))
@@ -451,6 +449,35 @@ def test_qlinear_int8_levels_mlp_down_sampled():
     rows = np.random.default_rng(6).choice(4608, 8, replace=False)
     n_band, dev = _qlinear_i8_case(m["X_dn"], m["W_dn"], 12288, 4, 2, seed=5, rows=rows)
     assert dev < 2e-2
+
+
+@pytest.mark.parametrize("layer,M,N,K,ba,bw", [("fp16", 139264, 136, 1024, 4, 4), ("int8", 70000, 136, 1024, 4, 3)])
+def test_large_activation_operand_tiles_walked_n_fastest(layer, M, N, K, ba, bw):
+    """Activation operands above 64 MiB (and above the weights) make the GEMMs
+    walk their output tiles N-fastest; random codes, sampled rows (the first,
+    the last and tiles in between) against the oracle."""
+    gen = torch.Generator(device="cuda").manual_seed(M)
+    a = torch.randint(0, 256, (M, K * ba // 8), dtype=torch.uint8, device="cuda", generator=gen)
+    w = torch.randint(0, 256, (N, K * bw // 8), dtype=torch.uint8, device="cuda", generator=gen)
+    s = torch.rand(M, device="cuda", generator=gen) + 0.5
+    rn = (torch.rand(N, device="cuda", generator=gen) + 0.5).to(torch.bfloat16)
+    fn = rbq.qlinear if layer == "fp16" else rbq.qlinear_int8_levels
+    y = fn(a, s, ba, w, rn, bw, K)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(M).choice(M, 40, replace=False)]))
+    idx = torch.as_tensor(rows).cuda()
+    la, _ = oracle.lloydmax_table(K, ba)
+    lw, _ = oracle.lloydmax_table(K, bw)
+    pa = _unpack(a[idx], ba, K)
+    pw = _unpack(w, bw, K)
+    got = bf16_to_numpy(y[idx])
+    if layer == "fp16":
+        ref = oracle.qlinear(pa, s.cpu().numpy()[rows], la, pw, bf16_to_numpy(rn), lw)
+        assert rel_frobenius(got, ref) < QLINEAR_RTOL
+    else:
+        ref = oracle.qlinear_int8_levels(pa, s.cpu().numpy()[rows], la, pw, bf16_to_numpy(rn), lw)
+        check_bf16_rounding(got, ref, "qlinear_int8_levels")
 
 
 def _int8_case(X, W, d, seed=0, rows=None):
