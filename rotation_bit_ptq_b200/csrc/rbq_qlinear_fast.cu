@@ -765,6 +765,11 @@ int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const 
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }
 
+// The TMA-fed GEMM on operands expanded beforehand (rbq_qlinear_int8_fast.cu).
+int qlinear_f16_operands_gemm(const uint16_t* af16, const float* s, const uint16_t* wf16, const uint16_t* rnorm,
+                              float inv_k, int M, int N, int K, uint16_t* Y, unsigned int* err, cudaStream_t st,
+                              int sms);
+
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
                         const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st) {
@@ -774,12 +779,25 @@ int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, cons
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaMemPool_t pool = qfast::workspace_pool(dev);
   if (!pool) return RBQ_ECUDA;
+  // 4-bit activation codes are expanded inside the GEMM by byte permutes at
+  // no cost to it; other widths cost the expansion warps more than the tensor
+  // core, so they get their own pass into fp16 and a GEMM that streams both
+  // operands by TMA -- while that fp16 copy (M*K*2 bytes) is at most 128 MiB,
+  // beyond which writing and re-reading it costs more than it saves.
+  const size_t a_f16_bytes = static_cast<size_t>(M) * K * 2;
+  const bool split = bits_a != 4 && a_f16_bytes <= (static_cast<size_t>(128) << 20);
   void* ws = nullptr;
-  e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K * 2, pool, st);
+  e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K * 2 + (split ? a_f16_bytes : 0), pool, st);
   if (e != cudaSuccess) return cuda_fail(e);
   uint16_t* wf16 = static_cast<uint16_t*>(ws);
   int rc = qfast::expand_weights(w_codes, bits_w, N, K, cw->levels_f16, wf16, st, sms);
-  if (rc == RBQ_OK) rc = qlinear_fast_gemm(a_codes, s, bits_a, wf16, rnorm, M, N, K, Y, ca, err, st, sms);
+  if (split) {
+    uint16_t* af16 = wf16 + static_cast<size_t>(N) * K;
+    if (rc == RBQ_OK) rc = qfast::expand_weights(a_codes, bits_a, M, K, ca->levels_f16, af16, st, sms);
+    if (rc == RBQ_OK) rc = qlinear_f16_operands_gemm(af16, s, wf16, rnorm, ca->inv_d, M, N, K, Y, err, st, sms);
+  } else if (rc == RBQ_OK) {
+    rc = qlinear_fast_gemm(a_codes, s, bits_a, wf16, rnorm, M, N, K, Y, ca, err, st, sms);
+  }
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
   return rc;

@@ -48,7 +48,10 @@ constexpr int kMmaWarp = 4, kTmaWarp = 5;
 
 struct Params {
   int M, N, K;
-  const float* scale;
+  const float* scale;         // W8A16: per-column scales
+  const float* s;             // qlinear: per-row norms
+  const uint16_t* rnorm;      // qlinear: BF16 per-column norms
+  float inv_k;                // qlinear: 1/K (the fp16 levels carry sqrt(K) each)
   uint16_t* Y;
   unsigned int* err;
 };
@@ -71,6 +74,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* 
   return mbar_warp_wait(bar, parity, &tl->abort);
 }
 
+// kQ = false: the W8A16 layer (bf16 operands, epilogue x scale[n]);
+// kQ = true: qlinear on codes expanded beforehand into fp16 levels (x sqrt(K)),
+// epilogue x s[m] r'[n] / K.
+template <bool kQ>
 __global__ void __launch_bounds__(kThreads, 1)
     qlinear_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const Params p) {
@@ -111,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, true);
+      constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, !kQ);
       const uint64_t desc0 = sdesc_k_sw128(smem_u32(ops));
       uint32_t s = 0, ph = 0, it = 0;
       bool ok = true;
@@ -170,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int mt = tile % ntiles_m, nt = tile / ntiles_m;
       const int m = mt * kBM + r;
+      const float rs = kQ ? ((m < p.M) ? p.s[m] * p.inv_k : 0.f) : 1.f;
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t v[32];
@@ -182,8 +190,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * __ldg(p.scale + nb + 2 * j),
-                                                           __uint_as_float(v[2 * j + 1]) * __ldg(p.scale + nb + 2 * j + 1));
+            float c0, c1;
+            if constexpr (kQ) {
+              const uint32_t rr = *reinterpret_cast<const uint32_t*>(p.rnorm + nb + 2 * j);
+              c0 = rs * __uint_as_float(rr << 16);
+              c1 = rs * __uint_as_float(rr & 0xFFFF0000u);
+            } else {
+              c0 = __ldg(p.scale + nb + 2 * j);
+              c1 = __ldg(p.scale + nb + 2 * j + 1);
+            }
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * c0, __uint_as_float(v[2 * j + 1]) * c1);
             packed[j] = *reinterpret_cast<const uint32_t*>(&h);
           }
           uint4* d4 = reinterpret_cast<uint4*>(dst);
@@ -193,8 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (nb + j < p.N)
-              dst[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * p.scale[nb + j]));
+            if (nb + j < p.N) {
+              const float c = kQ ? rs * __uint_as_float(static_cast<uint32_t>(p.rnorm[nb + j]) << 16) : p.scale[nb + j];
+              dst[j] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j]) * c));
+            }
         }
       }
       tc_fence_before();
@@ -275,14 +293,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 [rows, K] K-major, box = 64 x box_rows, 128B swizzle.
-int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int box_rows) {
+int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int box_rows, bool f16 = false) {
   auto fn = encode_fn();
   if (!fn) return RBQ_ECUDA;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box,
+  const CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<uint16_t*>(base), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
@@ -306,7 +325,49 @@ cudaMemPool_t workspace_pool(int dev) {
   return pools[dev];
 }
 
+// Launches the GEMM on two fp16/bf16 operands already in memory (K % 64 == 0).
+template <bool kQ>
+int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStream_t st, int sms) {
+  CUtensorMap mA, mB;
+  int rc = encode_bf16_map(&mA, A, p.M, p.K, kBM, kQ);
+  if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, kBN, kQ);
+  if (rc != RBQ_OK) return rc;
+  auto kern = qlinear_bf16_kernel<kQ>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int ntiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
+}
+
 }  // namespace q8fast
+
+// qlinear on expanded operands: `af16` [M, K] and `wf16` [N, K] fp16 levels x sqrt(K).
+int qlinear_f16_operands_gemm(const uint16_t* af16, const float* s, const uint16_t* wf16, const uint16_t* rnorm,
+                              float inv_k, int M, int N, int K, uint16_t* Y, unsigned int* err, cudaStream_t st,
+                              int sms) {
+  q8fast::Params p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.s = s;
+  p.rnorm = rnorm;
+  p.inv_k = inv_k;
+  p.Y = Y;
+  p.err = err;
+  return q8fast::launch_gemm<true>(af16, wf16, p, st, sms);
+}
 
 bool qlinear_int8_fast_eligible(int M, int N, int K) {
   return M >= 1 && N >= 8 && (N % 8) == 0 && K >= 64 && (K % 64) == 0;
@@ -336,32 +397,16 @@ int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float
     widen_int8_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(Wq, groups, wb);
   int rc = RBQ_OK;
   if ((e = cudaGetLastError()) != cudaSuccess) rc = cuda_fail(e);
-  CUtensorMap mA, mB;
-  if (rc == RBQ_OK) rc = encode_bf16_map(&mA, Xrot, M, K, kBM);
-  if (rc == RBQ_OK) rc = encode_bf16_map(&mB, wb, N, K, kBN);
   if (rc == RBQ_OK) {
-    Params p{M, N, K, scale, Y, err};
-    auto kern = qlinear_bf16_kernel;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
-    if (e != cudaSuccess) {
-      rc = cuda_fail(e);
-    } else {
-      const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
-      // programmatic dependent launch: the prologue overlaps the widening kernel's tail
-      cudaLaunchConfig_t cfg{};
-      cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = kSmem;
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
-      if (e == cudaSuccess) e = cudaGetLastError();
-      if (e != cudaSuccess) rc = cuda_fail(e);
-    }
+    Params p{};
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.scale = scale;
+    p.Y = Y;
+    p.err = err;
+    // programmatic dependent launch: the prologue overlaps the widening kernel's tail
+    rc = launch_gemm<false>(Xrot, wb, p, st, sms);
   }
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
