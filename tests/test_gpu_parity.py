@@ -453,9 +453,10 @@ def test_qlinear_int8_levels_mlp_down_sampled():
 
 @pytest.mark.parametrize("layer,M,N,K,ba,bw", [("fp16", 139264, 136, 1024, 4, 4), ("int8", 70000, 136, 1024, 4, 3)])
 def test_large_activation_operand_tiles_walked_n_fastest(layer, M, N, K, ba, bw):
-    """Activation operands above 64 MiB (and above the weights) make the GEMMs
-    walk their output tiles N-fastest; random codes, sampled rows (the first,
-    the last and tiles in between) against the oracle."""
+    """Activation operands larger than the weights (above 64 MiB for the
+    fp16-level kernel) make the GEMMs walk their output tiles N-fastest; random
+    codes, sampled rows (the first, the last and tiles in between) against the
+    oracle."""
     gen = torch.Generator(device="cuda").manual_seed(M)
     a = torch.randint(0, 256, (M, K * ba // 8), dtype=torch.uint8, device="cuda", generator=gen)
     w = torch.randint(0, 256, (N, K * bw // 8), dtype=torch.uint8, device="cuda", generator=gen)
