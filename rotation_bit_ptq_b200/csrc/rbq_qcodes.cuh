@@ -2,8 +2,8 @@
 // a row's codes in a code stage (as the TMA producer lands them), reading one
 // row's codes back, byte-permute helpers, and the host calls that build the
 // tensor maps and the weight workspace pool.  Used by the fp16-operand
-// qlinear kernel; the 8-bit-operand variant takes the byte permute, the
-// tensor-map encoder and the workspace pool.
+// qlinear kernel; the W8A16 and 8-bit-operand GEMMs take the byte permute,
+// the tensor-map encoder and the workspace pool.
 #pragma once
 
 #include <cuda.h>

@@ -684,6 +684,7 @@ int expand_weights(const uint8_t* codes, int bits, int rows, int K, const uint16
 cudaMemPool_t workspace_pool(int dev) {
   static cudaMemPool_t pools[kMaxDevices] = {};
   static std::mutex mu;
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
   if (!pools[dev]) {
     cudaMemPoolProps props{};

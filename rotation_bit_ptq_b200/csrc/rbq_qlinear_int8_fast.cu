@@ -28,15 +28,16 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
-#include <mutex>
-
 #include "rbq_internal.h"
+#include "rbq_qcodes.cuh"
 #include "rbq_sm100.cuh"
 
 namespace rbq {
 namespace q8fast {
 
 using namespace sm100;
+using qfast::encode_fn;
+using qfast::workspace_pool;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kATile = kBM * kBK * 2;          // 16 KB
@@ -279,19 +280,6 @@ __global__ void __launch_bounds__(256) widen_int8_kernel(const int8_t* q, long l
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 // bf16 [rows, K] K-major, box = 64 x box_rows, 128B swizzle.
 int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int box_rows, bool f16 = false) {
   auto fn = encode_fn();
@@ -305,24 +293,6 @@ int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
-}
-
-cudaMemPool_t workspace_pool(int dev) {
-  static cudaMemPool_t pools[kMaxDevices] = {};
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!pools[dev]) {
-    cudaMemPoolProps props{};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t pool = nullptr;
-    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
-    uint64_t keep = ~0ull;
-    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    pools[dev] = pool;
-  }
-  return pools[dev];
 }
 
 // Launches the GEMM on two fp16/bf16 operands already in memory (K % 64 == 0).
