@@ -257,6 +257,28 @@ int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int bits_a,
                         int M, int N, int K, uint16_t* Y, void* stream);
 
 /*
+ * qlinear_fp8_levels -- the same layer with each codebook's levels rounded to
+ * FP8 E4M3 (OCP E4M3FN, round to nearest even) and summed in fp32 on the FP8
+ * tensor cores (tcgen05 kind::f8f6f4):
+ *   e_b[j] = E4M3(beta_b * c_j),  beta_b = 2^(7 - floor(log2 max_j |c_j|))
+ *   Y[m, n] = bf16( s[m] * r'[n] * (sum_k e_w[q_nk] * e_a[p_mk]) / (beta_w * beta_a) )
+ * beta is a power of two, so the levels lose only their mantissa bits beyond
+ * the third (relative error <= 2^-4); the sum is fp32 (not exact).
+ * rbq_fp8_levels returns the E4M3 bytes and beta.  Arguments, layouts, limits,
+ * workspace and errors as qlinear_int8_levels.
+ */
+int qlinear_fp8_levels(const uint8_t* a_codes, const float* s, int bits_a,
+                       const uint8_t* w_codes, const uint16_t* rnorm, int bits_w,
+                       int M, int N, int K, uint16_t* Y, void* stream);
+
+/*
+ * rbq_fp8_levels -- the E4M3 levels qlinear_fp8_levels uses for (d, bits)
+ * (host only): levels HOST uint8[2^bits] E4M3 bytes (may be NULL), beta HOST
+ * double (may be NULL).  Returns RBQ_OK, RBQ_EINVAL or RBQ_ECONVERGE.
+ */
+int rbq_fp8_levels(int d, int bits, uint8_t* levels, double* beta);
+
+/*
  * rbq_int8_levels -- the integer levels qlinear_int8_levels uses for (d, bits)
  * (host only): levels HOST int8[2^bits] (may be NULL), alpha HOST double
  * (may be NULL).  Returns RBQ_OK, RBQ_EINVAL or RBQ_ECONVERGE.

@@ -45,6 +45,10 @@ qlinear.*              pure-Python triple loop; equal-code closed form
 qlinear.int8_levels    J. Max (1960) 16-level table rounded by hand
                        (tests/golden); grid bounds and antisymmetry; the
                        layer within its rounding bound of the exact one
+qlinear.e4m3_round     PyTorch's float8_e4m3fn conversion (library routine)
+qlinear.fp8_levels     the same Max table rounded to 3 mantissa bits by hand;
+                       power-of-two beta; the layer's triple loop, closed
+                       form and rounding bound
 =====================  ===================================================
 """
 
@@ -55,7 +59,8 @@ from .bf16 import round_to_bf16
 from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
                     quantize_weights_lloydmax, quantize_weights_int8,
                     quantize_weights_int8_asym, rotate_only, EPS)
-from .qlinear import qlinear, qlinear_int8, qlinear_int8_asym, int8_levels, qlinear_int8_levels
+from .qlinear import (qlinear, qlinear_int8, qlinear_int8_asym, int8_levels, qlinear_int8_levels,
+                      e4m3_round, fp8_levels, qlinear_fp8_levels)
 
 __all__ = [
     "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_rows", "rpbh_apply",
@@ -63,5 +68,6 @@ __all__ = [
     "round_to_bf16", "assign_codes", "pack_codes", "unpack_codes",
     "quantize_act", "quantize_weights_lloydmax", "quantize_weights_int8",
     "quantize_weights_int8_asym", "rotate_only", "EPS", "qlinear", "qlinear_int8",
-    "qlinear_int8_asym", "int8_levels", "qlinear_int8_levels",
+    "qlinear_int8_asym", "int8_levels", "qlinear_int8_levels", "e4m3_round", "fp8_levels",
+    "qlinear_fp8_levels",
 ]

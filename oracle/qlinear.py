@@ -21,6 +21,12 @@ codebook's levels c_j are put on a signed 8-bit grid,
 and y[m, n] = s_m · r'_n · (sum_k l_w[q_nk] · l_a[p_mk]) / (alpha_w · alpha_a),
 the sum an exact integer.
 
+FP8 variant (the same, for FP8 tensor cores): beta = 2^(7 - floor(log2 max|c|))
+(a power of two, so beta·max|c| lies in [128, 256)), e_j = E4M3(beta · c_j)
+rounded to nearest even (OCP E4M3FN: 3 mantissa bits, exponent bias 7,
+subnormals below 2^-6, largest finite 448), and
+y[m, n] = s_m · r'_n · (sum_k e_w[q_nk] · e_a[p_mk]) / (beta_w · beta_a).
+
 All are plain definitions; the oracle evaluates them with one matmul.
 """
 
@@ -65,3 +71,36 @@ def qlinear_int8_levels(a_codes, s, levels_a, w_codes, rnorm, levels_w):
     s = np.asarray(s, dtype=np.float64)
     r = np.asarray(rnorm, dtype=np.float64)
     return acc.astype(np.float64) * s[:, None] * r[None, :] / (alpha_a * alpha_w)
+
+
+def e4m3_round(x):
+    """Round fp64 values to the nearest FP8 E4M3FN value (ties to even);
+    magnitudes beyond 448 saturate to 448."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    out = np.zeros_like(a)
+    nz = a > 0
+    e = np.floor(np.log2(a[nz]))
+    e = np.maximum(e, -6.0)                  # below 2^-6 the spacing stays 2^-9 (subnormals)
+    step = np.exp2(e - 3.0)                  # 3 mantissa bits
+    out[nz] = np.rint(a[nz] / step) * step   # np.rint: round half to even
+    out = np.minimum(out, 448.0)
+    return np.copysign(out, x)
+
+
+def fp8_levels(levels):
+    """(e float64[L], beta): E4M3 values of beta·c, beta = 2^(7 - floor(log2 max|c|))."""
+    c = np.asarray(levels, dtype=np.float64)
+    beta = np.exp2(7.0 - np.floor(np.log2(np.max(np.abs(c)))))
+    return e4m3_round(beta * c), beta
+
+
+def qlinear_fp8_levels(a_codes, s, levels_a, w_codes, rnorm, levels_w):
+    """y = s_m r'_n (sum_k e_w[q_nk] e_a[p_mk]) / (beta_w beta_a) in fp64 (the
+    E4M3 products are exact in fp64, so this is the exact sum)."""
+    ea, beta_a = fp8_levels(levels_a)
+    ew, beta_w = fp8_levels(levels_w)
+    acc = ea[np.asarray(a_codes)] @ ew[np.asarray(w_codes)].T
+    s = np.asarray(s, dtype=np.float64)
+    r = np.asarray(rnorm, dtype=np.float64)
+    return acc * s[:, None] * r[None, :] / (beta_a * beta_w)

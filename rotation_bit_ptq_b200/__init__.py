@@ -57,6 +57,8 @@ SIGNATURES = {
     "qlinear_noalloc": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "qlinear_int8_levels": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
     "rbq_int8_levels": (_I, [_I, _I, _P, _P]),
+    "qlinear_fp8_levels": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "rbq_fp8_levels": (_I, [_I, _I, _P, _P]),
     "rbq_error_string": (ctypes.c_char_p, [_I]),
     "rbq_device_error": (_I, [_P]),
     "rbq_selftest_wait_limit": (_I, [_P, _P]),
@@ -297,6 +299,35 @@ def qlinear_int8_levels(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None,
     _check(lib().qlinear_int8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w),
                                      M, N, int(K), _ptr(out), _stream(stream)), "qlinear_int8_levels")
     return out
+
+
+def qlinear_fp8_levels(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, stream=None):
+    """qlinear with each codebook's levels rounded to FP8 E4M3 (times a power
+    of two) and summed in fp32 on the FP8 tensor cores:
+    y[m, n] = s_m r'_n sum_k e_w[q_nk] e_a[p_mk] / (beta_w beta_a), bfloat16 [M, N]
+    (see fp8_levels).  K a multiple of 128, N of 8."""
+    import torch
+    for t, n, dt in ((a_codes, "a_codes", torch.uint8), (s, "s", torch.float32),
+                     (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16)):
+        _need_cuda(t, n, dt)
+    M, N = a_codes.shape[0], w_codes.shape[0]
+    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
+        raise ValueError("code row widths do not match K and the bit widths")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _check(lib().qlinear_fp8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w),
+                                    M, N, int(K), _ptr(out), _stream(stream)), "qlinear_fp8_levels")
+    return out
+
+
+def fp8_levels(d, bits):
+    """(E4M3 bytes uint8[2^bits], beta) that qlinear_fp8_levels uses for
+    (d, bits): bytes = E4M3(beta * c), beta = 2^(7 - floor(log2 max |c|))."""
+    lv = np.empty(2 ** int(bits), dtype=np.uint8)
+    beta = ctypes.c_double(0.0)
+    _check(lib().rbq_fp8_levels(int(d), int(bits), lv.ctypes.data_as(_P), ctypes.byref(beta)), "rbq_fp8_levels")
+    return lv, beta.value
 
 
 def int8_levels(d, bits):

@@ -374,6 +374,39 @@ void int8_levels(const std::vector<double>& levels, std::vector<int8_t>& out, do
   *alpha = a;
 }
 
+// Round-to-nearest-even onto FP8 E4M3 (OCP "E4M3FN": 1 sign bit, 4 exponent
+// bits with bias 7, 3 mantissa bits, subnormals below 2^-6, largest finite
+// 448, no infinities) and encode; |x| above 448 saturates (never reached for
+// the scaled levels, which stay below 256).
+static uint8_t to_e4m3(double x) {
+  const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  double a = std::fabs(x);
+  if (a == 0.0) return sign;
+  int E = 0;
+  const double f = std::frexp(a, &E);          // a = f 2^E, f in [0.5, 1)
+  int e = E - 1;                               // a = m 2^e, m in [1, 2)
+  if (e < -6) {                                // subnormal: multiples of 2^-9
+    const double q = std::nearbyint(std::ldexp(a, 9));
+    if (q >= 8.0) return sign | (1u << 3);     // rounds up to the smallest normal
+    return sign | static_cast<uint8_t>(q);
+  }
+  double q = std::nearbyint(2.0 * f * 8.0);     // 8 .. 16
+  if (q == 16.0) { q = 8.0; ++e; }
+  if (e > 8 || (e == 8 && q > 14.0)) return sign | 0x7E;   // 448
+  return sign | static_cast<uint8_t>(((e + 7) << 3) | (static_cast<int>(q) - 8));
+}
+
+void fp8_levels(const std::vector<double>& levels, std::vector<uint8_t>& out, double* beta) {
+  double cmax = 0.0;
+  for (double c : levels) cmax = std::max(cmax, std::fabs(c));
+  int E = 0;
+  std::frexp(cmax, &E);                        // cmax in [2^(E-1), 2^E)
+  const double b = std::ldexp(1.0, 8 - E);     // b cmax in [128, 256)
+  out.assign(levels.size(), 0);
+  for (size_t j = 0; j < levels.size(); ++j) out[j] = to_e4m3(b * levels[j]);
+  *beta = b;
+}
+
 int codebook_device(int d, int bits, const CodebookDevice** out) {
   int dev;
   int rc = current_device(&dev);
@@ -404,6 +437,10 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
     int8_levels(levels, li, &cb->alpha);
     li.resize(256, 0);
     if ((rc = upload(li.data(), li.size(), &cb->levels_i8)) != RBQ_OK) { delete cb; return rc; }
+    std::vector<uint8_t> lf;
+    fp8_levels(levels, lf, &cb->beta);
+    lf.resize(256, 0);
+    if ((rc = upload(lf.data(), lf.size(), &cb->levels_e4m3)) != RBQ_OK) { delete cb; return rc; }
   }
   Grid grid;
   if ((rc = build_grid(bounds, &grid)) != RBQ_OK) { delete cb; return rc; }
@@ -423,6 +460,7 @@ int codebook_device(int d, int bits, const CodebookDevice** out) {
     cudaFree(cb->bounds);
     cudaFree(cb->levels_f16);
     cudaFree(cb->levels_i8);
+    cudaFree(cb->levels_e4m3);
     cudaFree(cb->grid);
     cudaFree(cb->grid_full);
     cudaFree(cb->grid_pad);
@@ -545,6 +583,19 @@ extern "C" int rbq_int8_levels(int d, int bits, int8_t* levels, double* alpha) {
   int8_levels(lv, li, &a);
   if (levels) std::memcpy(levels, li.data(), li.size());
   if (alpha) *alpha = a;
+  return RBQ_OK;
+}
+
+extern "C" int rbq_fp8_levels(int d, int bits, uint8_t* levels, double* beta) {
+  if (d <= 0 || bits < 1 || bits > 8) return RBQ_EINVAL;
+  std::vector<double> lv, bd;
+  const int rc = full_table(d, bits, lv, bd);
+  if (rc != RBQ_OK) return rc;
+  std::vector<uint8_t> lf;
+  double b = 0.0;
+  fp8_levels(lv, lf, &b);
+  if (levels) std::memcpy(levels, lf.data(), lf.size());
+  if (beta) *beta = b;
   return RBQ_OK;
 }
 

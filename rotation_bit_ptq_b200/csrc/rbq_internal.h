@@ -57,6 +57,11 @@ struct CodebookDevice {
   // RNE(alpha * level), alpha = 127 / max |level| (int8[256], zero padded).
   int8_t* levels_i8 = nullptr;
   double alpha = 0.0;
+  // qlinear_fp8_levels: levels times beta = 2^(7 - floor(log2 max |level|))
+  // rounded to FP8 E4M3 (round to nearest even), as E4M3 bytes (uint8[256],
+  // zero padded); the power-of-two beta leaves only the 3-bit mantissa rounding.
+  uint8_t* levels_e4m3 = nullptr;
+  double beta = 0.0;
   // Code-search grid: `grid_cells` + 1 cells centred at -R + n*2R/cells;
   // entry n = {boundary inside cell n or +inf, number of boundaries below
   // that cell}.  See build_grid() in rbq_host.cu.
@@ -90,6 +95,8 @@ int codebook_device(int d, int bits, const CodebookDevice** out);
 
 // The 8-bit integer levels of a codebook (see CodebookDevice::levels_i8).
 void int8_levels(const std::vector<double>& levels, std::vector<int8_t>& out, double* alpha);
+// The FP8 E4M3 levels of a codebook (see CodebookDevice::levels_e4m3).
+void fp8_levels(const std::vector<double>& levels, std::vector<uint8_t>& out, double* beta);
 
 // Records a CUDA error (for rbq_error_string) and maps it to RBQ_ECUDA.
 int cuda_fail(cudaError_t e);

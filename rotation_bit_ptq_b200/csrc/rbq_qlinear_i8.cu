@@ -1,4 +1,5 @@
-// qlinear_int8_levels: the quantised linear layer on the INT8 tensor cores.
+// qlinear_int8_levels / qlinear_fp8_levels: the quantised linear layer on the
+// 8-bit tensor cores.
 //
 //   OrbitQuant (hotelren.com/news/3376620) §2.2: with the rotation absorbed
 //   into the weights it cancels, y[m,n] = s_m r'_n sum_k C_w[q_nk] C_a[p_mk].
@@ -7,6 +8,11 @@
 //     y[m,n] = s_m r'_n (sum_k l_w[q_nk] l_a[p_mk]) / (alpha_w alpha_a),
 //   the sum exact in int32 (|sum| <= K 127^2 < 2^31 for K <= 32768), on
 //   tcgen05 kind::i8: twice the fp16 tensor rate and half the operand bytes.
+//   The FP8 form rounds beta c_j to E4M3 (beta a power of two, so only the
+//   3-bit mantissa rounding remains) and sums in fp32 on kind::f8f6f4:
+//     y[m,n] = s_m r'_n (sum_k e_w[q_nk] e_a[p_mk]) / (beta_w beta_a).
+//   Both run the same kernels; only the level bytes, the MMA kind and the
+//   accumulator type differ.
 //
 // Three kernels per call.
 // 1./2. expand_weights_i8_*: the weight codes [N, K*b/8] and the activation
@@ -62,15 +68,39 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T on signed 8-bit operands, int32 accumulate.
-__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format 0) and an
+// fp32 accumulator (D format 1), both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T on 8-bit operands: signed integers with an
+// int32 accumulator (kFp8 = false) or E4M3 with an fp32 one (kFp8 = true).
+template <bool kFp8>
+__device__ __forceinline__ void umma_8bit(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  if constexpr (kFp8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+
+// An accumulator word as fp32.
+template <bool kFp8>
+__device__ __forceinline__ float acc_value(uint32_t v) {
+  if constexpr (kFp8) return __uint_as_float(v);
+  else return __int2float_rn(static_cast<int>(v));
 }
 
 // The level bytes of codes 0..15 as four words (byte j of word w = level 4w+j).
@@ -119,9 +149,10 @@ struct __align__(8) Tail {
 
 constexpr size_t kSmem = 1024 + kAStages * kOpStage + sizeof(Tail) + 64;
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
-    qlinear_i8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const Params p) {
+    qlinear_8bit_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -158,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_i8(kBM, kBN);
+      constexpr uint32_t kIdesc = kFp8 ? idesc_e4m3(kBM, kBN) : idesc_i8(kBM, kBN);
       const uint64_t desc0 = sdesc_k_sw128(smem_u32(ops));
       uint32_t s = 0, ph = 0, it = 0;
       bool ok = true;
@@ -172,10 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);
           const uint64_t bd = ad + (kATile >> 4);
-          umma_i8(acc, ad, bd, kIdesc, ks != 0);
-          umma_i8(acc, ad + 2, bd + 2, kIdesc, 1u);            // +32 bytes = 32 values of K
-          umma_i8(acc, ad + 4, bd + 4, kIdesc, 1u);
-          umma_i8(acc, ad + 6, bd + 6, kIdesc, 1u);
+          umma_8bit<kFp8>(acc, ad, bd, kIdesc, ks != 0);
+          umma_8bit<kFp8>(acc, ad + 2, bd + 2, kIdesc, 1u);            // +32 bytes = 32 values of K
+          umma_8bit<kFp8>(acc, ad + 4, bd + 4, kIdesc, 1u);
+          umma_8bit<kFp8>(acc, ad + 6, bd + 6, kIdesc, 1u);
           umma_commit(&tl->empty[s]);
           if (++s == kAStages) { s = 0; ph ^= 1u; }
         }
@@ -234,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 16; ++j) {
             const uint32_t rr = *reinterpret_cast<const uint32_t*>(p.rnorm + nb + 2 * j);
             const float r0 = __uint_as_float(rr << 16), r1 = __uint_as_float(rr & 0xFFFF0000u);
-            const float f0 = __int2float_rn(static_cast<int>(v[2 * j]));
-            const float f1 = __int2float_rn(static_cast<int>(v[2 * j + 1]));
+            const float f0 = acc_value<kFp8>(v[2 * j]);
+            const float f1 = acc_value<kFp8>(v[2 * j + 1]);
             const __nv_bfloat162 h = __floats2bfloat162_rn(f0 * rs * r0, f1 * rs * r1);
             packed[j] = *reinterpret_cast<const uint32_t*>(&h);
           }
@@ -248,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) {
             if (nb + j < p.N) {
               const float rv = __uint_as_float(static_cast<uint32_t>(p.rnorm[nb + j]) << 16);
-              const float f = __int2float_rn(static_cast<int>(v[j]));
+              const float f = acc_value<kFp8>(v[j]);
               dst[j] = __bfloat16_as_ushort(__float2bfloat16_rn(f * rs * rv));
             }
           }
@@ -357,16 +388,16 @@ int encode_i8_map(CUtensorMap* map, const int8_t* base, int rows, int K, int box
 }
 
 // The GEMM on expanded int8 operands: activations `ai8` [M, K], weights `wi8` [N, K].
+template <bool kFp8>
 int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* rnorm, int M, int N, int K,
-             uint16_t* Y, const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err, cudaStream_t st,
-             int sms) {
+         uint16_t* Y, float inv_scale, unsigned int* err, cudaStream_t st, int sms) {
   Params p{};
   p.M = M;
   p.N = N;
   p.K = K;
   p.s = s;
   p.rnorm = rnorm;
-  p.inv_scale = static_cast<float>(1.0 / (ca->alpha * cw->alpha));
+  p.inv_scale = inv_scale;
   p.Y = Y;
   p.err = err;
   // walk N fastest when the int8 activations outweigh the weights: a wave of
@@ -377,7 +408,7 @@ int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* r
   int rc = encode_i8_map(&mA, ai8, M, K, kBM);
   if (rc != RBQ_OK) return rc;
   if ((rc = encode_i8_map(&mB, wi8, N, K, kBN)) != RBQ_OK) return rc;
-  auto kern = qlinear_i8_kernel;
+  auto kern = qlinear_8bit_kernel<kFp8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
@@ -401,9 +432,12 @@ int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* r
 
 using namespace rbq;
 
-extern "C" int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
-                                   const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
-                                   void* stream) {
+namespace {
+
+// The two 8-bit-level layers: validation, level tables, both expansions, GEMM.
+template <bool kFp8>
+int qlinear_8bit_levels(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
+                        const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y, void* stream) {
   if (M < 0 || N < 0 || K <= 0 || K % 128 || K > kMaxD) return RBQ_EINVAL;
   if (bits_a < 1 || bits_a > 8 || bits_w < 1 || bits_w > 8) return RBQ_EINVAL;
   if (N % 8 || (static_cast<long long>(K) * bits_a / 8) % 16) return RBQ_EINVAL;
@@ -427,12 +461,31 @@ extern "C" int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int b
   void* ws = nullptr;
   e = cudaMallocFromPoolAsync(&ws, (static_cast<size_t>(N) + M) * K, pool, st);
   if (e != cudaSuccess) return cuda_fail(e);
-  int8_t* wi8 = static_cast<int8_t*>(ws);
-  int8_t* ai8 = wi8 + static_cast<size_t>(N) * K;
-  rc = qi8::expand_weights(w_codes, bits_w, N, K, cw->levels_i8, wi8, st, sms);
-  if (rc == RBQ_OK) rc = qi8::expand_weights(a_codes, bits_a, M, K, ca->levels_i8, ai8, st, sms);
-  if (rc == RBQ_OK) rc = qi8::gemm(ai8, s, wi8, rnorm, M, N, K, Y, ca, cw, err, st, sms);
+  int8_t* wq = static_cast<int8_t*>(ws);
+  int8_t* aq = wq + static_cast<size_t>(N) * K;
+  // level bytes: two's-complement integers or E4M3 codes, expanded alike
+  const int8_t* lut_w = kFp8 ? reinterpret_cast<const int8_t*>(cw->levels_e4m3) : cw->levels_i8;
+  const int8_t* lut_a = kFp8 ? reinterpret_cast<const int8_t*>(ca->levels_e4m3) : ca->levels_i8;
+  const double scale = kFp8 ? ca->beta * cw->beta : ca->alpha * cw->alpha;
+  rc = qi8::expand_weights(w_codes, bits_w, N, K, lut_w, wq, st, sms);
+  if (rc == RBQ_OK) rc = qi8::expand_weights(a_codes, bits_a, M, K, lut_a, aq, st, sms);
+  if (rc == RBQ_OK)
+    rc = qi8::gemm<kFp8>(aq, s, wq, rnorm, M, N, K, Y, static_cast<float>(1.0 / scale), err, st, sms);
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
   return rc;
+}
+
+}  // namespace
+
+extern "C" int qlinear_int8_levels(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
+                                   const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
+                                   void* stream) {
+  return qlinear_8bit_levels<false>(a_codes, s, bits_a, w_codes, rnorm, bits_w, M, N, K, Y, stream);
+}
+
+extern "C" int qlinear_fp8_levels(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
+                                  const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
+                                  void* stream) {
+  return qlinear_8bit_levels<true>(a_codes, s, bits_a, w_codes, rnorm, bits_w, M, N, K, Y, stream);
 }

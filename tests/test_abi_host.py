@@ -158,7 +158,23 @@ def test_kernel_entry_points_validate_before_launch(lib):
     assert lib.qlinear_int8_levels(fake, fake, 4, fake, fake, 4, 8, 8, 32896, fake, None) == rbq.RBQ_EINVAL
     assert lib.qlinear_int8_levels(fake, None, 4, fake, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EINVAL
     assert lib.qlinear_int8_levels(odd, fake, 4, fake, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EALIGN
+    assert lib.qlinear_fp8_levels(None, None, 4, None, None, 4, 0, 8, 128, None, None) == rbq.RBQ_OK
+    assert lib.qlinear_fp8_levels(fake, fake, 4, fake, fake, 4, 8, 8, 192, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_fp8_levels(fake, fake, 4, fake, fake, 4, 8, 4, 128, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_fp8_levels(fake, fake, 4, odd, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EALIGN
     r.close()
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+def test_fp8_levels_match_oracle(lib, bits):
+    torch = pytest.importorskip("torch")
+    for d in (64, 3072, 12288):
+        lv, beta = rbq.fp8_levels(d, bits)
+        vals = torch.from_numpy(lv).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        ov, obeta = oracle.fp8_levels(oracle.lloydmax_table(d, bits)[0])
+        assert beta == obeta
+        assert np.array_equal(vals, ov)
+    assert lib.rbq_fp8_levels(64, 9, None, None) == rbq.RBQ_EINVAL
 
 
 @pytest.mark.parametrize("bits", range(1, 9))

@@ -436,6 +436,51 @@ def test_qlinear_int8_levels_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
     print(f"int8-level qlinear {M}x{N}x{K} W{bw}A{ba}: {n_band} in-band roundings, {dev:.2e} from exact levels")
 
 
+FP8_RTOL = 3e-3           # rel. Frobenius, fp32 sums of exact E4M3 products + BF16 output
+
+
+def _qlinear_fp8_case(X, W, d, bits_a, bits_w, seed=0, rows=None):
+    """qlinear_fp8_levels on the library's own codes vs the oracle's FP8 layer
+    (exact fp64 sums) on the same codes; returns (error vs oracle, deviation
+    from the exact-level layer)."""
+    r, _ = _rpbh(d, seed)
+    a_codes, s = rbq.rotate_quantize_act(r, _dense(X, "bf16"), bits_a)
+    w_codes, rn = rbq.quantize_weights(r, _dense(W, "bf16"), bits_w)
+    y = rbq.qlinear_fp8_levels(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    y_fp16 = rbq.qlinear(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
+    idx = torch.as_tensor(rows).cuda()
+    la, _ = oracle.lloydmax_table(d, bits_a)
+    lw, _ = oracle.lloydmax_table(d, bits_w)
+    pa = _unpack(a_codes[idx], bits_a, d)
+    pw = _unpack(w_codes, bits_w, d)
+    ref = oracle.qlinear_fp8_levels(pa, s.cpu().numpy()[rows], la, pw, bf16_to_numpy(rn), lw)
+    got = bf16_to_numpy(y[idx])
+    return rel_frobenius(got, ref), rel_frobenius(got, bf16_to_numpy(y_fp16[idx]))
+
+
+@pytest.mark.parametrize("M,N,K,ba,bw", [(1, 8, 128, 4, 4), (130, 136, 128, 4, 2), (257, 264, 384, 3, 3),
+                                         (64, 512, 256, 6, 4), (200, 128, 256, 8, 8), (300, 520, 256, 5, 7),
+                                         (129, 512, 1024, 4, 4), (260, 256, 640, 1, 5)])
+def test_qlinear_fp8_levels_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
+    g = np.random.default_rng(M * N + 2)
+    X = synth.to_bf16(g.standard_t(3, (M, K)).astype(np.float32))
+    W = synth.to_bf16((g.standard_normal((N, K)) * 0.02).astype(np.float32))
+    err, dev = _qlinear_fp8_case(X, W, K, ba, bw, seed=M)
+    print(f"fp8-level qlinear {M}x{N}x{K} W{bw}A{ba}: {err:.2e} vs oracle, {dev:.2e} from exact levels")
+    assert err < FP8_RTOL, err
+
+
+def test_qlinear_fp8_levels_attention_projection_sampled():
+    data = synth.attn_proj()
+    rows = np.random.default_rng(7).choice(4608, 32, replace=False)
+    err, dev = _qlinear_fp8_case(data["X"], data["W"], 3072, 4, 4, rows=rows)
+    print(f"fp8-level qlinear attn_proj W4A4: {err:.2e} vs oracle, {dev:.2e} from exact levels")
+    assert err < FP8_RTOL and dev < 5e-2, (err, dev)
+
+
 def test_qlinear_int8_levels_attention_projection_sampled():
     data = synth.attn_proj()
     rows = np.random.default_rng(5).choice(4608, 32, replace=False)

@@ -1,12 +1,15 @@
-"""Pins of the oracle's 8-bit integer-level layer (oracle.qlinear.int8_levels,
-oracle.qlinear.qlinear_int8_levels).
+"""Pins of the oracle's 8-bit-level layers (oracle.qlinear.int8_levels,
+qlinear_int8_levels, e4m3_round, fp8_levels, qlinear_fp8_levels).
 
 * the integer levels of J. Max's (1960) 4-, 8- and 16-level Gaussian
   quantisers, worked by hand from the published table (tests/golden);
 * grid invariants: |l| <= 127 with 127 reached, antisymmetry, order, and
   |l - alpha c| <= 1/2; the same integers for every d (alpha absorbs 1/sqrt(d));
 * the layer against a pure-Python triple loop, the equal-code closed form, and
-  the exact-level layer (oracle.qlinear) within the levels' rounding bound.
+  the exact-level layer (oracle.qlinear) within the levels' rounding bound;
+* FP8: E4M3 rounding against PyTorch's float8_e4m3fn conversion, the Max
+  tables rounded to 3 mantissa bits by hand (tests/golden), the power-of-two
+  scale, and the same loop, closed form and rounding bound.
 """
 
 import numpy as np
@@ -104,5 +107,74 @@ def test_within_rounding_bound_of_exact_levels(ba, bw):
     # C_w C_a - L_w L_a = C_w (C_a - L_a) + L_a (C_w - L_w), |L - C| <= 1/(2 alpha)
     per = np.abs(cw[q])[None, :, :] * 0.5 / aa + np.abs(la[p] / aa)[:, None, :] * 0.5 / oracle.int8_levels(cw)[1]
     bound = s[:, None] * rn[None, :] * per.sum(axis=2)
+    assert np.all(np.abs(y8 - y) <= bound * (1 + 1e-12))
+    assert np.any(y8 != y)
+
+
+# ---- the FP8 (E4M3) form ----------------------------------------------------
+
+def test_e4m3_rounding_matches_library_conversion():
+    torch = pytest.importorskip("torch")
+    x = np.concatenate([np.linspace(-448, 448, 20001), np.exp2(np.arange(-12, 8.8, 0.01)),
+                        -np.exp2(np.arange(-12, 8.8, 0.013)),
+                        [0.59375, 2.0 ** -10, 1.5 * 2.0 ** -10, 1.0625, 1.1875, 0.0]])
+    lib = torch.tensor(x, dtype=torch.float64).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_round(x), lib)
+
+
+def test_fp8_levels_of_max_1960_table():
+    for row in golden_rows("fp8_levels_max1960.txt"):
+        n = int(row[0])
+        want = np.array([float(v) for v in row[1].split()])
+        c, _, _ = oracle.lloydmax_unit(int(np.log2(n)))
+        e, beta = oracle.fp8_levels(c)
+        assert np.array_equal(e[n // 2:] / beta, want)
+        assert np.array_equal(e[: n // 2] / beta, -want[::-1])
+
+
+@pytest.mark.parametrize("bits", range(1, 9))
+def test_fp8_level_scale_and_bound(bits):
+    for d in (64, 3072, 12288):
+        c, _ = oracle.lloydmax_table(d, bits)
+        e, beta = oracle.fp8_levels(c)
+        assert beta == 2.0 ** np.round(np.log2(beta))
+        assert 128 <= beta * np.max(np.abs(c)) < 256
+        assert np.all(np.abs(e / beta - c) <= 2.0 ** -4 * np.abs(c))
+        assert np.array_equal(e, -e[::-1])
+
+
+def test_fp8_layer_against_triple_loop_and_closed_form():
+    g = np.random.default_rng(9)
+    K = 64
+    ca, _ = oracle.lloydmax_table(K, 4)
+    cw, _ = oracle.lloydmax_table(K, 3)
+    p = g.integers(0, 16, (3, K))
+    q = g.integers(0, 8, (4, K))
+    s = g.uniform(0.5, 2, 3)
+    rn = g.uniform(0.5, 2, 4)
+    y = oracle.qlinear_fp8_levels(p, s, ca, q, rn, cw)
+    ea, ba = oracle.fp8_levels(ca)
+    ew, bw = oracle.fp8_levels(cw)
+    assert np.allclose(y, _loop(p, s, ea, ba, q, rn, ew, bw), rtol=1e-14, atol=0)
+    pe = np.full((2, K), 11)
+    qe = np.full((2, K), 2)
+    ye = oracle.qlinear_fp8_levels(pe, s[:2], ca, qe, rn[:2], cw)
+    assert np.allclose(ye, s[:2, None] * rn[None, :2] * K * ea[11] * ew[2] / (ba * bw), rtol=1e-15, atol=0)
+
+
+def test_fp8_layer_within_rounding_bound_of_exact_levels():
+    g = np.random.default_rng(10)
+    K = 512
+    ca, _ = oracle.lloydmax_table(K, 4)
+    cw, _ = oracle.lloydmax_table(K, 4)
+    p = g.integers(0, 16, (6, K))
+    q = g.integers(0, 16, (7, K))
+    s = g.uniform(0.5, 2, 6)
+    rn = g.uniform(0.5, 2, 7)
+    y8 = oracle.qlinear_fp8_levels(p, s, ca, q, rn, cw)
+    y = oracle.qlinear(p, s, ca, q, rn, cw)
+    # each level within 2^-4 relative, so each product within (1 + 2^-4)^2 - 1
+    prod = np.abs(ca[p])[:, None, :] * np.abs(cw[q])[None, :, :]
+    bound = s[:, None] * rn[None, :] * prod.sum(axis=2) * ((1 + 2.0 ** -4) ** 2 - 1)
     assert np.all(np.abs(y8 - y) <= bound * (1 + 1e-12))
     assert np.any(y8 != y)
