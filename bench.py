@@ -419,11 +419,13 @@ def run_suite(dev, stream, pk):
         tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
         return {"us": round(us, 2), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / tc, 4)}
 
-    def i8_entry(us, M, N, K, us_fp16, y8, y16):
-        # int8 dense peak: the measured bf16 peak times the nominal int8:bf16 ratio (4.5 / 2.25)
-        tops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+    def i8_entry(us, M, N, K, us_fp16, y8, y16, fp8=False):
+        # int8 / fp8 dense peak: the measured bf16 peak times the nominal
+        # 8-bit:bf16 ratio (4.5 / 2.25)
+        ops = 2.0 * M * N * K / (us * 1e-6) / 1e12
         dev_ = float(torch.linalg.norm((y8.float() - y16.float())) / torch.linalg.norm(y16.float()))
-        return {"us": round(us, 2), "TOPS": round(tops, 1), "frac_int8": round(tops / (2 * tc), 4),
+        return {"us": round(us, 2), ("TFLOP/s" if fp8 else "TOPS"): round(ops, 1),
+                ("frac_fp8" if fp8 else "frac_int8"): round(ops / (2 * tc), 4),
                 "speedup_vs_fp16_levels": round(us_fp16 / us, 3), "rel_dev_from_exact_levels": round(dev_, 5)}
 
     # MLP pair: up 3072 -> 12288, down 12288 -> 3072, 4608 tokens
@@ -458,6 +460,15 @@ def run_suite(dev, stream, pk):
         e["qlinear_int8_levels down"] = i8_entry(
             _time_us(lambda: rbq.qlinear_int8_levels(ad, sd, ba, wd, nd, bw, 12288, yd8, stream=stream), stream),
             T, 3072, 12288, e["qlinear down 4608x3072x12288"]["us"], yd8, yd)
+        del yu8, yd8
+        yu8 = rbq.qlinear_fp8_levels(au, su, ba, wu, nu, bw, 3072)
+        yd8 = rbq.qlinear_fp8_levels(ad, sd, ba, wd, nd, bw, 12288)
+        e["qlinear_fp8_levels up"] = i8_entry(
+            _time_us(lambda: rbq.qlinear_fp8_levels(au, su, ba, wu, nu, bw, 3072, yu8, stream=stream), stream),
+            T, 12288, 3072, e["qlinear up 4608x12288x3072"]["us"], yu8, yu, fp8=True)
+        e["qlinear_fp8_levels down"] = i8_entry(
+            _time_us(lambda: rbq.qlinear_fp8_levels(ad, sd, ba, wd, nd, bw, 12288, yd8, stream=stream), stream),
+            T, 3072, 12288, e["qlinear down 4608x3072x12288"]["us"], yd8, yd, fp8=True)
         del yu8, yd8
         mlp[f"W{bw}A{ba}"] = e
     out["mlp_pair"] = mlp
@@ -621,7 +632,11 @@ def run_suite(dev, stream, pk):
     out["int8_levels_attn_proj_W4A4"] = i8_entry(
         _time_us(lambda: rbq.qlinear_int8_levels(a4, s4, 4, wc4, wn4, 4, 3072, y8, stream=stream), stream),
         4608, 3072, 3072, us16, y8, y16)
-    del y8, y16
+    yf = rbq.qlinear_fp8_levels(a4, s4, 4, wc4, wn4, 4, 3072)
+    out["fp8_levels_attn_proj_W4A4"] = i8_entry(
+        _time_us(lambda: rbq.qlinear_fp8_levels(a4, s4, 4, wc4, wn4, 4, 3072, yf, stream=stream), stream),
+        4608, 3072, 3072, us16, yf, y16, fp8=True)
+    del y8, y16, yf
     r.close()
     del X, W, y, wc4, wn4, a4, s4
     torch.cuda.synchronize()
