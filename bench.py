@@ -709,8 +709,12 @@ def run_kernel_only(args):
     dev = torch.device("cuda", 0)
     r = rbq.RPBH(D, SEED)
     if args.kernel_only in ("rotate_quantize", "rotate_only"):
+        d = args.dim or D
         tokens = args.tokens or 32768
-        X = to_bf16_tensor(synth.student_t_act(tokens, D, seed=SEED)[0], dev)
+        if d != D:
+            r.close()
+            r = rbq.RPBH(d, SEED)
+        X = to_bf16_tensor(synth.student_t_act(tokens, d, seed=SEED)[0], dev)
         for _ in range(args.launches):
             if args.kernel_only == "rotate_quantize":
                 rbq.rotate_quantize_act(r, X, BITS_A)
@@ -757,6 +761,7 @@ def main():
                                                    "qlinear_int8_levels", "qlinear_int8", "quantize_weights_int8"],
                     help="run one kernel on a profiling-sized case (for ncu) instead of the benchmark")
     ap.add_argument("--tokens", type=int, default=0)
+    ap.add_argument("--dim", type=int, default=0, help="--kernel-only rotate_*: input width (default 3072)")
     ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
     if args.kernel_only:
