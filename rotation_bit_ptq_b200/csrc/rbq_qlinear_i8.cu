@@ -20,7 +20,7 @@
 //    stream-ordered workspace (4-bit codes by byte permutes over a 16-byte
 //    register table, other widths through a byte table in shared memory).
 //    The activation part (M*K bytes) stays in L2 for the GEMM.
-// 3. qlinear_i8_kernel: persistent, one CTA per SM, 128 x 256 output
+// 3. qlinear_8bit_kernel: persistent, one CTA per SM, 128 x 256 output
 //    tiles, K slices of 128 int8 values (one 128-byte swizzle row per operand
 //    row, so a stage is 16 KB of activations + 32 KB of weights):
 //      warps 0..3  epilogue: TMEM lane quadrant, one output row per thread;
