@@ -617,9 +617,12 @@ __global__ void __launch_bounds__(256) expand_weights_kernel8(const uint8_t* cod
   }
 }
 
-// 4-bit codes: one thread per 32 codes (16 bytes in, 64 bytes out).
-__global__ void __launch_bounds__(256) expand_weights_kernel4x32(const uint4* codes, long long groups,
-                                                                const uint16_t* lut_g, uint4* out) {
+// 4-bit codes: a warp expands 128 words of 8 codes (512 bytes in, 2 KB out)
+// per step; lane l takes words l, l+32, l+64 and l+96 of the warp's range, so
+// every load and every store instruction of the warp covers contiguous memory
+// (128 and 512 bytes) instead of 16-byte pieces 64 bytes apart.
+__global__ void __launch_bounds__(256) expand_weights_kernel4(const uint32_t* codes, long long words,
+                                                             const uint16_t* lut_g, uint4* out) {
   Planes4 P;
   {
     uint16_t lut[16];
@@ -627,15 +630,24 @@ __global__ void __launch_bounds__(256) expand_weights_kernel4x32(const uint4* co
     for (int i = 0; i < 16; ++i) lut[i] = __ldg(lut_g + i);
     P = make_planes4(lut);
   }
-  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
-       g += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint4 v = __ldcs(codes + g);
-    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long base = (blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5)) * 128;
+       base < words; base += 128 * warps) {
+    uint32_t x[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t w[4];
-      expand8_4bit(x[i], P, w);
-      __stcg(out + 4 * g + i, make_uint4(w[0], w[1], w[2], w[3]));
+    for (int j = 0; j < 4; ++j) {
+      const long long g = base + 32 * j + lane;
+      x[j] = g < words ? __ldcs(codes + g) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long g = base + 32 * j + lane;
+      if (g < words) {
+        uint32_t w[4];
+        expand8_4bit(x[j], P, w);
+        __stcg(out + g, make_uint4(w[0], w[1], w[2], w[3]));
+      }
     }
   }
 }
@@ -644,12 +656,12 @@ template <int BITS>
 int launch_expand(const uint8_t* codes, int rows, int K, const uint16_t* lut, uint16_t* out, cudaStream_t st,
                   int sms) {
   if constexpr (BITS == 4) {
-    // K is a multiple of 128, so every row holds whole 32-code groups
-    const long long groups = static_cast<long long>(rows) * (K / 32);
-    long long blocks = (groups + 255) / 256;
+    // one 32-bit word of codes = 8 fp16 levels = one 16-byte output chunk
+    const long long words = static_cast<long long>(rows) * (K / 8);
+    long long blocks = (words + 1023) / 1024;               // 8 warps x 128 words
     if (blocks > 16LL * sms) blocks = 16LL * sms;
-    expand_weights_kernel4x32<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint4*>(codes),
-                                                                         groups, lut, reinterpret_cast<uint4*>(out));
+    expand_weights_kernel4<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes),
+                                                                      words, lut, reinterpret_cast<uint4*>(out));
   } else if constexpr (8 % BITS == 0) {
     const long long groups = static_cast<long long>(rows) * (K / 8);
     long long blocks = (groups + 255) / 256;

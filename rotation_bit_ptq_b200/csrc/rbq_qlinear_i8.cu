@@ -298,22 +298,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Weight codes [N, K*b/8] -> int8 levels [N, K].  4-bit: a thread per 32 codes
-// (16 bytes in, 32 out); other widths: a thread per 8 codes (b bytes in, 8
-// out).  K is a multiple of 128, so no group straddles two rows.
-__global__ void __launch_bounds__(256) expand_weights_i8_4bit(const uint4* codes, long long groups,
+// Codes [rows, K*b/8] -> 8-bit levels [rows, K].  4-bit: a warp expands 128
+// pairs of code words (16 codes each: 8 bytes in, 16 out) per step, lane l
+// taking pairs l, l+32, l+64, l+96 of the warp's range, so every load and store
+// instruction of the warp covers contiguous memory; other widths: a thread per
+// 8 codes (b bytes in, 8 out).  K is a multiple of 128, so no group straddles
+// two rows.
+__global__ void __launch_bounds__(256) expand_weights_i8_4bit(const uint2* codes, long long pairs,
                                                              const int8_t* lut_g, uint4* out) {
   __shared__ __align__(16) uint8_t lut[16];
   if (threadIdx.x < 16) lut[threadIdx.x] = static_cast<uint8_t>(lut_g[threadIdx.x]);
   __syncthreads();
   const Tab16 T = make_tab16(lut);
-  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
-       g += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint4 v = __ldcs(codes + g);
-    const uint2 w0 = expand8_4bit_i8(v.x, T), w1 = expand8_4bit_i8(v.y, T);
-    const uint2 w2 = expand8_4bit_i8(v.z, T), w3 = expand8_4bit_i8(v.w, T);
-    __stcg(out + 2 * g, make_uint4(w0.x, w0.y, w1.x, w1.y));
-    __stcg(out + 2 * g + 1, make_uint4(w2.x, w2.y, w3.x, w3.y));
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long base = (blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5)) * 128;
+       base < pairs; base += 128 * warps) {
+    uint2 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long g = base + 32 * j + lane;
+      v[j] = g < pairs ? __ldcs(codes + g) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long g = base + 32 * j + lane;
+      if (g < pairs) {
+        const uint2 w0 = expand8_4bit_i8(v[j].x, T), w1 = expand8_4bit_i8(v[j].y, T);
+        __stcg(out + g, make_uint4(w0.x, w0.y, w1.x, w1.y));
+      }
+    }
   }
 }
 
@@ -348,10 +362,10 @@ int expand_weights(const uint8_t* codes, int bits, int rows, int K, const int8_t
                    cudaStream_t st, int sms) {
   const long long elems = static_cast<long long>(rows) * K;
   if (bits == 4) {
-    const long long groups = elems / 32;
-    long long blocks = (groups + 255) / 256;
+    const long long pairs = elems / 16;                     // 16 codes: 8 bytes in, 16 out
+    long long blocks = (pairs + 1023) / 1024;               // 8 warps x 128 pairs
     if (blocks > 16LL * sms) blocks = 16LL * sms;
-    expand_weights_i8_4bit<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint4*>(codes), groups,
+    expand_weights_i8_4bit<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint2*>(codes), pairs,
                                                                       lut, reinterpret_cast<uint4*>(out));
   } else {
     const long long groups = elems / 8;
