@@ -783,12 +783,14 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     res = run_ours(args, rank, world)
-    if rank == 0 and not args.no_suite:
+    # The other workloads' kernel timings and the CPU baseline run at N = 1
+    # only: at N > 1 they would hold every rank's GPU at the closing barrier.
+    if world == 1 and not args.no_suite:
         import torch
         res["suite"] = run_suite(torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))),
                                  torch.cuda.current_stream(), peaks())
     if rank == 0:
-        if not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline:
             gbs, el, reps = oracle_rotq_gbs(T, 10.0)
             res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
                                    "sample": f"all {T} tokens x {reps} reps ({el:.1f} s), dense fp64 Pi (numpy)"}
