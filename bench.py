@@ -601,7 +601,7 @@ def run_suite(dev, stream, pk):
         del X, xr, codes, norms, R
     out["transform_ablation"] = abl
 
-    # Bit-width sweep (mixed per-layer widths): the
+    # Bit-width sweep (per-layer widths, OrbitQuant §4.2-§4.4): the
     # attention projection (4608 x 3072 x 3072) at every activation width
     # with 4-bit weights and every weight width with 4-bit activations.
     data = synth.attn_proj(seed=5)

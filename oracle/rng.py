@@ -3,7 +3,7 @@
 OrbitQuant §2.3 defines Pi_d = blkdiag(H_h D_1, ..., H_h D_{d/h}) · P_pi with
 Rademacher signs D_i and a random permutation P_pi, and §6.3 asks that the
 permutation be reproducible across platforms.  The pages name no generator,
-so this build fixes one (our reading; the pages cannot pin the choice):
+this oracle fixes one (a reading; the pages cannot pin the choice):
 
 * generator: SplitMix64 (G. Steele, D. Lea, C. Flood, "Fast splittable
   pseudorandom number generators", OOPSLA 2014): a Weyl sequence with

@@ -23,7 +23,7 @@ if not torch.cuda.is_available():
 
 import rotation_bit_ptq_b200 as rbq  # noqa: E402
 
-NORM_RTOL = 1e-5          # fp32 norm vs fp64 (spec bar)
+NORM_RTOL = 1e-5          # fp32 norm vs fp64 (the stated norm tolerance)
 QLINEAR_RTOL = 4e-3       # rel. Frobenius, fp16 operands + BF16 output (bar: 2e-2)
 QLINEAR8_RTOL = 3e-3      # rel. Frobenius, exact operands + BF16 output (bar: 2e-2)
 
