@@ -168,7 +168,7 @@ def test_kernel_entry_points_validate_before_launch(lib):
 @pytest.mark.parametrize("bits", range(1, 9))
 def test_fp8_levels_match_oracle(lib, bits):
     torch = pytest.importorskip("torch")
-    for d in (64, 3072, 12288):
+    for d in (64, 256, 1536, 3072, 4096, 8960, 12288, 16384):   # every width of the workloads
         lv, beta = rbq.fp8_levels(d, bits)
         vals = torch.from_numpy(lv).view(torch.float8_e4m3fn).to(torch.float64).numpy()
         ov, obeta = oracle.fp8_levels(oracle.lloydmax_table(d, bits)[0])
@@ -179,7 +179,7 @@ def test_fp8_levels_match_oracle(lib, bits):
 
 @pytest.mark.parametrize("bits", range(1, 9))
 def test_int8_levels_match_oracle(lib, bits):
-    for d in (64, 3072, 12288):
+    for d in (64, 256, 1536, 3072, 4096, 8960, 12288, 16384):   # every width of the workloads
         lv, alpha = rbq.int8_levels(d, bits)
         olv, oalpha = oracle.int8_levels(oracle.lloydmax_table(d, bits)[0])
         assert np.array_equal(lv.astype(np.int64), olv)
