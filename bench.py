@@ -667,6 +667,13 @@ def oracle_rotq_gbs(tokens, min_seconds, rank_seed=0):
     return act_bytes_per_token() * tokens * reps / el / 1e9, el, reps
 
 
+def oracle_rotq_gbs_single_thread(tokens, min_seconds):
+    """oracle_rotq_gbs with the BLAS thread pools limited to one thread."""
+    import threadpoolctl
+    with threadpoolctl.threadpool_limits(limits=1):
+        return oracle_rotq_gbs(tokens, min_seconds)
+
+
 def cpu_cores():
     try:
         import threadpoolctl
@@ -794,6 +801,10 @@ def main():
             gbs, el, reps = oracle_rotq_gbs(T, 10.0)
             res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
                                    "sample": f"all {T} tokens x {reps} reps ({el:.1f} s), dense fp64 Pi (numpy)"}
+            gbs1, el1, reps1 = oracle_rotq_gbs_single_thread(512, 3.0)
+            res["cpu_baseline"]["single_thread"] = {
+                "value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                "sample": f"512 of {T} tokens x {reps1} reps ({el1:.1f} s), BLAS limited to one thread"}
         print(json.dumps(res))
     if world > 1:
         import torch.distributed as dist
