@@ -215,6 +215,11 @@ int quantize_weights_int8_asym(const rbq_rpbh* r, const void* W, int dtype, int 
  *   M, N, K  tokens, output width, input width (K a multiple of 64)
  *   Y        device uint16 BF16 [M, N], row-major
  * Alignment: code arrays 16-byte, Y 16-byte, s/rnorm 4-byte.
+ * Workspace (K a multiple of 128, N of 8, 16-byte code rows): the weight codes
+ * are expanded per call into fp16 levels, N*K*2 bytes from a stream-ordered
+ * memory pool; activation widths other than 4 bits are expanded too, M*K*2
+ * more bytes, while that part is at most 128 MiB.  Other shapes run a
+ * general kernel that expands both operands tile by tile without a workspace.
  * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
  */
 int qlinear(const uint8_t* a_codes, const float* s, int bits_a,
@@ -290,8 +295,9 @@ int rbq_int8_levels(int d, int bits, int8_t* levels, double* alpha);
  * allocate device memory.  (The pages have no counterpart: this is a
  * deployment variant of the library, not a step of the method.)
  *
- * qlinear expands the weight codes into an fp16 workspace of N*K*2 bytes taken
- * from a stream-ordered memory pool on every call.  Callers that own all device
+ * qlinear expands the weight codes (and, at activation widths other than 4
+ * bits, the activation codes) into an fp16 workspace taken from a
+ * stream-ordered memory pool on every call.  Callers that own all device
  * memory through their own allocator, forbid allocation on their inference
  * thread, or run inside a process whose allocator is not CUDA's cannot accept
  * that.  This entry point allocates nothing: its workspace, its two level
