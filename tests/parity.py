@@ -136,3 +136,25 @@ def rel_frobenius(y, ref):
     y = np.asarray(y, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     return float(np.linalg.norm(y - ref) / np.linalg.norm(ref))
+
+
+# --------------------------------------------------------------------------
+# poisoned output buffers: every output the kernels are asked to write starts
+# as a value they never produce (0xAB bytes for codes and int8, NaN for BF16
+# and fp32), so a row or tile a kernel leaves unwritten fails its comparison
+# instead of passing on whatever stale bytes the allocator returned
+# --------------------------------------------------------------------------
+
+POISON_BYTE = 0xAB
+
+
+def poison(shape, dtype, device="cuda"):
+    import torch
+    if dtype in (torch.uint8, torch.int8):
+        t = torch.empty(shape, dtype=torch.uint8, device=device).fill_(POISON_BYTE)
+        return t if dtype == torch.uint8 else t.view(torch.int8)
+    if dtype in (torch.float32, torch.bfloat16, torch.float16):
+        return torch.full(shape, float("nan"), dtype=dtype, device=device)
+    if dtype == torch.int32:
+        return torch.full(shape, -0x54545455, dtype=dtype, device=device)
+    raise TypeError(f"no poison for {dtype}")

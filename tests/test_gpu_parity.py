@@ -13,7 +13,7 @@ import pytest
 import oracle
 import synth
 from parity import (bf16_to_numpy, check_bf16_rounding, check_codes, check_int8, check_int8_asym, check_rel,
-                    rel_frobenius, torch_bf16)
+                    poison, rel_frobenius, torch_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -46,12 +46,54 @@ def _unpack(t, bits, d):
     return oracle.unpack_codes(t.cpu().numpy(), bits, d)
 
 
+# Library calls with poisoned outputs (see parity.poison): every element the
+# comparison reads must have been written by the kernel.
+
+def rq_act(r, X, bits):
+    T, d = X.shape
+    return rbq.rotate_quantize_act(r, X, bits, codes=poison((T, d * bits // 8), torch.uint8),
+                                   norms=poison((T,), torch.float32))
+
+
+def rot_act(r, X, norms=None):
+    return rbq.rotate_act(r, X, out=poison(tuple(X.shape), torch.bfloat16), norms=norms)
+
+
+def qweights(r, W, bits, mode="lloydmax"):
+    N, d = W.shape
+    if mode == "lloydmax":
+        return rbq.quantize_weights(r, W, bits, mode, out=poison((N, d * bits // 8), torch.uint8),
+                                    aux=poison((N,), torch.bfloat16))
+    return rbq.quantize_weights(r, W, bits, mode, out=poison((N, d), torch.int8), aux=poison((N,), torch.float32))
+
+
+def _layer(fn, a_codes, s, ba, w_codes, rn, bw, K):
+    return fn(a_codes, s, ba, w_codes, rn, bw, K,
+              out=poison((a_codes.shape[0], w_codes.shape[0]), torch.bfloat16))
+
+
+def qlin(a_codes, s, ba, w_codes, rn, bw, K):
+    return _layer(rbq.qlinear, a_codes, s, ba, w_codes, rn, bw, K)
+
+
+def qlin_i8(a_codes, s, ba, w_codes, rn, bw, K):
+    return _layer(rbq.qlinear_int8_levels, a_codes, s, ba, w_codes, rn, bw, K)
+
+
+def qlin_fp8(a_codes, s, ba, w_codes, rn, bw, K):
+    return _layer(rbq.qlinear_fp8_levels, a_codes, s, ba, w_codes, rn, bw, K)
+
+
+def qlin_int8(xr, q, sc):
+    return rbq.qlinear_int8(xr, q, sc, out=poison((xr.shape[0], q.shape[0]), torch.bfloat16))
+
+
 def _act_parity(X, d, bits, seed=0, dtype="bf16", rows=None, Pi=None, r=None):
     """Run the kernel on all of X; compare rows `rows` (default all) with the oracle."""
     if r is None:
         r, Pi = _rpbh(d, seed)
     xt = _dense(X, dtype)
-    codes, norms = rbq.rotate_quantize_act(r, xt, bits)
+    codes, norms = rq_act(r, xt, bits)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
@@ -171,7 +213,7 @@ def test_pair_kernel_rotate_only(d):
     X, _ = synth.student_t_act(41, d, seed=d)
     r, Pi = _rpbh(d, 6)
     nr = torch.empty((41,), dtype=torch.float32, device="cuda")
-    xr = rbq.rotate_act(r, torch_bf16(X), norms=nr)
+    xr = rot_act(r, torch_bf16(X), norms=nr)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     ora = oracle.rotate_only(X.astype(np.float64), Pi)
@@ -184,7 +226,7 @@ def test_pair_kernel_weights_int8(d, n):
     W = synth.to_bf16(synth.gaussian_weights(synth.rng(12, d), n, d, outlier_frac=0.01).astype(np.float32))
     W[3] = 0.0
     r, Pi = _rpbh(d, 9)
-    q, sc = rbq.quantize_weights(r, torch_bf16(W), 8, mode="int8")
+    q, sc = qweights(r, torch_bf16(W), 8, mode="int8")
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi)
@@ -198,16 +240,16 @@ def test_weights_int8_per_tensor(d, n, dtype):
     W = synth.to_bf16(synth.gaussian_weights(synth.rng(13, d), n, d, outlier_frac=0.01).astype(np.float32))
     W[4] = 0.0
     r, Pi = _rpbh(d, 10)
-    q, sc = rbq.quantize_weights(r, _dense(W, dtype), 8, mode="int8_tensor")
+    q, sc = qweights(r, _dense(W, dtype), 8, mode="int8_tensor")
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi, per_tensor=True)
     check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
     # and the layer runs unchanged on it
     X = synth.to_bf16(np.random.default_rng(d).standard_normal((20, d)).astype(np.float32))
-    xr = rbq.rotate_act(r, torch_bf16(X)) if dtype == "bf16" else None
+    xr = rot_act(r, torch_bf16(X)) if dtype == "bf16" else None
     if xr is not None:
-        y = rbq.qlinear_int8(xr, q, sc)
+        y = qlin_int8(xr, q, sc)
         torch.cuda.synchronize()
         ref = oracle.qlinear_int8(bf16_to_numpy(xr), q.cpu().numpy().astype(np.float64),
                                   sc.cpu().numpy().astype(np.float64))
@@ -221,7 +263,9 @@ def test_weights_int8_asymmetric(d, n, dtype):
     W = synth.to_bf16(W)
     W[2] = 0.0
     r, Pi = _rpbh(d, 12)
-    q, sc, z = rbq.quantize_weights_int8_asym(r, _dense(W, dtype))
+    q, sc, z = rbq.quantize_weights_int8_asym(r, _dense(W, dtype), q=poison((n, d), torch.uint8),
+                                              scale=poison((n,), torch.float32),
+                                              zero_point=poison((n,), torch.uint8))
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     ora = oracle.quantize_weights_int8_asym(W.astype(np.float64), Pi)
@@ -229,8 +273,8 @@ def test_weights_int8_asymmetric(d, n, dtype):
                     z.cpu().numpy().astype(np.int64), ora)
     if n % 8 == 0 and dtype == "bf16":
         X = synth.to_bf16(np.random.default_rng(d + 1).standard_normal((24, d)).astype(np.float32))
-        xr = rbq.rotate_act(r, torch_bf16(X))
-        y = rbq.qlinear_int8_asym(xr, q, sc, z)
+        xr = rot_act(r, torch_bf16(X))
+        y = rbq.qlinear_int8_asym(xr, q, sc, z, out=poison((24, n), torch.bfloat16))
         torch.cuda.synchronize()
         assert rbq.device_error() == 0
         ref = oracle.qlinear_int8_asym(bf16_to_numpy(xr), q.cpu().numpy(), sc.cpu().numpy().astype(np.float64),
@@ -244,7 +288,7 @@ def test_pair_kernel_weights_wide_codebooks(bits):
     W = synth.attn_proj()["W"][:40].copy()
     W[2] = 0.0
     r, Pi = _rpbh(d, 0)
-    codes, rn = rbq.quantize_weights(r, torch_bf16(W), bits)
+    codes, rn = qweights(r, torch_bf16(W), bits)
     torch.cuda.synchronize()
     _, bounds = oracle.lloydmax_table(d, bits)
     ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
@@ -277,7 +321,7 @@ def test_ablation_handle_rotate_only(d):
     r = rbq.RPBH(d, 8, permute=False)
     perm, sg = r.export()
     Pi = oracle.rpbh_matrix(perm.astype(np.int64), sg.astype(np.int64))
-    xr = rbq.rotate_act(r, torch_bf16(X))
+    xr = rot_act(r, torch_bf16(X))
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     ora = oracle.rotate_only(X.astype(np.float64), Pi)
@@ -292,7 +336,7 @@ def test_ablation_handle_rotate_only(d):
 def test_rotate_only_bf16(d):
     X, _ = synth.student_t_act(200, d, seed=9)
     r, Pi = _rpbh(d, 4)
-    xr = rbq.rotate_act(r, torch_bf16(X))
+    xr = rot_act(r, torch_bf16(X))
     torch.cuda.synchronize()
     ora = oracle.rotate_only(X.astype(np.float64), Pi)
     n = check_bf16_rounding(bf16_to_numpy(xr), ora["xr"], "rotate-only")
@@ -306,7 +350,7 @@ def test_weights_lloydmax(bits):
     W = W.copy()
     W[5] = 0.0
     r, Pi = _rpbh(d, 0)
-    codes, rn = rbq.quantize_weights(r, torch_bf16(W), bits)
+    codes, rn = qweights(r, torch_bf16(W), bits)
     torch.cuda.synchronize()
     _, bounds = oracle.lloydmax_table(d, bits)
     ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
@@ -317,7 +361,7 @@ def test_weights_lloydmax(bits):
 def test_weights_tiny_fp32():
     W = synth.tiny()["W"]
     r, Pi = _rpbh(256, 0)
-    codes, rn = rbq.quantize_weights(r, _dense(W, "f32"), 4)
+    codes, rn = qweights(r, _dense(W, "f32"), 4)
     _, bounds = oracle.lloydmax_table(256, 4)
     ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
     check_codes(_unpack(codes, 4, 256), ora["codes"], ora["v"], bounds, 256)
@@ -332,7 +376,7 @@ def test_weights_int8(shape):
     W = synth.to_bf16(W)
     W[1] = 0.0
     r, Pi = _rpbh(d, 2)
-    q, sc = rbq.quantize_weights(r, torch_bf16(W), 8, mode="int8")
+    q, sc = qweights(r, torch_bf16(W), 8, mode="int8")
     torch.cuda.synchronize()
     ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi)
     n_mis = check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
@@ -345,9 +389,9 @@ def test_weights_int8(shape):
 
 def _qlinear_case(X, W, d, bits_a, bits_w, seed=0, rows=None, dtype="bf16"):
     r, Pi = _rpbh(d, seed)
-    a_codes, s = rbq.rotate_quantize_act(r, _dense(X, dtype), bits_a)
-    w_codes, rn = rbq.quantize_weights(r, _dense(W, dtype), bits_w)
-    y = rbq.qlinear(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    a_codes, s = rq_act(r, _dense(X, dtype), bits_a)
+    w_codes, rn = qweights(r, _dense(W, dtype), bits_w)
+    y = qlin(a_codes, s, bits_a, w_codes, rn, bits_w, d)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
@@ -405,10 +449,10 @@ def _qlinear_i8_case(X, W, d, bits_a, bits_w, seed=0, rows=None):
     layer on the same codes: BF16 outputs bit-exact outside the rounding band
     (the integer sum is exact on both sides, only the fp32 scaling differs)."""
     r, _ = _rpbh(d, seed)
-    a_codes, s = rbq.rotate_quantize_act(r, _dense(X, "bf16"), bits_a)
-    w_codes, rn = rbq.quantize_weights(r, _dense(W, "bf16"), bits_w)
-    y = rbq.qlinear_int8_levels(a_codes, s, bits_a, w_codes, rn, bits_w, d)
-    y_fp16 = rbq.qlinear(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    a_codes, s = rq_act(r, _dense(X, "bf16"), bits_a)
+    w_codes, rn = qweights(r, _dense(W, "bf16"), bits_w)
+    y = qlin_i8(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    y_fp16 = qlin(a_codes, s, bits_a, w_codes, rn, bits_w, d)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
@@ -439,15 +483,26 @@ def test_qlinear_int8_levels_ragged_shapes_and_bit_widths(M, N, K, ba, bw):
 FP8_RTOL = 3e-3           # rel. Frobenius, fp32 sums of exact E4M3 products + BF16 output
 
 
+# Each E4M3 level e_j / beta is within 2^-4 (half of a 3-bit mantissa step)
+# of the exact level c_j, so every product e_w e_a / (beta_w beta_a) is within
+# FP8_PRODUCT_REL = (1 + 2^-4)^2 - 1 of c_w c_a, and by the triangle
+# inequality |y_fp8 - y_exact| <= FP8_PRODUCT_REL * s_m r'_n sum_k |c_w| |c_a|
+# element by element.  That bound is on the sum of absolute products, not on
+# |y_exact| itself: with cancellation in the sum the relative deviation can
+# exceed FP8_PRODUCT_REL, so the test checks the absolute form.
+FP8_PRODUCT_REL = (1 + 2.0 ** -4) ** 2 - 1
+
+
 def _qlinear_fp8_case(X, W, d, bits_a, bits_w, seed=0, rows=None):
     """qlinear_fp8_levels on the library's own codes vs the oracle's FP8 layer
     (exact fp64 sums) on the same codes; returns (error vs oracle, deviation
-    from the exact-level layer)."""
+    from the exact-level layer) and checks the deviation against the bound
+    above (plus the kernel's own error against its oracle)."""
     r, _ = _rpbh(d, seed)
-    a_codes, s = rbq.rotate_quantize_act(r, _dense(X, "bf16"), bits_a)
-    w_codes, rn = rbq.quantize_weights(r, _dense(W, "bf16"), bits_w)
-    y = rbq.qlinear_fp8_levels(a_codes, s, bits_a, w_codes, rn, bits_w, d)
-    y_fp16 = rbq.qlinear(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    a_codes, s = rq_act(r, _dense(X, "bf16"), bits_a)
+    w_codes, rn = qweights(r, _dense(W, "bf16"), bits_w)
+    y = qlin_fp8(a_codes, s, bits_a, w_codes, rn, bits_w, d)
+    y_fp16 = qlin(a_codes, s, bits_a, w_codes, rn, bits_w, d)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
@@ -456,9 +511,15 @@ def _qlinear_fp8_case(X, W, d, bits_a, bits_w, seed=0, rows=None):
     lw, _ = oracle.lloydmax_table(d, bits_w)
     pa = _unpack(a_codes[idx], bits_a, d)
     pw = _unpack(w_codes, bits_w, d)
-    ref = oracle.qlinear_fp8_levels(pa, s.cpu().numpy()[rows], la, pw, bf16_to_numpy(rn), lw)
+    s_np, rn_np = s.cpu().numpy()[rows], bf16_to_numpy(rn)
+    ref = oracle.qlinear_fp8_levels(pa, s_np, la, pw, rn_np, lw)
     got = bf16_to_numpy(y[idx])
-    return rel_frobenius(got, ref), rel_frobenius(got, bf16_to_numpy(y_fp16[idx]))
+    exact = oracle.qlinear(pa, s_np, la, pw, rn_np, lw)
+    abs_sum = oracle.qlinear(pa, s_np, np.abs(la), pw, rn_np, np.abs(lw))
+    err = rel_frobenius(got, ref)
+    bound = FP8_PRODUCT_REL * np.linalg.norm(abs_sum) + err * np.linalg.norm(ref)
+    assert np.linalg.norm(got - exact) <= bound * (1 + 1e-9), (np.linalg.norm(got - exact), bound)
+    return err, rel_frobenius(got, bf16_to_numpy(y_fp16[idx]))
 
 
 @pytest.mark.parametrize("M,N,K,ba,bw", [(1, 8, 128, 4, 4), (130, 136, 128, 4, 2), (257, 264, 384, 3, 3),
@@ -478,9 +539,7 @@ def test_qlinear_fp8_levels_attention_projection_sampled():
     rows = np.random.default_rng(7).choice(4608, 32, replace=False)
     err, dev = _qlinear_fp8_case(data["X"], data["W"], 3072, 4, 4, rows=rows)
     print(f"fp8-level qlinear attn_proj W4A4: {err:.2e} vs oracle, {dev:.2e} from exact levels")
-    # each E4M3 level is within 2^-4 of the exact one, so each product within
-    # (1 + 2^-4)^2 - 1 = 12.9 %: the layer cannot move further than that
-    assert err < FP8_RTOL and dev < (1 + 2.0 ** -4) ** 2 - 1, (err, dev)
+    assert err < FP8_RTOL, err
 
 
 def test_qlinear_int8_levels_attention_projection_sampled():
@@ -510,7 +569,7 @@ def test_large_activation_operand_tiles_walked_n_fastest(layer, M, N, K, ba, bw)
     s = torch.rand(M, device="cuda", generator=gen) + 0.5
     rn = (torch.rand(N, device="cuda", generator=gen) + 0.5).to(torch.bfloat16)
     fn = rbq.qlinear if layer == "fp16" else rbq.qlinear_int8_levels
-    y = fn(a, s, ba, w, rn, bw, K)
+    y = fn(a, s, ba, w, rn, bw, K, out=poison((M, N), torch.bfloat16))
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(M).choice(M, 40, replace=False)]))
@@ -528,11 +587,58 @@ def test_large_activation_operand_tiles_walked_n_fastest(layer, M, N, K, ba, bw)
         check_bf16_rounding(got, ref, "qlinear_int8_levels")
 
 
+@pytest.mark.parametrize("n_out,d_in", [(1536, 1536), (8960, 1536), (1536, 8960)])
+def test_qlinear_video_w4a6_full_size_sampled(n_out, d_in):
+    """The video-DiT workload (Wan 2.1 1.3B shape, OrbitQuant §3.2, W4A6):
+    32760 tokens = 21 frames x 1560 patches, hidden 1536, MLP 8960.  The two
+    1536-wide layers expand their 6-bit activation codes in a pass of their
+    own (the fp16 copy, 32760 x 1536 x 2 = 100 MB, fits the split route); the
+    8960-wide down-projection's copy would be 587 MB, so its GEMM expands the
+    6-bit codes itself (the shared-memory level table route).  Every token is
+    quantised on the GPU; sampled rows (first, last, others) are compared."""
+    T = 32760
+    X = synth.video_act(d_in, layer=7)
+    assert X.shape == (T, d_in)
+    W = synth.video_weight(n_out, d_in, layer=7)
+    rows = np.unique(np.concatenate([[0, T - 1], np.random.default_rng(d_in + n_out).choice(T, 30, replace=False)]))
+    err, _, _ = _qlinear_case(X, W, d_in, 6, 4, seed=1000 + 7, rows=rows)
+    print(f"qlinear video {T}x{n_out}x{d_in} W4A6 rel. Frobenius error {err:.2e}")
+    assert err < QLINEAR_RTOL, err
+
+
+@pytest.mark.parametrize("bits_a,bits_w", [(1, 4), (2, 3), (3, 4), (5, 2), (6, 4), (7, 8), (8, 1)])
+def test_qlinear_in_kernel_expansion_every_activation_width(bits_a, bits_w):
+    """Activation widths other than 4 bits take the in-kernel expansion route
+    (a shared-memory level table inside the GEMM) once their fp16 copy would
+    exceed 128 MiB: 70000 x 1024 x 2 bytes = 137 MiB here.  Random codes,
+    sampled rows (the first, the last and tiles in between) against the
+    oracle."""
+    M, N, K = 70000, 136, 1024
+    assert M * K * 2 > 128 << 20
+    gen = torch.Generator(device="cuda").manual_seed(bits_a * 16 + bits_w)
+    a = torch.randint(0, 256, (M, K * bits_a // 8), dtype=torch.uint8, device="cuda", generator=gen)
+    w = torch.randint(0, 256, (N, K * bits_w // 8), dtype=torch.uint8, device="cuda", generator=gen)
+    s = torch.rand(M, device="cuda", generator=gen) + 0.5
+    rn = (torch.rand(N, device="cuda", generator=gen) + 0.5).to(torch.bfloat16)
+    y = qlin(a, s, bits_a, w, rn, bits_w, K)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    rows = np.unique(np.concatenate([[0, 127, 128, M - 1], np.random.default_rng(M).choice(M, 40, replace=False)]))
+    idx = torch.as_tensor(rows).cuda()
+    la, _ = oracle.lloydmax_table(K, bits_a)
+    lw, _ = oracle.lloydmax_table(K, bits_w)
+    ref = oracle.qlinear(_unpack(a[idx], bits_a, K), s.cpu().numpy()[rows], la, _unpack(w, bits_w, K),
+                         bf16_to_numpy(rn), lw)
+    err = rel_frobenius(bf16_to_numpy(y[idx]), ref)
+    print(f"qlinear in-kernel expansion W{bits_w}A{bits_a}: rel. Frobenius error {err:.2e}")
+    assert err < QLINEAR_RTOL, err
+
+
 def _int8_case(X, W, d, seed=0, rows=None):
     r, Pi = _rpbh(d, seed)
-    xr = rbq.rotate_act(r, torch_bf16(X))
-    q, sc = rbq.quantize_weights(r, torch_bf16(W), 8, mode="int8")
-    y = rbq.qlinear_int8(xr, q, sc)
+    xr = rot_act(r, torch_bf16(X))
+    q, sc = qweights(r, torch_bf16(W), 8, mode="int8")
+    y = qlin_int8(xr, q, sc)
     torch.cuda.synchronize()
     assert rbq.device_error() == 0
     rows = np.arange(X.shape[0]) if rows is None else np.asarray(rows)
