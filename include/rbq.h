@@ -300,9 +300,9 @@ int rbq_int8_levels(int d, int bits, int8_t* levels, double* alpha);
  * stream-ordered memory pool on every call.  Callers that own all device
  * memory through their own allocator, forbid allocation on their inference
  * thread, or run inside a process whose allocator is not CUDA's cannot accept
- * that.  This entry point allocates nothing: its workspace, its two level
- * tables and a fallback error word live in one fixed __device__ array of
- * 32 MiB + 1280 bytes inside the library, which every GPU that loads the
+ * that.  This entry point allocates nothing: its workspace, 16 slots for
+ * level tables and a fallback error word live in one fixed __device__ array
+ * of 32 MiB + 8448 bytes inside the library, which every GPU that loads the
  * library holds until the process exits.
  *   Arguments as qlinear, plus
  *   err   device uint32 the kernels OR a non-zero value into when a bounded
@@ -311,14 +311,19 @@ int rbq_int8_levels(int d, int bits, int8_t* levels, double* alpha);
  * Limits: N*K <= 16,777,216 (else RBQ_ESCRATCH, nothing launched); K a
  * multiple of 128, N a multiple of 8, K*bits_a/8 a multiple of 16 (else
  * RBQ_EINVAL).
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Every call uses the same array and the array
- * keeps the last call's contents, so calls whose work overlaps on the GPU (on
- * different streams, or from several host threads) race and corrupt each
- * other's results; serialise them on one stream.  Nothing in the array needs
- * to start at zero: each call rewrites the tables and every workspace element
- * it reads.
+ * Set-up happens inside calls: the first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current),
+ * and the first call on a device for each (K, bits) pair copies that level
+ * table from host memory into a free slot of the array, ordered on the call's
+ * stream before its kernels (with all 16 slots taken, slots are reused in
+ * turn).  Make those first calls before any stream capture; later calls with
+ * widths already in a slot launch the two kernels and copy nothing.  Every
+ * call uses the same array and the array keeps the last call's contents, so
+ * calls whose work overlaps on the GPU (on different streams, or from several
+ * host threads) race and corrupt each other's results; serialise them on one
+ * stream.  Nothing in the array needs to start at zero: a slot is written
+ * before its first use and each call's expansion writes every workspace
+ * element its GEMM reads.
  * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ESCRATCH, RBQ_ECONVERGE, RBQ_ECUDA.
  */
 int qlinear_noalloc(const uint8_t* a_codes, const float* s, int bits_a,
@@ -398,9 +403,15 @@ int rbq_layer_write(const char* path, const rbq_layer_info* info, const void* co
 
 /* rbq_layer_read -- read a layer file's info and, when the buffer pointers are
  * not NULL, its payload into HOST buffers sized by rbq_layer_sizes(info).
+ *   codes_cap, aux_cap, zp_cap  the capacities in bytes of the three buffers
+ *   (zp_cap is ignored by modes without zero points).  Before anything is
+ *   read into them the sizes that this file's own header gives are checked
+ *   against them: a file replaced since the caller sized its buffers returns
+ *   RBQ_EINVAL with the buffers untouched.
  * The checksum is verified whenever the payload is read.
  * Errors: RBQ_EINVAL, RBQ_EIO (missing, short, corrupt or foreign file). */
-int rbq_layer_read(const char* path, rbq_layer_info* info, void* codes, void* aux, void* zero_point);
+int rbq_layer_read(const char* path, rbq_layer_info* info, void* codes, uint64_t codes_cap, void* aux,
+                   uint64_t aux_cap, void* zero_point, uint64_t zp_cap);
 
 /* Text for a return code (static storage). */
 const char* rbq_error_string(int code);

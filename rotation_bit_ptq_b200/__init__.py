@@ -16,6 +16,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librbq.so")
+LIB_DEBUG_PATH = os.path.join(_HERE, "librbq_debug.so")
 
 RBQ_F32, RBQ_BF16 = 0, 1
 RBQ_LLOYDMAX, RBQ_INT8_SYM, RBQ_INT8_TENSOR = 0, 1, 2
@@ -46,7 +47,7 @@ SIGNATURES = {
     "rpbh_describe": (_I, [_P, _P, _P, _P, _P]),
     "rbq_layer_sizes": (_I, [_P, _P, _P, _P]),
     "rbq_layer_write": (_I, [ctypes.c_char_p, _P, _P, _P, _P]),
-    "rbq_layer_read": (_I, [ctypes.c_char_p, _P, _P, _P, _P]),
+    "rbq_layer_read": (_I, [ctypes.c_char_p, _P, _P, _U64, _P, _U64, _P, _U64]),
     "lloydmax_table": (_I, [_I, _I, _P, _P]),
     "rotate_quantize_act": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "quantize_weights": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
@@ -91,6 +92,29 @@ def lib():
     return _lib
 
 
+_debug_lib = None
+
+
+def debug_lib():
+    """librbq_debug.so: the same kernels built with RBQ_DEBUG, whose
+    device-side bounds checks on computed indices record into the device error
+    word instead of trapping.  Loaded beside librbq.so with the same
+    signatures, for tests and debugging only; its handles, codebook cache and
+    error word are its own.  Raises if it has not been built."""
+    global _debug_lib
+    if _debug_lib is None:
+        if not os.path.exists(LIB_DEBUG_PATH):
+            raise RuntimeError(f"{LIB_DEBUG_PATH} is missing: build it with "
+                               "`python -m rotation_bit_ptq_b200.build --debug`")
+        handle = ctypes.CDLL(LIB_DEBUG_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _debug_lib = handle
+    return _debug_lib
+
+
 def _check(rc, where):
     if rc != RBQ_OK:
         raise RBQError(rc, where)
@@ -114,6 +138,43 @@ def _need_cuda(t, name, dtype=None):
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need_shape(t, shape, name):
+    """Caller-supplied buffers must have exactly the shape the kernel writes or
+    reads; a short one would be overrun on the device."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def check_layer_shapes(M, N, K, bits_a, bits_w, a_shape, s_shape, w_shape, rn_shape, out_shape=None):
+    """Shapes of a quantised linear layer's operands (pure Python, no device):
+    a_codes [M, K*bits_a/8], s [M], w_codes [N, K*bits_w/8], rnorm [N],
+    out [M, N].  Raises ValueError on any mismatch."""
+    if K <= 0 or (K * bits_a) % 8 or (K * bits_w) % 8:
+        raise ValueError("K times each bit width must be a whole number of bytes")
+    if tuple(a_shape) != (M, K * bits_a // 8) or tuple(w_shape) != (N, K * bits_w // 8):
+        raise ValueError("code row widths do not match K and the bit widths")
+    if tuple(s_shape) != (M,):
+        raise ValueError(f"s must have shape ({M},), got {tuple(s_shape)}")
+    if tuple(rn_shape) != (N,):
+        raise ValueError(f"rnorm must have shape ({N},), got {tuple(rn_shape)}")
+    if out_shape is not None and tuple(out_shape) != (M, N):
+        raise ValueError(f"out must have shape ({M}, {N}), got {tuple(out_shape)}")
+
+
+def check_same_device(*tensors):
+    """Every operand of one call on one device (the library launches on the
+    device that is current, which the binding sets to that one)."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"operands are on different devices: {sorted(str(d) for d in devs)}")
+    return next(iter(devs)) if devs else None
+
+
+def _device_ctx(*tensors):
+    import torch
+    return torch.cuda.device(check_same_device(*tensors))
 
 
 def _dtype_code(t):
@@ -210,8 +271,11 @@ def rotate_quantize_act(rpbh, X, bits, codes=None, norms=None, stream=None):
         norms = torch.empty((T,), dtype=torch.float32, device=X.device)
     _need_cuda(codes, "codes", torch.uint8)
     _need_cuda(norms, "norms", torch.float32)
-    _check(lib().rotate_quantize_act(rpbh.handle, _ptr(X), _dtype_code(X), T, int(bits), _ptr(codes),
-                                     _ptr(norms), _stream(stream)), "rotate_quantize_act")
+    _need_shape(codes, (T, d * bits // 8), "codes")
+    _need_shape(norms, (T,), "norms")
+    with _device_ctx(X, codes, norms):
+        _check(lib().rotate_quantize_act(rpbh.handle, _ptr(X), _dtype_code(X), T, int(bits), _ptr(codes),
+                                         _ptr(norms), _stream(stream)), "rotate_quantize_act")
     return codes, norms
 
 
@@ -225,10 +289,13 @@ def rotate_act(rpbh, X, out=None, norms=None, stream=None):
     if out is None:
         out = torch.empty((T, d), dtype=torch.bfloat16, device=X.device)
     _need_cuda(out, "out", torch.bfloat16)
+    _need_shape(out, (T, d), "out")
     if norms is not None:
         _need_cuda(norms, "norms", torch.float32)
-    _check(lib().rotate_quantize_act(rpbh.handle, _ptr(X), _dtype_code(X), T, RBQ_ROTATE_ONLY, _ptr(out),
-                                     _ptr(norms), _stream(stream)), "rotate_quantize_act")
+        _need_shape(norms, (T,), "norms")
+    with _device_ctx(X, out, norms):
+        _check(lib().rotate_quantize_act(rpbh.handle, _ptr(X), _dtype_code(X), T, RBQ_ROTATE_ONLY, _ptr(out),
+                                         _ptr(norms), _stream(stream)), "rotate_quantize_act")
     return out
 
 
@@ -249,6 +316,7 @@ def quantize_weights(rpbh, W, bits, mode="lloydmax", out=None, aux=None, stream=
             aux = torch.empty((N,), dtype=torch.bfloat16, device=W.device)
         _need_cuda(out, "codes", torch.uint8)
         _need_cuda(aux, "rnorm", torch.bfloat16)
+        _need_shape(out, (N, d * bits // 8), "codes")
     elif mode in ("int8", "int8_tensor"):
         code, bits = (RBQ_INT8_SYM if mode == "int8" else RBQ_INT8_TENSOR), 8
         if out is None:
@@ -257,10 +325,13 @@ def quantize_weights(rpbh, W, bits, mode="lloydmax", out=None, aux=None, stream=
             aux = torch.empty((N,), dtype=torch.float32, device=W.device)
         _need_cuda(out, "q", torch.int8)
         _need_cuda(aux, "scale", torch.float32)
+        _need_shape(out, (N, d), "q")
     else:
         raise ValueError("mode must be 'lloydmax', 'int8' or 'int8_tensor'")
-    _check(lib().quantize_weights(rpbh.handle, _ptr(W), _dtype_code(W), N, code, int(bits), _ptr(out),
-                                  _ptr(aux), _stream(stream)), "quantize_weights")
+    _need_shape(aux, (N,), "rnorm" if mode == "lloydmax" else "scale")
+    with _device_ctx(W, out, aux):
+        _check(lib().quantize_weights(rpbh.handle, _ptr(W), _dtype_code(W), N, code, int(bits), _ptr(out),
+                                      _ptr(aux), _stream(stream)), "quantize_weights")
     return out, aux
 
 
@@ -271,13 +342,14 @@ def qlinear(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, stream=None
                      (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16)):
         _need_cuda(t, n, dt)
     M, N = a_codes.shape[0], w_codes.shape[0]
-    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
-        raise ValueError("code row widths do not match K and the bit widths")
+    check_layer_shapes(M, N, int(K), int(bits_a), int(bits_w), a_codes.shape, s.shape, w_codes.shape,
+                       rnorm.shape, None if out is None else out.shape)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
     _need_cuda(out, "out", torch.bfloat16)
-    _check(lib().qlinear(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M, N,
-                         int(K), _ptr(out), _stream(stream)), "qlinear")
+    with _device_ctx(a_codes, s, w_codes, rnorm, out):
+        _check(lib().qlinear(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M, N,
+                             int(K), _ptr(out), _stream(stream)), "qlinear")
     return out
 
 
@@ -291,13 +363,14 @@ def qlinear_int8_levels(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None,
                      (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16)):
         _need_cuda(t, n, dt)
     M, N = a_codes.shape[0], w_codes.shape[0]
-    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
-        raise ValueError("code row widths do not match K and the bit widths")
+    check_layer_shapes(M, N, int(K), int(bits_a), int(bits_w), a_codes.shape, s.shape, w_codes.shape,
+                       rnorm.shape, None if out is None else out.shape)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
     _need_cuda(out, "out", torch.bfloat16)
-    _check(lib().qlinear_int8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w),
-                                     M, N, int(K), _ptr(out), _stream(stream)), "qlinear_int8_levels")
+    with _device_ctx(a_codes, s, w_codes, rnorm, out):
+        _check(lib().qlinear_int8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm),
+                                         int(bits_w), M, N, int(K), _ptr(out), _stream(stream)), "qlinear_int8_levels")
     return out
 
 
@@ -311,13 +384,14 @@ def qlinear_fp8_levels(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out=None, 
                      (w_codes, "w_codes", torch.uint8), (rnorm, "rnorm", torch.bfloat16)):
         _need_cuda(t, n, dt)
     M, N = a_codes.shape[0], w_codes.shape[0]
-    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
-        raise ValueError("code row widths do not match K and the bit widths")
+    check_layer_shapes(M, N, int(K), int(bits_a), int(bits_w), a_codes.shape, s.shape, w_codes.shape,
+                       rnorm.shape, None if out is None else out.shape)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
     _need_cuda(out, "out", torch.bfloat16)
-    _check(lib().qlinear_fp8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w),
-                                    M, N, int(K), _ptr(out), _stream(stream)), "qlinear_fp8_levels")
+    with _device_ctx(a_codes, s, w_codes, rnorm, out):
+        _check(lib().qlinear_fp8_levels(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm),
+                                        int(bits_w), M, N, int(K), _ptr(out), _stream(stream)), "qlinear_fp8_levels")
     return out
 
 
@@ -352,12 +426,13 @@ def qlinear_noalloc(a_codes, s, bits_a, w_codes, rnorm, bits_w, K, out, err=None
     if err is not None:
         _need_cuda(err, "err", torch.int32)
     M, N = a_codes.shape[0], w_codes.shape[0]
-    if a_codes.shape[1] * 8 != K * bits_a or w_codes.shape[1] * 8 != K * bits_w:
-        raise ValueError("code row widths do not match K and the bit widths")
-    if tuple(out.shape) != (M, N):
-        raise ValueError("out must be [M, N]")
-    _check(lib().qlinear_noalloc(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w), M,
-                                 N, int(K), _ptr(out), _ptr(err), _stream(stream)), "qlinear_noalloc")
+    check_layer_shapes(M, N, int(K), int(bits_a), int(bits_w), a_codes.shape, s.shape, w_codes.shape,
+                       rnorm.shape, out.shape)
+    if err is not None and err.numel() < 1:
+        raise ValueError("err must hold one int32")
+    with _device_ctx(a_codes, s, w_codes, rnorm, out, err):
+        _check(lib().qlinear_noalloc(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes), _ptr(rnorm), int(bits_w),
+                                     M, N, int(K), _ptr(out), _ptr(err), _stream(stream)), "qlinear_noalloc")
     return out
 
 
@@ -371,11 +446,14 @@ def qlinear_int8(xrot, q, scale, out=None, stream=None):
     N = q.shape[0]
     if q.shape[1] != K:
         raise ValueError("q and xrot disagree on K")
+    _need_shape(scale, (N,), "scale")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=xrot.device)
     _need_cuda(out, "out", torch.bfloat16)
-    _check(lib().qlinear_int8(_ptr(xrot), _ptr(q), _ptr(scale), M, N, K, _ptr(out), _stream(stream)),
-           "qlinear_int8")
+    _need_shape(out, (M, N), "out")
+    with _device_ctx(xrot, q, scale, out):
+        _check(lib().qlinear_int8(_ptr(xrot), _ptr(q), _ptr(scale), M, N, K, _ptr(out), _stream(stream)),
+               "qlinear_int8")
     return out
 
 
@@ -393,8 +471,12 @@ def quantize_weights_int8_asym(rpbh, W, q=None, scale=None, zero_point=None, str
     _need_cuda(q, "q", torch.uint8)
     _need_cuda(scale, "scale", torch.float32)
     _need_cuda(zero_point, "zero_point", torch.uint8)
-    _check(lib().quantize_weights_int8_asym(rpbh.handle, _ptr(W), _dtype_code(W), N, _ptr(q), _ptr(scale),
-                                            _ptr(zero_point), _stream(stream)), "quantize_weights_int8_asym")
+    _need_shape(q, (N, d), "q")
+    _need_shape(scale, (N,), "scale")
+    _need_shape(zero_point, (N,), "zero_point")
+    with _device_ctx(W, q, scale, zero_point):
+        _check(lib().quantize_weights_int8_asym(rpbh.handle, _ptr(W), _dtype_code(W), N, _ptr(q), _ptr(scale),
+                                                _ptr(zero_point), _stream(stream)), "quantize_weights_int8_asym")
     return q, scale, zero_point
 
 
@@ -407,11 +489,17 @@ def qlinear_int8_asym(xrot, q, scale, zero_point, out=None, stream=None):
     _need_cuda(zero_point, "zero_point", torch.uint8)
     M, K = xrot.shape
     N = q.shape[0]
+    if q.shape[1] != K:
+        raise ValueError("q and xrot disagree on K")
+    _need_shape(scale, (N,), "scale")
+    _need_shape(zero_point, (N,), "zero_point")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=xrot.device)
     _need_cuda(out, "out", torch.bfloat16)
-    _check(lib().qlinear_int8_asym(_ptr(xrot), _ptr(q), _ptr(scale), _ptr(zero_point), M, N, K, _ptr(out),
-                                   _stream(stream)), "qlinear_int8_asym")
+    _need_shape(out, (M, N), "out")
+    with _device_ctx(xrot, q, scale, zero_point, out):
+        _check(lib().qlinear_int8_asym(_ptr(xrot), _ptr(q), _ptr(scale), _ptr(zero_point), M, N, K, _ptr(out),
+                                       _stream(stream)), "qlinear_int8_asym")
     return out
 
 
@@ -449,15 +537,16 @@ def load_layer(path, device=None):
     info), codes, aux, zero_point) -- numpy arrays, or torch tensors on
     `device` when given."""
     info = LayerInfo()
-    _check(lib().rbq_layer_read(os.fsencode(path), ctypes.byref(info), None, None, None), "rbq_layer_read")
+    _check(lib().rbq_layer_read(os.fsencode(path), ctypes.byref(info), None, 0, None, 0, None, 0), "rbq_layer_read")
     nc, na, nz = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
     _check(lib().rbq_layer_sizes(ctypes.byref(info), ctypes.byref(nc), ctypes.byref(na), ctypes.byref(nz)),
            "rbq_layer_sizes")
     c = np.empty(nc.value, dtype=np.uint8)
     a = np.empty(na.value, dtype=np.uint8)
     z = np.empty(nz.value, dtype=np.uint8) if nz.value else None
-    _check(lib().rbq_layer_read(os.fsencode(path), ctypes.byref(info), c.ctypes.data_as(_P), a.ctypes.data_as(_P),
-                                z.ctypes.data_as(_P) if z is not None else None), "rbq_layer_read")
+    _check(lib().rbq_layer_read(os.fsencode(path), ctypes.byref(info), c.ctypes.data_as(_P), c.nbytes,
+                                a.ctypes.data_as(_P), a.nbytes, z.ctypes.data_as(_P) if z is not None else None,
+                                z.nbytes if z is not None else 0), "rbq_layer_read")
     kind = {v: k for k, v in _LAYER_KINDS.items()}[info.mode]
     rows, d = info.rows, info.d
     if kind == "lloydmax":

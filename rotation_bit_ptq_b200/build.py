@@ -19,6 +19,11 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "librbq.so")
+# The same sources compiled with RBQ_DEBUG: device-side bounds checks on the
+# indices the kernels compute (see dbg_index in csrc/rbq_sm100.cuh) record
+# into the device error word instead of trapping.  Tests load it beside the
+# release library; the product path never does.
+LIB_DEBUG = os.path.join(PKG, "librbq_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -44,15 +49,19 @@ def _stale(obj, src, newest_header):
     return os.path.getmtime(src) > t or newest_header > t
 
 
-def build(verbose=False, ptxas_info=False, jobs=None):
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose=False, ptxas_info=False, jobs=None, debug=False):
+    """Compile every CUDA source for sm_100a and link librbq.so (or, with
+    debug=True, librbq_debug.so with -DRBQ_DEBUG, objects under _build/debug)."""
+    bdir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = LIB_DEBUG if debug else LIB
+    os.makedirs(bdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0.0)
-    extra = ["-Xptxas", "-v"] if ptxas_info else []
+    extra = (["-Xptxas", "-v"] if ptxas_info else []) + (["-DRBQ_DEBUG"] if debug else [])
     cmds = []
     objs = []
     for src in srcs:
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
         objs.append(obj)
         if ptxas_info or _stale(obj, src, newest_header):
             cmds.append([nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj])
@@ -67,16 +76,15 @@ def build(verbose=False, ptxas_info=False, jobs=None):
                 sys.stderr.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)
             if r.returncode:
                 raise RuntimeError(f"nvcc failed on {cmd[-3]}")
-    if cmds or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        link = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcudart_static", "-lrt", "-lpthread", "-ldl"]
+    if cmds or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        link = [nvcc(), *ARCH, "-shared", "-o", lib, *objs, "-lcudart_static", "-lrt", "-lpthread", "-ldl"]
         r = subprocess.run(link, capture_output=True, text=True)
         if verbose or r.returncode:
             sys.stderr.write(" ".join(link) + "\n" + r.stdout + r.stderr)
         if r.returncode:
-            raise RuntimeError("link of librbq.so failed")
-    return LIB
+            raise RuntimeError(f"link of {os.path.basename(lib)} failed")
+    return lib
 
 
 if __name__ == "__main__":
-    build(verbose="-v" in sys.argv, ptxas_info="--ptxas" in sys.argv)
-    print(LIB)
+    print(build(verbose="-v" in sys.argv, ptxas_info="--ptxas" in sys.argv, debug="--debug" in sys.argv))

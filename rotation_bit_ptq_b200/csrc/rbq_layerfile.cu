@@ -124,7 +124,8 @@ extern "C" int rbq_layer_write(const char* path, const rbq_layer_info* info, con
   return RBQ_OK;
 }
 
-extern "C" int rbq_layer_read(const char* path, rbq_layer_info* info, void* codes, void* aux, void* zero_point) {
+extern "C" int rbq_layer_read(const char* path, rbq_layer_info* info, void* codes, uint64_t codes_cap, void* aux,
+                              uint64_t aux_cap, void* zero_point, uint64_t zp_cap) {
   if (!path || !info) return RBQ_EINVAL;
   File f(path, "rb");
   if (!f.f) return RBQ_EIO;
@@ -145,6 +146,10 @@ extern "C" int rbq_layer_read(const char* path, rbq_layer_info* info, void* code
   *info = I;
   if (!codes && !aux && !zero_point) return RBQ_OK;                   // info only
   if (!codes || !aux || (nz && !zero_point)) return RBQ_EINVAL;
+  // The payload sizes come from this file's header; a file replaced since the
+  // caller sized its buffers (or buffers sized from another description)
+  // must not be read past their ends.
+  if (nc > codes_cap || na > aux_cap || nz > zp_cap) return RBQ_EINVAL;
   if (std::fread(codes, 1, nc, f.f) != nc) return RBQ_EIO;
   if (std::fread(aux, 1, na, f.f) != na) return RBQ_EIO;
   if (nz && std::fread(zero_point, 1, nz, f.f) != nz) return RBQ_EIO;

@@ -8,7 +8,7 @@
 // runtime that forbids allocation on its inference thread, or a plug-in loaded
 // into a process whose allocator is not the CUDA one.  This variant runs the
 // same two kernels (weight expansion, then the tcgen05 GEMM) but puts the
-// workspace, the two level tables and a fallback error word in one file-scope
+// workspace, the level tables and a fallback error word in one file-scope
 // __device__ array of fixed size.  Nothing is allocated on any call.
 //
 // The array's name, seen from host code, is a host-side stand-in and not a
@@ -19,7 +19,6 @@
 #include <cuda_fp16.h>
 
 #include <cmath>
-#include <cstring>
 #include <mutex>
 
 #include "rbq_internal.h"
@@ -36,12 +35,13 @@ int expand_weights(const uint8_t* codes, int bits, int rows, int K, const uint16
 
 namespace {
 
-// Layout of the array: [fp16 weights, up to kWorkspaceBytes][lut_a 256 x u16]
-// [lut_w 256 x u16][error word].
+// Layout of the array: [fp16 weights, up to kWorkspaceBytes][kLutSlots level
+// tables of 256 x u16][error word].
 constexpr size_t kWorkspaceBytes = size_t(32) << 20;          // N * K <= 16,777,216
-constexpr size_t kLutAOffset = kWorkspaceBytes;
-constexpr size_t kLutWOffset = kLutAOffset + 512;
-constexpr size_t kErrOffset = kLutWOffset + 512;
+constexpr int kLutSlots = 16;
+constexpr size_t kLutBytes = 512;
+constexpr size_t kLutOffset = kWorkspaceBytes;
+constexpr size_t kErrOffset = kLutOffset + kLutSlots * kLutBytes;
 constexpr size_t kScratchBytes = kErrOffset + 256;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -64,8 +64,9 @@ int scratch_address(int dev, unsigned char** out) {
 }
 
 // Host copies of the fp16 level tables (levels x sqrt(d), the scaling the
-// GEMM's epilogue undoes with 1/d), kept in a fixed table so that repeated
-// calls do not solve the Lloyd-Max conditions again.
+// GEMM's epilogue undoes with 1/d), kept so that repeated calls do not solve
+// the Lloyd-Max conditions again.  Entries are never moved or overwritten
+// while the cache has room; when it is full the last entry is reused.
 struct HostLut {
   int d = 0, bits = 0;
   uint16_t lut[256] = {};
@@ -73,12 +74,10 @@ struct HostLut {
 constexpr int kLutCache = 64;
 HostLut g_luts[kLutCache];
 int g_nluts = 0;
-std::mutex g_lut_mu;
 
-int host_lut(int d, int bits, uint16_t* out) {
-  std::lock_guard<std::mutex> lk(g_lut_mu);
+int host_lut(int d, int bits, const uint16_t** out) {
   for (int i = 0; i < g_nluts; ++i)
-    if (g_luts[i].d == d && g_luts[i].bits == bits) { std::memcpy(out, g_luts[i].lut, 512); return RBQ_OK; }
+    if (g_luts[i].d == d && g_luts[i].bits == bits) { *out = g_luts[i].lut; return RBQ_OK; }
   double levels[256], bounds[255];
   const int rc = lloydmax_table(d, bits, levels, bounds);
   if (rc != RBQ_OK) return rc;
@@ -90,7 +89,50 @@ int host_lut(int d, int bits, uint16_t* out) {
     const __half v = __float2half_rn(j < (1 << bits) ? static_cast<float>(levels[j] * sd) : 0.f);
     h.lut[j] = *reinterpret_cast<const uint16_t*>(&v);
   }
-  std::memcpy(out, h.lut, 512);
+  *out = h.lut;
+  return RBQ_OK;
+}
+
+// Which (d, bits) level table each of a device's slots holds.  A table is
+// copied into a slot on the first call that needs it on that device (ordered
+// on that call's stream before its kernels); later calls find it there and
+// copy nothing.  When every slot is taken, slots are reused in turn (never
+// the one the same call just took for its other operand).
+struct SlotKey {
+  int d = 0, bits = 0;
+};
+SlotKey g_slot_key[kMaxDevices][kLutSlots];
+int g_slot_next[kMaxDevices] = {};
+std::mutex g_slot_mu;
+
+int level_table_slot(int dev, unsigned char* base, int d, int bits, int avoid, cudaStream_t st, int* slot_out) {
+  std::lock_guard<std::mutex> lk(g_slot_mu);
+  SlotKey* keys = g_slot_key[dev];
+  for (int i = 0; i < kLutSlots; ++i)
+    if (keys[i].d == d && keys[i].bits == bits) { *slot_out = i; return RBQ_OK; }
+  int slot = -1;
+  for (int i = 0; i < kLutSlots && slot < 0; ++i)
+    if (keys[i].d == 0 && i != avoid) slot = i;
+  if (slot < 0) {
+    slot = g_slot_next[dev];
+    if (slot == avoid) slot = (slot + 1) % kLutSlots;
+    g_slot_next[dev] = (slot + 1) % kLutSlots;
+  }
+  const uint16_t* lut = nullptr;
+  int rc = host_lut(d, bits, &lut);
+  if (rc != RBQ_OK) return rc;
+  // A copy from pageable host memory returns once the source has been staged,
+  // so the host table may change afterwards; the device copy is ordered on
+  // `st` before the kernels that read the slot.
+  const cudaError_t e = cudaMemcpyAsync(base + kLutOffset + static_cast<size_t>(slot) * kLutBytes, lut, kLutBytes,
+                                        cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) {
+    keys[slot] = SlotKey{};
+    return cuda_fail(e);
+  }
+  keys[slot].d = d;
+  keys[slot].bits = bits;
+  *slot_out = slot;
   return RBQ_OK;
 }
 
@@ -122,20 +164,17 @@ extern "C" int qlinear_noalloc(const uint8_t* a_codes, const float* s, int bits_
   unsigned char* base = nullptr;
   int rc = scratch_address(dev, &base);
   if (rc != RBQ_OK) return rc;
-  uint16_t lut_a[256], lut_w[256];
-  if ((rc = host_lut(K, bits_a, lut_a)) != RBQ_OK) return rc;
-  if ((rc = host_lut(K, bits_w, lut_w)) != RBQ_OK) return rc;
-
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int slot_a = 0, slot_w = 0;
+  if ((rc = level_table_slot(dev, base, K, bits_a, -1, st, &slot_a)) != RBQ_OK) return rc;
+  if ((rc = level_table_slot(dev, base, K, bits_w, slot_a, st, &slot_w)) != RBQ_OK) return rc;
+
   uint16_t* wf16 = reinterpret_cast<uint16_t*>(base);
-  uint16_t* dlut_a = reinterpret_cast<uint16_t*>(base + kLutAOffset);
-  uint16_t* dlut_w = reinterpret_cast<uint16_t*>(base + kLutWOffset);
+  uint16_t* dlut_a = reinterpret_cast<uint16_t*>(base + kLutOffset + static_cast<size_t>(slot_a) * kLutBytes);
+  uint16_t* dlut_w = reinterpret_cast<uint16_t*>(base + kLutOffset + static_cast<size_t>(slot_w) * kLutBytes);
   unsigned int* werr = err ? err : reinterpret_cast<unsigned int*>(base + kErrOffset);
-  // The tables are rewritten on every call (a copy from pageable memory has
-  // left the stack buffers once cudaMemcpyAsync returns); the workspace needs
-  // no clearing because the expansion writes every element the GEMM reads.
-  if ((e = cudaMemcpyAsync(dlut_a, lut_a, 512, cudaMemcpyHostToDevice, st)) != cudaSuccess) return cuda_fail(e);
-  if ((e = cudaMemcpyAsync(dlut_w, lut_w, 512, cudaMemcpyHostToDevice, st)) != cudaSuccess) return cuda_fail(e);
+  // The workspace needs no clearing: the expansion writes every element the
+  // GEMM reads.
 
   CodebookDevice ca{};
   ca.d = K;

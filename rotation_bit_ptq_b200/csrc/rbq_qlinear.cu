@@ -48,6 +48,7 @@ struct QParams {
 
 struct __align__(8) SmemTail {
   uint64_t bar[kStages];
+  uint64_t drain;                  // abort path only: completion of the MMAs issued
   uint32_t tmem_slot;
   uint32_t pad;
   uint16_t lut_a[256];
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(128, 1) qgemm_kernel(QParams p) {
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&tail->bar[s], 1);
+    mbar_init(&tail->drain, 1);
     mbar_fence_init();
   }
   if (warp == 0) {
@@ -223,8 +225,9 @@ __global__ void __launch_bounds__(128, 1) qgemm_kernel(QParams p) {
         }
       }
     }
-  } else if (tid == 0) {
-    atomicOr(p.err, 1u);
+  } else {
+    if (tid == 0) atomicOr(p.err, 1u);
+    drain_after_abort(tid == 0, &tail->drain);    // `ok` is the same in every thread
   }
   tc_fence_before();
   __syncthreads();

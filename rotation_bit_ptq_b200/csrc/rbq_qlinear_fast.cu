@@ -105,6 +105,7 @@ struct __align__(8) Tail {
   uint64_t cempty[kMaxC];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t drain;                // abort path only: completion of the MMAs issued
   uint32_t tmem_slot;
   volatile uint32_t abort;
   uint16_t lut_a[256];
@@ -286,6 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tl->acc_full[a], 1);
       mbar_init(&tl->acc_empty[a], 128);
     }
+    mbar_init(&tl->drain, 1);
     tl->abort = 0u;
     mbar_fence_init();
   }
@@ -464,6 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (tl->abort) {                 // the same value in every thread after the barrier
+    drain_after_abort(warp == kMmaWarp && lane == 0, &tl->drain);
+    __syncthreads();
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

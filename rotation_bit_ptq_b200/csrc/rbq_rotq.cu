@@ -17,9 +17,12 @@
 #include <cuda_bf16.h>
 
 #include "rbq_internal.h"
+#include "rbq_sm100.cuh"
 
 namespace rbq {
 namespace {
+
+using sm100::dbg_index;
 
 enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3, kInt8Asym = 4 };
 
@@ -37,6 +40,7 @@ struct RotqParams {
   void* aux;             // float norms | bf16 row norms | float scales | float norms (optional)
   const float* fixed_scale;   // INT8: one scale for every row (not written back), else null
   uint8_t* zero_point;        // asymmetric INT8: uint8 zero point per row
+  unsigned int* err;          // device error word (debug builds' bounds checks)
 };
 
 template <typename Tin> __device__ __forceinline__ float to_f32(Tin v);
@@ -105,7 +109,7 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
 #pragma unroll
     for (int i = 0; i < 64; ++i) {
       const int k = 64 * b + i;
-      y[i] = p.sign[k] * rows[g * d + p.perm[k]];
+      y[i] = p.sign[k] * rows[g * d + dbg_index(static_cast<uint32_t>(p.perm[k]), static_cast<uint32_t>(d), p.err)];
     }
     fwht64(y);
     float acc = (MODE == kInt8Asym) ? -INFINITY : 0.f, acc2 = INFINITY;
@@ -261,6 +265,7 @@ struct Params {
   void* out;
   void* aux;
   const float* fixed_scale;  // INT8: one scale for every row (not written back), else null
+  unsigned int* err;         // device error word (debug builds' bounds checks)
 };
 
 __device__ __forceinline__ unsigned long long pk(float a, float b) {
@@ -428,7 +433,10 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
       const uint32_t base = stage_addr[st] + static_cast<uint32_t>(g * L::row_pitch(d));
 #pragma unroll
       for (int i4 = 0; i4 < 16; ++i4) {
-        const uint4 o = lds128(off_addr + 4 * (64 * b + 4 * (i4 ^ (b & 15))));
+        uint4 o = lds128(off_addr + 4 * (64 * b + 4 * (i4 ^ (b & 15))));
+        const uint32_t rb = 2u * static_cast<uint32_t>(d);
+        o = make_uint4(dbg_index(o.x, rb, p.err), dbg_index(o.y, rb, p.err), dbg_index(o.z, rb, p.err),
+                       dbg_index(o.w, rb, p.err));
         P[2 * i4] = pk(__uint_as_float(lds_u16(base + o.x) << 16), __uint_as_float(lds_u16(base + o.y) << 16));
         P[2 * i4 + 1] = pk(__uint_as_float(lds_u16(base + o.z) << 16), __uint_as_float(lds_u16(base + o.w) << 16));
       }
@@ -504,7 +512,6 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         const float kq = inv * (0.5f * p.grid_cells);
         const float cq = 0.5f * p.grid_cells + 8388608.0f;   // + 2^23: round(.) lands in the low bits
         const unsigned long long kq2 = pk(kq, kq), cq2 = pk(cq, cq), inv2 = pk(inv, inv);
-        const uint32_t gbase = grid_addr - 0x4B000000u * 8u;
         uint32_t w[2 * BITS];
 #pragma unroll
         for (int i = 0; i < 2 * BITS; ++i) w[i] = 0u;
@@ -516,7 +523,8 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int r = 2 * j + e;
-            const float2 ent = lds_f2(gbase + __float_as_uint(e ? q1 : q0) * 8u);
+            const float2 ent = lds_f2(grid_addr + 8u * dbg_index(__float_as_uint(e ? q1 : q0) - 0x4B000000u,
+                                                                 static_cast<uint32_t>(p.grid_n), p.err));
             const uint32_t code = static_cast<uint32_t>(__float_as_int(ent.y)) - set_ge(e ? v1 : v0, ent.x);
             const int bit = r * BITS, wi = bit >> 5, sh = bit & 31;
             if constexpr ((32 % BITS) == 0) {
@@ -547,7 +555,6 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         const float nrm = sqrtf(tot);
         const float inv = 1.0f / (nrm + 8e-12f);
         const float A = inv * p.grid_scale;
-        const uint32_t gbase = grid_addr - 0x4B000000u * 8u;
         uint32_t w[2 * BITS];
 #pragma unroll
         for (int i = 0; i < 2 * BITS; ++i) w[i] = 0u;
@@ -558,7 +565,8 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
           const float z = (r & 1) ? hi : lo;
           const float u = fma_sat(z, A, 0.5f);
           const float qf = fmaf(u, p.grid_cells, 8388608.0f);   // 2^23: round(u*NC) in the low bits
-          const float2 e = lds_f2(gbase + __float_as_uint(qf) * 8u);
+          const float2 e = lds_f2(grid_addr + 8u * dbg_index(__float_as_uint(qf) - 0x4B000000u,
+                                                             static_cast<uint32_t>(p.grid_n), p.err));
           // code = base + (v >= thr): the sign of z*inv - thr, as 0 / -1
           const int below = __float_as_int(fmaf(z, inv, -e.x)) >> 31;
           const uint32_t code = static_cast<uint32_t>(__float_as_int(e.y) + 1 + below);
@@ -747,6 +755,7 @@ int run_fast(const rbq_rpbh* r, int mode, int bits, long long rows, const void* 
   p.out = out;
   p.aux = aux;
   p.fixed_scale = fixed_scale;
+  if ((rc = device_error_word_ptr(&p.err)) != RBQ_OK) return rc;
   if (mode == kAct || mode == kWeightLM) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
@@ -795,6 +804,7 @@ int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X
   p->aux = aux;
   p->fixed_scale = fixed_scale;
   p->zero_point = nullptr;
+  if ((rc = device_error_word_ptr(&p->err)) != RBQ_OK) return rc;
   if (mode == kAct || mode == kWeightLM) {
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;

@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
         const uint32_t ss[4] = {sg.x, sg.y, sg.z, sg.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t a = rowA + oo[e];
+          const uint32_t a = rowA + dbg_index(oo[e], 2u * static_cast<uint32_t>(p.d), p.err);
           const float y0 = bf16_signed(lds_u16(a), ss[e]);
           const float y1 = bf16_signed(lds_u16(a + pitch8), ss[e]);
           R[4 * q4 + e] = pk(y0, y1);
@@ -312,7 +312,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       uint32_t w0[2 * BITS], w1[2 * BITS];
 #pragma unroll
       for (int i = 0; i < 2 * BITS; ++i) w0[i] = w1[i] = 0u;
-      const Enc enc(inv0, inv1, p.grid_cells, p.grid_scale, gbase);
+      Enc enc(inv0, inv1, p.grid_cells, p.grid_scale, gbase);
+#ifdef RBQ_DEBUG
+      enc.dbg_err = p.err;
+      enc.dbg_entries = static_cast<uint32_t>(guarded_grid_entries(p.grid_n));
+#endif
       // warp-uniform choice: encode_block reads tensor memory collectively
       if (__any_sync(0xffffffffu, bad0 || bad1)) {
         encode_block<BITS, true>(enc, tA, tB, bad0, bad1, w0, w1);

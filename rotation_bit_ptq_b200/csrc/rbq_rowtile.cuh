@@ -155,15 +155,30 @@ __device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
 struct Enc {
   float A0, A1, inv0, inv1, cells;
   uint32_t gbase;
+#ifdef RBQ_DEBUG
+  unsigned int* dbg_err = nullptr;     // debug builds: check every grid entry index
+  uint32_t dbg_entries = 0;
+#endif
   __device__ __forceinline__ Enc(float i0, float i1, float nc, float scale, uint32_t gb)
       : A0(i0 * scale), A1(i1 * scale), inv0(i0), inv1(i1), cells(nc), gbase(gb) {}
+  // Shared-memory address of the entry for the rounded grid coordinate qf
+  // (2^23 + n in the float's low bits; gbase already holds -2^23 entries and
+  // the guard entries before entry 0).
+  __device__ __forceinline__ uint32_t entry_addr(float qf) const {
+#ifdef RBQ_DEBUG
+    const uint32_t e = __float_as_uint(qf) - 0x4B000000u + static_cast<uint32_t>(kGridGuard);
+    return gbase + (0x4B000000u - static_cast<uint32_t>(kGridGuard)) * 8u + 8u * dbg_index(e, dbg_entries, dbg_err);
+#else
+    return gbase + __float_as_uint(qf) * 8u;
+#endif
+  }
   __device__ __forceinline__ void codes(unsigned long long z, uint32_t& c0, uint32_t& c1) const {
     float z0, z1;
     upk(z, z0, z1);
     const float qf0 = fmaf(fma_sat(z0, A0, 0.5f), cells, 8388608.0f);
     const float qf1 = fmaf(fma_sat(z1, A1, 0.5f), cells, 8388608.0f);
-    const float2 e0 = lds_f2(gbase + __float_as_uint(qf0) * 8u);
-    const float2 e1 = lds_f2(gbase + __float_as_uint(qf1) * 8u);
+    const float2 e0 = lds_f2(entry_addr(qf0));
+    const float2 e1 = lds_f2(entry_addr(qf1));
     const int below0 = __float_as_int(fmaf(z0, inv0, -e0.x)) >> 31;
     const int below1 = __float_as_int(fmaf(z1, inv1, -e1.x)) >> 31;
     c0 = static_cast<uint32_t>(__float_as_int(e0.y) + 1 + below0);

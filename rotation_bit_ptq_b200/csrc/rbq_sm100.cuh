@@ -12,6 +12,28 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- debug builds ------------------------------------------------------------
+// librbq_debug.so is compiled with RBQ_DEBUG: an index the kernels compute on
+// the device (a gather offset from a table, a code-grid entry from a float) is
+// checked against its bound before the access it feeds.  An index out of range
+// ORs kDebugBoundsBit into the library's device error word (rbq_device_error
+// then returns RBQ_EDEVICE) and is replaced by 0, so the access stays inside
+// its buffer.  Release builds return the index unchanged and compile the check
+// away.
+constexpr unsigned int kDebugBoundsBit = 1u << 20;
+__device__ __forceinline__ uint32_t dbg_index(uint32_t i, uint32_t bound, unsigned int* err) {
+#ifdef RBQ_DEBUG
+  if (i >= bound) {
+    atomicOr(err, kDebugBoundsBit);
+    return 0u;
+  }
+#else
+  (void)bound;
+  (void)err;
+#endif
+  return i;
+}
+
 // ---- mbarrier -------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -149,6 +171,23 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// Abort path of a CTA whose bounded wait gave up: work it already handed to
+// the asynchronous units may still be running -- MMAs writing tensor memory,
+// bulk copies writing shared memory.  The thread that issued the MMAs commits
+// them to `drain` (an mbarrier initialised with one arrival and used for
+// nothing else) and waits for it, bounded; every calling thread then spins for
+// about 40K SM cycles (~20 us) so that bulk copies still in flight land before
+// the CTA frees its tensor memory and exits.  Only the abort path calls it.
+__device__ __forceinline__ void drain_after_abort(bool mma_issuer, uint64_t* drain) {
+  if (mma_issuer) {
+    umma_commit(drain);
+    mbar_wait(drain, 0);
+  }
+  const long long t0 = clock64();
+  while (clock64() - t0 < 40000) {
+  }
 }
 
 // Instruction descriptor of kind::f16: fp32 accumulator, K-major A and B.

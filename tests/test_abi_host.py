@@ -234,3 +234,27 @@ def _check_grid_variant(d, bits, variant):
     nz = (np.clip(z * scale + np.float32(0.5), 0, 1) * np.float32(cells) + np.float32(2.0 ** 23)).astype(np.float32)
     nn = nz.view(np.int32) - 0x4B000000
     assert np.all(base[nn] + (z >= thr[nn]) == 2 ** (bits - 1))
+
+
+def test_binding_rejects_mismatched_layer_shapes():
+    """The binding checks every operand's length before a call reaches the
+    library: a short s or rnorm would be read past its end by the GEMM's
+    epilogue, and a wrong out shape written past its end."""
+    M, N, K, ba, bw = 100, 64, 256, 4, 3
+    good = dict(a_shape=(M, K * ba // 8), s_shape=(M,), w_shape=(N, K * bw // 8), rn_shape=(N,), out_shape=(M, N))
+    rbq.check_layer_shapes(M, N, K, ba, bw, **good)
+    for key, bad in (("s_shape", (M - 1,)), ("rn_shape", (N + 8,)), ("out_shape", (M, N - 8)),
+                     ("a_shape", (M, K * ba // 8 - 16)), ("w_shape", (N, K * 4 // 8)), ("s_shape", (M, 1))):
+        with pytest.raises(ValueError):
+            rbq.check_layer_shapes(M, N, K, ba, bw, **{**good, key: bad})
+    with pytest.raises(ValueError):
+        rbq.check_layer_shapes(M, N, 100, 3, bw, **good)            # 100 * 3 bits is not whole bytes
+
+
+def test_binding_rejects_operands_on_different_devices():
+    torch = pytest.importorskip("torch")
+    a = torch.zeros(4)
+    b = torch.zeros(4, device="meta")
+    with pytest.raises(ValueError):
+        rbq.check_same_device(a, b)
+    assert rbq.check_same_device(a, None, torch.ones(2)) == torch.device("cpu")

@@ -61,7 +61,7 @@ def test_corrupt_short_and_foreign_files(tmp_path):
 
     def read(p):
         return lib.rbq_layer_read(str(p).encode(), ctypes.byref(info), buf_c.ctypes.data_as(ctypes.c_void_p),
-                                  buf_a.ctypes.data_as(ctypes.c_void_p), None)
+                                  buf_c.nbytes, buf_a.ctypes.data_as(ctypes.c_void_p), buf_a.nbytes, None, 0)
 
     assert read(path) == rbq.RBQ_OK
     bad = bytearray(raw)
@@ -76,6 +76,35 @@ def test_corrupt_short_and_foreign_files(tmp_path):
     assert read(tmp_path / "e.rbq") == rbq.RBQ_EIO
     assert read(tmp_path / "missing.rbq") == rbq.RBQ_EIO
     assert b"layer file" in lib.rbq_error_string(rbq.RBQ_EIO)
+
+
+def test_read_rejects_a_file_larger_than_the_buffers(tmp_path):
+    """A caller sizes its buffers from an info-only read; if the file is then
+    replaced by one whose header asks for more bytes, the data read must refuse
+    (RBQ_EINVAL) and leave the buffers untouched instead of overrunning them."""
+    lib = rbq.lib()
+    path = tmp_path / "layer.rbq"
+    small, big = _arrays("int8", 8, 512), _arrays("int8", 16, 512, seed=1)
+    rbq.save_layer(path, rbq.RPBH(512, 3), "int8", small[0], small[1])
+    info = rbq.LayerInfo()
+    assert lib.rbq_layer_read(str(path).encode(), ctypes.byref(info), None, 0, None, 0, None, 0) == rbq.RBQ_OK
+    nc, na = ctypes.c_uint64(), ctypes.c_uint64()
+    assert lib.rbq_layer_sizes(ctypes.byref(info), ctypes.byref(nc), ctypes.byref(na), None) == rbq.RBQ_OK
+    buf_c = np.full(nc.value + 64, 0x5A, np.uint8)       # guard bytes past the sized part
+    buf_a = np.full(na.value + 64, 0x5A, np.uint8)
+    rbq.save_layer(path, rbq.RPBH(512, 3), "int8", big[0], big[1])          # swapped in between
+    rc = lib.rbq_layer_read(str(path).encode(), ctypes.byref(info), buf_c.ctypes.data_as(ctypes.c_void_p), nc.value,
+                            buf_a.ctypes.data_as(ctypes.c_void_p), na.value, None, 0)
+    assert rc == rbq.RBQ_EINVAL
+    assert np.all(buf_c == 0x5A) and np.all(buf_a == 0x5A)
+    # sized for the new file, the same call reads it
+    info2 = rbq.LayerInfo()
+    lib.rbq_layer_read(str(path).encode(), ctypes.byref(info2), None, 0, None, 0, None, 0)
+    lib.rbq_layer_sizes(ctypes.byref(info2), ctypes.byref(nc), ctypes.byref(na), None)
+    bc, ba = np.empty(nc.value, np.uint8), np.empty(na.value, np.uint8)
+    assert lib.rbq_layer_read(str(path).encode(), ctypes.byref(info2), bc.ctypes.data_as(ctypes.c_void_p), bc.nbytes,
+                              ba.ctypes.data_as(ctypes.c_void_p), ba.nbytes, None, 0) == rbq.RBQ_OK
+    assert np.array_equal(bc, big[0].view(np.uint8).reshape(-1))
 
 
 def test_layer_sizes_and_invalid_descriptions():
