@@ -47,6 +47,13 @@ METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
 
 
+def qlinear_algorithmic_bytes(M=T, N=D, K=D, bits_a=BITS_A, bits_w=BITS_W):
+    """Operand and result bytes of one qlinear call: activation codes, weight
+    codes, s (fp32), r' (BF16) and Y (BF16).  The fp16 weight workspace the
+    call writes and reads back (N*K*2 each way) is extra, reported beside it."""
+    return M * K * bits_a // 8 + N * K * bits_w // 8 + 4 * M + 2 * N + 2 * M * N
+
+
 def act_bytes_per_token(d=D, bits=BITS_A):
     return 2 * d + d * bits // 8 + 4
 
@@ -282,11 +289,24 @@ def run_ours(args, rank, world):
     tflops = flops * args.steps * world / (k2_ms * 1e-3) / 1e12
     wgbs = weight_bytes_per_row() * D * args.steps * world / (k1w_ms * 1e-3) / 1e9
 
-    # end to end through the public API with host buffers (every rank, its own shard)
-    e2e_ms, h2d, d2h = run_e2e(r, X_host, dev, stream, args)
-    (e2e_ms,), e2e_tokens = reduce_job([e2e_ms], T * args.steps, device=dev)
+    # end to end through the public API with host buffers (every rank, its own
+    # shard): the whole layer -- host X -> rotate_quantize_act -> qlinear (on
+    # the resident weight codes, quantised offline) -> host Y -- and, as a
+    # sub-key, the activation quantiser alone (host X -> codes and norms)
+    e2e_ms, h2d, d2h = run_e2e_layer(r, X_host, w_codes[0], rnorm[0], dev, stream, args)
+    act_ms, act_h2d, act_d2h = run_e2e(r, X_host, dev, stream, args)
+    (e2e_ms, act_ms), e2e_tokens = reduce_job([e2e_ms, act_ms], T * args.steps, device=dev)
     e2e = {"value": round(act_bytes_per_token() * e2e_tokens / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "what": "whole layer through the C ABI: host X (pinned) -> rotate_quantize_act -> qlinear -> host Y "
+                   "(BF16), every step's copies inside the timed region; value = activation bytes (2d + d*b/8 + 4 "
+                   "per token) per second, the headline metric's unit",
+           "tokens_per_s": round(e2e_tokens / (e2e_ms * 1e-3), 1),
+           "layer_TFLOP/s": round(2.0 * D * D * e2e_tokens / (e2e_ms * 1e-3) / 1e12, 2),
+           "rotate_quantize_only": {
+               "value": round(act_bytes_per_token() * e2e_tokens / (act_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": act_h2d, "d2h_bytes_per_step": act_d2h,
+               "what": "host X -> rotate_quantize_act -> host codes and norms"}}
 
     res = {
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
@@ -295,6 +315,9 @@ def run_ours(args, rank, world):
         "data": "synthetic (seeded; BF16 Student-t(3) activations with 1% outlier channels x30, N(0,0.02^2) weights)",
         "config": {"workload": WORKLOAD, "tokens_per_gpu": T, "d_in": D, "d_out": D, "bits_a": BITS_A,
                    "bits_w": BITS_W, "parallelism": f"replicas x{world} (tokens sharded, no collective)",
+                   "arithmetic": "rotate_quantize: BF16 in, fp32 transform and code search; qlinear: operand "
+                                 "tiles are fp16 levels x sqrt(d) expanded from the codes, fp32 accumulation, "
+                                 "BF16 out",
                    "l2": f"{nsets} rotating input sets ({nsets * per_set / 2**20:.0f} MiB > L2 {l2 / 2**20:.0f} MiB)"},
         "rotate_quantize": {"GB/s": round(gbs, 2), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
                             "avg_us": round(k1_avg_s * 1e6, 3)},
@@ -306,7 +329,10 @@ def run_ours(args, rank, world):
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": QLINEAR_DRAM_BYTES,
                      "peak_source": pk["source"] + " bf16 burst",
-                     "note": "achieved includes the per-call weight-code expansion launch"},
+                     "note": "achieved includes the per-call weight-code expansion launch; traffic is the ncu "
+                             "DRAM read + write of both launches (expansion + GEMM) of one call",
+                     "algorithmic_bytes": qlinear_algorithmic_bytes(),
+                     "workspace_round_trip_bytes": 2 * 2 * D * D},
         "roofline_rotate_quantize": {"kernel": "rotate_quantize_act", "bound": "hbm",
                                      "achieved": round(act_bytes / k1_avg_s / 1e9, 2), "peak": pk["hbm_gbs"],
                                      "unit": "GB/s", "frac": round(act_bytes / k1_avg_s / 1e9 / pk["hbm_gbs"], 4),
@@ -375,6 +401,61 @@ def run_e2e(r, X_host, dev, stream, args):
     b.record(stream)
     torch.cuda.synchronize()
     return a.elapsed_time(b), int(xh.numel() * 2), int(ch[0].numel() + nh[0].numel() * 4)
+
+
+def run_e2e_layer(r, X_host, w_codes, rnorm, dev, stream, args):
+    """The whole quantised layer through the public API from pinned host
+    memory: every step copies its input X host -> device, quantises it
+    (rotate_quantize_act), runs qlinear against the resident weight codes and
+    copies Y (BF16) back.  Two buffer sets and separate copy streams overlap
+    step i+1's upload and step i's download with the kernels; every step's
+    copies stay inside the timed region.  Returns (ms for args.steps steps,
+    H2D bytes per step, D2H bytes per step)."""
+    import torch
+    import rotation_bit_ptq_b200 as rbq
+    xh = torch.from_numpy(synth.bf16_bits(X_host).view(np.int16)).view(torch.bfloat16).pin_memory()
+    xd = [torch.empty_like(xh, device=dev) for _ in range(2)]
+    cd = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev) for _ in range(2)]
+    nd = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(2)]
+    yd = [torch.empty((T, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    yh = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    for e in downloaded:
+        e.record(s_out)
+
+    def one(i):
+        k = i % 2
+        s_in.wait_event(downloaded[k])              # the slot's previous Y is out
+        with torch.cuda.stream(s_in):
+            xd[k].copy_(xh, non_blocking=True)
+        uploaded[k].record(s_in)
+        stream.wait_event(uploaded[k])
+        rbq.rotate_quantize_act(r, xd[k], BITS_A, cd[k], nd[k], stream=stream)
+        rbq.qlinear(cd[k], nd[k], BITS_A, w_codes, rnorm, BITS_W, D, yd[k], stream=stream)
+        computed[k].record(stream)
+        s_out.wait_event(computed[k])
+        with torch.cuda.stream(s_out):
+            yh[k].copy_(yd[k], non_blocking=True)
+        downloaded[k].record(s_out)
+
+    for i in range(max(3, args.warmup)):
+        one(i)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    s_in.wait_event(a)
+    s_out.wait_event(a)
+    for i in range(args.steps):
+        one(i)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b), int(xh.numel() * 2), int(yh[0].numel() * 2)
 
 
 # ---------------------------------------------------------------------------
@@ -483,8 +564,15 @@ def run_suite(dev, stream, pk):
     rows = sum(o for _, o, _ in synth.INT8_DIT_SHAPES)
     block_quant_us = 0.0
     for name, n_out, d_in in synth.INT8_DIT_SHAPES:
-        if name in ("k", "v", "o"):          # same shape as q
-            block_quant_us += int8["q 4096->4096"]["quantize_weights_int8"]["us"]
+        if name in ("k", "v", "o"):          # same shape as q: the weight pass is timed, the layer is not repeated
+            W = to_bf16_tensor(synth.int8_dit_weight(0, name), dev)
+            r = rbq.RPBH(d_in, 100 + d_in)
+            q, sc = rbq.quantize_weights(r, W, 8, mode="int8")
+            us = _time_us(lambda: rbq.quantize_weights(r, W, 8, "int8", q, sc, stream=stream), stream)
+            block_quant_us += us
+            int8[f"{name} {d_in}->{n_out}"] = {"quantize_weights_int8": {"us": round(us, 2)}}
+            r.close()
+            del W, q, sc
             continue
         W = to_bf16_tensor(synth.int8_dit_weight(0, name), dev)
         X = to_bf16_tensor(synth.int8_dit_act(d_in), dev)
@@ -540,7 +628,9 @@ def run_suite(dev, stream, pk):
         "bf16_bytes": 2 * 32 * params, "int8_bytes": 32 * params + 4 * 32 * rows,
         "ratio": round((32 * params + 4 * 32 * rows) / (2 * 32 * params), 4),
         "pages_ratio": round(6.76 / 13.25, 4),
-        "quantize_weights_int8_ms_all_blocks": round(32 * block_quant_us * 1e-3, 3),
+        "quantize_weights_int8_ms_one_block": round(block_quant_us * 1e-3, 3),
+        "quantize_weights_int8_ms_all_blocks_derived": round(32 * block_quant_us * 1e-3, 3),
+        "derived": "all 32 blocks = 32 x the measured block (every block has the same six shapes)",
     }
     out["int8_dit"] = int8
 
