@@ -38,10 +38,13 @@ D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
 
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel as
 # it stands (profiles/qlinear_W4A4_4608x3072x3072.md,
-# profiles/rotate_quantize_act_d3072_T32768_A4.md).  The rotate-quantize
-# capture ran 32768 tokens; its bytes are scaled to this workload's 4608 by
-# the token count (its traffic grows in proportion to the tokens).
-QLINEAR_DRAM_BYTES = 26_068_224 + 79_872
+# profiles/rotate_quantize_act_d3072_T32768_A4.md).  qlinear: both launches of
+# one call (weight-code expansion + GEMM), caches flushed before each kernel,
+# so the GEMM reads the fp16 workspace back from DRAM and the 28 MB output is
+# still in L2 when it ends (its writes are not in the figure).  The
+# rotate-quantize capture ran 32768 tokens; its bytes are scaled to this
+# workload's 4608 by the token count (its traffic grows with the tokens).
+QLINEAR_DRAM_BYTES = (4_724_992 + 0) + (26_067_200 + 7_936)
 ROTQ_DRAM_BYTES = round((201_677_312 + 29_322_240) * 4608 / 32768)
 METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"

@@ -342,11 +342,10 @@ int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out) {
   auto* D = const_cast<RpbhDevice*>(rd);
   if (!D->pair_tab) {
     const int d = r->d;
-    std::vector<uint32_t> tab(2 * static_cast<size_t>(d));
+    std::vector<uint32_t> tab(static_cast<size_t>(d));
     for (int k = 0; k < d; ++k) {
       const uint32_t slot = pair_tab_slot(k / kH, k % kH);
-      tab[slot] = 2u * static_cast<uint32_t>(r->perm[k]);
-      tab[d + slot] = r->sign[k] < 0 ? 0x80000000u : 0u;
+      tab[slot] = 2u * static_cast<uint32_t>(r->perm[k]) | (r->sign[k] < 0 ? 0x80000000u : 0u);
     }
     uint32_t* dev = nullptr;
     if ((rc = upload(tab.data(), tab.size(), &dev)) != RBQ_OK) return rc;

@@ -21,9 +21,9 @@ struct RpbhDevice {
   bool ready = false;
   int32_t* perm = nullptr;        // pi(k), destination order
   float* sign = nullptr;          // D_k as +-1.0f, destination order
-  // Gather tables of the token-pair kernel (built on first use): d byte
-  // offsets 2 pi(k), then d sign words (0 or 0x80000000), both at
-  // pair_tab_slot(k / 64, k % 64).
+  // Gather table of the token-pair kernel (built on first use): for output
+  // position k, at pair_tab_slot(k / 64, k % 64), the byte offset 2 pi(k) of
+  // its source in a staged row with the sign D_k in bit 31 (set for -1).
   uint32_t* pair_tab = nullptr;
 };
 
@@ -86,8 +86,8 @@ constexpr int kMaxFullGridCells = 5000;
 
 // Returns the device tables of `r` on the current device, uploading on first use.
 int rpbh_device(const rbq_rpbh* r, const RpbhDevice** out);
-// Returns the token-pair kernel's gather tables of `r` on the current device
-// (2 d words, see RpbhDevice::pair_tab), building them on first use.
+// Returns the token-pair kernel's gather table of `r` on the current device
+// (d words, see RpbhDevice::pair_tab), building it on first use.
 int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out);
 // Returns the codebook of (d, bits) on the current device, computing and
 // uploading it on first use.

@@ -147,13 +147,16 @@ __global__ void __launch_bounds__(512) rotq_kernel(RotqParams p) {
     const float s = tok[g];
 
     if constexpr (kLloyd) {
-      const float inv = 1.0f / (s + 1e-12f);
+      // A row whose norm is not finite is encoded as the zero vector (every
+      // v = 0, code 2^(b-1)).
+      const bool fin = s < INFINITY;
+      const float inv = fin ? 1.0f / (s + 1e-12f) : 0.f;
       uint32_t w[2 * BITS];
 #pragma unroll
       for (int i = 0; i < 2 * BITS; ++i) w[i] = 0u;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const uint32_t c = code_of<BITS>(y[i] * inv, bnd);
+        const uint32_t c = code_of<BITS>(fin ? y[i] * inv : 0.f, bnd);
         const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
         w[wi] |= c << sh;
         if (sh + BITS > 32) w[wi + 1] |= c >> (32 - sh);
@@ -503,12 +506,16 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         // z here is 8x the rotated value (H unnormalised): v = z / (||z|| + 8 eps).
         // Grid over v in [-1, 1]: n = round((v + 1)/2 * NC) needs no clamp once
         // z is finite, which holds for every coordinate when ||z|| is finite.
+        // A row whose norm is not finite is encoded as the zero vector: z and
+        // the scale both 0, so every index lands on the middle cell (a NaN
+        // scale would turn into a NaN grid index).
         const float nrm = sqrtf(tot);
-        if (!(nrm < INFINITY)) {
+        const bool bad = !(nrm < INFINITY);
+        if (bad) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) P[j] = 0ull;
         }
-        const float inv = 1.0f / (nrm + 8e-12f);
+        const float inv = bad ? 0.f : 1.0f / (nrm + 8e-12f);
         const float kq = inv * (0.5f * p.grid_cells);
         const float cq = 0.5f * p.grid_cells + 8388608.0f;   // + 2^23: round(.) lands in the low bits
         const unsigned long long kq2 = pk(kq, kq), cq2 = pk(cq, cq), inv2 = pk(inv, inv);
@@ -552,8 +559,10 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         }
       } else if constexpr (kLloyd) {
         // Clamped grid (wide codebooks): u = sat(v/(2R) + 1/2), n = round(u NC).
+        // A row whose norm is not finite is encoded as the zero vector.
         const float nrm = sqrtf(tot);
-        const float inv = 1.0f / (nrm + 8e-12f);
+        const bool bad = !(nrm < INFINITY);
+        const float inv = bad ? 0.f : 1.0f / (nrm + 8e-12f);
         const float A = inv * p.grid_scale;
         uint32_t w[2 * BITS];
 #pragma unroll
@@ -562,7 +571,7 @@ __global__ void __launch_bounds__(384, 1) rotq_fast_kernel(Params p) {
         for (int r = 0; r < 64; ++r) {
           float lo, hi;
           upk(P[r >> 1], lo, hi);
-          const float z = (r & 1) ? hi : lo;
+          const float z = bad ? 0.f : ((r & 1) ? hi : lo);
           const float u = fma_sat(z, A, 0.5f);
           const float qf = fmaf(u, p.grid_cells, 8388608.0f);   // 2^23: round(u*NC) in the low bits
           const float2 e = lds_f2(grid_addr + 8u * dbg_index(__float_as_uint(qf) - 0x4B000000u,

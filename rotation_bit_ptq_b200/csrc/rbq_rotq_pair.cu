@@ -20,7 +20,7 @@
 // Data movement: whole rows arrive by bulk asynchronous copies (TMA, no
 // tensor map needed for contiguous rows), one row per lane of an issuing
 // warp, into a ring of tile slots, each completion counted on the slot's
-// mbarrier.  The gather tables and the code grid are copied first, so they are
+// mbarrier.  The gather table and the code grid are copied first, so they are
 // not queued behind the tiles.  The last warp done gathering from a slot
 // refills it with a later tile, so the next tiles stream in while the current
 // one is transformed and encoded.
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 127u) & ~127u;
   unsigned char* sm = smem_raw + (sbase - sraw);
-  const Layout L = layout(p.d, p.NS, p.grid_n);
+  const Layout L = layout(p.d, p.NS, p.grid_entries);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* red = full + p.NS;
   uint64_t* tabbar = red + 2 * p.NS;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     }
   };
 
-  // ---- prologue: the gather tables and the guarded code grid start streaming
+  // ---- prologue: the gather table and the guarded code grid start streaming
   //      first; the first tile follows once the barriers are visible to all
   //      (the other slots fill after it has landed, so that it is not slowed
   //      by them) ----
@@ -130,9 +130,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     for (int r = 0; r < 2 * NS; ++r) mbar_init(&red[r], p.nwarps);   // one arrival per warp
     mbar_init(tabbar, 1);
     mbar_fence_init();
-    const uint32_t gbytes = kLloyd ? 8u * static_cast<uint32_t>(guarded_grid_entries(p.grid_n)) : 0u;
-    mbar_arrive_expect_tx(tabbar, 8u * p.d + gbytes);
-    bulk_load(sbase + L.off, p.tab, 8u * p.d, tabbar);
+    const uint32_t gbytes = kLloyd ? 8u * static_cast<uint32_t>(p.grid_entries) : 0u;
+    mbar_arrive_expect_tx(tabbar, 4u * p.d + gbytes);
+    bulk_load(sbase + L.off, p.tab, 4u * p.d, tabbar);
     if (kLloyd) bulk_load(sbase + L.grid, p.grid, gbytes, tabbar);
   }
   {
@@ -161,9 +161,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   const int b = 4 * warp + j;                      // output block of this thread
   const int bx = b & 7;
   const uint32_t off_addr = sbase + L.off + 256u * b;
-  const uint32_t sgn_addr = sbase + L.sgn + 256u * b;
   const uint32_t part_addr = sbase + L.part;
-  const uint32_t gbase = sbase + L.grid + 8u * kGridGuard - 0x4B000000u * 8u;
+  const uint32_t gbase = sbase + L.grid + 8u * static_cast<uint32_t>(p.grid_first) - 0x4B000000u * 8u;
   const uint32_t pitch8 = 8u * pitch;
   // Tensor memory: each thread parks its pair's two half-blocks (2 x 64 words)
   // in its own lane; warps w, w+4, w+8 share a lane quarter, 128 columns each.
@@ -190,14 +189,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       for (int q4 = 0; q4 < 8; ++q4) {
         const uint32_t c = 16u * (static_cast<uint32_t>(8 * h + q4) ^ static_cast<uint32_t>(bx));
         const uint4 o = lds128(off_addr + c);
-        const uint4 sg = lds128(sgn_addr + c);
         const uint32_t oo[4] = {o.x, o.y, o.z, o.w};
-        const uint32_t ss[4] = {sg.x, sg.y, sg.z, sg.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t a = rowA + dbg_index(oo[e], 2u * static_cast<uint32_t>(p.d), p.err);
-          const float y0 = bf16_signed(lds_u16(a), ss[e]);
-          const float y1 = bf16_signed(lds_u16(a + pitch8), ss[e]);
+          // entry = source byte offset | sign << 31: the sign word S feeds the
+          // conversion, the entry minus S is the offset
+          const uint32_t S = oo[e] & 0x80000000u;
+          const uint32_t a = rowA + dbg_index(oo[e] - S, 2u * static_cast<uint32_t>(p.d), p.err);
+          const float y0 = bf16_signed(lds_u16(a), S);
+          const float y1 = bf16_signed(lds_u16(a + pitch8), S);
           R[4 * q4 + e] = pk(y0, y1);
           acc[e] = fma2(R[4 * q4 + e], R[4 * q4 + e], acc[e]);
         }
@@ -307,15 +307,19 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       // A non-finite row (or a padding row past T) is encoded as the zero
       // vector, which also keeps every grid index inside the table.
       const bool bad0 = !(tot[0] < INFINITY) || !ok0, bad1 = !(tot[1] < INFINITY) || !ok1;
-      // z is 8x the rotated value: v = z / (8 s + 8 eps)
-      const float inv0 = 1.0f / (8.0f * s0 + 8e-12f), inv1 = 1.0f / (8.0f * s1 + 8e-12f);
+      // z is 8x the rotated value: v = z / (8 s + 8 eps); a bad row's z is
+      // taken as 0 below and its scale as 0, so its v is exactly 0 (the
+      // middle cell, code 2^(b-1)) even when its norm is NaN
+      const float inv0 = bad0 ? 0.f : 1.0f / (8.0f * s0 + 8e-12f);
+      const float inv1 = bad1 ? 0.f : 1.0f / (8.0f * s1 + 8e-12f);
       uint32_t w0[2 * BITS], w1[2 * BITS];
 #pragma unroll
       for (int i = 0; i < 2 * BITS; ++i) w0[i] = w1[i] = 0u;
       Enc enc(inv0, inv1, p.grid_cells, p.grid_scale, gbase);
 #ifdef RBQ_DEBUG
       enc.dbg_err = p.err;
-      enc.dbg_entries = static_cast<uint32_t>(guarded_grid_entries(p.grid_n));
+      enc.dbg_entries = static_cast<uint32_t>(p.grid_entries);
+      enc.dbg_first = static_cast<uint32_t>(p.grid_first);
 #endif
       // warp-uniform choice: encode_block reads tensor memory collectively
       if (__any_sync(0xffffffffu, bad0 || bad1)) {
@@ -454,7 +458,7 @@ namespace {
 template <int MODE, int BITS>
 int launch_pair(const pairk::Params& p, cudaStream_t st) {
   auto kern = pairk::rotq_pair_kernel<MODE, BITS>;
-  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_n).total + 128;
+  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_entries).total + 128;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = rowtile::sm_count();
@@ -507,11 +511,12 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     const CodebookDevice* cb = nullptr;
     if ((rc = codebook_device(r->d, bits, &cb)) != RBQ_OK) return rc;
     p.grid = cb->grid_pad;
-    p.grid_n = cb->grid_cells + 1;
+    p.grid_entries = guarded_grid_entries(cb->grid_cells + 1);
+    p.grid_first = kGridGuard;
     p.grid_cells = static_cast<float>(cb->grid_cells);
     p.grid_scale = cb->grid_scale;
   }
-  p.NS = slots_that_fit(r->d, p.grid_n);
+  p.NS = slots_that_fit(r->d, p.grid_entries);
   if (p.NS < 2) return RBQ_ECONVERGE;
   switch (mode) {
     case kAct: return launch_pair_bits<kAct>(bits, p, st);

@@ -30,9 +30,10 @@ struct Params {
   int ntiles;                        // ceil(T / 16)
   int NS;                            // ring slots
   uint32_t pitch;                    // bytes per staged row (2d + 16)
-  const uint32_t* tab;               // 2 d words: offsets, then sign words (pair_tab_slot order)
-  const float2* grid;                // Lloyd-Max modes: guarded grid (kGridGuard entries each side)
-  int grid_n;                        // entries of the unguarded grid (cells + 1)
+  const uint32_t* tab;               // d words: source offset | sign << 31 (pair_tab_slot order)
+  const float2* grid;                // Lloyd-Max modes: the code grid as copied into shared memory
+  int grid_entries;                  // entries copied (even: one 16-byte-multiple bulk copy)
+  int grid_first;                    // index of cell 0 among them (guard entries before it)
   float grid_cells, grid_scale;      // cells, 1 / (2R)
   void* out;
   void* aux;
@@ -42,17 +43,16 @@ struct Params {
 
 // Shared-memory layout (bytes from the 128-aligned base).
 struct Layout {
-  uint32_t ring, off, sgn, grid, part, bars, total;
+  uint32_t ring, off, grid, part, bars, total;
 };
 
-__host__ __device__ inline Layout layout(int d, int NS, int grid_n) {
+__host__ __device__ inline Layout layout(int d, int NS, int grid_entries) {
   Layout L{};
   const uint32_t pitch = 2u * d + 16u;
   L.ring = 0;
   L.off = L.ring + NS * kRows * pitch;
-  L.sgn = L.off + 4u * d;
-  L.grid = L.sgn + 4u * d;
-  L.part = (L.grid + 8u * guarded_grid_entries(grid_n) + 15u) & ~15u;
+  L.grid = L.off + 4u * d;
+  L.part = (L.grid + 8u * grid_entries + 15u) & ~15u;
   L.bars = L.part + 4u * (2 * NS) * kRows * kMaxWarps;   // [2NS][16 tokens][12 warps]
   L.bars = (L.bars + 7u) & ~7u;
   // full[NS], red[2NS], tab | TMEM base
@@ -94,6 +94,7 @@ __device__ __forceinline__ uint32_t set_ge(float a, float b) {
   asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(d) : "f"(a), "f"(b));
   return d;
 }
+
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float d;
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -147,17 +148,22 @@ __device__ __forceinline__ uint32_t bf2_bits(float lo, float hi) {
 // Code of each half of a packed pair z (two tokens) from the shared-memory
 // grid over [-R, R] (every cell holds at most one boundary): u = sat(v/(2R) +
 // 1/2), n = round(u * cells) through the +2^23 trick, and the cell's entry
-// {boundary or +inf, count of boundaries below the cell} gives
-// code = count + (v >= boundary).  Values beyond +-R saturate into the end
-// cells, whose entries cover them.  (A grid over all of [-1, 1] would need no
-// clamp but is 20x larger, and its lookups cost more shared-memory wavefronts
-// than the clamp costs arithmetic: measured 2-5 % slower for 2-4 bits.)
+// {boundary or +inf, count of boundaries below the cell} gives code = count +
+// (v >= boundary), the compare taken as the sign of z*inv - boundary.  Values
+// beyond +-R saturate into the end cells, whose entries cover them.  Measured
+// alternatives: a grid over all of [-1, 1] needs no clamp but is 20x larger
+// and its lookups cost more shared-memory wavefronts than the clamp costs
+// arithmetic (2-5 % slower for 2-4 bits); a grid over |v| with a negative v's
+// code mirrored fits 128 bytes at 4 bits, so its lookups never conflict, but
+// its extra compare and XOR per value cost 7 %; v for both tokens in one
+// packed multiply with the cell index from it cost 2 %.
 struct Enc {
   float A0, A1, inv0, inv1, cells;
   uint32_t gbase;
 #ifdef RBQ_DEBUG
   unsigned int* dbg_err = nullptr;     // debug builds: check every grid entry index
   uint32_t dbg_entries = 0;
+  uint32_t dbg_first = 0;
 #endif
   __device__ __forceinline__ Enc(float i0, float i1, float nc, float scale, uint32_t gb)
       : A0(i0 * scale), A1(i1 * scale), inv0(i0), inv1(i1), cells(nc), gbase(gb) {}
@@ -166,8 +172,8 @@ struct Enc {
   // the guard entries before entry 0).
   __device__ __forceinline__ uint32_t entry_addr(float qf) const {
 #ifdef RBQ_DEBUG
-    const uint32_t e = __float_as_uint(qf) - 0x4B000000u + static_cast<uint32_t>(kGridGuard);
-    return gbase + (0x4B000000u - static_cast<uint32_t>(kGridGuard)) * 8u + 8u * dbg_index(e, dbg_entries, dbg_err);
+    const uint32_t e = __float_as_uint(qf) - 0x4B000000u + dbg_first;
+    return gbase + (0x4B000000u - dbg_first) * 8u + 8u * dbg_index(e, dbg_entries, dbg_err);
 #else
     return gbase + __float_as_uint(qf) * 8u;
 #endif
@@ -221,10 +227,10 @@ inline int sm_count() {
 }
 
 // Most ring slots that fit next to the tables (at least 2, at most 6), or 0.
-inline int slots_that_fit(int d, int grid_n) {
+inline int slots_that_fit(int d, int grid_entries) {
   int best = 0;
   for (int ns = 2; ns <= 6; ++ns)
-    if (layout(d, ns, grid_n).total + 128 <= kSmemLimit) best = ns;
+    if (layout(d, ns, grid_entries).total + 128 <= kSmemLimit) best = ns;
   return best;
 }
 

@@ -159,6 +159,36 @@ def test_zero_and_degenerate_rows():
     assert norms[0].item() == 0.0
 
 
+@pytest.mark.parametrize("d,bits,dtype", [(3072, 4, "bf16"), (1280, 6, "bf16"),     # token-pair kernel
+                                          (4096, 5, "bf16"),                       # register-staged, [-1,1] grid
+                                          (4096, 8, "bf16"),                       # register-staged, clamped grid
+                                          (512, 3, "f32")])                        # general kernel
+def test_non_finite_rows_encode_as_the_zero_vector(d, bits, dtype):
+    """A row holding NaN or +-Inf has no finite norm; the kernels encode it as
+    the zero vector (every code 2^(b-1)) and the other rows are unaffected."""
+    X, _ = synth.student_t_act(40, d, seed=d + bits)
+    X = X.copy()
+    X[3, 7] = np.nan
+    X[17, d - 1] = np.inf
+    X[18, 0] = -np.inf
+    X[38, :] = np.nan
+    bad = np.array([3, 17, 18, 38])
+    good = np.setdiff1d(np.arange(40), bad)
+    r, Pi = _rpbh(d, 11)
+    codes, norms = rq_act(r, _dense(X, dtype), bits)
+    w_codes, rn = qweights(r, _dense(X, dtype), bits)          # the same rows as weights
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    for c in (codes, w_codes):
+        g = _unpack(c, bits, d)
+        assert np.all(g[bad] == 2 ** (bits - 1))
+    _, bounds = oracle.lloydmax_table(d, bits)
+    ora = oracle.quantize_act(X[good].astype(np.float64), Pi, bounds)
+    check_codes(_unpack(codes, bits, d)[good], ora["codes"], ora["v"], bounds, d)
+    check_rel(norms.cpu().numpy()[good], ora["norms"], NORM_RTOL, "norms")
+    assert not np.any(np.isfinite(norms.cpu().numpy()[bad]))
+
+
 def test_attention_projection_full_size_sampled():
     data = synth.attn_proj()
     X = data["X"]
