@@ -637,6 +637,41 @@ def run_suite(dev, stream, pk):
     }
     out["int8_dit"] = int8
 
+    # The rotation fused into the producing matmul (OrbitQuant §6.2): the DiT
+    # block's MLP up-projection (4096 tokens, 4096 -> 16384, W8A16) whose GELU
+    # output is the down-projection's input, rotated at d = 16384.  Unfused:
+    # qlinear_int8 (BF16 y) -> GELU (a torch elementwise kernel, fp32 math on
+    # the BF16 tensor) -> rotate_act.  Fused: one qlinear_int8_rotate_next on
+    # the weight rows reordered (once, offline) by the next layer's permutation.
+    W = to_bf16_tensor(synth.int8_dit_weight(0, "up"), dev)
+    X = to_bf16_tensor(synth.int8_dit_act(4096), dev)
+    r, nxt = rbq.RPBH(4096, 100 + 4096), rbq.RPBH(16384, 200 + 16384)
+    xr = rbq.rotate_act(r, X)
+    q, sc = rbq.quantize_weights(r, W, 8, mode="int8")
+    qn, scn = rbq.rows_in_next_order(nxt, q), rbq.rows_in_next_order(nxt, sc)
+    y = torch.empty((4096, 16384), dtype=torch.bfloat16, device=dev)
+    g = torch.empty_like(y)
+    xn = torch.empty_like(y)
+
+    def unfused():
+        rbq.qlinear_int8(xr, q, sc, y, stream=stream)
+        torch.nn.functional.gelu(y, out=g)
+        rbq.rotate_act(nxt, g, xn, stream=stream)
+
+    us_un = _time_us(unfused, stream)
+    us_gemm = _time_us(lambda: rbq.qlinear_int8(xr, q, sc, y, stream=stream), stream)
+    us_rot = _time_us(lambda: rbq.rotate_act(nxt, g, xn, stream=stream), stream)
+    us_fused = _time_us(lambda: rbq.qlinear_int8_rotate_next(xr, qn, scn, nxt, "gelu", xn, stream=stream), stream)
+    out["fused_rotation_dit_mlp_up_into_down"] = {
+        "unfused_us": round(us_un, 2), "unfused_parts_us": {"qlinear_int8": round(us_gemm, 2),
+                                                            "gelu (torch)": round(us_un - us_gemm - us_rot, 2),
+                                                            "rotate_act d=16384": round(us_rot, 2)},
+        "fused_us": round(us_fused, 2), "speedup": round(us_un / us_fused, 3),
+        "fused_TFLOP/s": round(2.0 * 4096 * 16384 * 4096 / (us_fused * 1e-6) / 1e12, 1)}
+    r.close()
+    nxt.close()
+    del W, X, xr, q, sc, qn, scn, y, g, xn
+
     # video DiT W4A6: 32760 tokens (21 frames x 1560), hidden 1536, MLP 8960
     T = 32760
     vid = {}

@@ -363,6 +363,53 @@ int rbq_code_grid(int d, int bits, int variant, float* thr, int32_t* base, int* 
 int qlinear_int8_asym(const uint16_t* Xrot, const uint8_t* Wq, const float* scale, const uint8_t* zero_point,
                       int M, int N, int K, uint16_t* Y, void* stream);
 
+/* ---- the rotation fused into the producing matmul ---------------------------
+ * OrbitQuant §6.2 ("performance below expectations") points at fusing the
+ * rotation with the matrix-multiply kernels to cut memory traffic.  The
+ * rotation of a layer's input gathers it by pi across the whole row, which no
+ * output tile of the producing GEMM holds; with the producing layer's weight
+ * rows reordered offline by that pi, each 64 consecutive output columns are
+ * the inputs of one Hadamard block, and the producing GEMM's epilogue can
+ * finish the rotation. */
+#define RBQ_ACT_NONE 0
+#define RBQ_ACT_GELU 1   /* exact GELU: y Phi(y) = 0.5 y erfc(-y / sqrt 2) */
+
+/*
+ * rpbh_gather_rows -- the offline reordering: row k of dst = row pi(k) of src,
+ * k = 0..d-1, with pi the permutation of `r` (the handle of the layer that
+ * will consume the producing layer's output; OrbitQuant §2.3).
+ *   src, dst   DEVICE buffers of d rows of row_bytes each, not the same buffer
+ *   Use it on the producing layer's INT8 weight rows (row_bytes = K) and on
+ *   its per-row scales (row_bytes = 4).  Asynchronous on `stream`.
+ * Errors: RBQ_EINVAL, RBQ_ECUDA.
+ */
+int rpbh_gather_rows(const rbq_rpbh* r, const void* src, long long row_bytes, void* dst, void* stream);
+
+/*
+ * qlinear_int8_rotate_next -- the W8A16 layer of qlinear_int8 fused with the
+ * rotation of the next layer's input, in one GEMM:
+ *   y[m, j]          = scale[j] * sum_k q[j, k] * Xrot[m, k]   (the producing layer)
+ *   x[m, :]          = act(y[m, :])                             (RBQ_ACT_NONE: x = y)
+ *   Xrot_next[m, :]  = bf16( Pi_next x[m, :] )                  (the next layer's input,
+ *                                                                as rotate_act gives it)
+ * The epilogue takes each 64-column block of the accumulator (fp32), scales
+ * it, applies act and the signs D of the block, the 64-point Walsh-Hadamard
+ * transform and 1/8, and stores BF16 once: neither y nor x reaches memory.
+ *   Xrot              device BF16 [M, K], the producing layer's rotated input
+ *   Wq_next_order     device int8 [N, K]: row k = the layer's output channel
+ *                     pi_next(k) (rpbh_gather_rows on the quantize_weights rows)
+ *   scale_next_order  device fp32 [N], reordered the same way
+ *   next              the RPBH handle of the next layer; N = its d
+ *   activation        RBQ_ACT_NONE or RBQ_ACT_GELU (fp32, with CUDA's erfcf)
+ *   Xrot_next         device BF16 [M, N], row-major
+ * K a multiple of 64 (else RBQ_EINVAL).  Stream-ordered like qlinear_int8
+ * (same workspace).
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int qlinear_int8_rotate_next(const uint16_t* Xrot, const int8_t* Wq_next_order, const float* scale_next_order,
+                             int M, int K, const rbq_rpbh* next, int activation, uint16_t* Xrot_next,
+                             void* stream);
+
 /* ---- quantised layer files ------------------------------------------------
  * The pages' "quantized model file" (INT8-convrot, section 1): the quantised
  * weights, their quantisation parameters (scale, zero point or row norms) and

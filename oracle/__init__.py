@@ -23,6 +23,9 @@ Source pages, cited by title and section:
 * INT8 image-text model -- cloud.baidu.com/article/9432337, "how it works"
   (scale per tensor/channel).
 
+OrbitQuant §6.2 (fusing the rotation with the matmul kernels) adds the fused
+layer of ``fused.py``: a plain composition of the parts above.
+
 Pin status (what ties each function to something other than itself):
 
 =====================  ===================================================
@@ -49,6 +52,11 @@ qlinear.e4m3_round     PyTorch's float8_e4m3fn conversion (library routine)
 qlinear.fp8_levels     the same Max table rounded to 3 mantissa bits by hand;
                        power-of-two beta; the layer's triple loop, closed
                        form and rounding bound
+fused.gelu             y * Phi(y) with Phi from scipy.stats.norm (a library
+                       routine); odd-part identity gelu(y) - gelu(-y) = y;
+                       published values
+fused.qlinear_int8_    composition of pinned parts; a pure-Python triple
+  rotate_next          loop and an explicit dense Pi on a tiny case
 =====================  ===================================================
 """
 
@@ -61,6 +69,7 @@ from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
                     quantize_weights_int8_asym, rotate_only, EPS)
 from .qlinear import (qlinear, qlinear_int8, qlinear_int8_asym, int8_levels, qlinear_int8_levels,
                       e4m3_round, fp8_levels, qlinear_fp8_levels)
+from .fused import gelu, qlinear_int8_rotate_next
 
 __all__ = [
     "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_rows", "rpbh_apply",
@@ -69,5 +78,5 @@ __all__ = [
     "quantize_act", "quantize_weights_lloydmax", "quantize_weights_int8",
     "quantize_weights_int8_asym", "rotate_only", "EPS", "qlinear", "qlinear_int8",
     "qlinear_int8_asym", "int8_levels", "qlinear_int8_levels", "e4m3_round", "fp8_levels",
-    "qlinear_fp8_levels",
+    "qlinear_fp8_levels", "gelu", "qlinear_int8_rotate_next",
 ]

@@ -25,6 +25,8 @@ RBQ_OK, RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA, RBQ_ENOMEM, RBQ_ECONVERGE, RBQ_EDEVIC
 RBQ_ESCRATCH = -7
 RBQ_RPBH_NO_PERMUTATION, RBQ_RPBH_NO_SIGNS = 1, 2
 RBQ_EIO = -8
+RBQ_ACT_NONE, RBQ_ACT_GELU = 0, 1
+_ACTS = {None: RBQ_ACT_NONE, "none": RBQ_ACT_NONE, "gelu": RBQ_ACT_GELU}
 RBQ_LAYER_LLOYDMAX, RBQ_LAYER_INT8_SYM, RBQ_LAYER_INT8_TENSOR, RBQ_LAYER_INT8_ASYM = 0, 1, 2, 3
 _LAYER_KINDS = {"lloydmax": RBQ_LAYER_LLOYDMAX, "int8": RBQ_LAYER_INT8_SYM, "int8_tensor": RBQ_LAYER_INT8_TENSOR,
                 "int8_asym": RBQ_LAYER_INT8_ASYM}
@@ -64,6 +66,8 @@ SIGNATURES = {
     "rbq_device_error": (_I, [_P]),
     "rbq_selftest_wait_limit": (_I, [_P, _P]),
     "rbq_code_grid": (_I, [_I, _I, _I, _P, _P, _P, _P]),
+    "rpbh_gather_rows": (_I, [_P, _P, ctypes.c_longlong, _P, _P]),
+    "qlinear_int8_rotate_next": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P]),
 }
 
 _lib = None
@@ -500,6 +504,51 @@ def qlinear_int8_asym(xrot, q, scale, zero_point, out=None, stream=None):
     with _device_ctx(xrot, q, scale, zero_point, out):
         _check(lib().qlinear_int8_asym(_ptr(xrot), _ptr(q), _ptr(scale), _ptr(zero_point), M, N, K, _ptr(out),
                                        _stream(stream)), "qlinear_int8_asym")
+    return out
+
+
+def rows_in_next_order(next_rpbh, t, out=None, stream=None):
+    """The offline reordering for qlinear_int8_rotate_next: out[k] = t[pi(k)]
+    for the rows of a device tensor t [d, ...] (d = next_rpbh.d), pi the
+    permutation of the next layer's rotation (rpbh_gather_rows)."""
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+        raise ValueError("t must be a contiguous CUDA tensor")
+    if t.shape[0] != next_rpbh.d:
+        raise ValueError(f"t must have {next_rpbh.d} rows (the next layer's width)")
+    out = torch.empty_like(t) if out is None else out
+    if out.shape != t.shape or out.dtype != t.dtype or not out.is_contiguous() or out.data_ptr() == t.data_ptr():
+        raise ValueError("out must be a different contiguous tensor of t's shape and dtype")
+    row_bytes = t[0].numel() * t.element_size() if t.dim() > 1 else t.element_size()
+    with _device_ctx(t, out):
+        _check(lib().rpbh_gather_rows(next_rpbh.handle, _ptr(t), int(row_bytes), _ptr(out), _stream(stream)),
+               "rpbh_gather_rows")
+    return out
+
+
+def qlinear_int8_rotate_next(xrot, q_next_order, scale_next_order, next_rpbh, activation="gelu", out=None,
+                             stream=None):
+    """The W8A16 layer fused with the next layer's input rotation:
+    out = bf16(Pi_next act(scale_n sum_k q_nk x'_mk)) as bfloat16 [M, next.d];
+    q and scale in the next layer's permutation order (rows_in_next_order)."""
+    import torch
+    _need_cuda(xrot, "xrot", torch.bfloat16)
+    _need_cuda(q_next_order, "q_next_order", torch.int8)
+    _need_cuda(scale_next_order, "scale_next_order", torch.float32)
+    M, K = xrot.shape
+    N = next_rpbh.d
+    _need_shape(q_next_order, (N, K), "q_next_order")
+    _need_shape(scale_next_order, (N,), "scale_next_order")
+    if activation not in _ACTS:
+        raise ValueError("activation must be None, 'none' or 'gelu'")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xrot.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _need_shape(out, (M, N), "out")
+    with _device_ctx(xrot, q_next_order, scale_next_order, out):
+        _check(lib().qlinear_int8_rotate_next(_ptr(xrot), _ptr(q_next_order), _ptr(scale_next_order), M, K,
+                                              next_rpbh.handle, _ACTS[activation], _ptr(out), _stream(stream)),
+               "qlinear_int8_rotate_next")
     return out
 
 

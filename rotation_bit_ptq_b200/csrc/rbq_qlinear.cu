@@ -252,7 +252,8 @@ int launch_qgemm(const QParams& p, cudaStream_t st) {
 namespace rbq {
 bool qlinear_int8_fast_eligible(int M, int N, int K);
 int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float* scale, int M, int N, int K,
-                             uint16_t* Y, unsigned int* err, cudaStream_t st, const uint8_t* zero_point = nullptr);
+                             uint16_t* Y, unsigned int* err, cudaStream_t st, const uint8_t* zero_point = nullptr,
+                             const float* next_sign = nullptr, int act = 0);
 bool qlinear_fast_eligible(int M, int N, int K, int bits_a, int bits_w);
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,

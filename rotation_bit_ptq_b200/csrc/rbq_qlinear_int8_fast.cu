@@ -20,6 +20,11 @@
 //                  128B-swizzled K-major.
 //    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
 //    overlap the MMAs of tile i+1.
+//    Fused with the next layer's rotation (qlinear_int8_rotate_next, see
+//    rbq_fused.cu) the epilogue does more per element -- an activation, the
+//    signs, the 64-point Walsh-Hadamard transform on packed pairs -- so it runs
+//    on eight warps (0..3 and 6..9, two per TMEM lane quadrant), each thread
+//    finishing two of a tile's four 64-column blocks.
 //
 // Every mbarrier wait is bounded (see qlinear_fast); a thread whose wait runs
 // out raises the shared abort flag and records an error bit.
@@ -44,8 +49,22 @@ constexpr int kATile = kBM * kBK * 2;          // 16 KB
 constexpr int kBTile = kBN * kBK * 2;          // 32 KB
 constexpr int kStage = kATile + kBTile;        // 48 KB
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
+
+// Epilogue kinds.
+enum Epi {
+  kEpiScale = 0,        // W8A16: Y = bf16(acc * scale[n])
+  kEpiCodes = 1,        // qlinear on expanded code levels: Y = bf16(acc * s[m] r'[n] / K)
+  kEpiRotateNext = 2,   // W8A16 whose output feeds the next rotated layer: per 64-column
+                        // block, Y = bf16(H_64 D (act(acc * scale)) / 8), act = identity
+  kEpiRotateNextGelu = 3,   // the same with act = GELU
+};
+
+// Threads per CTA: 4 epilogue warps + MMA warp + TMA warp; the rotating
+// epilogues add 4 more epilogue warps (warps 6..9), two per TMEM lane
+// quadrant, so that each thread finishes two of a tile's four Hadamard blocks.
+__host__ __device__ constexpr int threads_for(int epi) { return epi >= kEpiRotateNext ? 320 : 192; }
+__host__ __device__ constexpr int epi_threads_for(int epi) { return epi >= kEpiRotateNext ? 256 : 128; }
 
 struct Params {
   int M, N, K;
@@ -53,9 +72,69 @@ struct Params {
   const float* s;             // qlinear: per-row norms
   const uint16_t* rnorm;      // qlinear: BF16 per-column norms
   float inv_k;                // qlinear: 1/K (the fp16 levels carry sqrt(K) each)
+  const float* next_sign;     // rotating epilogues: D of the next layer (+-1, output position order)
   uint16_t* Y;
   unsigned int* err;
 };
+
+// GELU(y) = y Phi(y) with the normal CDF from Abramowitz & Stegun (1964),
+// formula 7.1.26 (Hastings' rational approximation of erf, |error| <= 1.5e-7
+// for x >= 0): for x = |y| / sqrt 2, t = 1 / (1 + p x),
+// erfc(x) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-x^2), and
+// Phi(y) = 1 - erfc(x) / 2 for y >= 0, erfc(x) / 2 for y < 0.  Phi is within
+// 1e-7 of the exact value, far below the BF16 rounding of the layer's output.
+__device__ __forceinline__ float gelu_as7126(float y) {
+  const float x = fabsf(y) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+  float poly = fmaf(t, 1.061405429f, -1.453152027f);
+  poly = fmaf(t, poly, 1.421413741f);
+  poly = fmaf(t, poly, -0.284496736f);
+  poly = fmaf(t, poly, 0.254829592f);
+  const float half_erfc = 0.5f * t * poly * __expf(-x * x);
+  return y * (y >= 0.f ? 1.0f - half_erfc : half_erfc);
+}
+
+__device__ __forceinline__ unsigned long long pk2(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(unsigned long long r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ unsigned long long add_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long sub_f2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// In-place unnormalised 64-point Walsh-Hadamard transform (Sylvester order)
+// on the pairs P[i] = (z_i, z_{i+32}): strides 1..16 act on both halves of a
+// pair alike (one packed add/sub each), stride 32 combines the two halves.
+__device__ __forceinline__ void fwht64_pairs(unsigned long long (&P)[32]) {
+#pragma unroll
+  for (int len = 1; len < 32; len <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & len) == 0) {
+        const unsigned long long a = P[i], b = P[i + len];
+        P[i] = add_f2(a, b);
+        P[i + len] = sub_f2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float lo, hi;
+    upk2(P[i], lo, hi);
+    P[i] = pk2(lo + hi, lo - hi);        // (z_i, z_{i+32})
+  }
+}
 
 struct __align__(8) Tail {
   uint64_t full[kStages];
@@ -76,13 +155,17 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* 
   return mbar_warp_wait(bar, parity, &tl->abort);
 }
 
-// kQ = false: the W8A16 layer (bf16 operands, epilogue x scale[n]);
-// kQ = true: qlinear on codes expanded beforehand into fp16 levels (x sqrt(K)),
-// epilogue x s[m] r'[n] / K.
-template <bool kQ>
-__global__ void __launch_bounds__(kThreads, 1)
+// EPI = kEpiScale: the W8A16 layer (bf16 operands, epilogue x scale[n]);
+// kEpiCodes: qlinear on codes expanded beforehand into fp16 levels (x sqrt(K)),
+// epilogue x s[m] r'[n] / K; kEpiRotateNext: the W8A16 layer whose weight rows
+// come in the order of the next layer's permutation, its epilogue applying the
+// activation and the next layer's signs and 64-point Hadamard blocks.
+template <int EPI>
+__global__ void __launch_bounds__(threads_for(EPI), 1)
     qlinear_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const Params p) {
+  constexpr bool kQ = (EPI == kEpiCodes);
+  constexpr bool kRot = (EPI >= kEpiRotateNext);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -99,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tl->acc_full[a], 1);
-      mbar_init(&tl->acc_empty[a], 128);
+      mbar_init(&tl->acc_empty[a], epi_threads_for(EPI));
     }
     mbar_init(&tl->drain, 1);
     tl->abort = 0u;
@@ -168,8 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue ----------------
-    const int q = warp;                     // TMEM lane quadrant
+    const int q = warp & 3;                 // TMEM lane quadrant (warps 6..9: 2, 3, 0, 1)
     const int r = 32 * q + lane;            // row within the tile
+    const int eg = warp < 4 ? 0 : 1;        // rotating epilogues: which two of the four blocks
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
       const uint32_t a = it & 1u, use = it >> 1;
@@ -180,6 +264,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int mt = tile % ntiles_m, nt = tile / ntiles_m;
       const int m = mt * kBM + r;
+      if constexpr (kRot) {
+        // The tile's 256 columns are four whole blocks of the next layer's
+        // rotation (N % 64 == 0, tiles start at multiples of 256): column k is
+        // the producing layer's output channel pi(k), so block b of the next
+        // layer's rotated input is H_64 D_b act(y) over these 64 columns.
+        // This thread's warp group takes blocks 2 eg and 2 eg + 1.
+#pragma unroll 1
+        for (int blk = 2 * eg; blk < 2 * eg + 2; ++blk) {
+          uint32_t v0[32], v1[32];
+          __syncwarp();                   // the loads are warp-collective; rows past M only skip the stores
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + a * kBN + 64 * blk, v0);
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + a * kBN + 64 * blk + 32, v1);
+          tmem_wait_ld();
+          const int n0 = nt * kBN + 64 * blk;
+          if (m >= p.M || n0 >= p.N) continue;
+          unsigned long long P[32];       // (z_i, z_{i+32})
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float y0 = __uint_as_float(v0[i]) * __ldg(p.scale + n0 + i);
+            float y1 = __uint_as_float(v1[i]) * __ldg(p.scale + n0 + 32 + i);
+            if constexpr (EPI == kEpiRotateNextGelu) {
+              y0 = gelu_as7126(y0);
+              y1 = gelu_as7126(y1);
+            }
+            P[i] = pk2(y0 * __ldg(p.next_sign + n0 + i), y1 * __ldg(p.next_sign + n0 + 32 + i));
+          }
+          fwht64_pairs(P);
+          uint4* d4 = reinterpret_cast<uint4*>(p.Y + static_cast<long long>(m) * p.N + n0);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                float a0, a1, b0, b1;
+                upk2(P[8 * j + 2 * e], a0, a1);
+                upk2(P[8 * j + 2 * e + 1], b0, b1);
+                const __nv_bfloat162 h = half ? __floats2bfloat162_rn(a1 * 0.125f, b1 * 0.125f)
+                                              : __floats2bfloat162_rn(a0 * 0.125f, b0 * 0.125f);
+                w[e] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+              d4[4 * half + j] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tl->acc_empty[a]);
+        continue;
+      }
       const float rs = kQ ? ((m < p.M) ? p.s[m] * p.inv_k : 0.f) : 1.f;
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
@@ -302,19 +436,20 @@ int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int
 }
 
 // Launches the GEMM on two fp16/bf16 operands already in memory (K % 64 == 0).
-template <bool kQ>
+template <int EPI>
 int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStream_t st, int sms) {
+  constexpr bool kQ = (EPI == kEpiCodes);
   CUtensorMap mA, mB;
   int rc = encode_bf16_map(&mA, A, p.M, p.K, kBM, kQ);
   if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, kBN, kQ);
   if (rc != RBQ_OK) return rc;
-  auto kern = qlinear_bf16_kernel<kQ>;
+  auto kern = qlinear_bf16_kernel<EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int ntiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(threads_for(EPI), 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -342,15 +477,17 @@ int qlinear_f16_operands_gemm(const uint16_t* af16, const float* s, const uint16
   p.inv_k = inv_k;
   p.Y = Y;
   p.err = err;
-  return q8fast::launch_gemm<true>(af16, wf16, p, st, sms);
+  return q8fast::launch_gemm<q8fast::kEpiCodes>(af16, wf16, p, st, sms);
 }
 
 bool qlinear_int8_fast_eligible(int M, int N, int K) {
   return M >= 1 && N >= 8 && (N % 8) == 0 && K >= 64 && (K % 64) == 0;
 }
 
+// next_sign != null: the kEpiRotateNext epilogue (N % 64 == 0, act given).
 int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float* scale, int M, int N, int K,
-                             uint16_t* Y, unsigned int* err, cudaStream_t st, const uint8_t* zero_point) {
+                             uint16_t* Y, unsigned int* err, cudaStream_t st, const uint8_t* zero_point,
+                             const float* next_sign, int act) {
   using namespace q8fast;
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
@@ -379,10 +516,13 @@ int qlinear_int8_fast_launch(const uint16_t* Xrot, const int8_t* Wq, const float
     p.N = N;
     p.K = K;
     p.scale = scale;
+    p.next_sign = next_sign;
     p.Y = Y;
     p.err = err;
     // programmatic dependent launch: the prologue overlaps the widening kernel's tail
-    rc = launch_gemm<false>(Xrot, wb, p, st, sms);
+    if (!next_sign) rc = launch_gemm<kEpiScale>(Xrot, wb, p, st, sms);
+    else if (act == RBQ_ACT_GELU) rc = launch_gemm<kEpiRotateNextGelu>(Xrot, wb, p, st, sms);
+    else rc = launch_gemm<kEpiRotateNext>(Xrot, wb, p, st, sms);
   }
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
