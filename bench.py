@@ -52,8 +52,9 @@ WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x3
 
 def qlinear_algorithmic_bytes(M=T, N=D, K=D, bits_a=BITS_A, bits_w=BITS_W):
     """Operand and result bytes of one qlinear call: activation codes, weight
-    codes, s (fp32), r' (BF16) and Y (BF16).  The fp16 weight workspace the
-    call writes and reads back (N*K*2 each way) is extra, reported beside it."""
+    codes, s (fp32), r' (BF16) and Y (BF16).  The fp16 workspaces the call
+    writes and reads back (weights N*K*2 and activations M*K*2, each way) are
+    extra, reported beside it."""
     return M * K * bits_a // 8 + N * K * bits_w // 8 + 4 * M + 2 * N + 2 * M * N
 
 
@@ -332,17 +333,19 @@ def run_ours(args, rank, world):
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": QLINEAR_DRAM_BYTES,
                      "peak_source": pk["source"] + " bf16 burst",
-                     "note": "achieved includes the per-call weight-code expansion launch; traffic is the ncu "
-                             "DRAM read + write of both launches (expansion + GEMM) of one call",
+                     "note": "achieved includes the per-call code expansion launches (weights, activations); "
+                             "traffic is the ncu DRAM read + write of the three launches of one call "
+                             "(two expansions + GEMM)",
                      "algorithmic_bytes": qlinear_algorithmic_bytes(),
-                     "workspace_round_trip_bytes": 2 * 2 * D * D},
+                     "workspace_round_trip_bytes": 2 * 2 * (D * D + T * D)},
         "roofline_rotate_quantize": {"kernel": "rotate_quantize_act", "bound": "hbm",
                                      "achieved": round(act_bytes / k1_avg_s / 1e9, 2), "peak": pk["hbm_gbs"],
                                      "unit": "GB/s", "frac": round(act_bytes / k1_avg_s / 1e9 / pk["hbm_gbs"], 4),
                                      "traffic": ROTQ_DRAM_BYTES, "algorithmic_bytes": act_bytes,
                                      "peak_source": pk["source"]},
-        # steps: rotate-quantize, weights, weight-code expansion, GEMM; kernel passes likewise x nsets x reps
-        "gpu_launches": 4 * args.steps + 4 * kernel_reps * nsets,
+        # steps: rotate-quantize, weights, weight- and activation-code expansion, GEMM; kernel passes
+        # likewise x nsets x reps
+        "gpu_launches": 5 * args.steps + 5 * kernel_reps * nsets,
         "timing": ("per-kernel: CUDA graphs of %d launches over the rotating sets, replayed %d times; "
                    "ms_per_step: direct API calls" % (nsets, kernel_reps)) if kernel_graphs else
                   "per-kernel and ms_per_step: direct API calls",

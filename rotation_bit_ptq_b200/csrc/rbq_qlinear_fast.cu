@@ -5,13 +5,21 @@
 //   the weights (§2.1) cancels the online one, so
 //   y[m,n] = s_m r'_n sum_k C_w[q_nk] C_a[p_mk].
 //
-// Two kernels per call.
+// Code expansion: expand_codes_kernel turns
+// packed codes into fp16 levels (x sqrt(K)) in a stream-ordered workspace, an
+// HBM-bound pass over rows*K*(b/8 + 2) bytes with warp-contiguous loads and
+// stores.  Expanding each weight tile inside the GEMM instead would redo that
+// work for every tile of tokens and saturate the SM's integer pipe.
 //
-// 1. expand_weights_kernel(8): the weight codes are turned into fp16 levels
-//    (x sqrt(K)) once, into a stream-ordered workspace [N, K] -- an HBM-bound
-//    pass over N*K*(b/8 + 2) bytes.  Expanding each weight tile inside the
-//    GEMM instead would redo that work for every 128-row tile of tokens and
-//    saturate the SM's integer pipe.
+// Each call expands the weight codes [N, K]; then one of two routes:
+//  * activations whose fp16 copy (M*K*2 bytes) is at most 128 MiB are
+//    expanded the same way and the TMA-fed GEMM of rbq_qlinear_int8_fast.cu
+//    (on CTA pairs, epilogue s_m r'_n / K) multiplies the two fp16 operands;
+//  * larger activations stay packed and are expanded inside the GEMM below,
+//    which avoids writing and re-reading a copy that would not stay in L2.
+//
+// 1. expand_codes_kernel: the weight codes (and, first route, the activation
+//    codes in the same launch) to fp16 levels.
 // 2. qlinear_fast_kernel: each CTA (one per SM) walks a static list of
 //    128 x 256 output tiles.
 //      warps 0..3  epilogue: TMEM lane quadrant w, one output row per thread;
@@ -476,54 +484,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Weight codes [N, K*b/8] -> fp16 levels (x sqrt(K)) [N, K], one 64-code slice
-// per thread: read 8b bytes, write 128 bytes (both contiguous across threads).
-template <int BITS>
-__global__ void __launch_bounds__(256) expand_weights_kernel(const uint8_t* codes, long long rows, int K,
-                                                            const uint16_t* lut_g, uint16_t* out) {
-  __shared__ uint16_t lut[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = (i < (1 << BITS)) ? lut_g[i] : 0;
-  __syncthreads();
-  const Planes4 P = make_planes4(lut);
-  const int slices = K / kBK;
-  const long long items = rows * slices;
-  for (long long it = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; it < items;
-       it += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint2* src = reinterpret_cast<const uint2*>(codes + it * (8 * BITS));
-    uint32_t w[slice_words<BITS>()];
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) {
-      const uint2 v = __ldcs(src + i);
-      w[2 * i] = v.x;
-      w[2 * i + 1] = v.y;
-    }
-    uint4* dst = reinterpret_cast<uint4*>(out + it * kBK);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t o[4];
-      if constexpr (BITS == 4) {
-        expand8_4bit(w[c], P, o);
-      } else {
-        constexpr uint32_t mask = (1u << BITS) - 1u;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t pair = 0u;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int i = 8 * c + 2 * j + e;
-            const int bit = i * BITS, wi = bit >> 5, sh = bit & 31;
-            uint32_t code = w[wi] >> sh;
-            if (sh + BITS > 32) code |= w[wi + 1] << (32 - sh);
-            pair |= static_cast<uint32_t>(lut[code & mask]) << (16 * e);
-          }
-          o[j] = pair;
-        }
-      }
-      dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
-}
-
 // ---- host side ------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -594,107 +554,191 @@ int encode_f16_map(CUtensorMap* map, const uint16_t* base, int rows, int K) {
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
 }
 
-// Widths that divide 8 bits: one thread per 8 codes (BITS bytes in, 16 bytes
-// out), so a warp reads 32*BITS and writes 512 contiguous bytes.
-template <int BITS>
-__global__ void __launch_bounds__(256) expand_weights_kernel8(const uint8_t* codes, long long groups,
-                                                             const uint16_t* lut_g, uint16_t* out) {
-  __shared__ uint16_t lut[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = (i < (1 << BITS)) ? lut_g[i] : 0;
-  __syncthreads();
-  const Planes4 P = make_planes4(lut);
-  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < groups;
-       g += static_cast<long long>(gridDim.x) * blockDim.x) {
-    uint32_t w[4];
-    if constexpr (BITS == 4) {
-      expand8_4bit(__ldcs(reinterpret_cast<const uint32_t*>(codes) + g), P, w);
-    } else {
-      uint64_t x;
-      if constexpr (BITS == 8) x = __ldcs(reinterpret_cast<const unsigned long long*>(codes) + g);
-      else if constexpr (BITS == 2) x = __ldcs(reinterpret_cast<const unsigned short*>(codes) + g);
-      else x = codes[g];
-      constexpr uint32_t mask = (1u << BITS) - 1u;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        w[j] = static_cast<uint32_t>(lut[(x >> (2 * j * BITS)) & mask]) |
-               (static_cast<uint32_t>(lut[(x >> ((2 * j + 1) * BITS)) & mask]) << 16);
-    }
-    __stcg(reinterpret_cast<uint4*>(out) + g, make_uint4(w[0], w[1], w[2], w[3]));
-  }
-}
+// ---- code expansion ------------------------------------------------------
+// One job: `groups` groups of 8 codes (BITS bytes each; the packed rows are
+// contiguous and every row holds K/8 whole groups) -> 16 bytes of fp16
+// levels each.  One launch runs one or two jobs (a call's weights and
+// activations), each on its own range of blocks; every body is a grid-stride
+// loop over its job's blocks in which each warp's loads and stores cover
+// contiguous memory.
+struct ExpandJob {
+  const uint8_t* codes;
+  long long groups;
+  const uint16_t* lut;      // 2^bits fp16 levels
+  uint4* out;
+  int bits;
+  int blocks;               // blocks of the launch that run this job
+};
 
-// 4-bit codes: a warp expands 128 words of 8 codes (512 bytes in, 2 KB out)
-// per step; lane l takes words l, l+32, l+64 and l+96 of the warp's range, so
-// every load and every store instruction of the warp covers contiguous memory
-// (128 and 512 bytes) instead of 16-byte pieces 64 bytes apart.
-__global__ void __launch_bounds__(256) expand_weights_kernel4(const uint32_t* codes, long long words,
-                                                             const uint16_t* lut_g, uint4* out) {
+// 4-bit codes: a group is one 32-bit word.  A warp expands 128 words (512
+// bytes in, 2 KB out) per step; lane l takes words l, l+32, l+64 and l+96 of
+// the warp's range, so every load and store instruction of the warp is
+// contiguous (128 and 512 bytes), not 16-byte pieces 64 bytes apart.
+__device__ __forceinline__ void expand_job4(const ExpandJob& j, int jb) {
   Planes4 P;
   {
     uint16_t lut[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) lut[i] = __ldg(lut_g + i);
+    for (int i = 0; i < 16; ++i) lut[i] = __ldg(j.lut + i);
     P = make_planes4(lut);
   }
+  const uint32_t* codes = reinterpret_cast<const uint32_t*>(j.codes);
   const int lane = threadIdx.x & 31;
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  for (long long base = (blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5)) * 128;
-       base < words; base += 128 * warps) {
+  const long long warps = static_cast<long long>(j.blocks) * (blockDim.x >> 5);
+  for (long long base = (jb * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5)) * 128;
+       base < j.groups; base += 128 * warps) {
     uint32_t x[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const long long g = base + 32 * j + lane;
-      x[j] = g < words ? __ldcs(codes + g) : 0u;
+    for (int q = 0; q < 4; ++q) {
+      const long long g = base + 32 * q + lane;
+      x[q] = g < j.groups ? __ldcs(codes + g) : 0u;
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const long long g = base + 32 * j + lane;
-      if (g < words) {
+    for (int q = 0; q < 4; ++q) {
+      const long long g = base + 32 * q + lane;
+      if (g < j.groups) {
         uint32_t w[4];
-        expand8_4bit(x[j], P, w);
-        __stcg(out + g, make_uint4(w[0], w[1], w[2], w[3]));
+        expand8_4bit(x[q], P, w);
+        __stcg(j.out + g, make_uint4(w[0], w[1], w[2], w[3]));
       }
     }
   }
 }
 
+// Widths that divide 8 bits (1, 2, 8): one thread per group, the group read
+// as one 16-, 8- or 64-bit word, its 8 levels from the shared table.
 template <int BITS>
-int launch_expand(const uint8_t* codes, int rows, int K, const uint16_t* lut, uint16_t* out, cudaStream_t st,
-                  int sms) {
-  if constexpr (BITS == 4) {
-    // one 32-bit word of codes = 8 fp16 levels = one 16-byte output chunk
-    const long long words = static_cast<long long>(rows) * (K / 8);
-    long long blocks = (words + 1023) / 1024;               // 8 warps x 128 words
-    if (blocks > 16LL * sms) blocks = 16LL * sms;
-    expand_weights_kernel4<<<static_cast<int>(blocks), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes),
-                                                                      words, lut, reinterpret_cast<uint4*>(out));
-  } else if constexpr (8 % BITS == 0) {
-    const long long groups = static_cast<long long>(rows) * (K / 8);
-    long long blocks = (groups + 255) / 256;
-    if (blocks > 16LL * sms) blocks = 16LL * sms;
-    expand_weights_kernel8<BITS><<<static_cast<int>(blocks), 256, 0, st>>>(codes, groups, lut, out);
-  } else {
-    const long long items = static_cast<long long>(rows) * (K / kBK);
-    long long blocks = (items + 255) / 256;
-    if (blocks > 8LL * sms) blocks = 8LL * sms;
-    expand_weights_kernel<BITS><<<static_cast<int>(blocks), 256, 0, st>>>(codes, rows, K, lut, out);
+__device__ __forceinline__ void expand_job_div8(const ExpandJob& j, const uint16_t* lut, int jb) {
+  for (long long g = jb * static_cast<long long>(blockDim.x) + threadIdx.x; g < j.groups;
+       g += static_cast<long long>(j.blocks) * blockDim.x) {
+    uint64_t x;
+    if constexpr (BITS == 8) x = __ldcs(reinterpret_cast<const unsigned long long*>(j.codes) + g);
+    else if constexpr (BITS == 2) x = __ldcs(reinterpret_cast<const unsigned short*>(j.codes) + g);
+    else x = j.codes[g];
+    constexpr uint32_t mask = (1u << BITS) - 1u;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w[q] = static_cast<uint32_t>(lut[(x >> (2 * q * BITS)) & mask]) |
+             (static_cast<uint32_t>(lut[(x >> ((2 * q + 1) * BITS)) & mask]) << 16);
+    __stcg(j.out + g, make_uint4(w[0], w[1], w[2], w[3]));
   }
-  const cudaError_t e = cudaGetLastError();
+}
+
+// Widths that do not divide 8 bits (3, 5, 6, 7): one thread per group.  A
+// warp's 32 groups are 32*BITS contiguous bytes, loaded as words by the warp
+// into its shared buffer `wb` (so the loads are contiguous too) and read back
+// by each lane as the 64-bit window that holds its group.
+template <int BITS>
+__device__ __forceinline__ void expand_job_groups(const ExpandJob& j, const uint16_t* lut, uint32_t* wb, int jb) {
+  constexpr int kWords = 8 * BITS;                     // words of a warp's 32 groups
+  const uint32_t* codes = reinterpret_cast<const uint32_t*>(j.codes);
+  const int lane = threadIdx.x & 31;
+  const long long total_words = j.groups * BITS / 4;   // groups % 16 == 0 (K % 128 == 0)
+  const long long warps = static_cast<long long>(j.blocks) * (blockDim.x >> 5);
+  for (long long g0 = (jb * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5)) * 32; g0 < j.groups;
+       g0 += 32 * warps) {
+    const long long w0 = g0 * BITS / 4;                // g0 % 32 == 0: a whole word
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < (kWords + 31) / 32; ++q) {
+      const int i = 32 * q + lane;
+      if (i < kWords) wb[i] = (w0 + i < total_words) ? __ldcs(codes + w0 + i) : 0u;
+    }
+    __syncwarp();
+    const long long g = g0 + lane;
+    if (g < j.groups) {
+      // bytes [lane*BITS, lane*BITS + BITS) of the buffer; word wi + 2 only
+      // feeds bits above the group's 8*BITS (the buffer has 2 spare words)
+      const int byte = lane * BITS, wi = byte >> 2, sh = 8 * (byte & 3);
+      const uint64_t lo = (static_cast<uint64_t>(wb[wi + 1]) << 32) | wb[wi];
+      const uint64_t v = sh ? (lo >> sh) | (static_cast<uint64_t>(wb[wi + 2]) << (64 - sh)) : lo;
+      constexpr uint32_t mask = (1u << BITS) - 1u;
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o[q] = static_cast<uint32_t>(lut[(v >> (2 * q * BITS)) & mask]) |
+               (static_cast<uint32_t>(lut[(v >> ((2 * q + 1) * BITS)) & mask]) << 16);
+      __stcg(j.out + g, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+}
+
+// Blocks [0, j0.blocks) run job 0, the rest job 1 (j1.blocks may be 0).
+__global__ void __launch_bounds__(256) expand_codes_kernel(const ExpandJob j0, const ExpandJob j1) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ uint16_t lut[256];
+  __shared__ uint32_t buf[8][64 + 2];                  // per warp (expand_job_groups)
+  const bool second = static_cast<int>(blockIdx.x) >= j0.blocks;
+  const ExpandJob j = second ? j1 : j0;
+  const int jb = second ? static_cast<int>(blockIdx.x) - j0.blocks : static_cast<int>(blockIdx.x);
+  if (j.bits == 4) {                                   // block-uniform
+    expand_job4(j, jb);
+    return;
+  }
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) lut[i] = (i < (1 << j.bits)) ? j.lut[i] : 0;
+  __syncthreads();
+  uint32_t* wb = buf[threadIdx.x >> 5];
+  switch (j.bits) {
+    case 1: expand_job_div8<1>(j, lut, jb); break;
+    case 2: expand_job_div8<2>(j, lut, jb); break;
+    case 3: expand_job_groups<3>(j, lut, wb, jb); break;
+    case 5: expand_job_groups<5>(j, lut, wb, jb); break;
+    case 6: expand_job_groups<6>(j, lut, wb, jb); break;
+    case 7: expand_job_groups<7>(j, lut, wb, jb); break;
+    default: expand_job_div8<8>(j, lut, jb); break;
+  }
+}
+
+// ---- host side ------------------------------------------------------------
+
+// The job that expands `rows` rows of K codes of `bits` bits (K % 128 == 0).
+ExpandJob expand_job(const uint8_t* codes, int bits, int rows, int K, const uint16_t* lut, uint16_t* out, int sms) {
+  ExpandJob j{};
+  j.codes = codes;
+  j.groups = static_cast<long long>(rows) * (K / 8);
+  j.lut = lut;
+  j.out = reinterpret_cast<uint4*>(out);
+  j.bits = bits;
+  // 4-bit: 8 warps x 128 groups per block step; other widths 256 groups
+  long long blocks = bits == 4 ? (j.groups + 1023) / 1024 : (j.groups + 255) / 256;
+  if (blocks > 16LL * sms) blocks = 16LL * sms;
+  j.blocks = static_cast<int>(blocks);
+  return j;
+}
+
+// Launch with programmatic dependent launch allowed: the kernel waits
+// (griddep_wait) for the launch before it before touching memory, so only its
+// launch latency overlaps that launch's tail, and the GEMM after it waits for
+// it the same way.
+int launch_expand(const ExpandJob& j0, const ExpandJob& j1, cudaStream_t st) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(j0.blocks + j1.blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, expand_codes_kernel, j0, j1);
+  if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }
 
 int expand_weights(const uint8_t* codes, int bits, int rows, int K, const uint16_t* lut, uint16_t* out,
                    cudaStream_t st, int sms) {
-  switch (bits) {
-    case 1: return launch_expand<1>(codes, rows, K, lut, out, st, sms);
-    case 2: return launch_expand<2>(codes, rows, K, lut, out, st, sms);
-    case 3: return launch_expand<3>(codes, rows, K, lut, out, st, sms);
-    case 4: return launch_expand<4>(codes, rows, K, lut, out, st, sms);
-    case 5: return launch_expand<5>(codes, rows, K, lut, out, st, sms);
-    case 6: return launch_expand<6>(codes, rows, K, lut, out, st, sms);
-    case 7: return launch_expand<7>(codes, rows, K, lut, out, st, sms);
-    default: return launch_expand<8>(codes, rows, K, lut, out, st, sms);
-  }
+  ExpandJob none{};
+  return launch_expand(expand_job(codes, bits, rows, K, lut, out, sms), none, st);
+}
+
+// Weights and activations of one call in one launch.
+int expand_both(const uint8_t* w_codes, int bits_w, int N, const uint16_t* lut_w, uint16_t* wf16,
+                const uint8_t* a_codes, int bits_a, int M, const uint16_t* lut_a, uint16_t* af16, int K,
+                cudaStream_t st, int sms) {
+  return launch_expand(expand_job(w_codes, bits_w, N, K, lut_w, wf16, sms),
+                       expand_job(a_codes, bits_a, M, K, lut_a, af16, sms), st);
 }
 
 // A memory pool per device for the stream-ordered weight workspace; it keeps
@@ -798,24 +842,25 @@ int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, cons
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaMemPool_t pool = qfast::workspace_pool(dev);
   if (!pool) return RBQ_ECUDA;
-  // 4-bit activation codes are expanded inside the GEMM by byte permutes at
-  // no cost to it; other widths cost the expansion warps more than the tensor
-  // core, so they get their own pass into fp16 and a GEMM that streams both
-  // operands by TMA -- while that fp16 copy (M*K*2 bytes) is at most 128 MiB,
-  // beyond which writing and re-reading it costs more than it saves.
+  // The activation codes get their own pass into fp16 and the GEMM streams
+  // both operands by TMA on CTA pairs -- while that fp16 copy (M*K*2 bytes)
+  // is at most 128 MiB, beyond which writing and re-reading it costs more than
+  // it saves; larger activations are expanded inside the GEMM (qlinear_fast_kernel).
   const size_t a_f16_bytes = static_cast<size_t>(M) * K * 2;
-  const bool split = bits_a != 4 && a_f16_bytes <= (static_cast<size_t>(128) << 20);
+  const bool split = a_f16_bytes <= (static_cast<size_t>(128) << 20);
   void* ws = nullptr;
   e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K * 2 + (split ? a_f16_bytes : 0), pool, st);
   if (e != cudaSuccess) return cuda_fail(e);
   uint16_t* wf16 = static_cast<uint16_t*>(ws);
-  int rc = qfast::expand_weights(w_codes, bits_w, N, K, cw->levels_f16, wf16, st, sms);
+  int rc = RBQ_OK;
   if (split) {
     uint16_t* af16 = wf16 + static_cast<size_t>(N) * K;
-    if (rc == RBQ_OK) rc = qfast::expand_weights(a_codes, bits_a, M, K, ca->levels_f16, af16, st, sms);
+    rc = qfast::expand_both(w_codes, bits_w, N, cw->levels_f16, wf16, a_codes, bits_a, M, ca->levels_f16, af16, K,
+                            st, sms);
     if (rc == RBQ_OK) rc = qlinear_f16_operands_gemm(af16, s, wf16, rnorm, ca->inv_d, M, N, K, Y, err, st, sms);
-  } else if (rc == RBQ_OK) {
-    rc = qlinear_fast_gemm(a_codes, s, bits_a, wf16, rnorm, M, N, K, Y, ca, err, st, sms);
+  } else {
+    rc = qfast::expand_weights(w_codes, bits_w, N, K, cw->levels_f16, wf16, st, sms);
+    if (rc == RBQ_OK) rc = qlinear_fast_gemm(a_codes, s, bits_a, wf16, rnorm, M, N, K, Y, ca, err, st, sms);
   }
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);

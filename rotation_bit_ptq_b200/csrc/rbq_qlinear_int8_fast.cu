@@ -9,15 +9,20 @@
 // 1. widen_int8_kernel: q [N, K] int8 -> bf16 [N, K] in a stream-ordered
 //    workspace.  Integers up to 127 are exact in bf16, so the tensor core sees
 //    the same values; an HBM pass over 3 N K bytes.
-// 2. qlinear_bf16_kernel: persistent tcgen05 GEMM, one CTA per SM, 128 x 256
-//    output tiles, K slices of 64.
-//      warps 0..3  epilogue: TMEM lane quadrant w, one output row per thread;
-//                  multiply by scale[n], round to BF16, store.
-//      warp 4      MMA issuer: one thread, four 128x256x16 kind::f16 (bf16)
-//                  MMAs per slice from shared memory, one commit per slice.
-//      warp 5      TMA producer: x' tile (128 x 64) and weight tile
-//                  (256 x 64) of each slice into a 4-stage ring, both
-//                  128B-swizzled K-major.
+// 2. qlinear_bf16_kernel: persistent tcgen05 GEMM, K slices of 64, on CTA
+//    pairs (256 x 256 output tiles, cta_group::2) when there is more than one
+//    128-row tile of rows, else one CTA per SM (128 x 256 tiles).
+//      warps 0..3  epilogue: TMEM lane quadrant w, one output row of this
+//                  CTA's 128 per thread; multiply by scale[n], round to BF16,
+//                  store.
+//      warp 4      MMA issuer (the even CTA's, for a pair): one thread, four
+//                  kind::f16 (bf16) MMAs per slice from shared memory, one
+//                  commit per slice (to both CTAs' stage barriers).
+//      warp 5      TMA producer: this CTA's x' tile (128 x 64) and its part
+//                  of the weight tile (256 x 64, or 128 x 64 for a pair) of
+//                  each slice into the ring (4 stages of 48 KB, or 6 of 32
+//                  KB), both 128B-swizzled K-major.  No multicast: a pair's
+//                  weight tile is split between the two CTAs, not copied.
 //    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
 //    overlap the MMAs of tile i+1.
 //    Fused with the next layer's rotation (qlinear_int8_rotate_next, see
@@ -46,10 +51,27 @@ using qfast::workspace_pool;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kATile = kBM * kBK * 2;          // 16 KB
-constexpr int kBTile = kBN * kBK * 2;          // 32 KB
-constexpr int kStage = kATile + kBTile;        // 48 KB
-constexpr int kStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
+
+// Tile geometry.  Single-SM tiles are 128 x 256: the CTA holds the whole
+// 256 x 64 weight tile of each K slice (4 stages of 48 KB).  CTA-pair tiles
+// are 256 x 256: one thread of the even CTA issues each MMA for both SMs
+// (cta_group::2, M = 256), each CTA holds its own 128 rows of x' and 128 of
+// the 256 weight rows (6 stages of 32 KB), and each CTA's tensor memory
+// receives its own 128 output rows.  The pair does the same MMA work per SM
+// with a third fewer operand bytes arriving per K slice, and the freed shared
+// memory deepens the ring.
+template <bool PAIR>
+struct Geom {
+  static constexpr int kTileM = PAIR ? 2 * kBM : kBM;     // output rows per tile
+  static constexpr int kBNc = PAIR ? kBN / 2 : kBN;       // weight rows loaded per CTA
+  static constexpr int kBTile = kBNc * kBK * 2;           // 16 KB / 32 KB
+  static constexpr int kStage = kATile + kBTile;          // 32 KB / 48 KB
+  static constexpr int kStages = PAIR ? 6 : 4;
+};
+static_assert(Geom<true>::kStages * Geom<true>::kStage == Geom<false>::kStages * Geom<false>::kStage,
+              "both geometries use the same shared memory");
 
 // Epilogue kinds.
 enum Epi {
@@ -137,8 +159,8 @@ __device__ __forceinline__ void fwht64_pairs(unsigned long long (&P)[32]) {
 }
 
 struct __align__(8) Tail {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;                // abort path only: completion of the MMAs issued
@@ -146,7 +168,7 @@ struct __align__(8) Tail {
   volatile uint32_t abort;
 };
 
-constexpr size_t kSmem = 1024 + kStages * kStage + sizeof(Tail) + 64;
+constexpr size_t kSmem = 1024 + Geom<false>::kStages * Geom<false>::kStage + sizeof(Tail) + 64;
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Tail* tl) {
   return mbar_wait_or_abort(bar, parity, &tl->abort);
@@ -160,40 +182,58 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Tail* 
 // epilogue x s[m] r'[n] / K; kEpiRotateNext: the W8A16 layer whose weight rows
 // come in the order of the next layer's permutation, its epilogue applying the
 // activation and the next layer's signs and 64-point Hadamard blocks.
-template <int EPI>
+// PAIR: the kernel runs on clusters of two CTAs (see Geom).
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(threads_for(EPI), 1)
     qlinear_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const Params p) {
+  using G = Geom<PAIR>;
+  constexpr int kS = G::kStages;
   constexpr bool kQ = (EPI == kEpiCodes);
   constexpr bool kRot = (EPI >= kEpiRotateNext);
+  constexpr uint32_t kEpiWarps = epi_threads_for(EPI) / 32;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  Tail* tl = reinterpret_cast<Tail*>(ops + kStages * kStage);
+  Tail* tl = reinterpret_cast<Tail*>(ops + kS * G::kStage);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ntiles_m = (p.M + kBM - 1) / kBM, ntiles_n = (p.N + kBN - 1) / kBN;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;       // CTA within the pair
+  const int tile0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int tstep = PAIR ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+  const int ntiles_m = (p.M + G::kTileM - 1) / G::kTileM, ntiles_n = (p.N + kBN - 1) / kBN;
   const int ntiles = ntiles_m * ntiles_n;
   const int KT = p.K / kBK;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(&tl->full[s], 1);
       mbar_init(&tl->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tl->acc_full[a], 1);
-      mbar_init(&tl->acc_empty[a], epi_threads_for(EPI));
+      // one arrival per epilogue warp (of both CTAs for a pair: the even CTA's
+      // MMA thread waits for both halves of the accumulator to be drained)
+      mbar_init(&tl->acc_empty[a], (PAIR ? 2u : 1u) * kEpiWarps);
     }
     mbar_init(&tl->drain, 1);
     tl->abort = 0u;
     mbar_fence_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&tl->tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&tl->tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&tl->tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // A pair's barriers are signalled from both CTAs: both must be initialised.
+  if constexpr (PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tl->tmem_slot;
   // The prologue above reads only constant tables; the operands (written by
@@ -202,49 +242,78 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
   griddep_launch_dependents();
 
   if (warp == kMmaWarp) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t kIdesc = idesc_f16(kBM, kBN, !kQ);
+    // ---------------- MMA issuer (the even CTA's, for a pair) ----------------
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdesc = idesc_f16(G::kTileM, kBN, !kQ);
       const uint64_t desc0 = sdesc_k_sw128(smem_u32(ops));
       uint32_t s = 0, ph = 0, it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++it) {
         const uint32_t a = it & 1u, use = it >> 1;
-        if (use >= 1 && !wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, tl)) { ok = false; break; }
+        if (use >= 1) {
+          const bool got = PAIR ? mbar_wait_or_abort_cl(&tl->acc_empty[a], (use - 1) & 1, &tl->abort)
+                                : wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, tl);
+          if (!got) { ok = false; break; }
+        }
         tc_fence_after();
         const uint32_t acc = tmem + a * kBN;
         for (int kb = 0; kb < KT; ++kb) {
           if (!wait_or_abort(&tl->full[s], ph, tl)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(kStage)) >> 4);
+          const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(G::kStage)) >> 4);
           const uint64_t bd = ad + (kATile >> 4);
-          umma_f16(acc, ad, bd, kIdesc, kb != 0);
-          umma_f16(acc, ad + 2, bd + 2, kIdesc, 1u);           // +32 bytes of K per step
-          umma_f16(acc, ad + 4, bd + 4, kIdesc, 1u);
-          umma_f16(acc, ad + 6, bd + 6, kIdesc, 1u);
-          umma_commit(&tl->empty[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; }
+          if constexpr (PAIR) {
+            umma_f16_pair(acc, ad, bd, kIdesc, kb != 0);
+            umma_f16_pair(acc, ad + 2, bd + 2, kIdesc, 1u);      // +32 bytes of K per step
+            umma_f16_pair(acc, ad + 4, bd + 4, kIdesc, 1u);
+            umma_f16_pair(acc, ad + 6, bd + 6, kIdesc, 1u);
+            umma_commit_pair(&tl->empty[s], 3);                  // stage s of both CTAs
+          } else {
+            umma_f16(acc, ad, bd, kIdesc, kb != 0);
+            umma_f16(acc, ad + 2, bd + 2, kIdesc, 1u);
+            umma_f16(acc, ad + 4, bd + 4, kIdesc, 1u);
+            umma_f16(acc, ad + 6, bd + 6, kIdesc, 1u);
+            umma_commit(&tl->empty[s]);
+          }
+          if (++s == kS) { s = 0; ph ^= 1u; }
         }
-        if (ok) umma_commit(&tl->acc_full[a]);
+        if (ok) {
+          if constexpr (PAIR)
+            umma_commit_pair(&tl->acc_full[a], 3);
+          else
+            umma_commit(&tl->acc_full[a]);
+        }
       }
       if (!ok) atomicOr(p.err, 2u);
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA producer ----------------
+    // For a pair each CTA loads its own 128 rows of x' and its half of the
+    // weight rows; both CTAs' bytes are counted on the even CTA's barrier,
+    // which only the even CTA's producer arms.
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       uint32_t s = 0, ph = 0;
       bool first = true, ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
         const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+        const int m0 = mt * G::kTileM + static_cast<int>(rank) * kBM;
+        const int n0 = nt * kBN + static_cast<int>(rank) * G::kBNc;
         for (int kb = 0; kb < KT; ++kb) {
           if (!first && !wait_or_abort(&tl->empty[s], ph ^ 1u, tl)) { ok = false; break; }
-          uint8_t* st = ops + s * kStage;
-          mbar_arrive_expect_tx(&tl->full[s], kStage);
-          tma_load_2d(st, &tmA, kb * kBK, mt * kBM, &tl->full[s]);
-          tma_load_2d(st + kATile, &tmB, kb * kBK, nt * kBN, &tl->full[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; first = false; }
+          uint8_t* st = ops + s * G::kStage;
+          if constexpr (PAIR) {
+            if (rank == 0) mbar_arrive_expect_tx(&tl->full[s], 2 * G::kStage);
+            const uint32_t bar = mapa_shared(&tl->full[s], 0);
+            tma_load_2d_pair(st, &tmA, kb * kBK, m0, bar);
+            tma_load_2d_pair(st + kATile, &tmB, kb * kBK, n0, bar);
+          } else {
+            mbar_arrive_expect_tx(&tl->full[s], G::kStage);
+            tma_load_2d(st, &tmA, kb * kBK, m0, &tl->full[s]);
+            tma_load_2d(st + kATile, &tmB, kb * kBK, n0, &tl->full[s]);
+          }
+          if (++s == kS) { s = 0; ph ^= 1u; first = false; }
         }
       }
       if (!ok) atomicOr(p.err, 16u);
@@ -252,10 +321,21 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
   } else {
     // ---------------- epilogue ----------------
     const int q = warp & 3;                 // TMEM lane quadrant (warps 6..9: 2, 3, 0, 1)
-    const int r = 32 * q + lane;            // row within the tile
+    const int r = 32 * q + lane;            // row within this CTA's 128 rows of the tile
     const int eg = warp < 4 ? 0 : 1;        // rotating epilogues: which two of the four blocks
+    // Accumulator drained: one arrival per warp, on the even CTA's barrier.
+    auto release_acc = [&](uint32_t a) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(&tl->acc_empty[a], 0));
+        else
+          mbar_arrive(&tl->acc_empty[a]);
+      }
+    };
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    for (int tile = tile0; tile < ntiles; tile += tstep, ++it) {
       const uint32_t a = it & 1u, use = it >> 1;
       if (!warp_wait(&tl->acc_full[a], use & 1, tl)) {
         if (lane == 0) atomicOr(p.err, 4u);
@@ -263,7 +343,7 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
       }
       tc_fence_after();
       const int mt = tile % ntiles_m, nt = tile / ntiles_m;
-      const int m = mt * kBM + r;
+      const int m = mt * G::kTileM + static_cast<int>(rank) * kBM + r;
       if constexpr (kRot) {
         // The tile's 256 columns are four whole blocks of the next layer's
         // rotation (N % 64 == 0, tiles start at multiples of 256): column k is
@@ -310,8 +390,7 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
             }
           }
         }
-        tc_fence_before();
-        mbar_arrive(&tl->acc_empty[a]);
+        release_acc(a);
         continue;
       }
       const float rs = kQ ? ((m < p.M) ? p.s[m] * p.inv_k : 0.f) : 1.f;
@@ -352,20 +431,25 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
             }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tl->acc_empty[a]);
+      release_acc(a);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (tl->abort) {                 // the same value in every thread after the barrier
-    drain_after_abort(warp == kMmaWarp && lane == 0, &tl->drain);
+    drain_after_abort(warp == kMmaWarp && lane == 0 && rank == 0, &tl->drain, PAIR);
     __syncthreads();
   }
+  // Neither CTA of a pair leaves while the other may still signal its
+  // barriers or the MMAs may still read its shared memory.
+  if constexpr (PAIR) cluster_sync();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
@@ -435,29 +519,82 @@ int encode_bf16_map(CUtensorMap* map, const uint16_t* base, int rows, int K, int
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
 }
 
-// Launches the GEMM on two fp16/bf16 operands already in memory (K % 64 == 0).
+// Resident clusters of two for the pair kernel on device `dev` (0: none
+// could be co-scheduled), queried once per device.
+template <int EPI>
+int pair_clusters(int dev) {
+  static int cached[kMaxDevices] = {};        // 0 = not yet asked; else clusters + 1
+  if (cached[dev]) return cached[dev] - 1;
+  auto kern = qlinear_bf16_kernel<EPI, true>;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(threads_for(EPI), 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached[dev] = n + 1;
+  return n;
+}
+
+// Launches the GEMM on two fp16/bf16 operands already in memory (K % 64 == 0):
+// on CTA pairs (256 x 256 tiles) when there is more than one 128-row tile of
+// rows and the device can co-schedule pairs, else on single SMs.
 template <int EPI>
 int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStream_t st, int sms) {
   constexpr bool kQ = (EPI == kEpiCodes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return RBQ_EINVAL;
+  bool pair = p.M > kBM;
+  if (pair) {
+    e = cudaFuncSetAttribute(qlinear_bf16_kernel<EPI, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem));
+    if (e != cudaSuccess) return cuda_fail(e);
+    pair = pair_clusters<EPI>(dev) >= 1;
+  }
+  const int tile_m = pair ? Geom<true>::kTileM : Geom<false>::kTileM;
   CUtensorMap mA, mB;
   int rc = encode_bf16_map(&mA, A, p.M, p.K, kBM, kQ);
-  if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, kBN, kQ);
+  if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, pair ? Geom<true>::kBNc : Geom<false>::kBNc, kQ);
   if (rc != RBQ_OK) return rc;
-  auto kern = qlinear_bf16_kernel<EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
-  if (e != cudaSuccess) return cuda_fail(e);
-  const int ntiles = ((p.M + kBM - 1) / kBM) * ((p.N + kBN - 1) / kBN);
+  const int ntiles = ((p.M + tile_m - 1) / tile_m) * ((p.N + kBN - 1) / kBN);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
   cfg.blockDim = dim3(threads_for(EPI), 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+  if (pair) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    int clusters = pair_clusters<EPI>(dev);           // persistent: as many pairs as are resident at once
+    if (clusters > ntiles) clusters = ntiles;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, qlinear_bf16_kernel<EPI, true>, mA, mB, p);
+  } else {
+    auto kern = qlinear_bf16_kernel<EPI, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    if (e != cudaSuccess) return cuda_fail(e);
+    cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }

@@ -1,4 +1,4 @@
-// Rotate-then-quantise for BF16 rows of width 1024..3072 (d a multiple of
+// Rotate-then-quantise for BF16 rows of width 1024..16384 (d a multiple of
 // 256): the token-pair kernel.
 //
 //   OrbitQuant (hotelren.com/news/3376620) §2.2 / §2.1: x' = Pi_d x, s = ||x'||,
@@ -7,15 +7,19 @@
 //   §4: rotate, scale = max|w'|/127, round.  Rotate-only: x' in BF16.
 //   Pi_d = blkdiag(H_64 D_1, ..., H_64 D_{d/64}) · P_pi (OrbitQuant §2.3).
 //
-// Work unit: a tile of 16 token rows.  Thread (p, b) owns output block b of
-// the token pair (p, p+8), p = 0..7, holding the pair's values as packed
-// fp32x2 registers, so every butterfly stage is one packed add/sub per pair.
+// Work unit: a tile of R = 2P token rows, P = 8 pairs for d <= 3072 and 4, 2
+// or 1 for wider rows (whatever keeps two ring slots in shared memory).
+// Thread (p, b) owns output block b of the token pair (p, p+P), p < P,
+// holding the pair's values as packed fp32x2 registers, so every butterfly
+// stage is one packed add/sub per pair.
 // It gathers and transforms one 32-position half-block at a time (strides
 // 1..16), parks both halves in its own lane of tensor memory, and runs the
 // last stage (stride 32) inside the encoding loop as it reads them back; the
-// smaller live register set leaves room for many loads in flight.  A warp covers 8 pairs x 4 blocks; the 8 lanes that share
-// a block read the same source position of 8 different rows, which a 16-byte
-// row padding puts in 8 different banks.
+// smaller live register set leaves room for many loads in flight.  A warp
+// covers P pairs x 32/P blocks; the P lanes that share a block read the same
+// source position of P different rows, which a 16-byte row padding puts in P
+// different banks.  Threads whose block is past d/64 (when 32/P does not
+// divide the block count) only join the warp's collective steps.
 //
 // Data movement: whole rows arrive by bulk asynchronous copies (TMA, no
 // tensor map needed for contiguous rows), one row per lane of an issuing
@@ -84,13 +88,14 @@ __device__ __forceinline__ void encode_block(const Enc& enc, uint32_t tA, uint32
   }
 }
 
-template <int MODE, int BITS>
+template <int MODE, int BITS, int P>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) {
+  constexpr int kTR = 2 * P;                       // rows per tile
   extern __shared__ unsigned char smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 127u) & ~127u;
   unsigned char* sm = smem_raw + (sbase - sraw);
-  const Layout L = layout(p.d, p.NS, p.grid_entries);
+  const Layout L = layout(p.d, p.NS, p.grid_entries, kTR);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* red = full + p.NS;
   uint64_t* tabbar = red + 2 * p.NS;
@@ -100,7 +105,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   const int NS = p.NS;
 
   const uint32_t pitch = p.pitch;
-  const uint32_t slot_bytes = kRows * pitch;
+  const uint32_t slot_bytes = kTR * pitch;
   const uint32_t ring = sbase + L.ring;
 
   // The bulk copies of tile `tile` into slot `slot`, shared out over the
@@ -111,8 +116,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   int n_issued = 0;
   auto issue_rows = [&](int tile, int slot) {
     const uint32_t row_bytes = 2u * static_cast<uint32_t>(p.d);
-    const long long r0 = static_cast<long long>(tile) * kRows;
-    const int rows = static_cast<int>(min(static_cast<long long>(kRows), p.T - r0));
+    const long long r0 = static_cast<long long>(tile) * kTR;
+    const int rows = static_cast<int>(min(static_cast<long long>(kTR), p.T - r0));
     ++n_issued;
     if (tid == 0) mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(rows) * row_bytes);
     for (int r = warp + p.nwarps * lane; r < rows; r += 32 * p.nwarps) {
@@ -137,7 +142,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   }
   {
     float* part = reinterpret_cast<float*>(sm + L.part);
-    for (int i = tid; i < (2 * NS) * kRows * kMaxWarps; i += blockDim.x) part[i] = 0.f;
+    for (int i = tid; i < (2 * NS) * kTR * kMaxWarps; i += blockDim.x) part[i] = 0.f;
   }
   __syncwarp();
   if (warp == 0) {
@@ -157,13 +162,16 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   if (!mbar_wait(tabbar, 0)) atomicOr(p.err, 256u);
 
   // ---------------- consumers ----------------
-  const int j = lane >> 3, pp = lane & 7;          // lane = 8 j + p
-  const int b = 4 * warp + j;                      // output block of this thread
+  const int j = lane / P, pp = lane % P;           // lane = P j + p
+  const int b = (32 / P) * warp + j;               // output block of this thread
+  // With 8 pairs the host keeps d % 256 == 0, so every block is a whole
+  // warp's; otherwise the last warp may hold lanes past the last block.
+  const bool act = (P == 8) || b < p.nblk;
   const int bx = b & 7;
-  const uint32_t off_addr = sbase + L.off + 256u * b;
+  const uint32_t off_addr = sbase + L.off + 256u * (act ? b : 0);
   const uint32_t part_addr = sbase + L.part;
   const uint32_t gbase = sbase + L.grid + 8u * static_cast<uint32_t>(p.grid_first) - 0x4B000000u * 8u;
-  const uint32_t pitch8 = 8u * pitch;
+  const uint32_t pitchP = static_cast<uint32_t>(P) * pitch;   // token p to token p + P
   // Tensor memory: each thread parks its pair's two half-blocks (2 x 64 words)
   // in its own lane; warps w, w+4, w+8 share a lane quarter, 128 columns each.
   const uint32_t tA = *tmem_slot + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 128u * (warp >> 2);
@@ -178,42 +186,48 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       for (int s2 = 1; s2 < NS; ++s2)
         if (blockIdx.x + s2 * static_cast<int>(gridDim.x) < p.ntiles) issue_rows(blockIdx.x + s2 * gridDim.x, s2);
 
-    // ---- gather x[pi(k)] with D_k folded in (tokens p, p+8), one half-block
+    // ---- gather x[pi(k)] with D_k folded in (tokens p, p+P), one half-block
     //      at a time; butterfly strides 1..16 inside each half; park in TMEM ----
     const uint32_t rowA = ring + s * slot_bytes + pp * pitch;
     unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       unsigned long long R[32];
+      if (act) {
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const uint32_t c = 16u * (static_cast<uint32_t>(8 * h + q4) ^ static_cast<uint32_t>(bx));
-        const uint4 o = lds128(off_addr + c);
-        const uint32_t oo[4] = {o.x, o.y, o.z, o.w};
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const uint32_t c = 16u * (static_cast<uint32_t>(8 * h + q4) ^ static_cast<uint32_t>(bx));
+          const uint4 o = lds128(off_addr + c);
+          const uint32_t oo[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          // entry = source byte offset | sign << 31: the sign word S feeds the
-          // conversion, the entry minus S is the offset
-          const uint32_t S = oo[e] & 0x80000000u;
-          const uint32_t a = rowA + dbg_index(oo[e] - S, 2u * static_cast<uint32_t>(p.d), p.err);
-          const float y0 = bf16_signed(lds_u16(a), S);
-          const float y1 = bf16_signed(lds_u16(a + pitch8), S);
-          R[4 * q4 + e] = pk(y0, y1);
-          acc[e] = fma2(R[4 * q4 + e], R[4 * q4 + e], acc[e]);
+          for (int e = 0; e < 4; ++e) {
+            // entry = source byte offset | sign << 31: the sign word S feeds the
+            // conversion, the entry minus S is the offset
+            const uint32_t S = oo[e] & 0x80000000u;
+            const uint32_t a = rowA + dbg_index(oo[e] - S, 2u * static_cast<uint32_t>(p.d), p.err);
+            const float y0 = bf16_signed(lds_u16(a), S);
+            const float y1 = bf16_signed(lds_u16(a + pitchP), S);
+            R[4 * q4 + e] = pk(y0, y1);
+            acc[e] = fma2(R[4 * q4 + e], R[4 * q4 + e], acc[e]);
+          }
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) R[i] = 0ull;      // a lane past the last block: zeros
       }
       if (h == 1) {
         if constexpr (MODE != kInt8) {
-          // ||x||^2 partials of both tokens (||Pi x|| = ||x||): 4 lanes share a pair
+          // ||x||^2 partials of both tokens (||Pi x|| = ||x||): 32/P lanes share a pair
           float a0, a1;
           upk(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), a0, a1);
-          a0 += __shfl_xor_sync(0xffffffffu, a0, 8);
-          a1 += __shfl_xor_sync(0xffffffffu, a1, 8);
-          a0 += __shfl_xor_sync(0xffffffffu, a0, 16);
-          a1 += __shfl_xor_sync(0xffffffffu, a1, 16);
+#pragma unroll
+          for (int o = P; o < 32; o <<= 1) {
+            a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+          }
           if (j == 0) {
-            sts_f32(part_addr + 4u * ((rb * kRows + pp) * kMaxWarps + warp), a0);
-            sts_f32(part_addr + 4u * ((rb * kRows + pp + 8) * kMaxWarps + warp), a1);
+            sts_f32(part_addr + 4u * ((rb * kTR + pp) * kMaxWarps + warp), a0);
+            sts_f32(part_addr + 4u * ((rb * kTR + pp + P) * kMaxWarps + warp), a1);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&red[rb]);
@@ -262,13 +276,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
           m1 = fmaxf(m1, fmaxf(fabsf(z1), fabsf(y1)));
         }
       }
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 8));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 8));
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 16));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 16));
+#pragma unroll
+      for (int o = P; o < 32; o <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
       if (j == 0) {
-        sts_f32(part_addr + 4u * ((rb * kRows + pp) * kMaxWarps + warp), m0);
-        sts_f32(part_addr + 4u * ((rb * kRows + pp + 8) * kMaxWarps + warp), m1);
+        sts_f32(part_addr + 4u * ((rb * kTR + pp) * kMaxWarps + warp), m0);
+        sts_f32(part_addr + 4u * ((rb * kTR + pp + P) * kMaxWarps + warp), m1);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&red[rb]);
@@ -283,7 +298,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     float tot[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint32_t pa = part_addr + 4u * ((rb * kRows + pp + 8 * h) * kMaxWarps);
+      const uint32_t pa = part_addr + 4u * ((rb * kTR + pp + P * h) * kMaxWarps);
       const uint4 q0 = lds128(pa), q1 = lds128(pa + 16), q2 = lds128(pa + 32);
       const float v[12] = {__uint_as_float(q0.x), __uint_as_float(q0.y), __uint_as_float(q0.z),
                            __uint_as_float(q0.w), __uint_as_float(q1.x), __uint_as_float(q1.y),
@@ -299,8 +314,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       }
     }
 
-    const long long t0 = static_cast<long long>(tile) * kRows + pp, t1 = t0 + 8;
-    const bool ok0 = t0 < p.T, ok1 = t1 < p.T;
+    const long long t0 = static_cast<long long>(tile) * kTR + pp, t1 = t0 + P;
+    const bool ok0 = act && t0 < p.T, ok1 = act && t1 < p.T;   // rows to store
 
     if constexpr (kLloyd) {
       const float s0 = sqrtf(tot[0]), s1 = sqrtf(tot[1]);      // ||x|| = ||Pi x||
@@ -434,7 +449,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   // threads may have left the loop at different tiles, this bounds the exit).
   tc_fence_before();
   __syncthreads();
-  if (warp + p.nwarps * lane < kRows) {
+  if (warp + p.nwarps * lane < kTR) {
     bool ok = true;
     for (int s = 0; s < NS; ++s) {
       const int uses = n_issued > s ? (n_issued - 1 - s) / NS + 1 : 0;
@@ -455,10 +470,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
 
 namespace {
 
-template <int MODE, int BITS>
+template <int MODE, int BITS, int P>
 int launch_pair(const pairk::Params& p, cudaStream_t st) {
-  auto kern = pairk::rotq_pair_kernel<MODE, BITS>;
-  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_entries).total + 128;
+  auto kern = pairk::rotq_pair_kernel<MODE, BITS, P>;
+  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_entries, 2 * P).total + 128;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = rowtile::sm_count();
@@ -466,24 +481,52 @@ int launch_pair(const pairk::Params& p, cudaStream_t st) {
   return rowtile::launch_pdl(kern, grid, p.nwarps * 32, smem, st, p);
 }
 
+template <int MODE, int BITS>
+int launch_pair_p(int P, const pairk::Params& p, cudaStream_t st) {
+  switch (P) {
+    case 8: return launch_pair<MODE, BITS, 8>(p, st);
+    case 4: return launch_pair<MODE, BITS, 4>(p, st);
+    case 2: return launch_pair<MODE, BITS, 2>(p, st);
+    default: return launch_pair<MODE, BITS, 1>(p, st);
+  }
+}
+
 template <int MODE>
-int launch_pair_bits(int bits, const pairk::Params& p, cudaStream_t st) {
+int launch_pair_bits(int bits, int P, const pairk::Params& p, cudaStream_t st) {
   switch (bits) {
-    case 1: return launch_pair<MODE, 1>(p, st);
-    case 2: return launch_pair<MODE, 2>(p, st);
-    case 3: return launch_pair<MODE, 3>(p, st);
-    case 4: return launch_pair<MODE, 4>(p, st);
-    case 5: return launch_pair<MODE, 5>(p, st);
-    case 6: return launch_pair<MODE, 6>(p, st);
-    case 7: return launch_pair<MODE, 7>(p, st);
-    case 8: return launch_pair<MODE, 8>(p, st);
+    case 1: return launch_pair_p<MODE, 1>(P, p, st);
+    case 2: return launch_pair_p<MODE, 2>(P, p, st);
+    case 3: return launch_pair_p<MODE, 3>(P, p, st);
+    case 4: return launch_pair_p<MODE, 4>(P, p, st);
+    case 5: return launch_pair_p<MODE, 5>(P, p, st);
+    case 6: return launch_pair_p<MODE, 6>(P, p, st);
+    case 7: return launch_pair_p<MODE, 7>(P, p, st);
+    case 8: return launch_pair_p<MODE, 8>(P, p, st);
     default: return RBQ_EINVAL;
   }
 }
 
 }  // namespace
 
-bool rotq_pair_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d % 256 == 0 && d >= 1024 && d <= 3072; }
+bool rotq_pair_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d % 256 == 0 && d >= 1024 && d <= 16384; }
+
+// Pairs per tile for width d: the most (8, 4, 2 or 1) whose CTA has at most
+// kMaxWarps warps and whose ring keeps at least two slots next to the tables;
+// 0 when none fits.  Sets the ring slots and warps.
+int pair_geometry(int d, int grid_entries, int* NS, int* nwarps) {
+  const int nblk = d / kH;
+  for (int P = 8; P >= 1; P >>= 1) {
+    const int w = (P * nblk + 31) / 32;
+    if (w > rowtile::kMaxWarps) continue;
+    const int ns = rowtile::slots_that_fit(d, grid_entries, 2 * P);
+    if (ns >= 2) {
+      *NS = ns;
+      *nwarps = w;
+      return P;
+    }
+  }
+  return 0;
+}
 
 // Returns RBQ_ECONVERGE when the tables do not fit (the caller then uses
 // another kernel); any other code is the call's result.
@@ -498,8 +541,6 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
   p.T = rows;
   p.d = r->d;
   p.nblk = r->d / kH;
-  p.nwarps = p.nblk / 4;
-  p.ntiles = static_cast<int>((rows + kRows - 1) / kRows);
   p.pitch = 2u * static_cast<uint32_t>(r->d) + 16u;
   p.tab = tab;
   p.out = out;
@@ -516,13 +557,14 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     p.grid_cells = static_cast<float>(cb->grid_cells);
     p.grid_scale = cb->grid_scale;
   }
-  p.NS = slots_that_fit(r->d, p.grid_entries);
-  if (p.NS < 2) return RBQ_ECONVERGE;
+  const int P = pair_geometry(r->d, p.grid_entries, &p.NS, &p.nwarps);
+  if (P == 0) return RBQ_ECONVERGE;
+  p.ntiles = static_cast<int>((rows + 2 * P - 1) / (2 * P));
   switch (mode) {
-    case kAct: return launch_pair_bits<kAct>(bits, p, st);
-    case kWeightLM: return launch_pair_bits<kWeightLM>(bits, p, st);
-    case kInt8: return launch_pair<kInt8, 8>(p, st);
-    default: return launch_pair<kRotate, 8>(p, st);
+    case kAct: return launch_pair_bits<kAct>(bits, P, p, st);
+    case kWeightLM: return launch_pair_bits<kWeightLM>(bits, P, p, st);
+    case kInt8: return launch_pair_p<kInt8, 8>(P, p, st);
+    default: return launch_pair_p<kRotate, 8>(P, p, st);
   }
 }
 

@@ -19,15 +19,17 @@ using namespace sm100;
 
 enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
 
-constexpr int kRows = 16;            // tokens per tile
-constexpr int kMaxWarps = 12;        // partial-sum columns per token (d <= 3072)
+// A tile holds R = 2P token rows (P token pairs): 16 rows for d <= 3072, and
+// 8, 4 or 2 rows for wider rows, so that a double-buffered ring still fits.
+constexpr int kMaxRows = 16;
+constexpr int kMaxWarps = 12;        // partial-sum columns per token (warps of the CTA)
 constexpr size_t kSmemLimit = 227 * 1024;
 
 struct Params {
   const __nv_bfloat16* X;
   long long T;
   int d, nblk, nwarps;               // warps of the CTA
-  int ntiles;                        // ceil(T / 16)
+  int ntiles;                        // ceil(T / R)
   int NS;                            // ring slots
   uint32_t pitch;                    // bytes per staged row (2d + 16)
   const uint32_t* tab;               // d words: source offset | sign << 31 (pair_tab_slot order)
@@ -46,14 +48,14 @@ struct Layout {
   uint32_t ring, off, grid, part, bars, total;
 };
 
-__host__ __device__ inline Layout layout(int d, int NS, int grid_entries) {
+__host__ __device__ inline Layout layout(int d, int NS, int grid_entries, int R) {
   Layout L{};
   const uint32_t pitch = 2u * d + 16u;
   L.ring = 0;
-  L.off = L.ring + NS * kRows * pitch;
+  L.off = L.ring + NS * R * pitch;
   L.grid = L.off + 4u * d;
   L.part = (L.grid + 8u * grid_entries + 15u) & ~15u;
-  L.bars = L.part + 4u * (2 * NS) * kRows * kMaxWarps;   // [2NS][16 tokens][12 warps]
+  L.bars = L.part + 4u * (2 * NS) * R * kMaxWarps;       // [2NS][R tokens][12 warps]
   L.bars = (L.bars + 7u) & ~7u;
   // full[NS], red[2NS], tab | TMEM base
   L.total = L.bars + 8u * (NS + 2 * NS + 1) + 8u;
@@ -226,11 +228,12 @@ inline int sm_count() {
   return n;
 }
 
-// Most ring slots that fit next to the tables (at least 2, at most 6), or 0.
-inline int slots_that_fit(int d, int grid_entries) {
+// Most ring slots of R-row tiles that fit next to the tables (at least 2, at
+// most 6), or 0.
+inline int slots_that_fit(int d, int grid_entries, int R) {
   int best = 0;
   for (int ns = 2; ns <= 6; ++ns)
-    if (layout(d, ns, grid_entries).total + 128 <= kSmemLimit) best = ns;
+    if (layout(d, ns, grid_entries, R).total + 128 <= kSmemLimit) best = ns;
   return best;
 }
 

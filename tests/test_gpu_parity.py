@@ -123,17 +123,19 @@ def test_all_bit_widths_ragged_tokens(bits, dtype):
 
 @pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_fast_path_all_bit_widths(bits):
-    # d = 1024 takes the fast kernel (4 tokens per CTA); 257 tokens leave a
-    # ragged last group
-    X, _ = synth.student_t_act(257, 1024, seed=10 + bits)
-    _act_parity(X, 1024, bits, seed=bits)
+    # d = 1088 (17 blocks, not a multiple of 256) takes the register-staged
+    # kernel (4 tokens per CTA); 257 tokens leave a ragged last group
+    X, _ = synth.student_t_act(257, 1088, seed=10 + bits)
+    _act_parity(X, 1088, bits, seed=bits)
 
 
-@pytest.mark.parametrize("d,T,bits", [(8960, 37, 3), (12288, 9, 5), (16384, 5, 7), (1024, 1, 4),
-                                      (2048, 4099, 2)])
+@pytest.mark.parametrize("d,T,bits", [(4160, 37, 3), (8896, 9, 5), (16320, 5, 7), (1088, 1, 4),
+                                      (2112, 4099, 2)])
 def test_fast_path_widths(d, T, bits):
-    # 8960 = 140 blocks: 2 tokens per CTA, 280 threads padded to 288;
-    # 16384: 1 token per CTA; 4099 tokens: many groups per CTA
+    # widths that are multiples of 64 but not of 256 take the register-staged
+    # kernel: 4160 = 65 blocks (4 tokens per CTA, padded lanes); 8896 = 139
+    # blocks (2 tokens per CTA); 16320: 1 token per CTA; 4099 tokens: many
+    # groups per CTA
     X, _ = synth.student_t_act(T, d, seed=d + T)
     rows = None if T < 600 else np.random.default_rng(0).choice(T, 64, replace=False)
     _act_parity(X, d, bits, seed=d, rows=rows)
@@ -159,9 +161,10 @@ def test_zero_and_degenerate_rows():
     assert norms[0].item() == 0.0
 
 
-@pytest.mark.parametrize("d,bits,dtype", [(3072, 4, "bf16"), (1280, 6, "bf16"),     # token-pair kernel
-                                          (4096, 5, "bf16"),                       # register-staged, [-1,1] grid
-                                          (4096, 8, "bf16"),                       # register-staged, clamped grid
+@pytest.mark.parametrize("d,bits,dtype", [(3072, 4, "bf16"), (1280, 6, "bf16"),     # token-pair kernel, 8 pairs
+                                          (4096, 5, "bf16"), (12288, 8, "bf16"),   # token-pair kernel, 4 / 1 pairs
+                                          (4160, 5, "bf16"),                       # register-staged, [-1,1] grid
+                                          (4160, 8, "bf16"),                       # register-staged, clamped grid
                                           (512, 3, "f32")])                        # general kernel
 def test_non_finite_rows_encode_as_the_zero_vector(d, bits, dtype):
     """A row holding NaN or +-Inf has no finite norm; the kernels encode it as
@@ -251,6 +254,61 @@ def test_pair_kernel_rotate_only(d):
     check_rel(nr.cpu().numpy(), np.linalg.norm(ora["xr"], axis=1), NORM_RTOL, "rotate-only norms")
 
 
+# Wider rows: tiles of 8, 4 or 2 rows (4, 2 or 1 token pairs per tile), as
+# many as keep two ring slots next to the gather table.  3328 and 8960 leave
+# the CTA's last warp with lanes past the last block; the long cases wrap the
+# ring of slots and the norm barriers several times per CTA.
+@pytest.mark.parametrize("d,T,bits", [(4096, 8 * 148 * 3 + 5, 4), (3328, 45, 6), (5120, 19, 5), (8960, 37, 2),
+                                      (8960, 4 * 148 * 2 + 3, 6), (12288, 2 * 148 * 4 + 1, 4), (16384, 19, 3),
+                                      (16384, 7, 8)])
+def test_pair_kernel_wide_rows(d, T, bits):
+    X, _ = synth.student_t_act(T, d, seed=d + bits)
+    rows = None
+    if T > 64:
+        rows = np.unique(np.concatenate([[0, 1, 7, 8, T - 1, T - 2],
+                                         np.random.default_rng(d).choice(T, 40, replace=False)]))
+    _act_parity(X, d, bits, seed=d + 1, rows=rows)
+
+
+@pytest.mark.parametrize("d,n,bits", [(4096, 21, 4), (8960, 13, 3), (16384, 9, 2)])
+def test_pair_kernel_wide_rows_weights(d, n, bits):
+    W = synth.to_bf16(synth.gaussian_weights(synth.rng(15, d), n, d, outlier_frac=0.01).astype(np.float32))
+    W[1] = 0.0
+    r, Pi = _rpbh(d, 14)
+    codes, rn = qweights(r, torch_bf16(W), bits)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    _, bounds = oracle.lloydmax_table(d, bits)
+    ora = oracle.quantize_weights_lloydmax(W.astype(np.float64), Pi, bounds)
+    check_codes(_unpack(codes, bits, d), ora["codes"], ora["v"], bounds, d)
+    check_bf16_rounding(bf16_to_numpy(rn), ora["rnorm"], "row norms")
+
+
+@pytest.mark.parametrize("d,n", [(4096, 37), (12288, 11), (8960, 5)])
+def test_pair_kernel_wide_rows_int8(d, n):
+    W = synth.to_bf16(synth.gaussian_weights(synth.rng(16, d), n, d, outlier_frac=0.01).astype(np.float32))
+    W[2] = 0.0
+    r, Pi = _rpbh(d, 15)
+    q, sc = qweights(r, torch_bf16(W), 8, mode="int8")
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.quantize_weights_int8(W.astype(np.float64), Pi)
+    check_int8(q.cpu().numpy().astype(np.int64), sc.cpu().numpy().astype(np.float64), ora)
+
+
+@pytest.mark.parametrize("d,T", [(4096, 45), (8960, 11), (16384, 6)])
+def test_pair_kernel_wide_rows_rotate_only(d, T):
+    X, _ = synth.student_t_act(T, d, seed=d)
+    r, Pi = _rpbh(d, 16)
+    nr = torch.empty((T,), dtype=torch.float32, device="cuda")
+    xr = rot_act(r, torch_bf16(X), norms=nr)
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    ora = oracle.rotate_only(X.astype(np.float64), Pi)
+    check_bf16_rounding(bf16_to_numpy(xr), ora["xr"], "rotate-only")
+    check_rel(nr.cpu().numpy(), np.linalg.norm(ora["xr"], axis=1), NORM_RTOL, "rotate-only norms")
+
+
 @pytest.mark.parametrize("d,n", [(1024, 33), (3072, 50)])
 def test_pair_kernel_weights_int8(d, n):
     W = synth.to_bf16(synth.gaussian_weights(synth.rng(12, d), n, d, outlier_frac=0.01).astype(np.float32))
@@ -264,7 +322,8 @@ def test_pair_kernel_weights_int8(d, n):
 
 
 @pytest.mark.parametrize("d,n,dtype", [(1024, 40, "bf16"), (3072, 56, "bf16"),    # token-pair kernel
-                                       (4096, 40, "bf16"),                         # register-staged kernel
+                                       (4096, 40, "bf16"),                         # token-pair kernel, 4 pairs
+                                       (4160, 40, "bf16"),                         # register-staged kernel
                                        (512, 37, "f32")])                          # general kernel
 def test_weights_int8_per_tensor(d, n, dtype):
     W = synth.to_bf16(synth.gaussian_weights(synth.rng(13, d), n, d, outlier_frac=0.01).astype(np.float32))
