@@ -39,13 +39,13 @@ D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel as
 # it stands (profiles/qlinear_W4A4_4608x3072x3072.md,
 # profiles/rotate_quantize_act_d3072_T32768_A4.md).  qlinear: both launches of
-# one call (weight-code expansion + GEMM), caches flushed before each kernel,
-# so the GEMM reads the fp16 workspace back from DRAM and the 28 MB output is
-# still in L2 when it ends (its writes are not in the figure).  The
+# one call (code expansion of weights and activations + GEMM), caches flushed
+# before each kernel, so the GEMM reads both fp16 workspaces back from DRAM
+# and most of the 28 MB output is still in L2 when it ends.  The
 # rotate-quantize capture ran 32768 tokens; its bytes are scaled to this
 # workload's 4608 by the token count (its traffic grows with the tokens).
-QLINEAR_DRAM_BYTES = (4_724_992 + 0) + (26_067_200 + 7_936)
-ROTQ_DRAM_BYTES = round((201_677_312 + 29_322_240) * 4608 / 32768)
+QLINEAR_DRAM_BYTES = (11_848_448 + 176_640) + (47_262_720 + 4_477_696)
+ROTQ_DRAM_BYTES = round((201_408_768 + 28_317_440) * 4608 / 32768)
 METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
 
@@ -333,9 +333,9 @@ def run_ours(args, rank, world):
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": QLINEAR_DRAM_BYTES,
                      "peak_source": pk["source"] + " bf16 burst",
-                     "note": "achieved includes the per-call code expansion launches (weights, activations); "
-                             "traffic is the ncu DRAM read + write of the three launches of one call "
-                             "(two expansions + GEMM)",
+                     "note": "achieved includes the per-call code expansion launch (weights and activations); "
+                             "traffic is the ncu DRAM read + write of the two launches of one call "
+                             "(expansion + GEMM)",
                      "algorithmic_bytes": qlinear_algorithmic_bytes(),
                      "workspace_round_trip_bytes": 2 * 2 * (D * D + T * D)},
         "roofline_rotate_quantize": {"kernel": "rotate_quantize_act", "bound": "hbm",
@@ -343,9 +343,9 @@ def run_ours(args, rank, world):
                                      "unit": "GB/s", "frac": round(act_bytes / k1_avg_s / 1e9 / pk["hbm_gbs"], 4),
                                      "traffic": ROTQ_DRAM_BYTES, "algorithmic_bytes": act_bytes,
                                      "peak_source": pk["source"]},
-        # steps: rotate-quantize, weights, weight- and activation-code expansion, GEMM; kernel passes
-        # likewise x nsets x reps
-        "gpu_launches": 5 * args.steps + 5 * kernel_reps * nsets,
+        # steps: rotate-quantize, weights, code expansion (weights and activations, one launch), GEMM;
+        # kernel passes likewise x nsets x reps
+        "gpu_launches": 4 * args.steps + 4 * kernel_reps * nsets,
         "timing": ("per-kernel: CUDA graphs of %d launches over the rotating sets, replayed %d times; "
                    "ms_per_step: direct API calls" % (nsets, kernel_reps)) if kernel_graphs else
                   "per-kernel and ms_per_step: direct API calls",

@@ -559,6 +559,11 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
   }
   const int P = pair_geometry(r->d, p.grid_entries, &p.NS, &p.nwarps);
   if (P == 0) return RBQ_ECONVERGE;
+  // With pi = identity (the ablation handle) the source of step i of every
+  // block sits at the same offset of consecutive 128-byte blocks, i.e. in one
+  // bank: with fewer than 8 pairs a warp's 32/P blocks would all conflict.
+  // The register-staged kernel, whose staging spreads the blocks, takes it.
+  if (P < 8 && (r->flags & RBQ_RPBH_NO_PERMUTATION)) return RBQ_ECONVERGE;
   p.ntiles = static_cast<int>((rows + 2 * P - 1) / (2 * P));
   switch (mode) {
     case kAct: return launch_pair_bits<kAct>(bits, P, p, st);

@@ -392,7 +392,8 @@ def test_pair_kernel_weights_wide_codebooks(bits):
 # --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("d,T,bits,permute,signs", [(3072, 37, 4, False, True), (1024, 20, 2, False, True),
-                                                    (3072, 19, 3, True, False), (512, 33, 4, False, False)])
+                                                    (3072, 19, 3, True, False), (512, 33, 4, False, False),
+                                                    (12288, 9, 4, False, True), (8960, 11, 3, True, False)])
 def test_ablation_handles_quantize(d, T, bits, permute, signs):
     X, _ = synth.student_t_act(T, d, seed=d + bits)
     r = rbq.RPBH(d, 21, permute=permute, signs=signs)
