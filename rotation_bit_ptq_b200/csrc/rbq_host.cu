@@ -355,6 +355,28 @@ int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out) {
   return RBQ_OK;
 }
 
+int rpbh_pair_tables16(const rbq_rpbh* r, const uint16_t** out) {
+  if (r->d > 16384) return RBQ_EINVAL;
+  const RpbhDevice* rd = nullptr;
+  int rc = rpbh_device(r, &rd);
+  if (rc != RBQ_OK) return rc;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto* D = const_cast<RpbhDevice*>(rd);
+  if (!D->pair_tab16) {
+    const int d = r->d;
+    std::vector<uint16_t> tab(static_cast<size_t>(d));
+    for (int k = 0; k < d; ++k) {
+      const uint32_t slot = pair_tab16_slot(k / kH, k % kH);
+      tab[slot] = static_cast<uint16_t>(2u * static_cast<uint32_t>(r->perm[k]) | (r->sign[k] < 0 ? 0x8000u : 0u));
+    }
+    uint16_t* dev = nullptr;
+    if ((rc = upload(tab.data(), tab.size(), &dev)) != RBQ_OK) return rc;
+    D->pair_tab16 = dev;
+  }
+  *out = D->pair_tab16;
+  return RBQ_OK;
+}
+
 // The grid with kGridGuard copies of each end entry outside it, padded with
 // one more copy of the last entry to an even count.
 std::vector<float2> guarded(const std::vector<float2>& lut) {
@@ -540,6 +562,7 @@ extern "C" void rpbh_free(rbq_rpbh* r) {
     cudaFree(D.perm);
     cudaFree(D.sign);
     cudaFree(D.pair_tab);
+    cudaFree(D.pair_tab16);
   }
   delete r;
 }

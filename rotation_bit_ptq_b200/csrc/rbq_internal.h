@@ -25,6 +25,9 @@ struct RpbhDevice {
   // position k, at pair_tab_slot(k / 64, k % 64), the byte offset 2 pi(k) of
   // its source in a staged row with the sign D_k in bit 31 (set for -1).
   uint32_t* pair_tab = nullptr;
+  // The same in 16 bits for wide rows (d <= 16384), at pair_tab16_slot(k / 64,
+  // k % 64): the byte offset 2 pi(k) (< 2^15) with D_k in bit 15.
+  uint16_t* pair_tab16 = nullptr;
 };
 
 // Slot of output position (block b, index i) in the token-pair kernel's
@@ -32,6 +35,12 @@ struct RpbhDevice {
 // the four blocks a warp reads hit four different bank quads.
 __host__ __device__ inline uint32_t pair_tab_slot(int b, int i) {
   return 64u * b + 4u * ((static_cast<uint32_t>(i) >> 2) ^ (static_cast<uint32_t>(b) & 7u)) + (i & 3);
+}
+
+// The same for the 16-bit table: 8 entries per 16-byte chunk, the chunk
+// index XORed with b & 7.
+__host__ __device__ inline uint32_t pair_tab16_slot(int b, int i) {
+  return 64u * b + 8u * ((static_cast<uint32_t>(i) >> 3) ^ (static_cast<uint32_t>(b) & 7u)) + (i & 7);
 }
 
 }  // namespace rbq
@@ -89,6 +98,8 @@ int rpbh_device(const rbq_rpbh* r, const RpbhDevice** out);
 // Returns the token-pair kernel's gather table of `r` on the current device
 // (d words, see RpbhDevice::pair_tab), building it on first use.
 int rpbh_pair_tables(const rbq_rpbh* r, const uint32_t** out);
+// The 16-bit gather table (d <= 16384; see RpbhDevice::pair_tab16).
+int rpbh_pair_tables16(const rbq_rpbh* r, const uint16_t** out);
 // Returns the codebook of (d, bits) on the current device, computing and
 // uploading it on first use.
 int codebook_device(int d, int bits, const CodebookDevice** out);

@@ -88,14 +88,15 @@ __device__ __forceinline__ void encode_block(const Enc& enc, uint32_t tA, uint32
   }
 }
 
-template <int MODE, int BITS, int P>
+template <int MODE, int BITS, int P, bool TAB16>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) {
   constexpr int kTR = 2 * P;                       // rows per tile
+  constexpr uint32_t kTabBytes = TAB16 ? 2u : 4u;  // per gather-table entry
   extern __shared__ unsigned char smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 127u) & ~127u;
   unsigned char* sm = smem_raw + (sbase - sraw);
-  const Layout L = layout(p.d, p.NS, p.grid_entries, kTR);
+  const Layout L = layout(p.d, p.NS, p.grid_entries, kTR, kTabBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* red = full + p.NS;
   uint64_t* tabbar = red + 2 * p.NS;
@@ -136,8 +137,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     mbar_init(tabbar, 1);
     mbar_fence_init();
     const uint32_t gbytes = kLloyd ? 8u * static_cast<uint32_t>(p.grid_entries) : 0u;
-    mbar_arrive_expect_tx(tabbar, 4u * p.d + gbytes);
-    bulk_load(sbase + L.off, p.tab, 4u * p.d, tabbar);
+    mbar_arrive_expect_tx(tabbar, kTabBytes * p.d + gbytes);
+    bulk_load(sbase + L.off, p.tab, kTabBytes * p.d, tabbar);
     if (kLloyd) bulk_load(sbase + L.grid, p.grid, gbytes, tabbar);
   }
   {
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   // warp's; otherwise the last warp may hold lanes past the last block.
   const bool act = (P == 8) || b < p.nblk;
   const int bx = b & 7;
-  const uint32_t off_addr = sbase + L.off + 256u * (act ? b : 0);
+  const uint32_t off_addr = sbase + L.off + 64u * kTabBytes * (act ? b : 0);
   const uint32_t part_addr = sbase + L.part;
   const uint32_t gbase = sbase + L.grid + 8u * static_cast<uint32_t>(p.grid_first) - 0x4B000000u * 8u;
   const uint32_t pitchP = static_cast<uint32_t>(P) * pitch;   // token p to token p + P
@@ -193,7 +194,26 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       unsigned long long R[32];
-      if (act) {
+      if (act && TAB16) {
+        // 16-bit entries, 8 per 16-byte chunk: byte offset | sign << 15
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const uint32_t c = 16u * (static_cast<uint32_t>(4 * h + q8) ^ static_cast<uint32_t>(bx));
+          const uint4 o = lds128(off_addr + c);
+          const uint32_t ww[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t w = ww[e >> 1];
+            const uint32_t S = (e & 1) ? (w & 0x80000000u) : ((w << 16) & 0x80000000u);
+            const uint32_t off = ((e & 1) ? (w >> 16) : w) & 0x7FFFu;
+            const uint32_t a = rowA + dbg_index(off, 2u * static_cast<uint32_t>(p.d), p.err);
+            const float y0 = bf16_signed(lds_u16(a), S);
+            const float y1 = bf16_signed(lds_u16(a + pitchP), S);
+            R[8 * q8 + e] = pk(y0, y1);
+            acc[e & 3] = fma2(R[8 * q8 + e], R[8 * q8 + e], acc[e & 3]);
+          }
+        }
+      } else if (act) {
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
           const uint32_t c = 16u * (static_cast<uint32_t>(8 * h + q4) ^ static_cast<uint32_t>(bx));
@@ -470,10 +490,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
 
 namespace {
 
-template <int MODE, int BITS, int P>
+template <int MODE, int BITS, int P, bool TAB16>
 int launch_pair(const pairk::Params& p, cudaStream_t st) {
-  auto kern = pairk::rotq_pair_kernel<MODE, BITS, P>;
-  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_entries, 2 * P).total + 128;
+  auto kern = pairk::rotq_pair_kernel<MODE, BITS, P, TAB16>;
+  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_entries, 2 * P, TAB16 ? 2 : 4).total + 128;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = rowtile::sm_count();
@@ -481,27 +501,30 @@ int launch_pair(const pairk::Params& p, cudaStream_t st) {
   return rowtile::launch_pdl(kern, grid, p.nwarps * 32, smem, st, p);
 }
 
+// The 16-bit table is instantiated only for 2-pair tiles, the one geometry
+// that needs it (widths of about 11000 to 12288; 1-pair tiles fit the 32-bit
+// table up to 16384).
 template <int MODE, int BITS>
-int launch_pair_p(int P, const pairk::Params& p, cudaStream_t st) {
+int launch_pair_p(int P, bool tab16, const pairk::Params& p, cudaStream_t st) {
   switch (P) {
-    case 8: return launch_pair<MODE, BITS, 8>(p, st);
-    case 4: return launch_pair<MODE, BITS, 4>(p, st);
-    case 2: return launch_pair<MODE, BITS, 2>(p, st);
-    default: return launch_pair<MODE, BITS, 1>(p, st);
+    case 8: return launch_pair<MODE, BITS, 8, false>(p, st);
+    case 4: return launch_pair<MODE, BITS, 4, false>(p, st);
+    case 2: return tab16 ? launch_pair<MODE, BITS, 2, true>(p, st) : launch_pair<MODE, BITS, 2, false>(p, st);
+    default: return launch_pair<MODE, BITS, 1, false>(p, st);
   }
 }
 
 template <int MODE>
-int launch_pair_bits(int bits, int P, const pairk::Params& p, cudaStream_t st) {
+int launch_pair_bits(int bits, int P, bool tab16, const pairk::Params& p, cudaStream_t st) {
   switch (bits) {
-    case 1: return launch_pair_p<MODE, 1>(P, p, st);
-    case 2: return launch_pair_p<MODE, 2>(P, p, st);
-    case 3: return launch_pair_p<MODE, 3>(P, p, st);
-    case 4: return launch_pair_p<MODE, 4>(P, p, st);
-    case 5: return launch_pair_p<MODE, 5>(P, p, st);
-    case 6: return launch_pair_p<MODE, 6>(P, p, st);
-    case 7: return launch_pair_p<MODE, 7>(P, p, st);
-    case 8: return launch_pair_p<MODE, 8>(P, p, st);
+    case 1: return launch_pair_p<MODE, 1>(P, tab16, p, st);
+    case 2: return launch_pair_p<MODE, 2>(P, tab16, p, st);
+    case 3: return launch_pair_p<MODE, 3>(P, tab16, p, st);
+    case 4: return launch_pair_p<MODE, 4>(P, tab16, p, st);
+    case 5: return launch_pair_p<MODE, 5>(P, tab16, p, st);
+    case 6: return launch_pair_p<MODE, 6>(P, tab16, p, st);
+    case 7: return launch_pair_p<MODE, 7>(P, tab16, p, st);
+    case 8: return launch_pair_p<MODE, 8>(P, tab16, p, st);
     default: return RBQ_EINVAL;
   }
 }
@@ -511,18 +534,22 @@ int launch_pair_bits(int bits, int P, const pairk::Params& p, cudaStream_t st) {
 bool rotq_pair_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d % 256 == 0 && d >= 1024 && d <= 16384; }
 
 // Pairs per tile for width d: the most (8, 4, 2 or 1) whose CTA has at most
-// kMaxWarps warps and whose ring keeps at least two slots next to the tables;
-// 0 when none fits.  Sets the ring slots and warps.
-int pair_geometry(int d, int grid_entries, int* NS, int* nwarps) {
+// kMaxWarps warps and whose ring keeps at least two slots next to the tables,
+// with the 32-bit gather table if it fits, else (2 pairs) the 16-bit one; 0
+// when none fits.  Sets the ring slots, the warps and the table width.
+int pair_geometry(int d, int grid_entries, int* NS, int* nwarps, bool* tab16) {
   const int nblk = d / kH;
   for (int P = 8; P >= 1; P >>= 1) {
     const int w = (P * nblk + 31) / 32;
     if (w > rowtile::kMaxWarps) continue;
-    const int ns = rowtile::slots_that_fit(d, grid_entries, 2 * P);
-    if (ns >= 2) {
-      *NS = ns;
-      *nwarps = w;
-      return P;
+    for (int t16 = 0; t16 < (P == 2 ? 2 : 1); ++t16) {
+      const int ns = rowtile::slots_that_fit(d, grid_entries, 2 * P, t16 ? 2 : 4);
+      if (ns >= 2) {
+        *NS = ns;
+        *nwarps = w;
+        *tab16 = t16 != 0;
+        return P;
+      }
     }
   }
   return 0;
@@ -533,20 +560,17 @@ int pair_geometry(int d, int grid_entries, int* NS, int* nwarps) {
 int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
                      cudaStream_t st, const float* fixed_scale) {
   using namespace pairk;
-  const uint32_t* tab = nullptr;
-  int rc = rpbh_pair_tables(r, &tab);
-  if (rc != RBQ_OK) return rc;
   Params p{};
   p.X = static_cast<const __nv_bfloat16*>(X);
   p.T = rows;
   p.d = r->d;
   p.nblk = r->d / kH;
   p.pitch = 2u * static_cast<uint32_t>(r->d) + 16u;
-  p.tab = tab;
   p.out = out;
   p.aux = aux;
   p.fixed_scale = fixed_scale;
-  if ((rc = device_error_word_ptr(&p.err)) != RBQ_OK) return rc;
+  int rc = device_error_word_ptr(&p.err);
+  if (rc != RBQ_OK) return rc;
   const bool lloyd = (mode == kAct || mode == kWeightLM);
   if (lloyd) {
     const CodebookDevice* cb = nullptr;
@@ -557,19 +581,29 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     p.grid_cells = static_cast<float>(cb->grid_cells);
     p.grid_scale = cb->grid_scale;
   }
-  const int P = pair_geometry(r->d, p.grid_entries, &p.NS, &p.nwarps);
+  bool tab16 = false;
+  const int P = pair_geometry(r->d, p.grid_entries, &p.NS, &p.nwarps, &tab16);
   if (P == 0) return RBQ_ECONVERGE;
   // With pi = identity (the ablation handle) the source of step i of every
   // block sits at the same offset of consecutive 128-byte blocks, i.e. in one
   // bank: with fewer than 8 pairs a warp's 32/P blocks would all conflict.
   // The register-staged kernel, whose staging spreads the blocks, takes it.
   if (P < 8 && (r->flags & RBQ_RPBH_NO_PERMUTATION)) return RBQ_ECONVERGE;
+  if (tab16) {
+    const uint16_t* t = nullptr;
+    if ((rc = rpbh_pair_tables16(r, &t)) != RBQ_OK) return rc;
+    p.tab = t;
+  } else {
+    const uint32_t* t = nullptr;
+    if ((rc = rpbh_pair_tables(r, &t)) != RBQ_OK) return rc;
+    p.tab = t;
+  }
   p.ntiles = static_cast<int>((rows + 2 * P - 1) / (2 * P));
   switch (mode) {
-    case kAct: return launch_pair_bits<kAct>(bits, P, p, st);
-    case kWeightLM: return launch_pair_bits<kWeightLM>(bits, P, p, st);
-    case kInt8: return launch_pair_p<kInt8, 8>(P, p, st);
-    default: return launch_pair_p<kRotate, 8>(P, p, st);
+    case kAct: return launch_pair_bits<kAct>(bits, P, tab16, p, st);
+    case kWeightLM: return launch_pair_bits<kWeightLM>(bits, P, tab16, p, st);
+    case kInt8: return launch_pair_p<kInt8, 8>(P, tab16, p, st);
+    default: return launch_pair_p<kRotate, 8>(P, tab16, p, st);
   }
 }
 

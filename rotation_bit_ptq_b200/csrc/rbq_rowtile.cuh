@@ -32,7 +32,8 @@ struct Params {
   int ntiles;                        // ceil(T / R)
   int NS;                            // ring slots
   uint32_t pitch;                    // bytes per staged row (2d + 16)
-  const uint32_t* tab;               // d words: source offset | sign << 31 (pair_tab_slot order)
+  const void* tab;                   // d entries: source byte offset | sign in the top bit, 32-bit
+                                     // (pair_tab_slot order) or 16-bit (pair_tab16_slot order)
   const float2* grid;                // Lloyd-Max modes: the code grid as copied into shared memory
   int grid_entries;                  // entries copied (even: one 16-byte-multiple bulk copy)
   int grid_first;                    // index of cell 0 among them (guard entries before it)
@@ -48,12 +49,13 @@ struct Layout {
   uint32_t ring, off, grid, part, bars, total;
 };
 
-__host__ __device__ inline Layout layout(int d, int NS, int grid_entries, int R) {
+// tab_bytes: bytes per gather-table entry (4, or 2 for the 16-bit table).
+__host__ __device__ inline Layout layout(int d, int NS, int grid_entries, int R, int tab_bytes) {
   Layout L{};
   const uint32_t pitch = 2u * d + 16u;
   L.ring = 0;
   L.off = L.ring + NS * R * pitch;
-  L.grid = L.off + 4u * d;
+  L.grid = L.off + static_cast<uint32_t>(tab_bytes) * d;
   L.part = (L.grid + 8u * grid_entries + 15u) & ~15u;
   L.bars = L.part + 4u * (2 * NS) * R * kMaxWarps;       // [2NS][R tokens][12 warps]
   L.bars = (L.bars + 7u) & ~7u;
@@ -230,10 +232,10 @@ inline int sm_count() {
 
 // Most ring slots of R-row tiles that fit next to the tables (at least 2, at
 // most 6), or 0.
-inline int slots_that_fit(int d, int grid_entries, int R) {
+inline int slots_that_fit(int d, int grid_entries, int R, int tab_bytes) {
   int best = 0;
   for (int ns = 2; ns <= 6; ++ns)
-    if (layout(d, ns, grid_entries, R).total + 128 <= kSmemLimit) best = ns;
+    if (layout(d, ns, grid_entries, R, tab_bytes).total + 128 <= kSmemLimit) best = ns;
   return best;
 }
 

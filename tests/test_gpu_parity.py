@@ -255,12 +255,14 @@ def test_pair_kernel_rotate_only(d):
 
 
 # Wider rows: tiles of 8, 4 or 2 rows (4, 2 or 1 token pairs per tile), as
-# many as keep two ring slots next to the gather table.  3328 and 8960 leave
-# the CTA's last warp with lanes past the last block; the long cases wrap the
-# ring of slots and the norm barriers several times per CTA.
+# many as keep two ring slots next to the gather table; 12288 (and 11520 at 8
+# bits, whose code grid is larger) take 4-row tiles with the 16-bit gather
+# table.  3328, 8960 and 11520 leave the CTA's
+# last warp with lanes past the last block; the long cases wrap the ring of
+# slots and the norm barriers several times per CTA.
 @pytest.mark.parametrize("d,T,bits", [(4096, 8 * 148 * 3 + 5, 4), (3328, 45, 6), (5120, 19, 5), (8960, 37, 2),
-                                      (8960, 4 * 148 * 2 + 3, 6), (12288, 2 * 148 * 4 + 1, 4), (16384, 19, 3),
-                                      (16384, 7, 8)])
+                                      (8960, 4 * 148 * 2 + 3, 6), (12288, 4 * 148 * 3 + 1, 4), (12288, 21, 7),
+                                      (11520, 37, 8), (11520, 29, 5), (16384, 19, 3), (16384, 7, 8)])
 def test_pair_kernel_wide_rows(d, T, bits):
     X, _ = synth.student_t_act(T, d, seed=d + bits)
     rows = None
