@@ -355,35 +355,44 @@ def run_ours(args, rank, world):
     return res
 
 
+E2E_SLOTS = 3
+
+
 def run_e2e(r, X_host, dev, stream, args):
     """rotate_quantize_act through the public API from pinned host memory:
     every step copies its input X host -> device, runs the kernel and copies
-    the codes and norms back.  Two buffer sets and separate copy streams let
-    step i+1's upload overlap step i's kernel and download (PCIe moves both
-    directions at once); every step's copies stay inside the timed region.
-    Returns (ms for args.steps steps, H2D bytes per step, D2H bytes per step)."""
+    the codes and norms back.  Three buffer sets and separate copy streams let
+    step i+1's upload overlap step i's kernel and step i-1's download (PCIe
+    moves both directions at once): an upload waits only for the kernel that
+    last read its input buffer, a kernel only for its upload and for the
+    download that last read its output buffers.  Every step's copies stay
+    inside the timed region.  Returns (ms for args.steps steps, H2D bytes per
+    step, D2H bytes per step)."""
     import torch
     import rotation_bit_ptq_b200 as rbq
+    S = E2E_SLOTS
     xh = torch.from_numpy(synth.bf16_bits(X_host).view(np.int16)).view(torch.bfloat16).pin_memory()
-    xd = [torch.empty_like(xh, device=dev) for _ in range(2)]
-    cd = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev) for _ in range(2)]
-    nd = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(2)]
-    ch = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8).pin_memory() for _ in range(2)]
-    nh = [torch.empty((T,), dtype=torch.float32).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(xh, device=dev) for _ in range(S)]
+    cd = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev) for _ in range(S)]
+    nd = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(S)]
+    ch = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8).pin_memory() for _ in range(S)]
+    nh = [torch.empty((T,), dtype=torch.float32).pin_memory() for _ in range(S)]
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    uploaded = [torch.cuda.Event() for _ in range(2)]
-    computed = [torch.cuda.Event() for _ in range(2)]
-    downloaded = [torch.cuda.Event() for _ in range(2)]
-    for e in downloaded:
-        e.record(s_out)
+    uploaded = [torch.cuda.Event() for _ in range(S)]
+    computed = [torch.cuda.Event() for _ in range(S)]
+    downloaded = [torch.cuda.Event() for _ in range(S)]
+    for k in range(S):
+        computed[k].record(stream)
+        downloaded[k].record(s_out)
 
     def one(i):
-        k = i % 2
-        s_in.wait_event(downloaded[k])              # the slot's previous results are out
+        k = i % S
+        s_in.wait_event(computed[k])                # the slot's input buffer is no longer read
         with torch.cuda.stream(s_in):
             xd[k].copy_(xh, non_blocking=True)
         uploaded[k].record(s_in)
         stream.wait_event(uploaded[k])
+        stream.wait_event(downloaded[k])            # the slot's previous results are out
         rbq.rotate_quantize_act(r, xd[k], BITS_A, cd[k], nd[k], stream=stream)
         computed[k].record(stream)
         s_out.wait_event(computed[k])
@@ -413,32 +422,36 @@ def run_e2e_layer(r, X_host, w_codes, rnorm, dev, stream, args):
     """The whole quantised layer through the public API from pinned host
     memory: every step copies its input X host -> device, quantises it
     (rotate_quantize_act), runs qlinear against the resident weight codes and
-    copies Y (BF16) back.  Two buffer sets and separate copy streams overlap
-    step i+1's upload and step i's download with the kernels; every step's
-    copies stay inside the timed region.  Returns (ms for args.steps steps,
-    H2D bytes per step, D2H bytes per step)."""
+    copies Y (BF16) back.  Three buffer sets and separate copy streams overlap
+    step i+1's upload and step i-1's download with step i's kernels (the same
+    dependencies as run_e2e); every step's copies stay inside the timed
+    region.  Returns (ms for args.steps steps, H2D bytes per step, D2H bytes
+    per step)."""
     import torch
     import rotation_bit_ptq_b200 as rbq
+    S = E2E_SLOTS
     xh = torch.from_numpy(synth.bf16_bits(X_host).view(np.int16)).view(torch.bfloat16).pin_memory()
-    xd = [torch.empty_like(xh, device=dev) for _ in range(2)]
-    cd = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev) for _ in range(2)]
-    nd = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(2)]
-    yd = [torch.empty((T, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    yh = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(xh, device=dev) for _ in range(S)]
+    cd = [torch.empty((T, D * BITS_A // 8), dtype=torch.uint8, device=dev) for _ in range(S)]
+    nd = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in range(S)]
+    yd = [torch.empty((T, D), dtype=torch.bfloat16, device=dev) for _ in range(S)]
+    yh = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(S)]
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    uploaded = [torch.cuda.Event() for _ in range(2)]
-    computed = [torch.cuda.Event() for _ in range(2)]
-    downloaded = [torch.cuda.Event() for _ in range(2)]
-    for e in downloaded:
-        e.record(s_out)
+    uploaded = [torch.cuda.Event() for _ in range(S)]
+    computed = [torch.cuda.Event() for _ in range(S)]
+    downloaded = [torch.cuda.Event() for _ in range(S)]
+    for k in range(S):
+        computed[k].record(stream)
+        downloaded[k].record(s_out)
 
     def one(i):
-        k = i % 2
-        s_in.wait_event(downloaded[k])              # the slot's previous Y is out
+        k = i % S
+        s_in.wait_event(computed[k])                # the slot's input buffer is no longer read
         with torch.cuda.stream(s_in):
             xd[k].copy_(xh, non_blocking=True)
         uploaded[k].record(s_in)
         stream.wait_event(uploaded[k])
+        stream.wait_event(downloaded[k])            # the slot's previous Y is out
         rbq.rotate_quantize_act(r, xd[k], BITS_A, cd[k], nd[k], stream=stream)
         rbq.qlinear(cd[k], nd[k], BITS_A, w_codes, rnorm, BITS_W, D, yd[k], stream=stream)
         computed[k].record(stream)

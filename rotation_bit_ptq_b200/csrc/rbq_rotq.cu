@@ -824,11 +824,11 @@ int prepare(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X
 
 }  // namespace
 
-// The token-pair kernel (rbq_rotq_pair.cu): BF16 rows, d = 1024..3072 in
+// The token-pair kernel (rbq_rotq_pair.cu): BF16 rows, d = 1024..16384 in
 // steps of 256.  RBQ_ECONVERGE from the launch means "not this kernel".
 bool rotq_pair_eligible(int dtype, int d);
 int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
-                     cudaStream_t st, const float* fixed_scale = nullptr);
+                     cudaStream_t st, const float* fixed_scale = nullptr, uint8_t* zero_point = nullptr);
 
 namespace {
 
@@ -937,6 +937,11 @@ extern "C" int quantize_weights_int8_asym(const rbq_rpbh* r, const void* W, int 
   if (d_out == 0) return RBQ_OK;
   if (!W || !q || !scale || !zero_point) return RBQ_EINVAL;
   if (!aligned(W, 16) || !aligned(q, 16) || !aligned(scale, 4)) return RBQ_EALIGN;
+  if (rotq_pair_eligible(dtype, r->d)) {
+    const int prc = rotq_pair_launch(r, kInt8Asym, 8, d_out, W, q, scale, static_cast<cudaStream_t>(stream),
+                                     nullptr, zero_point);
+    if (prc != RBQ_ECONVERGE) return prc;
+  }
   RotqParams p;
   int rc = prepare(r, kInt8Asym, 8, d_out, W, q, scale, &p);
   if (rc != RBQ_OK) return rc;

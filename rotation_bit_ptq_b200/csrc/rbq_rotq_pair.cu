@@ -92,11 +92,13 @@ template <int MODE, int BITS, int P, bool TAB16>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) {
   constexpr int kTR = 2 * P;                       // rows per tile
   constexpr uint32_t kTabBytes = TAB16 ? 2u : 4u;  // per gather-table entry
+  constexpr bool kAsym = (MODE == kInt8Asym);
+  constexpr int kParts = kAsym ? 2 : 1;             // partial-result arrays (max, min)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 127u) & ~127u;
   unsigned char* sm = smem_raw + (sbase - sraw);
-  const Layout L = layout(p.d, p.NS, p.grid_entries, kTR, kTabBytes);
+  const Layout L = layout(p.d, p.NS, p.grid_entries, kTR, kTabBytes, kParts);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* red = full + p.NS;
   uint64_t* tabbar = red + 2 * p.NS;
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   }
   {
     float* part = reinterpret_cast<float*>(sm + L.part);
-    for (int i = tid; i < (2 * NS) * kTR * kMaxWarps; i += blockDim.x) part[i] = 0.f;
+    for (int i = tid; i < kParts * (2 * NS) * kTR * kMaxWarps; i += blockDim.x) part[i] = 0.f;
   }
   __syncwarp();
   if (warp == 0) {
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
   const int bx = b & 7;
   const uint32_t off_addr = sbase + L.off + 64u * kTabBytes * (act ? b : 0);
   const uint32_t part_addr = sbase + L.part;
+  const uint32_t part2_addr = part_addr + 4u * (2 * NS) * kTR * kMaxWarps;   // asymmetric INT8: the minima
   const uint32_t gbase = sbase + L.grid + 8u * static_cast<uint32_t>(p.grid_first) - 0x4B000000u * 8u;
   const uint32_t pitchP = static_cast<uint32_t>(P) * pitch;   // token p to token p + P
   // Tensor memory: each thread parks its pair's two half-blocks (2 x 64 words)
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
         for (int i = 0; i < 32; ++i) R[i] = 0ull;      // a lane past the last block: zeros
       }
       if (h == 1) {
-        if constexpr (MODE != kInt8) {
+        if constexpr (MODE != kInt8 && !kAsym) {
           // ||x||^2 partials of both tokens (||Pi x|| = ||x||): 32/P lanes share a pair
           float a0, a1;
           upk(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), a0, a1);
@@ -276,9 +279,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     }
     tmem_wait_st();
 
-    if constexpr (MODE == kInt8) {
-      // max |z| needs the last butterfly stage: z_i = A_i + B_i, z_{i+32} = A_i - B_i
-      float m0 = 0.f, m1 = 0.f;
+    if constexpr (MODE == kInt8 || kAsym) {
+      // max |z| (asymmetric: max z and min z, both widened to contain 0) needs
+      // the last butterfly stage: z_i = A_i + B_i, z_{i+32} = A_i - B_i
+      float m0 = 0.f, m1 = 0.f, n0 = 0.f, n1 = 0.f;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t va[32], vb[32];
@@ -292,18 +296,33 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
           float z0, z1, y0, y1;
           upk(add2(a, bb), z0, z1);
           upk(sub2(a, bb), y0, y1);
-          m0 = fmaxf(m0, fmaxf(fabsf(z0), fabsf(y0)));
-          m1 = fmaxf(m1, fmaxf(fabsf(z1), fabsf(y1)));
+          if constexpr (kAsym) {
+            m0 = fmaxf(m0, fmaxf(z0, y0));
+            m1 = fmaxf(m1, fmaxf(z1, y1));
+            n0 = fminf(n0, fminf(z0, y0));
+            n1 = fminf(n1, fminf(z1, y1));
+          } else {
+            m0 = fmaxf(m0, fmaxf(fabsf(z0), fabsf(y0)));
+            m1 = fmaxf(m1, fmaxf(fabsf(z1), fabsf(y1)));
+          }
         }
       }
 #pragma unroll
       for (int o = P; o < 32; o <<= 1) {
         m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
         m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+        if constexpr (kAsym) {
+          n0 = fminf(n0, __shfl_xor_sync(0xffffffffu, n0, o));
+          n1 = fminf(n1, __shfl_xor_sync(0xffffffffu, n1, o));
+        }
       }
       if (j == 0) {
         sts_f32(part_addr + 4u * ((rb * kTR + pp) * kMaxWarps + warp), m0);
         sts_f32(part_addr + 4u * ((rb * kTR + pp + P) * kMaxWarps + warp), m1);
+        if constexpr (kAsym) {
+          sts_f32(part2_addr + 4u * ((rb * kTR + pp) * kMaxWarps + warp), n0);
+          sts_f32(part2_addr + 4u * ((rb * kTR + pp + P) * kMaxWarps + warp), n1);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&red[rb]);
@@ -315,16 +334,27 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
     // slot can take the tile NS steps ahead (the barrier's release/acquire
     // orders those reads before the asynchronous overwrite).
     if (tile + NS * static_cast<int>(gridDim.x) < p.ntiles) issue_rows(tile + NS * gridDim.x, s);
-    float tot[2];
+    float tot[2], tot2[2];                         // tot2: asymmetric INT8 min z
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      if constexpr (kAsym) {
+        const uint32_t pa = part2_addr + 4u * ((rb * kTR + pp + P * h) * kMaxWarps);
+        const uint4 q0 = lds128(pa), q1 = lds128(pa + 16), q2 = lds128(pa + 32);
+        const uint32_t u[12] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w, q2.x, q2.y, q2.z, q2.w};
+        float m = __uint_as_float(u[0]);
+#pragma unroll
+        for (int w = 1; w < 12; ++w) m = fminf(m, __uint_as_float(u[w]));
+        tot2[h] = m;
+      } else {
+        tot2[h] = 0.f;
+      }
       const uint32_t pa = part_addr + 4u * ((rb * kTR + pp + P * h) * kMaxWarps);
       const uint4 q0 = lds128(pa), q1 = lds128(pa + 16), q2 = lds128(pa + 32);
       const float v[12] = {__uint_as_float(q0.x), __uint_as_float(q0.y), __uint_as_float(q0.z),
                            __uint_as_float(q0.w), __uint_as_float(q1.x), __uint_as_float(q1.y),
                            __uint_as_float(q1.z), __uint_as_float(q1.w), __uint_as_float(q2.x),
                            __uint_as_float(q2.y), __uint_as_float(q2.z), __uint_as_float(q2.w)};
-      if constexpr (MODE == kInt8) {
+      if constexpr (MODE == kInt8 || kAsym) {
         float m = v[0];
 #pragma unroll
         for (int w = 1; w < 12; ++w) m = fmaxf(m, v[w]);
@@ -415,6 +445,63 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
         if (ok0 && !p.fixed_scale) static_cast<float*>(p.aux)[t0] = sc0;
         if (ok1 && !p.fixed_scale) static_cast<float*>(p.aux)[t1] = sc1;
       }
+    } else if constexpr (kAsym) {
+      // the row's range [min w', max w'] widened to contain 0, 255 steps:
+      // scale = (hi - lo) / 255, zero point = round(-lo / scale) in 0..255,
+      // q = clamp(round(w' / scale) + zero point, 0, 255), w' = z / 8
+      float sc[2], rc[2];
+      int zp[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float hi = tot[h] * 0.125f, lo = tot2[h] * 0.125f;
+        sc[h] = (hi - lo) / 255.0f;
+        rc[h] = (sc[h] > 0.f) ? 1.0f / sc[h] : 0.f;
+        zp[h] = (sc[h] > 0.f) ? min(255, max(0, __float2int_rn(-lo * rc[h]))) : 0;
+      }
+      uint8_t* out = static_cast<uint8_t*>(p.out) + 64 * b;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t va[32], vb[32];
+        __syncwarp();
+        tmem_ld32(tA + 32u * c, va);
+        tmem_ld32(tB + 32u * c, vb);
+        tmem_wait_ld();
+        uint32_t qa0[4] = {0u, 0u, 0u, 0u}, qa1[4] = {0u, 0u, 0u, 0u};   // positions 16c + k
+        uint32_t qb0[4] = {0u, 0u, 0u, 0u}, qb1[4] = {0u, 0u, 0u, 0u};   // positions 32 + 16c + k
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const unsigned long long a = pk_u(va[2 * k], va[2 * k + 1]), bb = pk_u(vb[2 * k], vb[2 * k + 1]);
+          float z0, z1, y0, y1;
+          upk(add2(a, bb), z0, z1);
+          upk(sub2(a, bb), y0, y1);
+          const int sh = 8 * (k & 3);
+          const auto code = [&](float z, int h) {
+            return static_cast<uint32_t>(sc[h] > 0.f ? min(255, max(0, __float2int_rn(z * 0.125f * rc[h]) + zp[h])) : 0);
+          };
+          qa0[k >> 2] |= code(z0, 0) << sh;
+          qa1[k >> 2] |= code(z1, 1) << sh;
+          qb0[k >> 2] |= code(y0, 0) << sh;
+          qb1[k >> 2] |= code(y1, 1) << sh;
+        }
+        if (ok0) {
+          __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 16 * c), make_uint4(qa0[0], qa0[1], qa0[2], qa0[3]));
+          __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 32 + 16 * c), make_uint4(qb0[0], qb0[1], qb0[2], qb0[3]));
+        }
+        if (ok1) {
+          __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 16 * c), make_uint4(qa1[0], qa1[1], qa1[2], qa1[3]));
+          __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 32 + 16 * c), make_uint4(qb1[0], qb1[1], qb1[2], qb1[3]));
+        }
+      }
+      if (b == 0) {
+        if (ok0) {
+          static_cast<float*>(p.aux)[t0] = sc[0];
+          p.zero_point[t0] = static_cast<uint8_t>(zp[0]);
+        }
+        if (ok1) {
+          static_cast<float*>(p.aux)[t1] = sc[1];
+          p.zero_point[t1] = static_cast<uint8_t>(zp[1]);
+        }
+      }
     } else {   // kRotate: x' = z / 8 in BF16
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + 64 * b;
 #pragma unroll
@@ -493,7 +580,8 @@ namespace {
 template <int MODE, int BITS, int P, bool TAB16>
 int launch_pair(const pairk::Params& p, cudaStream_t st) {
   auto kern = pairk::rotq_pair_kernel<MODE, BITS, P, TAB16>;
-  const size_t smem = rowtile::layout(p.d, p.NS, p.grid_entries, 2 * P, TAB16 ? 2 : 4).total + 128;
+  const size_t smem =
+      rowtile::layout(p.d, p.NS, p.grid_entries, 2 * P, TAB16 ? 2 : 4, MODE == rowtile::kInt8Asym ? 2 : 1).total + 128;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_fail(e);
   const int sms = rowtile::sm_count();
@@ -537,13 +625,13 @@ bool rotq_pair_eligible(int dtype, int d) { return dtype == RBQ_BF16 && d % 256 
 // kMaxWarps warps and whose ring keeps at least two slots next to the tables,
 // with the 32-bit gather table if it fits, else (2 pairs) the 16-bit one; 0
 // when none fits.  Sets the ring slots, the warps and the table width.
-int pair_geometry(int d, int grid_entries, int* NS, int* nwarps, bool* tab16) {
+int pair_geometry(int d, int grid_entries, int nparts, int* NS, int* nwarps, bool* tab16) {
   const int nblk = d / kH;
   for (int P = 8; P >= 1; P >>= 1) {
     const int w = (P * nblk + 31) / 32;
     if (w > rowtile::kMaxWarps) continue;
     for (int t16 = 0; t16 < (P == 2 ? 2 : 1); ++t16) {
-      const int ns = rowtile::slots_that_fit(d, grid_entries, 2 * P, t16 ? 2 : 4);
+      const int ns = rowtile::slots_that_fit(d, grid_entries, 2 * P, t16 ? 2 : 4, nparts);
       if (ns >= 2) {
         *NS = ns;
         *nwarps = w;
@@ -558,7 +646,7 @@ int pair_geometry(int d, int grid_entries, int* NS, int* nwarps, bool* tab16) {
 // Returns RBQ_ECONVERGE when the tables do not fit (the caller then uses
 // another kernel); any other code is the call's result.
 int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, const void* X, void* out, void* aux,
-                     cudaStream_t st, const float* fixed_scale) {
+                     cudaStream_t st, const float* fixed_scale, uint8_t* zero_point) {
   using namespace pairk;
   Params p{};
   p.X = static_cast<const __nv_bfloat16*>(X);
@@ -569,6 +657,7 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
   p.out = out;
   p.aux = aux;
   p.fixed_scale = fixed_scale;
+  p.zero_point = zero_point;
   int rc = device_error_word_ptr(&p.err);
   if (rc != RBQ_OK) return rc;
   const bool lloyd = (mode == kAct || mode == kWeightLM);
@@ -582,7 +671,7 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     p.grid_scale = cb->grid_scale;
   }
   bool tab16 = false;
-  const int P = pair_geometry(r->d, p.grid_entries, &p.NS, &p.nwarps, &tab16);
+  const int P = pair_geometry(r->d, p.grid_entries, mode == kInt8Asym ? 2 : 1, &p.NS, &p.nwarps, &tab16);
   if (P == 0) return RBQ_ECONVERGE;
   // With pi = identity (the ablation handle) the source of step i of every
   // block sits at the same offset of consecutive 128-byte blocks, i.e. in one
@@ -603,6 +692,7 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     case kAct: return launch_pair_bits<kAct>(bits, P, tab16, p, st);
     case kWeightLM: return launch_pair_bits<kWeightLM>(bits, P, tab16, p, st);
     case kInt8: return launch_pair_p<kInt8, 8>(P, tab16, p, st);
+    case kInt8Asym: return launch_pair_p<kInt8Asym, 8>(P, tab16, p, st);
     default: return launch_pair_p<kRotate, 8>(P, tab16, p, st);
   }
 }

@@ -17,7 +17,7 @@ namespace rowtile {
 
 using namespace sm100;
 
-enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3 };
+enum Mode { kAct = 0, kWeightLM = 1, kInt8 = 2, kRotate = 3, kInt8Asym = 4 };
 
 // A tile holds R = 2P token rows (P token pairs): 16 rows for d <= 3072, and
 // 8, 4 or 2 rows for wider rows, so that a double-buffered ring still fits.
@@ -42,6 +42,7 @@ struct Params {
   void* aux;
   unsigned int* err;
   const float* fixed_scale;          // INT8: one scale for every row (not written back), else null
+  uint8_t* zero_point;               // asymmetric INT8: one per row
 };
 
 // Shared-memory layout (bytes from the 128-aligned base).
@@ -49,15 +50,16 @@ struct Layout {
   uint32_t ring, off, grid, part, bars, total;
 };
 
-// tab_bytes: bytes per gather-table entry (4, or 2 for the 16-bit table).
-__host__ __device__ inline Layout layout(int d, int NS, int grid_entries, int R, int tab_bytes) {
+// tab_bytes: bytes per gather-table entry (4, or 2 for the 16-bit table);
+// nparts: partial-result arrays (2 for the asymmetric INT8 mode: max and min).
+__host__ __device__ inline Layout layout(int d, int NS, int grid_entries, int R, int tab_bytes, int nparts) {
   Layout L{};
   const uint32_t pitch = 2u * d + 16u;
   L.ring = 0;
   L.off = L.ring + NS * R * pitch;
   L.grid = L.off + static_cast<uint32_t>(tab_bytes) * d;
   L.part = (L.grid + 8u * grid_entries + 15u) & ~15u;
-  L.bars = L.part + 4u * (2 * NS) * R * kMaxWarps;       // [2NS][R tokens][12 warps]
+  L.bars = L.part + 4u * nparts * (2 * NS) * R * kMaxWarps;   // nparts x [2NS][R tokens][12 warps]
   L.bars = (L.bars + 7u) & ~7u;
   // full[NS], red[2NS], tab | TMEM base
   L.total = L.bars + 8u * (NS + 2 * NS + 1) + 8u;
@@ -232,10 +234,10 @@ inline int sm_count() {
 
 // Most ring slots of R-row tiles that fit next to the tables (at least 2, at
 // most 6), or 0.
-inline int slots_that_fit(int d, int grid_entries, int R, int tab_bytes) {
+inline int slots_that_fit(int d, int grid_entries, int R, int tab_bytes, int nparts) {
   int best = 0;
   for (int ns = 2; ns <= 6; ++ns)
-    if (layout(d, ns, grid_entries, R, tab_bytes).total + 128 <= kSmemLimit) best = ns;
+    if (layout(d, ns, grid_entries, R, tab_bytes, nparts).total + 128 <= kSmemLimit) best = ns;
   return best;
 }
 

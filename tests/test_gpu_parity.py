@@ -347,7 +347,9 @@ def test_weights_int8_per_tensor(d, n, dtype):
         assert rel_frobenius(bf16_to_numpy(y), ref) < QLINEAR8_RTOL
 
 
-@pytest.mark.parametrize("d,n,dtype", [(1024, 40, "bf16"), (4096, 24, "bf16"), (512, 37, "f32")])
+@pytest.mark.parametrize("d,n,dtype", [(1024, 40, "bf16"), (3072, 37, "bf16"), (4096, 24, "bf16"),
+                                       (8960, 13, "bf16"), (12288, 9, "bf16"),   # token-pair kernel
+                                       (4160, 11, "bf16"), (512, 37, "f32")])   # general kernel
 def test_weights_int8_asymmetric(d, n, dtype):
     W = synth.gaussian_weights(synth.rng(14, d), n, d, outlier_frac=0.01).astype(np.float32)
     W[: n // 2] += 0.01                      # some rows skewed, so zero points vary
