@@ -90,6 +90,7 @@ __host__ __device__ constexpr int epi_threads_for(int epi) { return epi >= kEpiR
 
 struct Params {
   int M, N, K;
+  int order;                  // tile order (TileOrder)
   const float* scale;         // W8A16: per-column scales
   const float* s;             // qlinear: per-row norms
   const uint16_t* rnorm;      // qlinear: BF16 per-column norms
@@ -155,6 +156,35 @@ __device__ __forceinline__ void fwht64_pairs(unsigned long long (&P)[32]) {
     float lo, hi;
     upk2(P[i], lo, hi);
     P[i] = pk2(lo + hi, lo - hi);        // (z_i, z_{i+32})
+  }
+}
+
+// Order in which a CTA (pair) walks its output tiles, chosen on the host so
+// that the operand panels a wave of CTAs touches stay in L2:
+//   kOrderM  M fastest: a wave shares a few weight panels; the activation
+//            operand is read once if it stays in L2 (it fits in half of it);
+//   kOrderN  N fastest: a wave shares a few activation panels; for weights
+//            that fit in half of L2 (read once) and a larger activation
+//            operand (streamed once instead of once per column of tiles);
+//   kOrderGrouped  neither fits: groups of kGroupM row panels, N fastest
+//            inside a group, so a wave touches about kGroupM activation and
+//            ~waves/kGroupM weight panels.
+enum TileOrder { kOrderM = 0, kOrderN = 1, kOrderGrouped = 2 };
+constexpr int kGroupM = 8;
+
+__device__ __forceinline__ void tile_coords(int tile, int ntiles_m, int ntiles_n, int order, int& mt, int& nt) {
+  if (order == kOrderM) {
+    mt = tile % ntiles_m;
+    nt = tile / ntiles_m;
+  } else if (order == kOrderN) {
+    mt = tile / ntiles_n;
+    nt = tile % ntiles_n;
+  } else {
+    const int per_group = kGroupM * ntiles_n;
+    const int g = tile / per_group, r = tile - g * per_group;
+    const int m0 = g * kGroupM, gm = min(kGroupM, ntiles_m - m0);
+    mt = m0 + r % gm;
+    nt = r / gm;
   }
 }
 
@@ -297,7 +327,8 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
       uint32_t s = 0, ph = 0;
       bool first = true, ok = true;
       for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
-        const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+        int mt, nt;
+        tile_coords(tile, ntiles_m, ntiles_n, p.order, mt, nt);
         const int m0 = mt * G::kTileM + static_cast<int>(rank) * kBM;
         const int n0 = nt * kBN + static_cast<int>(rank) * G::kBNc;
         for (int kb = 0; kb < KT; ++kb) {
@@ -342,7 +373,8 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
         break;
       }
       tc_fence_after();
-      const int mt = tile % ntiles_m, nt = tile / ntiles_m;
+      int mt, nt;
+      tile_coords(tile, ntiles_m, ntiles_n, p.order, mt, nt);
       const int m = mt * G::kTileM + static_cast<int>(rank) * kBM + r;
       if constexpr (kRot) {
         // The tile's 256 columns are four whole blocks of the next layer's
@@ -564,6 +596,19 @@ int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStrea
     pair = pair_clusters<EPI>(dev) >= 1;
   }
   const int tile_m = pair ? Geom<true>::kTileM : Geom<false>::kTileM;
+  Params q = p;
+  {
+    // the operand panels that can stay in L2 (half of it, the rest for the
+    // output and the other operand's panels in flight)
+    int l2 = 0;
+    if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0) l2 = 126 << 20;
+    const long long half = static_cast<long long>(l2) / 2;
+    const long long a_bytes = 2LL * p.M * p.K, b_bytes = 2LL * p.N * p.K;
+    if (b_bytes <= half && a_bytes > b_bytes) q.order = kOrderN;
+    else if (a_bytes <= half) q.order = kOrderM;
+    else if (b_bytes <= half) q.order = kOrderN;
+    else q.order = kOrderGrouped;
+  }
   CUtensorMap mA, mB;
   int rc = encode_bf16_map(&mA, A, p.M, p.K, kBM, kQ);
   if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, pair ? Geom<true>::kBNc : Geom<false>::kBNc, kQ);
@@ -587,13 +632,13 @@ int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStrea
     int clusters = pair_clusters<EPI>(dev);           // persistent: as many pairs as are resident at once
     if (clusters > ntiles) clusters = ntiles;
     cfg.gridDim = dim3(2 * clusters, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, qlinear_bf16_kernel<EPI, true>, mA, mB, p);
+    e = cudaLaunchKernelEx(&cfg, qlinear_bf16_kernel<EPI, true>, mA, mB, q);
   } else {
     auto kern = qlinear_bf16_kernel<EPI, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
     if (e != cudaSuccess) return cuda_fail(e);
     cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
-    e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+    e = cudaLaunchKernelEx(&cfg, kern, mA, mB, q);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
