@@ -20,17 +20,21 @@
 //    stream-ordered workspace (4-bit codes by byte permutes over a 16-byte
 //    register table, other widths through a byte table in shared memory).
 //    The activation part (M*K bytes) stays in L2 for the GEMM.
-// 3. qlinear_8bit_kernel: persistent, one CTA per SM, 128 x 256 output
-//    tiles, K slices of 128 int8 values (one 128-byte swizzle row per operand
-//    row, so a stage is 16 KB of activations + 32 KB of weights):
+// 3. qlinear_8bit_kernel: persistent, on CTA pairs (256 x 256 output tiles,
+//    cta_group::2, 6 stages of 32 KB per CTA: 16 KB of activations and half
+//    the weight tile) when there is more than one 128-row tile of rows, else
+//    one CTA per SM (128 x 256 tiles, 4 stages of 48 KB); K slices of 128
+//    int8 values (one 128-byte swizzle row per operand row):
 //      warps 0..3  epilogue: TMEM lane quadrant, one output row per thread;
 //                  int32 -> fp32, times s_m r'_n / (alpha_w alpha_a), BF16.
-//      warp 4      MMA issuer (one thread): four 128x256x32 kind::i8 MMAs
-//                  per slice (+32 bytes of K per step) into one of two int32
-//                  TMEM accumulators, so the epilogue of tile i overlaps the
-//                  MMAs of tile i+1.
-//      warp 5      TMA producer (one thread): both operand tiles of each slice
-//                  into a 4-stage ring, 128B-swizzled K-major.
+//      warp 4      MMA issuer (one thread; the even CTA's for a pair): four
+//                  kind::i8 MMAs per slice (+32 bytes of K per step) into one
+//                  of two int32 TMEM accumulators, so the epilogue of tile i
+//                  overlaps the MMAs of tile i+1.
+//      warp 5      TMA producer (one thread): this CTA's operand tiles of
+//                  each slice into the ring, 128B-swizzled K-major; no
+//                  multicast (a pair splits the weight tile, it does not
+//                  copy it).
 // (Expanding the activation codes inside the GEMM, as the fp16 qlinear kernel
 // does, measured slower here: at twice the tensor rate the expansion warps
 // set the pace, 57.3 vs 51.4 us at 4608 x 3072 x 3072 W4A4.)
@@ -55,11 +59,27 @@ using qfast::prmt;
 
 constexpr int kBM = 128, kBN = 256, kBK = 128;  // K values per slice (= bytes per operand row)
 constexpr int kATile = kBM * kBK;               // 16 KB int8 activation tile
-constexpr int kBTile = kBN * kBK;               // 32 KB int8 weight tile
-constexpr int kOpStage = kATile + kBTile;       // 48 KB per operand stage
-constexpr int kAStages = 4;                     // operand stages
+constexpr int kMaxStages = 6;
 constexpr int kThreads = 192;                   // 6 warps
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
+
+// Single-SM tiles are 128 x 256 (the CTA holds the whole 256 x 128 weight
+// tile of a slice, 4 stages of 48 KB); CTA-pair tiles are 256 x 256 (each CTA
+// holds its 128 activation rows and 128 of the 256 weight rows, 6 stages of
+// 32 KB; one thread of the even CTA issues the cta_group::2 MMAs), as in the
+// fp16 GEMM of rbq_qlinear_int8_fast.cu.  At twice the fp16 tensor rate the
+// single SM's 48 KB per slice arrive too slowly; the pair halves the weight
+// bytes per SM.
+template <bool PAIR>
+struct Geom {
+  static constexpr int kTileM = PAIR ? 2 * kBM : kBM;
+  static constexpr int kBNc = PAIR ? kBN / 2 : kBN;       // weight rows loaded per CTA
+  static constexpr int kBTile = kBNc * kBK;               // 16 KB / 32 KB
+  static constexpr int kStage = kATile + kBTile;          // 32 KB / 48 KB
+  static constexpr int kStages = PAIR ? 6 : 4;
+};
+static_assert(Geom<true>::kStages * Geom<true>::kStage == Geom<false>::kStages * Geom<false>::kStage,
+              "both geometries use the same shared memory");
 
 // Instruction descriptor of kind::i8: s32 accumulator (D format 2), signed
 // 8-bit A and B (format 1), both K-major, N>>3 at bit 17, M>>4 at bit 24.
@@ -91,6 +111,26 @@ __device__ __forceinline__ void umma_8bit(uint32_t tmem_d, uint64_t adesc, uint6
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+}
+// The same over a CTA pair (M = 256), issued by one thread of the even CTA.
+template <bool kFp8>
+__device__ __forceinline__ void umma_8bit_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  if constexpr (kFp8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
   }
@@ -139,8 +179,8 @@ struct Params {
 };
 
 struct __align__(8) Tail {
-  uint64_t full[kAStages];
-  uint64_t empty[kAStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;                // abort path only: completion of the MMAs issued
@@ -148,91 +188,133 @@ struct __align__(8) Tail {
   volatile uint32_t abort;
 };
 
-constexpr size_t kSmem = 1024 + kAStages * kOpStage + sizeof(Tail) + 64;
+constexpr size_t kSmem = 1024 + Geom<false>::kStages * Geom<false>::kStage + sizeof(Tail) + 64;
 
-template <bool kFp8>
+template <bool kFp8, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     qlinear_8bit_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const Params p) {
+  using G = Geom<PAIR>;
+  constexpr int kS = G::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* ops = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  Tail* tl = reinterpret_cast<Tail*>(ops + kAStages * kOpStage);
+  Tail* tl = reinterpret_cast<Tail*>(ops + kS * G::kStage);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ntiles_m = (p.M + kBM - 1) / kBM, ntiles_n = (p.N + kBN - 1) / kBN;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;       // CTA within the pair
+  const int tile0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int tstep = PAIR ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
+  const int ntiles_m = (p.M + G::kTileM - 1) / G::kTileM, ntiles_n = (p.N + kBN - 1) / kBN;
   const int ntiles = ntiles_m * ntiles_n;
   const int KS = p.K / kBK;
   volatile uint32_t* abort = &tl->abort;
 
   if (tid == 0) {
-    for (int s = 0; s < kAStages; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(&tl->full[s], 1);
       mbar_init(&tl->empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tl->acc_full[a], 1);
-      mbar_init(&tl->acc_empty[a], 128);
+      mbar_init(&tl->acc_empty[a], PAIR ? 8 : 4);    // one arrival per epilogue warp (of both CTAs)
     }
     mbar_init(&tl->drain, 1);
     tl->abort = 0u;
     mbar_fence_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&tl->tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(&tl->tmem_slot, 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&tl->tmem_slot, 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // A pair's barriers are signalled from both CTAs: both must be initialised.
+  if constexpr (PAIR)
+    cluster_sync();
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tl->tmem_slot;
   griddep_wait();
   griddep_launch_dependents();
 
   if (warp == kMmaWarp) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t kIdesc = kFp8 ? idesc_e4m3(kBM, kBN) : idesc_i8(kBM, kBN);
+    // ---------------- MMA issuer (the even CTA's, for a pair) ----------------
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdesc = kFp8 ? idesc_e4m3(G::kTileM, kBN) : idesc_i8(G::kTileM, kBN);
       const uint64_t desc0 = sdesc_k_sw128(smem_u32(ops));
       uint32_t s = 0, ph = 0, it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep, ++it) {
         const uint32_t a = it & 1u, use = it >> 1;
-        if (use >= 1 && !mbar_wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, abort)) { ok = false; break; }
+        if (use >= 1) {
+          const bool got = PAIR ? mbar_wait_or_abort_cl(&tl->acc_empty[a], (use - 1) & 1, abort)
+                                : mbar_wait_or_abort(&tl->acc_empty[a], (use - 1) & 1, abort);
+          if (!got) { ok = false; break; }
+        }
         tc_fence_after();
         const uint32_t acc = tmem + a * kBN;
         for (int ks = 0; ks < KS; ++ks) {
           if (!mbar_wait_or_abort(&tl->full[s], ph, abort)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(kOpStage)) >> 4);
+          const uint64_t ad = desc0 + ((s * static_cast<uint32_t>(G::kStage)) >> 4);
           const uint64_t bd = ad + (kATile >> 4);
-          umma_8bit<kFp8>(acc, ad, bd, kIdesc, ks != 0);
-          umma_8bit<kFp8>(acc, ad + 2, bd + 2, kIdesc, 1u);            // +32 bytes = 32 values of K
-          umma_8bit<kFp8>(acc, ad + 4, bd + 4, kIdesc, 1u);
-          umma_8bit<kFp8>(acc, ad + 6, bd + 6, kIdesc, 1u);
-          umma_commit(&tl->empty[s]);
-          if (++s == kAStages) { s = 0; ph ^= 1u; }
+          if constexpr (PAIR) {
+            umma_8bit_pair<kFp8>(acc, ad, bd, kIdesc, ks != 0);
+            umma_8bit_pair<kFp8>(acc, ad + 2, bd + 2, kIdesc, 1u);     // +32 bytes = 32 values of K
+            umma_8bit_pair<kFp8>(acc, ad + 4, bd + 4, kIdesc, 1u);
+            umma_8bit_pair<kFp8>(acc, ad + 6, bd + 6, kIdesc, 1u);
+            umma_commit_pair(&tl->empty[s], 3);                          // stage s of both CTAs
+          } else {
+            umma_8bit<kFp8>(acc, ad, bd, kIdesc, ks != 0);
+            umma_8bit<kFp8>(acc, ad + 2, bd + 2, kIdesc, 1u);
+            umma_8bit<kFp8>(acc, ad + 4, bd + 4, kIdesc, 1u);
+            umma_8bit<kFp8>(acc, ad + 6, bd + 6, kIdesc, 1u);
+            umma_commit(&tl->empty[s]);
+          }
+          if (++s == kS) { s = 0; ph ^= 1u; }
         }
-        if (ok) umma_commit(&tl->acc_full[a]);
+        if (ok) {
+          if constexpr (PAIR)
+            umma_commit_pair(&tl->acc_full[a], 3);
+          else
+            umma_commit(&tl->acc_full[a]);
+        }
       }
       if (!ok) atomicOr(p.err, 2u);
     }
   } else if (warp == kTmaWarp) {
     // ---------------- TMA producer ----------------
+    // For a pair each CTA loads its own activation rows and its half of the
+    // weight rows; both CTAs' bytes are counted on the even CTA's barrier.
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
       uint32_t s = 0, ph = 0;
       bool first = true, ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
         const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
         const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
+        const int m0 = mt * G::kTileM + static_cast<int>(rank) * kBM;
+        const int n0 = nt * kBN + static_cast<int>(rank) * G::kBNc;
         for (int ks = 0; ks < KS; ++ks) {
           if (!first && !mbar_wait_or_abort(&tl->empty[s], ph ^ 1u, abort)) { ok = false; break; }
-          uint8_t* st = ops + s * kOpStage;
-          mbar_arrive_expect_tx(&tl->full[s], kOpStage);
-          tma_load_2d(st, &tmA, ks * kBK, mt * kBM, &tl->full[s]);
-          tma_load_2d(st + kATile, &tmB, ks * kBK, nt * kBN, &tl->full[s]);
-          if (++s == kAStages) { s = 0; ph ^= 1u; first = false; }
+          uint8_t* st = ops + s * G::kStage;
+          if constexpr (PAIR) {
+            if (rank == 0) mbar_arrive_expect_tx(&tl->full[s], 2 * G::kStage);
+            const uint32_t bar = mapa_shared(&tl->full[s], 0);
+            tma_load_2d_pair(st, &tmA, ks * kBK, m0, bar);
+            tma_load_2d_pair(st + kATile, &tmB, ks * kBK, n0, bar);
+          } else {
+            mbar_arrive_expect_tx(&tl->full[s], G::kStage);
+            tma_load_2d(st, &tmA, ks * kBK, m0, &tl->full[s]);
+            tma_load_2d(st + kATile, &tmB, ks * kBK, n0, &tl->full[s]);
+          }
+          if (++s == kS) { s = 0; ph ^= 1u; first = false; }
         }
       }
       if (!ok) atomicOr(p.err, 16u);
@@ -240,9 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------- epilogue ----------------
     const int q = warp;                     // TMEM lane quadrant
-    const int r = 32 * q + lane;            // row within the tile
+    const int r = 32 * q + lane;            // row within this CTA's 128 rows of the tile
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    for (int tile = tile0; tile < ntiles; tile += tstep, ++it) {
       const uint32_t a = it & 1u, use = it >> 1;
       if (!mbar_warp_wait(&tl->acc_full[a], use & 1, abort)) {   // warp-uniform: tmem loads follow
         if (lane == 0) atomicOr(p.err, 4u);
@@ -251,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
       const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
-      const int m = mt * kBM + r;
+      const int m = mt * G::kTileM + static_cast<int>(rank) * kBM + r;
       const float rs = (m < p.M) ? p.s[m] * p.inv_scale : 0.f;
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
@@ -287,20 +369,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // accumulator drained: one arrival per warp, on the even CTA's barrier
       tc_fence_before();
-      mbar_arrive(&tl->acc_empty[a]);
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(&tl->acc_empty[a], 0));
+        else
+          mbar_arrive(&tl->acc_empty[a]);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (tl->abort) {                 // the same value in every thread after the barrier
-    drain_after_abort(warp == kMmaWarp && lane == 0, &tl->drain);
+    drain_after_abort(warp == kMmaWarp && lane == 0 && rank == 0, &tl->drain, PAIR);
     __syncthreads();
   }
+  // Neither CTA of a pair leaves while the other may still signal its
+  // barriers or the MMAs may still read its shared memory.
+  if constexpr (PAIR) cluster_sync();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
   }
 }
 
@@ -407,7 +502,34 @@ int encode_i8_map(CUtensorMap* map, const int8_t* base, int rows, int K, int box
   return r == CUDA_SUCCESS ? RBQ_OK : RBQ_ECUDA;
 }
 
-// The GEMM on expanded int8 operands: activations `ai8` [M, K], weights `wi8` [N, K].
+// Resident clusters of two for the pair kernel on device `dev` (0: none
+// could be co-scheduled), queried once per device.
+template <bool kFp8>
+int pair_clusters(int dev) {
+  static int cached[kMaxDevices] = {};        // 0 = not yet asked; else clusters + 1
+  if (cached[dev]) return cached[dev] - 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, qlinear_8bit_kernel<kFp8, true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached[dev] = n + 1;
+  return n;
+}
+
+// The GEMM on expanded int8 operands: activations `ai8` [M, K], weights `wi8`
+// [N, K]; on CTA pairs when there is more than one 128-row tile of rows.
 template <bool kFp8>
 int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* rnorm, int M, int N, int K,
          uint16_t* Y, float inv_scale, unsigned int* err, cudaStream_t st, int sms) {
@@ -424,25 +546,49 @@ int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* r
   // CTAs then shares a few activation tiles and sweeps the (smaller) weights
   // (measured 2 % faster on 32760 x 8960 x 1536, 20 % on 32760 x 1536 x 8960)
   p.n_fast = M > N;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return RBQ_EINVAL;
+  bool pair = M > kBM;
+  if (pair) {
+    e = cudaFuncSetAttribute(qlinear_8bit_kernel<kFp8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem));
+    if (e != cudaSuccess) return cuda_fail(e);
+    pair = pair_clusters<kFp8>(dev) >= 1;
+  }
+  const int tile_m = pair ? Geom<true>::kTileM : Geom<false>::kTileM;
   CUtensorMap mA, mB;
   int rc = encode_i8_map(&mA, ai8, M, K, kBM);
   if (rc != RBQ_OK) return rc;
-  if ((rc = encode_i8_map(&mB, wi8, N, K, kBN)) != RBQ_OK) return rc;
-  auto kern = qlinear_8bit_kernel<kFp8>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
-  if (e != cudaSuccess) return cuda_fail(e);
-  const int ntiles = ((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+  if ((rc = encode_i8_map(&mB, wi8, N, K, pair ? Geom<true>::kBNc : Geom<false>::kBNc)) != RBQ_OK) return rc;
+  const int ntiles = ((M + tile_m - 1) / tile_m) * ((N + kBN - 1) / kBN);
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+  if (pair) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    int clusters = pair_clusters<kFp8>(dev);          // persistent: as many pairs as are resident at once
+    if (clusters > ntiles) clusters = ntiles;
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, qlinear_8bit_kernel<kFp8, true>, mA, mB, p);
+  } else {
+    auto kern = qlinear_8bit_kernel<kFp8, false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+    if (e != cudaSuccess) return cuda_fail(e);
+    cfg.gridDim = dim3(ntiles < sms ? ntiles : sms, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kern, mA, mB, p);
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e == cudaSuccess ? RBQ_OK : cuda_fail(e);
 }
