@@ -57,6 +57,11 @@ fused.gelu             y * Phi(y) with Phi from scipy.stats.norm (a library
                        published values
 fused.qlinear_int8_    composition of pinned parts; a pure-Python triple
   rotate_next          loop and an explicit dense Pi on a tiny case
+fused.qlinear_         the same on the code layer: a pure-Python triple
+  rotate_next          loop over the levels and an explicit dense Pi
+quant.quantize_        steps 2-4 alone: quantize_rotated(Pi x) reproduces
+  rotated              quantize_act(x, Pi) exactly; brute-force nearest
+                       level on a tiny case
 =====================  ===================================================
 """
 
@@ -64,19 +69,19 @@ from .rng import splitmix64, rpbh_draw
 from .rpbh import hadamard, rpbh_matrix, rpbh_rows, rpbh_apply
 from .lloydmax import lloydmax_unit, lloydmax_table, lloydmax_distortion_unit
 from .bf16 import round_to_bf16
-from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act,
+from .quant import (assign_codes, pack_codes, unpack_codes, quantize_act, quantize_rotated,
                     quantize_weights_lloydmax, quantize_weights_int8,
                     quantize_weights_int8_asym, rotate_only, EPS)
 from .qlinear import (qlinear, qlinear_int8, qlinear_int8_asym, int8_levels, qlinear_int8_levels,
                       e4m3_round, fp8_levels, qlinear_fp8_levels)
-from .fused import gelu, qlinear_int8_rotate_next
+from .fused import gelu, qlinear_int8_rotate_next, qlinear_rotate_next
 
 __all__ = [
     "splitmix64", "rpbh_draw", "hadamard", "rpbh_matrix", "rpbh_rows", "rpbh_apply",
     "lloydmax_unit", "lloydmax_table", "lloydmax_distortion_unit",
     "round_to_bf16", "assign_codes", "pack_codes", "unpack_codes",
-    "quantize_act", "quantize_weights_lloydmax", "quantize_weights_int8",
+    "quantize_act", "quantize_rotated", "quantize_weights_lloydmax", "quantize_weights_int8",
     "quantize_weights_int8_asym", "rotate_only", "EPS", "qlinear", "qlinear_int8",
     "qlinear_int8_asym", "int8_levels", "qlinear_int8_levels", "e4m3_round", "fp8_levels",
-    "qlinear_fp8_levels", "gelu", "qlinear_int8_rotate_next",
+    "qlinear_fp8_levels", "gelu", "qlinear_int8_rotate_next", "qlinear_rotate_next",
 ]

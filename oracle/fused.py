@@ -12,6 +12,10 @@ layer's permutation is what the parity test checks):
     x_next  = act(y)                               act = identity or GELU
     x'_next = Pi_next x_next                       (rotate_only, before BF16 rounding)
 
+The same with the code layer of OrbitQuant §2.2 as the producer (y = s_m r'_n
+sum_k C_w[q_nk] C_a[p_mk]), whose output the next layer then quantises from
+x'_next with steps 2-4 only (quant.quantize_rotated).
+
 GELU is the exact one (the page's synthetic MLP inputs are "GELU-shaped"; no
 page fixes a variant): gelu(y) = y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)),
 evaluated as 0.5 y erfc(-y / sqrt 2), which has no cancellation for negative y.
@@ -22,7 +26,7 @@ import math
 import numpy as np
 from scipy.special import erfc
 
-from .qlinear import qlinear_int8
+from .qlinear import qlinear, qlinear_int8
 from .quant import rotate_only
 
 
@@ -35,5 +39,12 @@ def gelu(y):
 def qlinear_int8_rotate_next(xr, q, scale, Pi_next, activation="gelu"):
     """x'_next = Pi_next act(qlinear_int8(x', q, scale)) in fp64 (unrounded)."""
     y = qlinear_int8(xr, q, scale)
+    x = gelu(y) if activation == "gelu" else y
+    return rotate_only(x, Pi_next)["xr"]
+
+
+def qlinear_rotate_next(a_codes, s, levels_a, w_codes, rnorm, levels_w, Pi_next, activation="gelu"):
+    """x'_next = Pi_next act(qlinear(codes...)) in fp64 (unrounded)."""
+    y = qlinear(a_codes, s, levels_a, w_codes, rnorm, levels_w)
     x = gelu(y) if activation == "gelu" else y
     return rotate_only(x, Pi_next)["xr"]

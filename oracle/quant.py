@@ -65,6 +65,18 @@ def _direction_quantise(Xr, bounds, eps):
     return assign_codes(V, bounds), norms, V
 
 
+def quantize_rotated(Xr, bounds, eps=EPS):
+    """OrbitQuant §2.2 steps 2-4 on rows that are already rotated (x' = Pi x
+    computed elsewhere, e.g. by the producing layer): s = ||x'||, codes of
+    x'/(s + eps).
+
+    Returns dict(codes int64[T,d], norms fp64[T], v fp64[T,d]).
+    """
+    Xr = np.asarray(Xr, dtype=np.float64)
+    codes, norms, V = _direction_quantise(Xr, bounds, eps)
+    return {"codes": codes, "norms": norms, "v": V}
+
+
 def quantize_act(X, Pi, bounds, eps=EPS):
     """OrbitQuant §2.2 steps 1-4 on each row of X.
 

@@ -55,3 +55,51 @@ def test_published_erf_approximation_meets_its_bound():
     t = 1.0 / (1.0 + p * x)
     poly = t * (a[0] + t * (a[1] + t * (a[2] + t * (a[3] + t * a[4]))))
     assert np.max(np.abs(poly * np.exp(-x * x) - erfc(x))) <= 1.5e-7
+
+
+def test_code_layer_fused_against_a_triple_loop_and_dense_rotation():
+    g = np.random.default_rng(4)
+    M, K, N, ba, bw = 3, 64, 128, 3, 2
+    levels_a, _ = oracle.lloydmax_table(K, ba)
+    levels_w, _ = oracle.lloydmax_table(K, bw)
+    a = g.integers(0, 2 ** ba, (M, K))
+    w = g.integers(0, 2 ** bw, (N, K))
+    s = g.random(M) + 0.5
+    rn = g.random(N) + 0.5
+    perm, signs = oracle.rpbh_draw(N, 10)
+    Pi = oracle.rpbh_matrix(perm, signs)
+    for act in ("gelu", "none"):
+        got = oracle.qlinear_rotate_next(a, s, levels_a, w, rn, levels_w, Pi, activation=act)
+        ref = np.zeros((M, N))
+        for m in range(M):
+            x = []
+            for j in range(N):
+                yj = s[m] * rn[j] * sum(float(levels_w[w[j, k]]) * float(levels_a[a[m, k]]) for k in range(K))
+                x.append(0.5 * yj * (1 + math.erf(yj / math.sqrt(2))) if act == "gelu" else yj)
+            for r in range(N):
+                ref[m, r] = sum(Pi[r, c] * x[c] for c in range(N))
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_quantize_rotated_is_steps_two_to_four_of_quantize_act():
+    """Rotating first and quantising the rotated rows gives exactly what
+    quantize_act gives from the unrotated rows (same norms, directions, codes);
+    on a tiny case every code is the brute-force nearest level."""
+    g = np.random.default_rng(5)
+    d, bits = 256, 4
+    X = g.standard_normal((9, d)) * np.linspace(0.1, 10, 9)[:, None]
+    X[4] = 0.0
+    perm, signs = oracle.rpbh_draw(d, 2)
+    Pi = oracle.rpbh_matrix(perm, signs)
+    levels, bounds = oracle.lloydmax_table(d, bits)
+    full = oracle.quantize_act(X, Pi, bounds)
+    part = oracle.quantize_rotated(oracle.rpbh_apply(Pi, X), bounds)
+    assert np.array_equal(part["codes"], full["codes"])
+    assert np.array_equal(part["norms"], full["norms"])
+    assert np.array_equal(part["v"], full["v"])
+    v = part["v"]
+    nearest = np.argmin(np.abs(v[..., None] - levels[None, None, :]), axis=-1)
+    tie = np.isclose(np.abs(v[..., None] - levels).min(-1),
+                     np.sort(np.abs(v[..., None] - levels), axis=-1)[..., 1], rtol=0, atol=1e-15)
+    assert np.array_equal(part["codes"][~tie], nearest[~tie])
+    assert np.all(part["codes"][4] == 2 ** (bits - 1))
