@@ -688,6 +688,52 @@ def run_suite(dev, stream, pk):
     nxt.close()
     del W, X, xr, q, sc, qn, scn, y, g, xn
 
+    # The same fusion on the code layer (OrbitQuant §2.2): the MLP pair's
+    # up-projection (4608 tokens, 3072 -> 12288, W2A4) whose GELU output is the
+    # down-projection's input, quantised at d = 12288 with 4-bit codes.
+    # Unfused: qlinear (BF16 y) -> GELU (torch) -> rotate_quantize_act.
+    # Fused: qlinear_rotate_next (the rotation in the epilogue, BF16 x') ->
+    # quantize_rotated (norm and codes only).
+    m = synth.mlp()
+    Xu, Wu = to_bf16_tensor(m["X_up"], dev), to_bf16_tensor(m["W_up"], dev)
+    ru, nxt = rbq.RPBH(3072, 11), rbq.RPBH(12288, 12)
+    au, su = rbq.rotate_quantize_act(ru, Xu, 4)
+    wu, nu = rbq.quantize_weights(ru, Wu, 2)
+    wn, nn_ = rbq.rows_in_next_order(nxt, wu), rbq.rows_in_next_order(nxt, nu)
+    y = torch.empty((4608, 12288), dtype=torch.bfloat16, device=dev)
+    g = torch.empty_like(y)
+    xn = torch.empty_like(y)
+    cn = torch.empty((4608, 12288 * 4 // 8), dtype=torch.uint8, device=dev)
+    sn = torch.empty((4608,), dtype=torch.float32, device=dev)
+
+    def unfused_codes():
+        rbq.qlinear(au, su, 4, wu, nu, 2, 3072, y, stream=stream)
+        torch.nn.functional.gelu(y, out=g)
+        rbq.rotate_quantize_act(nxt, g, 4, cn, sn, stream=stream)
+
+    def fused_codes():
+        rbq.qlinear_rotate_next(au, su, 4, wn, nn_, 2, 3072, nxt, "gelu", xn, stream=stream)
+        rbq.quantize_rotated(xn, 4, cn, sn, stream=stream)
+
+    us_un = _time_us(unfused_codes, stream)
+    us_gemm = _time_us(lambda: rbq.qlinear(au, su, 4, wu, nu, 2, 3072, y, stream=stream), stream)
+    us_rq = _time_us(lambda: rbq.rotate_quantize_act(nxt, g, 4, cn, sn, stream=stream), stream)
+    us_fused = _time_us(fused_codes, stream)
+    us_fgemm = _time_us(lambda: rbq.qlinear_rotate_next(au, su, 4, wn, nn_, 2, 3072, nxt, "gelu", xn,
+                                                        stream=stream), stream)
+    us_qr = _time_us(lambda: rbq.quantize_rotated(xn, 4, cn, sn, stream=stream), stream)
+    out["fused_rotation_mlp_w2a4_up_into_down_a4"] = {
+        "unfused_us": round(us_un, 2),
+        "unfused_parts_us": {"qlinear": round(us_gemm, 2), "gelu (torch)": round(us_un - us_gemm - us_rq, 2),
+                             "rotate_quantize_act d=12288": round(us_rq, 2)},
+        "fused_us": round(us_fused, 2),
+        "fused_parts_us": {"qlinear_rotate_next": round(us_fgemm, 2), "quantize_rotated d=12288": round(us_qr, 2)},
+        "speedup": round(us_un / us_fused, 3),
+        "quantize_rotated": rotq_entry(us_qr, 4608, 12288, 4)}
+    ru.close()
+    nxt.close()
+    del m, Xu, Wu, au, su, wu, nu, wn, nn_, y, g, xn, cn, sn
+
     # video DiT W4A6: 32760 tokens (21 frames x 1560), hidden 1536, MLP 8960
     T = 32760
     vid = {}

@@ -400,7 +400,8 @@ int rpbh_gather_rows(const rbq_rpbh* r, const void* src, long long row_bytes, vo
  *                     pi_next(k) (rpbh_gather_rows on the quantize_weights rows)
  *   scale_next_order  device fp32 [N], reordered the same way
  *   next              the RPBH handle of the next layer; N = its d
- *   activation        RBQ_ACT_NONE or RBQ_ACT_GELU (fp32, with CUDA's erfcf)
+ *   activation        RBQ_ACT_NONE or RBQ_ACT_GELU (fp32; the normal CDF by
+ *                     Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7)
  *   Xrot_next         device BF16 [M, N], row-major
  * K a multiple of 64 (else RBQ_EINVAL).  Stream-ordered like qlinear_int8
  * (same workspace).
@@ -409,6 +410,48 @@ int rpbh_gather_rows(const rbq_rpbh* r, const void* src, long long row_bytes, vo
 int qlinear_int8_rotate_next(const uint16_t* Xrot, const int8_t* Wq_next_order, const float* scale_next_order,
                              int M, int K, const rbq_rpbh* next, int activation, uint16_t* Xrot_next,
                              void* stream);
+
+/*
+ * qlinear_rotate_next -- the code layer of qlinear fused with the rotation of
+ * the next layer's input (OrbitQuant §6.2 on the §2.2 layer):
+ *   y[m, j]          = s[m] r'[j] sum_k C_w[q_jk] C_a[p_mk]   (the producing layer)
+ *   Xrot_next[m, :]  = bf16( Pi_next act(y[m, :]) )
+ * as qlinear_int8_rotate_next does for the W8A16 layer; the next layer then
+ * finishes its quantiser with quantize_rotated (no gather, no butterfly).
+ *   a_codes, s, bits_a     the producing layer's activation codes and norms, as
+ *                          for qlinear (M rows, K = its input width)
+ *   w_codes_next_order     device uint8 [N, K*bits_w/8]: row k = the layer's
+ *                          output channel pi_next(k) (rpbh_gather_rows on the
+ *                          quantize_weights rows, row_bytes = K*bits_w/8)
+ *   rnorm_next_order       device BF16 [N], reordered the same way (row_bytes 2)
+ *   next                   the next layer's RPBH handle; N = its d
+ *   activation             RBQ_ACT_NONE or RBQ_ACT_GELU
+ *   Xrot_next              device BF16 [M, N], row-major
+ * K a multiple of 128 with K*bits_a/8 a multiple of 16, N a multiple of 64
+ * (else RBQ_EINVAL).  Stream-ordered like qlinear (its workspace holds both
+ * operands' fp16 levels).
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int qlinear_rotate_next(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes_next_order,
+                        const uint16_t* rnorm_next_order, int bits_w, int M, int K, const rbq_rpbh* next,
+                        int activation, uint16_t* Xrot_next, void* stream);
+
+/*
+ * quantize_rotated -- OrbitQuant §2.2 steps 2-4 on rows that are already
+ * rotated (x' = Pi_d x, e.g. from qlinear_rotate_next or rotate_act):
+ * s = ||x'||, codes of x' / (s + 1e-12) in the Lloyd-Max codebook of
+ * N(0, 1/d), packed as rotate_quantize_act packs them.
+ *   Xrot       device BF16 [T, d] (dtype must be RBQ_BF16), row-major
+ *   d          the row width (a multiple of 64; selects the codebook)
+ *   bits       1..8
+ *   codes_out  device uint8 [T, d*bits/8], 8-byte aligned
+ *   norms_out  device fp32 [T]
+ * A row whose norm is not finite is encoded as the zero vector (every code
+ * 2^(bits-1)) and its norm is stored as computed.  Asynchronous on `stream`.
+ * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
+ */
+int quantize_rotated(const void* Xrot, int dtype, int T, int d, int bits, void* codes_out, float* norms_out,
+                     void* stream);
 
 /* ---- quantised layer files ------------------------------------------------
  * The pages' "quantized model file" (INT8-convrot, section 1): the quantised

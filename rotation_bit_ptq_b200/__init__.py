@@ -68,6 +68,8 @@ SIGNATURES = {
     "rbq_code_grid": (_I, [_I, _I, _I, _P, _P, _P, _P]),
     "rpbh_gather_rows": (_I, [_P, _P, ctypes.c_longlong, _P, _P]),
     "qlinear_int8_rotate_next": (_I, [_P, _P, _P, _I, _I, _P, _I, _P, _P]),
+    "qlinear_rotate_next": (_I, [_P, _P, _I, _P, _P, _I, _I, _I, _P, _I, _P, _P]),
+    "quantize_rotated": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
 }
 
 _lib = None
@@ -550,6 +552,57 @@ def qlinear_int8_rotate_next(xrot, q_next_order, scale_next_order, next_rpbh, ac
                                               next_rpbh.handle, _ACTS[activation], _ptr(out), _stream(stream)),
                "qlinear_int8_rotate_next")
     return out
+
+
+def qlinear_rotate_next(a_codes, s, bits_a, w_codes_next_order, rnorm_next_order, bits_w, K, next_rpbh,
+                        activation="gelu", out=None, stream=None):
+    """The code layer of qlinear fused with the next layer's input rotation:
+    out = bf16(Pi_next act(s_m r'_n sum_k C_w[q_nk] C_a[p_mk])) as bfloat16
+    [M, next.d]; the weight codes and r' in the next layer's permutation order
+    (rows_in_next_order).  quantize_rotated then gives that layer's codes."""
+    import torch
+    for t, n, dt in ((a_codes, "a_codes", torch.uint8), (s, "s", torch.float32),
+                     (w_codes_next_order, "w_codes_next_order", torch.uint8),
+                     (rnorm_next_order, "rnorm_next_order", torch.bfloat16)):
+        _need_cuda(t, n, dt)
+    M = a_codes.shape[0]
+    N = next_rpbh.d
+    _need_shape(a_codes, (M, K * bits_a // 8), "a_codes")
+    _need_shape(s, (M,), "s")
+    _need_shape(w_codes_next_order, (N, K * bits_w // 8), "w_codes_next_order")
+    _need_shape(rnorm_next_order, (N,), "rnorm_next_order")
+    if activation not in _ACTS:
+        raise ValueError("activation must be None, 'none' or 'gelu'")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _need_cuda(out, "out", torch.bfloat16)
+    _need_shape(out, (M, N), "out")
+    with _device_ctx(a_codes, s, w_codes_next_order, rnorm_next_order, out):
+        _check(lib().qlinear_rotate_next(_ptr(a_codes), _ptr(s), int(bits_a), _ptr(w_codes_next_order),
+                                         _ptr(rnorm_next_order), int(bits_w), M, int(K), next_rpbh.handle,
+                                         _ACTS[activation], _ptr(out), _stream(stream)),
+               "qlinear_rotate_next")
+    return out
+
+
+def quantize_rotated(xrot, bits, codes=None, norms=None, stream=None):
+    """OrbitQuant §2.2 steps 2-4 on already rotated BF16 rows [T, d]: packed
+    codes uint8[T, d*bits/8] and norms float32[T]."""
+    import torch
+    _need_cuda(xrot, "xrot", torch.bfloat16)
+    T, d = xrot.shape
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=xrot.device)
+    if norms is None:
+        norms = torch.empty((T,), dtype=torch.float32, device=xrot.device)
+    _need_cuda(codes, "codes", torch.uint8)
+    _need_cuda(norms, "norms", torch.float32)
+    _need_shape(codes, (T, d * bits // 8), "codes")
+    _need_shape(norms, (T,), "norms")
+    with _device_ctx(xrot, codes, norms):
+        _check(lib().quantize_rotated(_ptr(xrot), _dtype_code(xrot), T, d, int(bits), _ptr(codes), _ptr(norms),
+                                      _stream(stream)), "quantize_rotated")
+    return codes, norms
 
 
 def _host_bytes(t):

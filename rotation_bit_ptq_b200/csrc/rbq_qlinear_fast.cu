@@ -831,7 +831,7 @@ int qlinear_fast_gemm(const uint8_t* a_codes, const float* s, int bits_a, const 
 // The TMA-fed GEMM on operands expanded beforehand (rbq_qlinear_int8_fast.cu).
 int qlinear_f16_operands_gemm(const uint16_t* af16, const float* s, const uint16_t* wf16, const uint16_t* rnorm,
                               float inv_k, int M, int N, int K, uint16_t* Y, unsigned int* err, cudaStream_t st,
-                              int sms);
+                              int sms, const float* next_sign = nullptr, int act = 0);
 
 int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
                         const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
@@ -862,6 +862,33 @@ int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, cons
     rc = qfast::expand_weights(w_codes, bits_w, N, K, cw->levels_f16, wf16, st, sms);
     if (rc == RBQ_OK) rc = qlinear_fast_gemm(a_codes, s, bits_a, wf16, rnorm, M, N, K, Y, ca, err, st, sms);
   }
+  e = cudaFreeAsync(ws, st);
+  if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
+  return rc;
+}
+
+// qlinear whose epilogue finishes the next layer's rotation (next_sign: its D
+// in output order; the weight rows and r' in its permutation's order): always
+// the expanded-operand route, whatever the activations' size.
+int qlinear_rotate_next_launch(const uint8_t* a_codes, const float* s, int bits_a, const uint8_t* w_codes,
+                               const uint16_t* rnorm, int bits_w, int M, int N, int K, uint16_t* Y,
+                               const CodebookDevice* ca, const CodebookDevice* cw, unsigned int* err,
+                               cudaStream_t st, const float* next_sign, int act) {
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaMemPool_t pool = qfast::workspace_pool(dev);
+  if (!pool) return RBQ_ECUDA;
+  void* ws = nullptr;
+  e = cudaMallocFromPoolAsync(&ws, (static_cast<size_t>(N) + M) * K * 2, pool, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  uint16_t* wf16 = static_cast<uint16_t*>(ws);
+  uint16_t* af16 = wf16 + static_cast<size_t>(N) * K;
+  int rc = qfast::expand_both(w_codes, bits_w, N, cw->levels_f16, wf16, a_codes, bits_a, M, ca->levels_f16, af16, K,
+                              st, sms);
+  if (rc == RBQ_OK)
+    rc = qlinear_f16_operands_gemm(af16, s, wf16, rnorm, ca->inv_d, M, N, K, Y, err, st, sms, next_sign, act);
   e = cudaFreeAsync(ws, st);
   if (rc == RBQ_OK && e != cudaSuccess) rc = cuda_fail(e);
   return rc;

@@ -80,7 +80,14 @@ enum Epi {
   kEpiRotateNext = 2,   // W8A16 whose output feeds the next rotated layer: per 64-column
                         // block, Y = bf16(H_64 D (act(acc * scale)) / 8), act = identity
   kEpiRotateNextGelu = 3,   // the same with act = GELU
+  kEpiCodesRotateNext = 4,      // qlinear on expanded code levels whose output feeds the next rotated
+                                // layer: y = acc * s[m] r'[n] / K, then as kEpiRotateNext
+  kEpiCodesRotateNextGelu = 5,  // the same with act = GELU
 };
+__host__ __device__ constexpr bool epi_codes(int epi) { return epi == kEpiCodes || epi >= kEpiCodesRotateNext; }
+__host__ __device__ constexpr bool epi_gelu(int epi) {
+  return epi == kEpiRotateNextGelu || epi == kEpiCodesRotateNextGelu;
+}
 
 // Threads per CTA: 4 epilogue warps + MMA warp + TMA warp; the rotating
 // epilogues add 4 more epilogue warps (warps 6..9), two per TMEM lane
@@ -106,6 +113,8 @@ struct Params {
 // erfc(x) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-x^2), and
 // Phi(y) = 1 - erfc(x) / 2 for y >= 0, erfc(x) / 2 for y < 0.  Phi is within
 // 1e-7 of the exact value, far below the BF16 rounding of the layer's output.
+// (A reciprocal by Newton-Raphson on the FMA pipe instead of the division
+// measured no faster.)
 __device__ __forceinline__ float gelu_as7126(float y) {
   const float x = fabsf(y) * 0.70710678118654752f;
   const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
@@ -219,7 +228,7 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
                         const Params p) {
   using G = Geom<PAIR>;
   constexpr int kS = G::kStages;
-  constexpr bool kQ = (EPI == kEpiCodes);
+  constexpr bool kQ = epi_codes(EPI);
   constexpr bool kRot = (EPI >= kEpiRotateNext);
   constexpr uint32_t kEpiWarps = epi_threads_for(EPI) / 32;
   extern __shared__ uint8_t smem_raw[];
@@ -391,12 +400,19 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
           tmem_wait_ld();
           const int n0 = nt * kBN + 64 * blk;
           if (m >= p.M || n0 >= p.N) continue;
+          // per-column factor: the W8A16 scale, or r'_n (BF16) for the code layer,
+          // whose per-row factor s_m / K comes in rs
+          const auto colf = [&](int n) {
+            if constexpr (kQ) return __uint_as_float(static_cast<uint32_t>(__ldg(p.rnorm + n)) << 16);
+            else return __ldg(p.scale + n);
+          };
+          const float rs = kQ ? p.s[m] * p.inv_k : 1.f;
           unsigned long long P[32];       // (z_i, z_{i+32})
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            float y0 = __uint_as_float(v0[i]) * __ldg(p.scale + n0 + i);
-            float y1 = __uint_as_float(v1[i]) * __ldg(p.scale + n0 + 32 + i);
-            if constexpr (EPI == kEpiRotateNextGelu) {
+            float y0 = __uint_as_float(v0[i]) * rs * colf(n0 + i);
+            float y1 = __uint_as_float(v1[i]) * rs * colf(n0 + 32 + i);
+            if constexpr (epi_gelu(EPI)) {
               y0 = gelu_as7126(y0);
               y1 = gelu_as7126(y1);
             }
@@ -583,7 +599,7 @@ int pair_clusters(int dev) {
 // rows and the device can co-schedule pairs, else on single SMs.
 template <int EPI>
 int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStream_t st, int sms) {
-  constexpr bool kQ = (EPI == kEpiCodes);
+  constexpr bool kQ = epi_codes(EPI);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -646,10 +662,12 @@ int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStrea
 
 }  // namespace q8fast
 
-// qlinear on expanded operands: `af16` [M, K] and `wf16` [N, K] fp16 levels x sqrt(K).
+// qlinear on expanded operands: `af16` [M, K] and `wf16` [N, K] fp16 levels x
+// sqrt(K).  next_sign != null: the epilogue finishes the next layer's rotation
+// (N % 64 == 0, the weight rows in the next permutation's order, act given).
 int qlinear_f16_operands_gemm(const uint16_t* af16, const float* s, const uint16_t* wf16, const uint16_t* rnorm,
                               float inv_k, int M, int N, int K, uint16_t* Y, unsigned int* err, cudaStream_t st,
-                              int sms) {
+                              int sms, const float* next_sign, int act) {
   q8fast::Params p{};
   p.M = M;
   p.N = N;
@@ -657,9 +675,12 @@ int qlinear_f16_operands_gemm(const uint16_t* af16, const float* s, const uint16
   p.s = s;
   p.rnorm = rnorm;
   p.inv_k = inv_k;
+  p.next_sign = next_sign;
   p.Y = Y;
   p.err = err;
-  return q8fast::launch_gemm<q8fast::kEpiCodes>(af16, wf16, p, st, sms);
+  if (!next_sign) return q8fast::launch_gemm<q8fast::kEpiCodes>(af16, wf16, p, st, sms);
+  if (act == RBQ_ACT_GELU) return q8fast::launch_gemm<q8fast::kEpiCodesRotateNextGelu>(af16, wf16, p, st, sms);
+  return q8fast::launch_gemm<q8fast::kEpiCodesRotateNext>(af16, wf16, p, st, sms);
 }
 
 bool qlinear_int8_fast_eligible(int M, int N, int K) {

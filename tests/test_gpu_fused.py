@@ -107,3 +107,94 @@ def test_fused_layer_dit_mlp_up_into_down_sampled():
     err = rel_frobenius(bf16_to_numpy(y[idx]), ref)
     print(f"fused DiT MLP up -> down rotation: rel. Frobenius error {err:.2e}")
     assert err < FUSED_RTOL, err
+
+
+# --------------------------------------------------------------------------
+# The code layer (OrbitQuant §2.2) fused with the next rotation, and the
+# next layer's quantiser on the rotated rows (quantize_rotated)
+# --------------------------------------------------------------------------
+
+from parity import check_codes, check_rel  # noqa: E402
+
+QLINEAR_RTOL = 4e-3        # rel. Frobenius, fp16 operands + BF16 output (bar: 2e-2)
+NORM_RTOL = 1e-5
+
+
+def _unpack(codes, bits, d):
+    return oracle.unpack_codes(codes.cpu().numpy(), bits, d)
+
+
+def _fused_codes_case(M, K, N, ba, bw, act, seed=0):
+    g = np.random.default_rng(M * 5 + K + N + ba + bw + seed)
+    X = synth.to_bf16(g.standard_t(3, (M, K)).astype(np.float32))
+    W = synth.to_bf16(synth.gaussian_weights(g, N, K, outlier_frac=0.01))
+    r, nxt = rbq.RPBH(K, seed + 3), rbq.RPBH(N, seed + 2000)
+    a, s = rbq.rotate_quantize_act(r, torch_bf16(X), ba)
+    w, rn = rbq.quantize_weights(r, torch_bf16(W), bw)
+    wn, rnn = rbq.rows_in_next_order(nxt, w), rbq.rows_in_next_order(nxt, rn)
+    y = rbq.qlinear_rotate_next(a, s, ba, wn, rnn, bw, K, nxt, activation=act, out=poison((M, N), torch.bfloat16))
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    la, _ = oracle.lloydmax_table(K, ba)
+    lw, _ = oracle.lloydmax_table(K, bw)
+    ref = oracle.qlinear_rotate_next(_unpack(a, ba, K), s.cpu().numpy().astype(np.float64), la, _unpack(w, bw, K),
+                                     rn.float().cpu().numpy().astype(np.float64), lw, _pi(N, seed + 2000),
+                                     activation=act)
+    got = bf16_to_numpy(y)
+    assert np.all(np.isfinite(got))
+    return rel_frobenius(got, ref), (a, s, w, rn, r, nxt, y)
+
+
+@pytest.mark.parametrize("M,K,N,ba,bw,act", [(1, 128, 64, 4, 4, "gelu"), (130, 256, 512, 4, 2, "gelu"),
+                                             (77, 384, 1024, 3, 3, "none"), (300, 512, 1536, 6, 4, "gelu"),
+                                             (257, 1024, 320, 2, 4, "none")])
+def test_fused_code_layer_ragged_shapes(M, K, N, ba, bw, act):
+    err, _ = _fused_codes_case(M, K, N, ba, bw, act)
+    print(f"fused W{bw}A{ba} -> rotation {M}x{K}->{N} act={act}: rel. Frobenius error {err:.2e}")
+    assert err < QLINEAR_RTOL, err
+
+
+@pytest.mark.parametrize("d,T,bits", [(64, 3, 1), (512, 40, 8), (1024, 37, 4), (3072, 130, 2), (3072, 65, 3),
+                                      (1536, 33, 6), (12288, 9, 5), (16384, 4, 7)])
+def test_quantize_rotated_matches_the_oracle(d, T, bits):
+    X, _ = synth.student_t_act(T, d, seed=d + bits)
+    X = X.copy()
+    X[0] = 0.0                                  # zero row: s = 0, every code 2^(b-1)
+    if T > 2:
+        X[2, 5] = np.nan                        # non-finite row: encoded as the zero vector
+    r = rbq.RPBH(d, 31)
+    xr = rbq.rotate_act(r, torch_bf16(X))
+    codes, norms = rbq.quantize_rotated(xr, bits, codes=poison((T, d * bits // 8), torch.uint8),
+                                        norms=poison((T,), torch.float32))
+    torch.cuda.synchronize()
+    assert rbq.device_error() == 0
+    g = _unpack(codes, bits, d)
+    assert np.all(g[0] == 2 ** (bits - 1)) and norms[0].item() == 0.0
+    good = np.arange(T) if T <= 2 else np.setdiff1d(np.arange(T), [2])
+    if T > 2:
+        assert np.all(g[2] == 2 ** (bits - 1))
+    _, bounds = oracle.lloydmax_table(d, bits)
+    ora = oracle.quantize_rotated(bf16_to_numpy(xr)[good], bounds)
+    check_codes(g[good], ora["codes"], ora["v"], bounds, d)
+    check_rel(norms.cpu().numpy()[good], ora["norms"], NORM_RTOL, "quantize_rotated norms")
+
+
+def test_fused_code_pipeline_against_the_unfused_one():
+    """The next layer's codes through the fused path (qlinear_rotate_next, then
+    quantize_rotated) and through the unfused one (qlinear, GELU, then
+    rotate_quantize_act) differ only where the two paths' BF16 roundings (of
+    x' in the first, of y and GELU(y) in the second) move a value across a
+    decision boundary: few codes, each by one level."""
+    M, K, N, ba, bw = 256, 1024, 3072, 4, 4
+    err, (a, s, w, rn, r, nxt, y) = _fused_codes_case(M, K, N, ba, bw, "gelu", seed=9)
+    assert err < QLINEAR_RTOL
+    c_f, s_f = rbq.quantize_rotated(y, 4)
+    y_un = rbq.qlinear(a, s, ba, w, rn, bw, K)
+    x_un = torch.nn.functional.gelu(y_un.float()).to(torch.bfloat16)
+    c_u, s_u = rbq.rotate_quantize_act(nxt, x_un, 4)
+    torch.cuda.synchronize()
+    g_f, g_u = _unpack(c_f, 4, N), _unpack(c_u, 4, N)
+    diff = g_f != g_u
+    assert diff.mean() < 0.02, diff.mean()
+    assert np.all(np.abs(g_f[diff] - g_u[diff]) == 1)
+    check_rel(s_f.cpu().numpy(), s_u.cpu().numpy(), 1e-2, "norms, fused vs unfused")
