@@ -50,6 +50,7 @@
 #include "rbq_internal.h"
 #include "rbq_qcodes.cuh"
 #include "rbq_sm100.cuh"
+#include "rbq_tiles.cuh"
 
 namespace rbq {
 namespace qi8 {
@@ -175,7 +176,7 @@ struct Params {
   float inv_scale;
   uint16_t* Y;
   unsigned int* err;
-  int n_fast;                 // tile order: N fastest (the activation operand is the larger)
+  int order;                  // tile order (tiles::TileOrder)
 };
 
 struct __align__(8) Tail {
@@ -297,8 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t s = 0, ph = 0;
       bool first = true, ok = true;
       for (int tile = tile0; tile < ntiles && ok; tile += tstep) {
-        const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
-        const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
+        int mt, nt;
+        tiles::tile_coords(tile, ntiles_m, ntiles_n, p.order, mt, nt);
         const int m0 = mt * G::kTileM + static_cast<int>(rank) * kBM;
         const int n0 = nt * kBN + static_cast<int>(rank) * G::kBNc;
         for (int ks = 0; ks < KS; ++ks) {
@@ -331,8 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int mt = p.n_fast ? tile / ntiles_n : tile % ntiles_m;
-      const int nt = p.n_fast ? tile % ntiles_n : tile / ntiles_m;
+      int mt, nt;
+      tiles::tile_coords(tile, ntiles_m, ntiles_n, p.order, mt, nt);
       const int m = mt * G::kTileM + static_cast<int>(rank) * kBM + r;
       const float rs = (m < p.M) ? p.s[m] * p.inv_scale : 0.f;
 #pragma unroll 1
@@ -542,10 +543,6 @@ int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* r
   p.inv_scale = inv_scale;
   p.Y = Y;
   p.err = err;
-  // walk N fastest when the int8 activations outweigh the weights: a wave of
-  // CTAs then shares a few activation tiles and sweeps the (smaller) weights
-  // (measured 2 % faster on 32760 x 8960 x 1536, 20 % on 32760 x 1536 x 8960)
-  p.n_fast = M > N;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -558,6 +555,7 @@ int gemm(const int8_t* ai8, const float* s, const int8_t* wi8, const uint16_t* r
     pair = pair_clusters<kFp8>(dev) >= 1;
   }
   const int tile_m = pair ? Geom<true>::kTileM : Geom<false>::kTileM;
+  p.order = tiles::tile_order(dev, 1LL * M * K, 1LL * N * K);
   CUtensorMap mA, mB;
   int rc = encode_i8_map(&mA, ai8, M, K, kBM);
   if (rc != RBQ_OK) return rc;

@@ -41,6 +41,7 @@
 #include "rbq_internal.h"
 #include "rbq_qcodes.cuh"
 #include "rbq_sm100.cuh"
+#include "rbq_tiles.cuh"
 
 namespace rbq {
 namespace q8fast {
@@ -48,6 +49,8 @@ namespace q8fast {
 using namespace sm100;
 using qfast::encode_fn;
 using qfast::workspace_pool;
+using tiles::tile_coords;
+using tiles::tile_order;
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr int kATile = kBM * kBK * 2;          // 16 KB
@@ -165,35 +168,6 @@ __device__ __forceinline__ void fwht64_pairs(unsigned long long (&P)[32]) {
     float lo, hi;
     upk2(P[i], lo, hi);
     P[i] = pk2(lo + hi, lo - hi);        // (z_i, z_{i+32})
-  }
-}
-
-// Order in which a CTA (pair) walks its output tiles, chosen on the host so
-// that the operand panels a wave of CTAs touches stay in L2:
-//   kOrderM  M fastest: a wave shares a few weight panels; the activation
-//            operand is read once if it stays in L2 (it fits in half of it);
-//   kOrderN  N fastest: a wave shares a few activation panels; for weights
-//            that fit in half of L2 (read once) and a larger activation
-//            operand (streamed once instead of once per column of tiles);
-//   kOrderGrouped  neither fits: groups of kGroupM row panels, N fastest
-//            inside a group, so a wave touches about kGroupM activation and
-//            ~waves/kGroupM weight panels.
-enum TileOrder { kOrderM = 0, kOrderN = 1, kOrderGrouped = 2 };
-constexpr int kGroupM = 8;
-
-__device__ __forceinline__ void tile_coords(int tile, int ntiles_m, int ntiles_n, int order, int& mt, int& nt) {
-  if (order == kOrderM) {
-    mt = tile % ntiles_m;
-    nt = tile / ntiles_m;
-  } else if (order == kOrderN) {
-    mt = tile / ntiles_n;
-    nt = tile % ntiles_n;
-  } else {
-    const int per_group = kGroupM * ntiles_n;
-    const int g = tile / per_group, r = tile - g * per_group;
-    const int m0 = g * kGroupM, gm = min(kGroupM, ntiles_m - m0);
-    mt = m0 + r % gm;
-    nt = r / gm;
   }
 }
 
@@ -613,18 +587,7 @@ int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStrea
   }
   const int tile_m = pair ? Geom<true>::kTileM : Geom<false>::kTileM;
   Params q = p;
-  {
-    // the operand panels that can stay in L2 (half of it, the rest for the
-    // output and the other operand's panels in flight)
-    int l2 = 0;
-    if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0) l2 = 126 << 20;
-    const long long half = static_cast<long long>(l2) / 2;
-    const long long a_bytes = 2LL * p.M * p.K, b_bytes = 2LL * p.N * p.K;
-    if (b_bytes <= half && a_bytes > b_bytes) q.order = kOrderN;
-    else if (a_bytes <= half) q.order = kOrderM;
-    else if (b_bytes <= half) q.order = kOrderN;
-    else q.order = kOrderGrouped;
-  }
+  q.order = tile_order(dev, 2LL * p.M * p.K, 2LL * p.N * p.K);
   CUtensorMap mA, mB;
   int rc = encode_bf16_map(&mA, A, p.M, p.K, kBM, kQ);
   if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, pair ? Geom<true>::kBNc : Geom<false>::kBNc, kQ);
