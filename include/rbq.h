@@ -217,9 +217,10 @@ int quantize_weights_int8_asym(const rbq_rpbh* r, const void* W, int dtype, int 
  * Alignment: code arrays 16-byte, Y 16-byte, s/rnorm 4-byte.
  * Workspace (K a multiple of 128, N of 8, 16-byte code rows): the weight codes
  * are expanded per call into fp16 levels, N*K*2 bytes from a stream-ordered
- * memory pool; activation widths other than 4 bits are expanded too, M*K*2
- * more bytes, while that part is at most 128 MiB.  Other shapes run a
- * general kernel that expands both operands tile by tile without a workspace.
+ * memory pool, and the activation codes too, M*K*2 more bytes, while that
+ * part is at most 2 GiB (beyond it the GEMM expands them itself).  Other
+ * shapes run a general kernel that expands both operands tile by tile
+ * without a workspace.
  * Errors: RBQ_EINVAL, RBQ_EALIGN, RBQ_ECUDA.
  */
 int qlinear(const uint8_t* a_codes, const float* s, int bits_a,

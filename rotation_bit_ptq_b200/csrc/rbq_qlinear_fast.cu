@@ -12,11 +12,12 @@
 // work for every tile of tokens and saturate the SM's integer pipe.
 //
 // Each call expands the weight codes [N, K]; then one of two routes:
-//  * activations whose fp16 copy (M*K*2 bytes) is at most 128 MiB are
+//  * activations whose fp16 copy (M*K*2 bytes) is at most 2 GiB are
 //    expanded the same way and the TMA-fed GEMM of rbq_qlinear_int8_fast.cu
 //    (on CTA pairs, epilogue s_m r'_n / K) multiplies the two fp16 operands;
-//  * larger activations stay packed and are expanded inside the GEMM below,
-//    which avoids writing and re-reading a copy that would not stay in L2.
+//  * larger activations stay packed and are expanded inside the GEMM below
+//    (as does the allocation-free entry point), which needs no workspace for
+//    them.
 //
 // 1. expand_codes_kernel: the weight codes (and, first route, the activation
 //    codes in the same launch) to fp16 levels.
@@ -843,11 +844,12 @@ int qlinear_fast_launch(const uint8_t* a_codes, const float* s, int bits_a, cons
   cudaMemPool_t pool = qfast::workspace_pool(dev);
   if (!pool) return RBQ_ECUDA;
   // The activation codes get their own pass into fp16 and the GEMM streams
-  // both operands by TMA on CTA pairs -- while that fp16 copy (M*K*2 bytes)
-  // is at most 128 MiB, beyond which writing and re-reading it costs more than
-  // it saves; larger activations are expanded inside the GEMM (qlinear_fast_kernel).
+  // both operands by TMA on CTA pairs -- faster than expanding them inside the
+  // GEMM at every measured size (587 MB of fp16 activations included) -- while
+  // that copy (M*K*2 bytes) is at most 2 GiB of workspace; beyond it the
+  // activations are expanded inside the GEMM (qlinear_fast_kernel).
   const size_t a_f16_bytes = static_cast<size_t>(M) * K * 2;
-  const bool split = a_f16_bytes <= (static_cast<size_t>(128) << 20);
+  const bool split = a_f16_bytes <= (static_cast<size_t>(2048) << 20);
   void* ws = nullptr;
   e = cudaMallocFromPoolAsync(&ws, static_cast<size_t>(N) * K * 2 + (split ? a_f16_bytes : 0), pool, st);
   if (e != cudaSuccess) return cuda_fail(e);

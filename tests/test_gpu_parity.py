@@ -653,8 +653,8 @@ def test_qlinear_int8_levels_mlp_down_sampled():
 
 @pytest.mark.parametrize("layer,M,N,K,ba,bw", [("fp16", 139264, 136, 1024, 4, 4), ("int8", 70000, 136, 1024, 4, 3)])
 def test_large_activation_operand_tiles_walked_n_fastest(layer, M, N, K, ba, bw):
-    """Activation operands larger than the weights (above 64 MiB for the
-    fp16-level kernel) make the GEMMs walk their output tiles N-fastest; random
+    """Activation operands larger than the weights, with weights that fit in
+    half of L2, make the pair GEMMs walk their output tiles N-fastest; random
     codes, sampled rows (the first, the last and tiles in between) against the
     oracle."""
     gen = torch.Generator(device="cuda").manual_seed(M)
@@ -684,12 +684,11 @@ def test_large_activation_operand_tiles_walked_n_fastest(layer, M, N, K, ba, bw)
 @pytest.mark.parametrize("n_out,d_in", [(1536, 1536), (8960, 1536), (1536, 8960)])
 def test_qlinear_video_w4a6_full_size_sampled(n_out, d_in):
     """The video-DiT workload (Wan 2.1 1.3B shape, OrbitQuant §3.2, W4A6):
-    32760 tokens = 21 frames x 1560 patches, hidden 1536, MLP 8960.  The two
-    1536-wide layers expand their 6-bit activation codes in a pass of their
-    own (the fp16 copy, 32760 x 1536 x 2 = 100 MB, fits the split route); the
-    8960-wide down-projection's copy would be 587 MB, so its GEMM expands the
-    6-bit codes itself (the shared-memory level table route).  Every token is
-    quantised on the GPU; sampled rows (first, last, others) are compared."""
+    32760 tokens = 21 frames x 1560 patches, hidden 1536, MLP 8960.  Every
+    layer expands its 6-bit activation codes in a pass of its own (fp16
+    copies of 100 MB and, for the 8960-wide down-projection, 587 MB) before
+    the pair GEMM.  Every token is quantised on the GPU; sampled rows (first,
+    last, others) are compared."""
     T = 32760
     X = synth.video_act(d_in, layer=7)
     assert X.shape == (T, d_in)
@@ -702,13 +701,13 @@ def test_qlinear_video_w4a6_full_size_sampled(n_out, d_in):
 
 @pytest.mark.parametrize("bits_a,bits_w", [(1, 4), (2, 3), (3, 4), (5, 2), (6, 4), (7, 8), (8, 1)])
 def test_qlinear_in_kernel_expansion_every_activation_width(bits_a, bits_w):
-    """Activation widths other than 4 bits take the in-kernel expansion route
-    (a shared-memory level table inside the GEMM) once their fp16 copy would
-    exceed 128 MiB: 70000 x 1024 x 2 bytes = 137 MiB here.  Random codes,
-    sampled rows (the first, the last and tiles in between) against the
-    oracle."""
-    M, N, K = 70000, 136, 1024
-    assert M * K * 2 > 128 << 20
+    """Activations whose fp16 copy would exceed 2 GiB take the in-kernel
+    expansion route (the codes expanded inside the GEMM: byte permutes at 2,
+    3 and 4 bits, a shared-memory level table otherwise): 1.1 M x 1024 x 2
+    bytes = 2.25 GB here.  Random codes, sampled rows (the first, the last and
+    tiles in between) against the oracle."""
+    M, N, K = 1_100_000, 136, 1024
+    assert M * K * 2 > 2 << 30
     gen = torch.Generator(device="cuda").manual_seed(bits_a * 16 + bits_w)
     a = torch.randint(0, 256, (M, K * bits_a // 8), dtype=torch.uint8, device="cuda", generator=gen)
     w = torch.randint(0, 256, (N, K * bits_w // 8), dtype=torch.uint8, device="cuda", generator=gen)

@@ -81,3 +81,34 @@ def test_noalloc_matches_qlinear_on_two_calls_in_a_row():
         print(f"qlinear_noalloc {M}x{N}x{K} W{bw}A{ba}: rel. Frobenius vs qlinear {e:.2e}, "
               f"{int(np.sum(got_np != ref_np))} differing elements")
         assert e < QLINEAR_RTOL, e
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("ba,bw", [(1, 4), (2, 3), (3, 4), (4, 4), (5, 2), (6, 4), (7, 8), (8, 1)])
+def test_noalloc_against_the_oracle_every_activation_width(ba, bw):
+    """qlinear_noalloc always expands the activation codes inside the GEMM (it
+    has no workspace for them), so it is also where that route meets the
+    oracle at sizes below qlinear's 2 GiB switch: random codes, ragged M and
+    N, every activation width."""
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import oracle
+    from parity import bf16_to_numpy, rel_frobenius
+    M, N, K = 300, 264, 1024
+    gen = torch.Generator(device="cuda").manual_seed(ba * 16 + bw)
+    a = torch.randint(0, 256, (M, K * ba // 8), dtype=torch.uint8, device="cuda", generator=gen)
+    w = torch.randint(0, 256, (N, K * bw // 8), dtype=torch.uint8, device="cuda", generator=gen)
+    s = torch.rand(M, device="cuda", generator=gen) + 0.5
+    rn = (torch.rand(N, device="cuda", generator=gen) + 0.5).to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rbq.qlinear_noalloc(a, s, ba, w, rn, bw, K, y, err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0 and rbq.device_error() == 0
+    la, _ = oracle.lloydmax_table(K, ba)
+    lw, _ = oracle.lloydmax_table(K, bw)
+    ref = oracle.qlinear(oracle.unpack_codes(a.cpu().numpy(), ba, K), s.cpu().numpy(), la,
+                         oracle.unpack_codes(w.cpu().numpy(), bw, K), bf16_to_numpy(rn), lw)
+    e = rel_frobenius(bf16_to_numpy(y), ref)
+    assert e < QLINEAR_RTOL, e
