@@ -154,26 +154,26 @@ __global__ void __launch_bounds__(kQRMaxWarps * 32, 1) quantize_rotated_kernel(c
     for (int c = lane; c < chunks; c += 32) {
       const uint4 v = rowtile::lds128(rbase + 16u * c);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint64_t packed = 0;
+      uint32_t pw[2] = {0u, 0u};                    // the chunk's 8 codes, LSB first (8*BITS bits)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float a = bad ? 0.f : __uint_as_float(w[j] << 16);
         const float b = bad ? 0.f : __uint_as_float(w[j] & 0xFFFF0000u);
         uint32_t c0, c1;
         enc.codes(rowtile::pk(a, b), c0, c1);
-        packed |= static_cast<uint64_t>(c0) << (2 * j * BITS);
-        packed |= static_cast<uint64_t>(c1) << ((2 * j + 1) * BITS);
+        rowtile::put_code<BITS>(pw, 2 * j, c0);
+        rowtile::put_code<BITS>(pw, 2 * j + 1, c1);
       }
       unsigned char* dst = out + static_cast<long long>(c) * BITS;
       if constexpr (BITS == 8) {
-        __stcs(reinterpret_cast<unsigned long long*>(dst), static_cast<unsigned long long>(packed));
+        __stcs(reinterpret_cast<uint2*>(dst), make_uint2(pw[0], pw[1]));
       } else if constexpr (BITS == 4) {
-        __stcs(reinterpret_cast<unsigned int*>(dst), static_cast<unsigned int>(packed));
+        __stcs(reinterpret_cast<unsigned int*>(dst), pw[0]);
       } else if constexpr (BITS == 2) {
-        __stcs(reinterpret_cast<unsigned short*>(dst), static_cast<unsigned short>(packed));
+        __stcs(reinterpret_cast<unsigned short*>(dst), static_cast<unsigned short>(pw[0]));
       } else {
 #pragma unroll
-        for (int q = 0; q < BITS; ++q) dst[q] = static_cast<unsigned char>(packed >> (8 * q));
+        for (int q = 0; q < BITS; ++q) dst[q] = static_cast<unsigned char>(pw[q >> 2] >> (8 * (q & 3)));
       }
     }
     if (lane == 0) p.norms[t] = s;

@@ -162,6 +162,24 @@ def test_kernel_entry_points_validate_before_launch(lib):
     assert lib.qlinear_fp8_levels(fake, fake, 4, fake, fake, 4, 8, 8, 192, fake, None) == rbq.RBQ_EINVAL
     assert lib.qlinear_fp8_levels(fake, fake, 4, fake, fake, 4, 8, 4, 128, fake, None) == rbq.RBQ_EINVAL
     assert lib.qlinear_fp8_levels(fake, fake, 4, odd, fake, 4, 8, 8, 128, fake, None) == rbq.RBQ_EALIGN
+    # the rotation fused into the code layer, and the quantiser on rotated rows
+    nx = rbq.RPBH(512, 1)
+    n = nx.handle
+    assert lib.qlinear_rotate_next(None, None, 4, None, None, 4, 0, 128, n, rbq.RBQ_ACT_GELU, None, None) == rbq.RBQ_OK
+    assert lib.qlinear_rotate_next(fake, fake, 4, fake, fake, 4, 8, 128, None, 0, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_rotate_next(fake, fake, 4, fake, fake, 4, 8, 96, n, 0, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_rotate_next(fake, fake, 9, fake, fake, 4, 8, 128, n, 0, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_rotate_next(fake, fake, 4, fake, fake, 4, 8, 128, n, 2, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_rotate_next(fake, fake, 4, fake, None, 4, 8, 128, n, 0, fake, None) == rbq.RBQ_EINVAL
+    assert lib.qlinear_rotate_next(fake, fake, 4, odd, fake, 4, 8, 128, n, 0, fake, None) == rbq.RBQ_EALIGN
+    assert lib.quantize_rotated(None, rbq.RBQ_BF16, 0, 256, 4, None, None, None) == rbq.RBQ_OK
+    assert lib.quantize_rotated(fake, rbq.RBQ_F32, 4, 256, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_rotated(fake, rbq.RBQ_BF16, 4, 200, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_rotated(fake, rbq.RBQ_BF16, 4, 256, 0, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_rotated(fake, rbq.RBQ_BF16, -1, 256, 4, fake, fake, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_rotated(fake, rbq.RBQ_BF16, 4, 256, 4, fake, None, None) == rbq.RBQ_EINVAL
+    assert lib.quantize_rotated(odd, rbq.RBQ_BF16, 4, 256, 4, fake, fake, None) == rbq.RBQ_EALIGN
+    nx.close()
     r.close()
 
 
