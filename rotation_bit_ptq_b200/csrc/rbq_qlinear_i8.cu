@@ -32,9 +32,9 @@
 //                  of two int32 TMEM accumulators, so the epilogue of tile i
 //                  overlaps the MMAs of tile i+1.
 //      warp 5      TMA producer (one thread): this CTA's operand tiles of
-//                  each slice into the ring, 128B-swizzled K-major; no
-//                  multicast (a pair splits the weight tile, it does not
-//                  copy it).
+//                  each slice into the ring, 128B-swizzled K-major (a pair
+//                  splits the weight tile between its CTAs, each loading
+//                  its own part).
 // (Expanding the activation codes inside the GEMM, as the fp16 qlinear kernel
 // does, measured slower here: at twice the tensor rate the expansion warps
 // set the pace, 57.3 vs 51.4 us at 4608 x 3072 x 3072 W4A4.)

@@ -21,8 +21,8 @@
 //      warp 5      TMA producer: this CTA's x' tile (128 x 64) and its part
 //                  of the weight tile (256 x 64, or 128 x 64 for a pair) of
 //                  each slice into the ring (4 stages of 48 KB, or 6 of 32
-//                  KB), both 128B-swizzled K-major.  No multicast: a pair's
-//                  weight tile is split between the two CTAs, not copied.
+//                  KB), both 128B-swizzled K-major.  A pair's weight tile
+//                  is split between the two CTAs, each loading its part.
 //    Two TMEM accumulators (2 x 256 columns) let the epilogue of tile i
 //    overlap the MMAs of tile i+1.
 //    Fused with the next layer's rotation (qlinear_int8_rotate_next, see

@@ -92,7 +92,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// ---- TMA (bulk tensor copies, no multicast) ----------------------------------
+// ---- TMA (bulk tensor copies into this CTA's own shared memory) -------------
 // 2D tile global -> shared, completion counted on `bar` in bytes.  `tmap` is a
 // CUtensorMap passed as a __grid_constant__ kernel parameter.
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
@@ -232,8 +232,8 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // 2D tile global -> this CTA's shared memory, completion counted in bytes on
-// an mbarrier of either CTA of the pair (shared::cluster address).  No
-// multicast: each CTA loads only its own half of a pair's operands.
+// an mbarrier of either CTA of the pair (shared::cluster address).  Each CTA
+// loads only its own half of a pair's operands, into its own shared memory.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const void* tmap, int x, int y, uint32_t bar_cluster) {
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
