@@ -45,7 +45,7 @@ D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
 # rotate-quantize capture ran 32768 tokens; its bytes are scaled to this
 # workload's 4608 by the token count (its traffic grows with the tokens).
 QLINEAR_DRAM_BYTES = (11_848_704 + 453_120) + (47_240_448 + 3_493_632)
-ROTQ_DRAM_BYTES = round((201_408_512 + 27_977_216) * 4608 / 32768)
+ROTQ_DRAM_BYTES = round((201_406_720 + 28_677_376) * 4608 / 32768)
 METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
 

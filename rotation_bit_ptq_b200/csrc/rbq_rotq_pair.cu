@@ -394,8 +394,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
       }
       const long long cp = static_cast<long long>(p.d) * BITS / 8;
       unsigned char* out = static_cast<unsigned char*>(p.out) + static_cast<long long>(b) * 8 * BITS;
-      if (ok0) store_codes<BITS>(out + t0 * cp, w0);
-      if (ok1) store_codes<BITS>(out + t1 * cp, w1);
+      if (ok0) store_codes<BITS>(out + t0 * cp, w0, p.st256 != 0);
+      if (ok1) store_codes<BITS>(out + t1 * cp, w1, p.st256 != 0);
       if (b == 0) {
         if (MODE == kAct) {
           if (ok0) static_cast<float*>(p.aux)[t0] = s0;
@@ -688,6 +688,9 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     p.tab = t;
   }
   p.ntiles = static_cast<int>((rows + 2 * P - 1) / (2 * P));
+  // 32-byte code stores need every row's block start 32-byte aligned
+  p.st256 = (lloyd && reinterpret_cast<uintptr_t>(out) % 32 == 0 &&
+             (static_cast<long long>(r->d) * bits / 8) % 32 == 0) ? 1 : 0;
   switch (mode) {
     case kAct: return launch_pair_bits<kAct>(bits, P, tab16, p, st);
     case kWeightLM: return launch_pair_bits<kWeightLM>(bits, P, tab16, p, st);

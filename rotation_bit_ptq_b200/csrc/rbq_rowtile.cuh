@@ -43,6 +43,7 @@ struct Params {
   unsigned int* err;
   const float* fixed_scale;          // INT8: one scale for every row (not written back), else null
   uint8_t* zero_point;               // asymmetric INT8: one per row
+  int st256;                         // output rows 32-byte aligned: 32-byte stores allowed
 };
 
 // Shared-memory layout (bytes from the 128-aligned base).
@@ -210,8 +211,26 @@ __device__ __forceinline__ void put_code(uint32_t* w, int i, uint32_t code) {
   }
 }
 
+// 32 bytes (eight words) to global memory in one streaming store; dst must be
+// 32-byte aligned.
+__device__ __forceinline__ void st_v8_cs(void* dst, const uint32_t* w) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// One block's codes (8*BITS bytes) of one row.  wide: dst is 32-byte aligned,
+// so 4- and 8-bit codes go out as 32-byte stores -- the four lanes of a warp
+// that hold one row's consecutive blocks then write whole 128-byte lines.
 template <int BITS>
-__device__ __forceinline__ void store_codes(unsigned char* dst, const uint32_t* w) {
+__device__ __forceinline__ void store_codes(unsigned char* dst, const uint32_t* w, bool wide = false) {
+  if constexpr ((BITS % 4) == 0) {
+    if (wide) {
+#pragma unroll
+      for (int i = 0; i < BITS / 4; ++i) st_v8_cs(dst + 32 * i, w + 8 * i);
+      return;
+    }
+  }
   if constexpr ((BITS % 2) == 0) {
 #pragma unroll
     for (int i = 0; i < BITS / 2; ++i)
