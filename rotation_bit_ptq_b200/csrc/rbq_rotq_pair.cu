@@ -527,19 +527,30 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) rotq_pair_kernel(Params p) 
           ub0[k2] = bf2_bits(y[0][0] * 0.125f, y[1][0] * 0.125f);
           ub1[k2] = bf2_bits(y[0][1] * 0.125f, y[1][1] * 0.125f);
         }
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        if (p.st256) {                 // 32-byte aligned rows: one store per 16 values
           if (ok0) {
-            __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 16 * c) + q,
-                   make_uint4(ua0[4 * q], ua0[4 * q + 1], ua0[4 * q + 2], ua0[4 * q + 3]));
-            __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 32 + 16 * c) + q,
-                   make_uint4(ub0[4 * q], ub0[4 * q + 1], ub0[4 * q + 2], ub0[4 * q + 3]));
+            st_v8_cs(out + t0 * p.d + 16 * c, ua0);
+            st_v8_cs(out + t0 * p.d + 32 + 16 * c, ub0);
           }
           if (ok1) {
-            __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 16 * c) + q,
-                   make_uint4(ua1[4 * q], ua1[4 * q + 1], ua1[4 * q + 2], ua1[4 * q + 3]));
-            __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 32 + 16 * c) + q,
-                   make_uint4(ub1[4 * q], ub1[4 * q + 1], ub1[4 * q + 2], ub1[4 * q + 3]));
+            st_v8_cs(out + t1 * p.d + 16 * c, ua1);
+            st_v8_cs(out + t1 * p.d + 32 + 16 * c, ub1);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            if (ok0) {
+              __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 16 * c) + q,
+                     make_uint4(ua0[4 * q], ua0[4 * q + 1], ua0[4 * q + 2], ua0[4 * q + 3]));
+              __stcs(reinterpret_cast<uint4*>(out + t0 * p.d + 32 + 16 * c) + q,
+                     make_uint4(ub0[4 * q], ub0[4 * q + 1], ub0[4 * q + 2], ub0[4 * q + 3]));
+            }
+            if (ok1) {
+              __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 16 * c) + q,
+                     make_uint4(ua1[4 * q], ua1[4 * q + 1], ua1[4 * q + 2], ua1[4 * q + 3]));
+              __stcs(reinterpret_cast<uint4*>(out + t1 * p.d + 32 + 16 * c) + q,
+                     make_uint4(ub1[4 * q], ub1[4 * q + 1], ub1[4 * q + 2], ub1[4 * q + 3]));
+            }
           }
         }
       }
@@ -688,9 +699,10 @@ int rotq_pair_launch(const rbq_rpbh* r, int mode, int bits, long long rows, cons
     p.tab = t;
   }
   p.ntiles = static_cast<int>((rows + 2 * P - 1) / (2 * P));
-  // 32-byte code stores need every row's block start 32-byte aligned
-  p.st256 = (lloyd && reinterpret_cast<uintptr_t>(out) % 32 == 0 &&
-             (static_cast<long long>(r->d) * bits / 8) % 32 == 0) ? 1 : 0;
+  // 32-byte stores need every row's block start 32-byte aligned (rotate-only
+  // rows are 2d bytes, a multiple of 512)
+  p.st256 = (reinterpret_cast<uintptr_t>(out) % 32 == 0 &&
+             ((lloyd && (static_cast<long long>(r->d) * bits / 8) % 32 == 0) || mode == kRotate)) ? 1 : 0;
   switch (mode) {
     case kAct: return launch_pair_bits<kAct>(bits, P, tab16, p, st);
     case kWeightLM: return launch_pair_bits<kWeightLM>(bits, P, tab16, p, st);
