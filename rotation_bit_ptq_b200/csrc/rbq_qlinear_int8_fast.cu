@@ -108,7 +108,15 @@ struct Params {
   const float* next_sign;     // rotating epilogues: D of the next layer (+-1, output position order)
   uint16_t* Y;
   unsigned int* err;
+  int y32;                    // Y 32-byte aligned with N % 16 == 0: 32-byte output stores
 };
+
+// 32 bytes (eight words) to global memory in one store; dst 32-byte aligned.
+__device__ __forceinline__ void st_v8(void* dst, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
 
 // GELU(y) = y Phi(y) with the normal CDF from Abramowitz & Stegun (1964),
 // formula 7.1.26 (Hastings' rational approximation of erf, |error| <= 1.5e-7
@@ -440,10 +448,17 @@ __global__ void __launch_bounds__(threads_for(EPI), 1)
             const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * c0, __uint_as_float(v[2 * j + 1]) * c1);
             packed[j] = *reinterpret_cast<const uint32_t*>(&h);
           }
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          // a lane writes 64 bytes of its own row: as two 32-byte stores each
+          // fills whole sectors (16-byte stores leave every piece alone in one)
+          if (p.y32) {
+            st_v8(dst, packed);
+            st_v8(dst + 16, packed + 8);
+          } else {
+            uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            for (int j = 0; j < 4; ++j)
+              d4[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
@@ -588,6 +603,7 @@ int launch_gemm(const uint16_t* A, const uint16_t* B, const Params& p, cudaStrea
   const int tile_m = pair ? Geom<true>::kTileM : Geom<false>::kTileM;
   Params q = p;
   q.order = tile_order(dev, 2LL * p.M * p.K, 2LL * p.N * p.K);
+  q.y32 = (reinterpret_cast<uintptr_t>(p.Y) % 32 == 0 && p.N % 16 == 0) ? 1 : 0;
   CUtensorMap mA, mB;
   int rc = encode_bf16_map(&mA, A, p.M, p.K, kBM, kQ);
   if (rc == RBQ_OK) rc = encode_bf16_map(&mB, B, p.N, p.K, pair ? Geom<true>::kBNc : Geom<false>::kBNc, kQ);
