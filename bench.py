@@ -37,14 +37,14 @@ import synth  # noqa: E402
 D, T, BITS_A, BITS_W, SEED = 3072, 4608, 4, 4, 0
 
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel as
-# it stands (profiles/qlinear_W4A4_4608x3072x3072.md,
-# profiles/rotate_quantize_act_d3072_T32768_A4.md).  qlinear: both launches of
-# one call (code expansion of weights and activations + GEMM), caches flushed
-# before each kernel, so the GEMM reads both fp16 workspaces back from DRAM
-# and most of the 28 MB output is still in L2 when it ends.  The
+# it stands (profiles/rotate_quantize_act_d3072_T32768_A4.md), or None once
+# the kernel has changed since its counters were taken.  qlinear: the last
+# capture of both launches of one call (code expansion + GEMM, caches flushed
+# before each) gave (11_848_704 + 453_120) + (47_240_448 + 3_493_632) bytes;
+# the GEMM's output stores changed after it, so no figure is reported.  The
 # rotate-quantize capture ran 32768 tokens; its bytes are scaled to this
 # workload's 4608 by the token count (its traffic grows with the tokens).
-QLINEAR_DRAM_BYTES = (11_848_704 + 453_120) + (47_240_448 + 3_493_632)
+QLINEAR_DRAM_BYTES = None
 ROTQ_DRAM_BYTES = round((201_406_720 + 28_677_376) * 4608 / 32768)
 METRIC = "rotate_quantize GB/s (% HBM peak); qlinear TFLOP/s (% BF16 TC peak)"
 WORKLOAD = "attn_proj d=3072 T=4608 W4A4 h=64 (Student-t(3) acts, 1% channels x30; N(0,0.02^2) weights)"
@@ -334,8 +334,8 @@ def run_ours(args, rank, world):
                      "frac": round(flops / k2_avg_s / 1e12 / pk["bf16_tflops"], 4), "traffic": QLINEAR_DRAM_BYTES,
                      "peak_source": pk["source"] + " bf16 burst",
                      "note": "achieved includes the per-call code expansion launch (weights and activations); "
-                             "traffic is the ncu DRAM read + write of the two launches of one call "
-                             "(expansion + GEMM)",
+                             "traffic (the ncu DRAM read + write of the two launches of one call) is null: "
+                             "the GEMM's epilogue changed after the last capture",
                      "algorithmic_bytes": qlinear_algorithmic_bytes(),
                      "workspace_round_trip_bytes": 2 * 2 * (D * D + T * D)},
         "roofline_rotate_quantize": {"kernel": "rotate_quantize_act", "bound": "hbm",
